@@ -1,0 +1,582 @@
+#!/usr/bin/env python
+"""Benchmark of layerwise QK-Norm on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+A step is one fused QK-Norm pass (qknorm_fwd: Algorithm 1 Phases A-C for Q
+and K, launch chosen by the selector) over the 13B-shaped prefill batch:
+T = 8192 tokens per GPU, Dq = Dk = 5120, bf16, P = 4, eps = 1e-6. Tokens are
+independent, so N GPUs each run their own batch (weak scaling, no collective
+on the data path); value = algorithmic bytes of all ranks / max-over-ranks
+device time. The split path, the decode latencies and the GQA shapes are
+measured after the timed region and reported beside it.
+
+--impl reference times the float64 CPU oracle (the only reference this
+method has) on the same workload, a bounded sample of rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import qknorm_workloads as W  # noqa: E402
+
+METRIC = "QK-Norm GB/s and % of B200 HBM peak (prefill); μs/call at decode T≤64"
+HEADLINE = "prefill13b"
+FALLBACK_HBM_GBS = 6650.0
+
+# dram bytes per launch of the headline kernel from one ncu capture, and the
+# hash of the kernel sources it was taken with (None until captured).
+NCU_TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the decode / GQA / split measurements after the timed region")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def kernel_src_sha() -> str:
+    csrc = os.path.join(ROOT, "qk_norm_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs: STREAM-style copy)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier measurement on this pool)"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ----------------------------------------------------------------------------- distributed
+
+class Dist:
+    """Rank bookkeeping. Under torchrun (WORLD_SIZE > 1) an NCCL process group
+    with a short timeout carries the barriers and the max-over-ranks reduction."""
+
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, value: float, device) -> float:
+        if self.pg is None:
+            return value
+        import torch
+        t = torch.tensor([value], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def shard_tokens(T_global: int, world: int, rank: int):
+    """Contiguous token range [start, stop) of this rank (the remainder goes to
+    the first ranks)."""
+    base, rem = divmod(T_global, world)
+    start = rank * base + min(rank, rem)
+    return start, start + base + (1 if rank < rem else 0)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sync_boost": 0x10,
+        "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML absent: report it instead of clocks
+            self.error = f"{type(e).__name__}: {e}"
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        return False
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples), "source": "NVML, sampled during the timed region"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+def nvml_index(torch, device) -> int:
+    """NVML index of a CUDA device (honours CUDA_VISIBLE_DEVICES)."""
+    fn = getattr(torch.cuda, "_get_nvml_device_index", None)
+    try:
+        return int(fn(device)) if fn else int(device.index or 0)
+    except Exception:
+        return int(device.index or 0)
+
+
+# ----------------------------------------------------------------------------- native arm
+
+class Fused:
+    """Raw C-ABI call of qknorm_fwd for one buffer set (no per-call Python
+    marshalling beyond ctypes)."""
+
+    def __init__(self, qk, bufs, T, Dq, Dk, P, eps, dtype_code, stream):
+        q, k, gq, gk, oq, ok = bufs
+        self.fn = qk.lib.qknorm_fwd
+        self.args = (q.data_ptr(), k.data_ptr(), gq.data_ptr(), gk.data_ptr(), oq.data_ptr(),
+                     ok.data_ptr(), T, Dq, Dk, P, eps, dtype_code, stream)
+        self.qk = qk
+
+    def __call__(self):
+        st = self.fn(*self.args)
+        if st != 0:
+            raise RuntimeError(f"qknorm_fwd: {self.qk.qknorm_status_string(st)} "
+                               f"{self.qk.qknorm_last_error()}")
+
+
+def device_inputs(torch, wl, T, device, row0=0):
+    """q, k (bf16 or fp32) drawn on the device with the workload's recipe, and
+    gamma; rows start at row0."""
+    from qknorm_workloads import gen_gamma
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    q = W.gen_device_workload(wl, "q", T, device, row0)
+    k = W.gen_device_workload(wl, "k", T, device, row0)
+    return q, k, dev(gen_gamma(wl, "q")), dev(gen_gamma(wl, "k"))
+
+
+def time_launches(torch, calls, steps, stream):
+    """Run `calls` round-robin for `steps` launches; returns (total_ms, [per-launch ms])."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        calls[i % len(calls)]()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    t1.synchronize()
+    return t0.elapsed_time(t1), [a.elapsed_time(b) for a, b in ev]
+
+
+def latency_us(torch, qk, wl, T, device, n_eager=400, n_graph=100, graph_reps=10):
+    """µs per qknorm_fwd call at a small T: back-to-back eager launches through
+    ctypes, and the same calls replayed from a CUDA graph."""
+    stream = torch.cuda.current_stream(device)
+    q, k, gq, gk = device_inputs(torch, wl, T, device)
+    bufs = (q, k, gq, gk, torch.empty_like(q), torch.empty_like(k))
+    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    f = Fused(qk, bufs, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+    for _ in range(50):
+        f()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n_eager):
+        f()
+    t1.record(stream)
+    t1.synchronize()
+    eager = t0.elapsed_time(t1) * 1000.0 / n_eager
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fc = Fused(qk, bufs, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt,
+                   torch.cuda.current_stream(device).cuda_stream)
+        for _ in range(n_graph):
+            fc()
+    g.replay()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(graph_reps):
+        g.replay()
+    t1.record(stream)
+    t1.synchronize()
+    graph = t0.elapsed_time(t1) * 1000.0 / (n_graph * graph_reps)
+    del g
+    return {"eager_us": round(eager, 3), "graph_us": round(graph, 3)}
+
+
+def throughput(torch, qk, wl, T, device, sets, steps=50):
+    """GB/s of the fused path on T tokens with `sets` rotating buffer sets."""
+    stream = torch.cuda.current_stream(device)
+    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    q, k, gq, gk = device_inputs(torch, wl, T, device)
+    calls = []
+    for s in range(sets):
+        qs, ks = (q, k) if s == 0 else (q.clone(), k.clone())
+        calls.append(Fused(qk, (qs, ks, gq, gk, torch.empty_like(q), torch.empty_like(k)), T,
+                           wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream))
+    for i in range(10):
+        calls[i % sets]()
+    torch.cuda.synchronize()
+    _, per = time_launches(torch, calls, steps, stream)
+    ms = statistics.mean(per)
+    nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes)
+    return {"T": T, "us_per_call": round(ms * 1000, 3), "GB_s": round(nbytes / ms / 1e6, 1),
+            "algorithmic_bytes": nbytes, "buffer_sets": sets}
+
+
+def split_path(torch, qk, device, peak, steps=20):
+    """The split path (stats + apply for Q and K: 4 launches) and the fused path
+    on the large-prefill workload, T = 65536, D = 4096, P = 8, bf16."""
+    wl = W.WORKLOADS["split_large"]
+    T = wl.Ts[0]
+    stream = torch.cuda.current_stream(device)
+    h = stream.cuda_stream
+    q, k, gq, gk = device_inputs(torch, wl, T, device)
+    oq, ok, aq, ak = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(q), torch.empty_like(k))
+    sq = torch.empty((T, wl.P), dtype=torch.float32, device=device)
+    sk = torch.empty_like(sq)
+    L = qk.lib
+    D, P, eps = wl.Dq, wl.P, wl.eps
+
+    def check(st):
+        if st != 0:
+            raise RuntimeError(qk.qknorm_status_string(st))
+
+    def stats_q():
+        check(L.qknorm_partial_sumsq(q.data_ptr(), sq.data_ptr(), T, D, P, 1, h))
+
+    def stats_k():
+        check(L.qknorm_partial_sumsq(k.data_ptr(), sk.data_ptr(), T, D, P, 1, h))
+
+    def apply_q():
+        check(L.qknorm_apply(q.data_ptr(), gq.data_ptr(), sq.data_ptr(), aq.data_ptr(), T, D, P, eps, 1, h))
+
+    def apply_k():
+        check(L.qknorm_apply(k.data_ptr(), gk.data_ptr(), sk.data_ptr(), ak.data_ptr(), T, D, P, eps, 1, h))
+
+    fused = Fused(qk, (q, k, gq, gk, oq, ok), T, D, D, P, eps, 1, h)
+    seq = [stats_q, stats_k, apply_q, apply_k]
+    for _ in range(3):
+        for c in seq + [fused]:
+            c()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(aq.view(torch.int16), oq.view(torch.int16)) and
+                torch.equal(ak.view(torch.int16), ok.view(torch.int16)))
+    _, per_split = time_launches(torch, seq, 4 * steps, stream)
+    _, per_fused = time_launches(torch, [fused], steps, stream)
+    st_ms = statistics.mean(per_split[0::4] + per_split[1::4])
+    ap_ms = statistics.mean(per_split[2::4] + per_split[3::4])
+    split_ms = 2 * st_ms + 2 * ap_ms
+    fused_ms = statistics.mean(per_fused)
+    b_split = 2 * W.split_bytes(T, D, P, 2)
+    b_fused = W.fused_bytes(T, D, D, 2)
+    b_stats = W.stats_bytes(T, D, P, 2)
+    b_apply = W.apply_bytes(T, D, P, 2)
+    return {
+        "workload": wl.note, "fused_equals_split_bitwise": same,
+        "split": {"ms_per_step": round(split_ms, 4), "GB_s": round(b_split / split_ms / 1e6, 1),
+                  "pct_hbm_peak": round(100 * b_split / split_ms / 1e6 / peak, 1),
+                  "algorithmic_bytes": b_split,
+                  "stats_kernel": {"us": round(st_ms * 1000, 2),
+                                   "GB_s": round(b_stats / st_ms / 1e6, 1)},
+                  "apply_kernel": {"us": round(ap_ms * 1000, 2),
+                                   "GB_s": round(b_apply / ap_ms / 1e6, 1)}},
+        "fused": {"ms_per_step": round(fused_ms, 4), "GB_s": round(b_fused / fused_ms / 1e6, 1),
+                  "pct_hbm_peak": round(100 * b_fused / fused_ms / 1e6 / peak, 1),
+                  "algorithmic_bytes": b_fused},
+    }
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_rows_rate(wl, n_rows, nthreads, target_s):
+    """Run the float64 oracle on n_rows tokens of Q and K until target_s has
+    passed; returns (passes, seconds)."""
+    import oracle
+    orc = oracle.get()
+    rows = np.arange(n_rows)
+    q, k = W.gen_rows(wl, "q", rows), W.gen_rows(wl, "k", rows)
+    gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
+    eps = float(np.float32(wl.eps))
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=nthreads)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            return passes, el
+
+
+def cpu_baseline(wl, T, target_s=10.0):
+    cores = host_cores()
+    n = min(T, 2048)
+    passes, el = oracle_rows_rate(wl, n, cores, target_s)
+    nbytes = passes * W.fused_bytes(n, wl.Dq, wl.Dk, wl.elem_bytes)
+    return {"value": round(nbytes / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of the {T} tokens (Q and K rows), {passes} passes in {el:.1f} s, "
+                      f"float64 C oracle with OpenMP over tokens on {cores} threads ({cpu_model()})",
+            "tokens_per_s": round(passes * n / el, 1)}
+
+
+def config_of(wl, T, world):
+    return {"workload": wl.note, "T_per_gpu": T, "global_tokens": T * world, "Dq": wl.Dq,
+            "Dk": wl.Dk, "P": wl.P, "eps": wl.eps, "storage": wl.dtype,
+            "accumulation": "fp32", "parallelism": f"token-sharded dp{world} (no collective)",
+            "l2": "inputs larger than L2: two rotating buffer sets of 336 MB each"}
+
+
+def run_reference(args, dist):
+    """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
+    if dist.rank != 0:
+        return 0
+    wl = W.WORKLOADS[HEADLINE]
+    T = wl.Ts[0]
+    cores = host_cores()
+    # Calibrate: rows per step so that warmup + steps take about two minutes.
+    p, el = oracle_rows_rate(wl, 64, cores, 0.5)
+    per_row = el / (p * 64)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(T, max(16, budget / per_row)))
+    import oracle
+    orc = oracle.get()
+    rows = np.arange(n)
+    q, k = W.gen_rows(wl, "q", rows), W.gen_rows(wl, "k", rows)
+    gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
+    eps = float(np.float32(wl.eps))
+    for _ in range(args.warmup):
+        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=cores)
+    el = time.perf_counter() - t0
+    nbytes = W.fused_bytes(n, wl.Dq, wl.Dk, wl.elem_bytes)
+    value = args.steps * nbytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1000 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, T, args.gpus),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} of the {T} tokens (Q and K rows) per step, float64 C "
+                                   f"oracle, OpenMP over tokens on {cores} threads ({cpu_model()})"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_native(args, dist):
+    import torch
+    import qk_norm_attention_b200 as qk
+
+    device = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(device)
+    dist.init("nccl")
+    wl = W.WORKLOADS[HEADLINE]
+    T = wl.Ts[0]                       # tokens per GPU (weak scaling)
+    row0, _ = shard_tokens(T * dist.world, dist.world, dist.rank)
+    stream = torch.cuda.current_stream(device)
+    peak, peak_src = hbm_peak()
+    dt = qk.QKNORM_BF16
+
+    q, k, gq, gk = device_inputs(torch, wl, T, device, row0)
+    sets = [(q, k), (q.clone(), k.clone())]
+    calls = [Fused(qk, (a, b, gq, gk, torch.empty_like(a), torch.empty_like(b)), T, wl.Dq, wl.Dk,
+                   wl.P, wl.eps, dt, stream.cuda_stream) for a, b in sets]
+    plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, dt)
+    for i in range(max(3, args.warmup)):
+        calls[i % 2]()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(nvml_index(torch, device)) as clk:
+        total_ms, per = time_launches(torch, calls, args.steps, stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = dist.max(total_ms / args.steps, device)
+    kern_ms = dist.max(statistics.mean(per), device)
+    nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes)
+    value = dist.world * nbytes / step_ms / 1e6          # GB/s, all ranks
+    achieved = nbytes / kern_ms / 1e6                    # GB/s, one launch
+
+    # End to end through the same C ABI: pinned host -> device, kernel, device -> host.
+    e2e_steps = max(3, min(args.steps, 30))
+    qh, kh = q.cpu().pin_memory(), k.cpu().pin_memory()
+    oqh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    okh = torch.empty(k.shape, dtype=k.dtype).pin_memory()
+    qd, kd = sets[1]
+    oqd, okd = (torch.empty_like(q), torch.empty_like(k))
+    f = Fused(qk, (qd, kd, gq, gk, oqd, okd), T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        f()
+        oqh.copy_(oqd, non_blocking=True)
+        okh.copy_(okd, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    e2e_ms = dist.max(e0.elapsed_time(e1) / e2e_steps, device)
+    h2d = (qh.numel() + kh.numel()) * qh.element_size()
+    d2h = (oqh.numel() + okh.numel()) * oqh.element_size()
+    del qh, kh, oqh, okh
+
+    extras = {}
+    if dist.rank == 0 and not args.no_extras:
+        dec = W.WORKLOADS["decode"]
+        extras["decode_us_per_call"] = {str(t): latency_us(torch, qk, dec, t, device) for t in dec.Ts}
+        gqa = W.WORKLOADS["gqa"]
+        extras["gqa"] = {"us_per_call": {str(t): latency_us(torch, qk, gqa, t, device)
+                                         for t in gqa.Ts if t <= 256},
+                         "T4096": throughput(torch, qk, gqa, 4096, device, sets=4)}
+        extras["gqa"]["T4096"]["pct_hbm_peak"] = round(100 * extras["gqa"]["T4096"]["GB_s"] / peak, 1)
+        extras["split_large"] = split_path(torch, qk, device, peak)
+    dist.barrier()
+
+    traffic = None
+    if NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"]:
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    line = {
+        "impl": "native",
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(wl, T, dist.world),
+        "pct_hbm_peak": round(100 * value / dist.world / peak, 2),
+        "tokens_per_s": round(dist.world * T / step_ms * 1000, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "fused_cta (qknorm_fwd)", "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "kernel_us": round(kern_ms * 1000, 3)},
+        "e2e": {"value": round(dist.world * nbytes / e2e_ms / 1e6, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
+                "path": "pinned host -> device copies, qknorm_fwd, device -> pinned host"},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "plan": plan,
+    }
+    line.update(extras)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, T)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("--steps must be >= 1 and --warmup >= 0")
+    dist = Dist()
+    if args.impl == "reference":
+        return run_reference(args, dist)
+    return run_native(args, dist)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,192 @@
+/*
+ * qknorm.h -- C ABI of libqknorm.so: layerwise Query-Key RMSNorm (QK-Norm)
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (SwiftQK technical review, "SwiftQK: When Normalization
+ * Becomes the Bottleneck of Tensor Parallelism", "Prerequisites", Eq. (1) and
+ * the layerwise QK-Norm paragraph): for every token t and each of the two
+ * tensors X in {Q, K}, with width D and learned weight gamma,
+ *
+ *     y[t,j] = x[t,j] * gamma[j] / sqrt( (1/D) * sum_j x[t,j]^2 + eps ).
+ *
+ * The mean of squares is formed the way Section 3, Algorithm 1 decomposes
+ * it: the width is cut into P equal logical shards, each shard's sum of
+ * squares S[t,p] is the only statistic (Phase A), the P scalars are added
+ * (Phase B), and x * gamma is formed independently of that sum (Phase B,
+ * compute path) before the factor is applied (Phase C). All accumulation is
+ * fp32 (Section 4, numerical precision). Here the P shards are slices of one
+ * row in one GPU's memory; nothing is exchanged between GPUs.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers on the current CUDA device unless stated.
+ *   The caller owns every buffer. The library allocates nothing and keeps
+ *   no state besides per-device caches of launch parameters.
+ * - Tensors are dense row-major: x[T, D] (row t starts at x + t*D), gamma[D]
+ *   fp32, stats[T, P] fp32 (row t holds S[t,0..P-1]).
+ * - dtype selects the storage type of x and y: QKNORM_F32 or QKNORM_BF16.
+ *   Accumulation and the factor are always fp32. y is rounded to nearest
+ *   even from fp32, once.
+ * - stream is a cudaStream_t (0 = legacy default stream). Calls only
+ *   enqueue work; none synchronises the host.
+ * - Every pointer must be 16-byte aligned, and the shard width D/P must be a
+ *   multiple of 8 (bf16) or 4 (fp32) elements, so that every row and shard
+ *   starts on a 16-byte vector.
+ * - An output may be the same buffer as its own input (exact in-place); any
+ *   other overlap between an output and any other buffer is rejected.
+ * - T == 0 returns QKNORM_OK and launches nothing.
+ * - Arguments are checked before anything is launched; a failed check
+ *   launches nothing and returns one of the codes below. A CUDA error at
+ *   launch returns QKNORM_ERR_CUDA; qknorm_last_error() gives its text.
+ *
+ * Reduction order (identical in every kernel of this library, so the fused
+ * path and the split path give bit-identical outputs): a shard of nv
+ * 16-byte vectors (8 bf16 or 4 fp32 values) is covered by K = ceil(nv/256)
+ * groups; group k, lane l (0..31) sums, in increasing i, the per-vector sums
+ * of squares of vectors v = 32k + l + 32Ki; the 32 lane sums are combined by
+ * an xor butterfly (16, 8, 4, 2, 1); the K group sums are added in order of
+ * k, giving S[t,p]; the P shard sums are added in order of p. A vector's sum
+ * of squares is e0*e0 followed by fused multiply-adds of e1..e_last.
+ * Then r = rsqrt(S / D + eps) and y = (x * gamma) * r, each step fp32.
+ */
+#ifndef QKNORM_H
+#define QKNORM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QKNORM_API __attribute__((visibility("default")))
+#else
+#define QKNORM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QKNORM_F32 = 0,
+    QKNORM_BF16 = 1
+} qknorm_dtype;
+
+typedef enum {
+    QKNORM_OK = 0,
+    QKNORM_ERR_INVALID_ARG = 1, /* null pointer with T > 0, T < 0, D <= 0, P <= 0,
+                                   D % P != 0, eps < 0 or not finite, overlapping
+                                   buffers */
+    QKNORM_ERR_MISALIGNED = 2,  /* a pointer not 16-byte aligned */
+    QKNORM_ERR_UNSUPPORTED = 3, /* unknown dtype, or D/P not a multiple of the
+                                   16-byte vector (8 bf16 / 4 fp32 elements) */
+    QKNORM_ERR_CUDA = 4         /* the CUDA runtime reported an error */
+} qknorm_status;
+
+/*
+ * qknorm_fwd -- the single-pass fused QK-Norm of Q and K.
+ *
+ * Algorithm 1 (Phases A, B and C) for every token of both tensors, in one
+ * launch: each element of q and k is read once from HBM and each element of
+ * out_q and out_k written once; the per-shard statistics never leave the SM.
+ *
+ *   q       [T, Dq] input, dtype          out_q [T, Dq] output, dtype
+ *   k       [T, Dk] input, dtype          out_k [T, Dk] output, dtype
+ *   gamma_q [Dq] fp32, gamma_k [Dk] fp32
+ *   T       tokens (rows); Dq, Dk widths; P logical shards of each width
+ *           (Dq/P and Dk/P are the shard widths)
+ *   eps     added to the mean of squares inside the root (Eq. (1))
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+               void *out_q, void *out_k, int64_t T, int32_t Dq, int32_t Dk, int32_t P,
+               float eps, int32_t dtype, void *stream);
+
+/*
+ * qknorm_partial_sumsq -- the statistics half of the split path.
+ *
+ * Algorithm 1, Phase A for one tensor: stats[t*P + p] = fp32 sum of
+ * squares of shard p of row t (the scalar each rank publishes to its IPC
+ * slot in the review's multi-GPU form), in the reduction order above.
+ *   x [T, D] input, dtype; stats [T, P] fp32 output.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int32_t P,
+                         int32_t dtype, void *stream);
+
+/*
+ * qknorm_apply -- the apply half of the split path.
+ *
+ * Algorithm 1, Phases B and C for one tensor, given the statistics:
+ * S = stats[t,0] + ... + stats[t,P-1] (in order of p), r = rsqrt(S/D + eps),
+ * out[t,j] = (x[t,j] * gamma[j]) * r. A caller that already holds combined
+ * per-token sums passes them as stats [T, 1] with P = 1.
+ *   x [T, D] input, dtype; gamma [D] fp32; stats [T, P] fp32; out [T, D].
+ * With stats from qknorm_partial_sumsq, out equals qknorm_fwd's bit for bit.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_apply(const void *x, const float *gamma, const float *stats, void *out,
+                 int64_t T, int32_t D, int32_t P, float eps, int32_t dtype, void *stream);
+
+/* Static text for a qknorm_status value ("unknown status" otherwise). */
+QKNORM_API const char *qknorm_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread ("" if none). */
+QKNORM_API const char *qknorm_last_error(void);
+
+/* Kernel variants of qknorm_fwd, for qknorm_plan_fwd and qknorm_force_variant. */
+typedef enum {
+    QKNORM_VARIANT_AUTO = -1,
+    QKNORM_VARIANT_CTA = 0,     /* CTA per token: one warp per (shard, group), row
+                                   held in registers, persistent grid, next token
+                                   prefetched when a CTA has more than one */
+    QKNORM_VARIANT_WARP = 1,    /* warp per token: one warp walks all shards of a
+                                   token, then re-reads the row to apply */
+    QKNORM_VARIANT_GENERIC = 2  /* CTA per token, any shape: warps loop over the
+                                   shard groups, re-read the row to apply */
+} qknorm_variant;
+
+/* A launch plan chosen by the selector (host-side description). */
+typedef struct {
+    int32_t variant;     /* qknorm_variant */
+    int32_t block;       /* threads per CTA */
+    int64_t grid;        /* CTAs */
+    int32_t vmax;        /* 16-byte vectors per lane per (shard, group); 0 if looped */
+    int32_t prefetch;    /* 1 if a CTA prefetches its next token */
+    int32_t groups_q;    /* K for a Q shard */
+    int32_t groups_k;    /* K for a K shard */
+} qknorm_plan;
+
+/*
+ * qknorm_plan_fwd -- the selector, as a pure host function (no CUDA call).
+ *
+ * Chooses the kernel variant, block and grid for qknorm_fwd given the shape
+ * and the device's SM count and resident-CTA count for the chosen kernel
+ * (num_sms, blocks_per_sm; pass <= 0 for blocks_per_sm to let the plan use
+ * its block-size-only estimate). Honours qknorm_force_variant. Returns
+ * QKNORM_OK and fills *plan, or an argument error code.
+ */
+QKNORM_API int qknorm_plan_fwd(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
+                    int32_t num_sms, int32_t blocks_per_sm, qknorm_plan *plan);
+
+/*
+ * qknorm_force_variant -- process-wide override of the selector for tests and
+ * benchmarks: variant (QKNORM_VARIANT_AUTO restores automatic choice) and,
+ * if grid > 0, the CTA count of a persistent launch. A forced variant that
+ * cannot run a shape makes qknorm_fwd return QKNORM_ERR_UNSUPPORTED.
+ * Not thread-safe with concurrent qknorm_fwd calls. Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_force_variant(int32_t variant, int64_t grid);
+
+/*
+ * qknorm_launch_plan -- the plan qknorm_fwd would use on the current device
+ * (queries the SM count and occupancy; no kernel runs). Returns a status.
+ */
+QKNORM_API int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
+                       qknorm_plan *plan);
+
+/* ABI version of this header (major * 100 + minor). */
+QKNORM_API int qknorm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNORM_H */

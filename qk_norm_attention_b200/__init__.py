@@ -1,0 +1,215 @@
+"""Layerwise Query-Key RMSNorm (QK-Norm) on NVIDIA B200: Python binding.
+
+A thin ctypes layer over ``libqknorm.so`` (C ABI in ``include/qknorm.h``).
+It only checks tensor metadata and passes pointers, sizes and the current
+CUDA stream; every step of the computation runs in the library's CUDA
+kernels. There is no CPU fallback: importing this package fails loudly if the
+library has not been built (``python qk_norm_attention_b200/csrc/build_lib.py``).
+
+Entry points (same names as the C ABI):
+
+* ``qknorm_fwd(q, k, gamma_q, gamma_k, P, eps, out_q=None, out_k=None)``:
+  the fused single-pass QK-Norm of Q [T, Dq] and K [T, Dk].
+* ``qknorm_partial_sumsq(x, P, stats=None)``: per-shard fp32 sums of squares,
+  stats [T, P].
+* ``qknorm_apply(x, gamma, stats, eps, out=None)``: the factor from stats and
+  (x * gamma) * r.
+
+Tensors are CUDA tensors, row-major contiguous, fp32 or bf16 for x/y and fp32
+for gamma and stats. Calls are asynchronous on ``torch.cuda.current_stream()``
+(or the ``stream`` argument).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libqknorm.so")
+
+QKNORM_F32, QKNORM_BF16 = 0, 1
+QKNORM_OK = 0
+QKNORM_ERR_INVALID_ARG = 1
+QKNORM_ERR_MISALIGNED = 2
+QKNORM_ERR_UNSUPPORTED = 3
+QKNORM_ERR_CUDA = 4
+
+VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC = -1, 0, 1, 2
+VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic"}
+
+_DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16}
+
+
+class QKNormError(RuntimeError):
+    """A libqknorm call returned a non-OK status."""
+
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{fn}: {qknorm_status_string(status)} (status {status})"
+        if detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+class QKNormPlan(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("grid", ctypes.c_int64), ("vmax", ctypes.c_int32),
+                ("prefetch", ctypes.c_int32), ("groups_q", ctypes.c_int32),
+                ("groups_k", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIBRARY):
+        raise ImportError(
+            f"libqknorm.so not found at {LIBRARY}; build it with "
+            "`python qk_norm_attention_b200/csrc/build_lib.py` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIBRARY)
+    vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    lib.qknorm_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32, vp]
+    lib.qknorm_partial_sumsq.argtypes = [vp, vp, i64, i32, i32, i32, vp]
+    lib.qknorm_apply.argtypes = [vp, vp, vp, vp, i64, i32, i32, f32, i32, vp]
+    for fn in (lib.qknorm_fwd, lib.qknorm_partial_sumsq, lib.qknorm_apply):
+        fn.restype = ctypes.c_int
+    lib.qknorm_status_string.argtypes = [ctypes.c_int]
+    lib.qknorm_status_string.restype = ctypes.c_char_p
+    lib.qknorm_last_error.argtypes = []
+    lib.qknorm_last_error.restype = ctypes.c_char_p
+    lib.qknorm_plan_fwd.argtypes = [i64, i32, i32, i32, i32, i32, i32, ctypes.POINTER(QKNormPlan)]
+    lib.qknorm_plan_fwd.restype = ctypes.c_int
+    lib.qknorm_launch_plan.argtypes = [i64, i32, i32, i32, i32, ctypes.POINTER(QKNormPlan)]
+    lib.qknorm_launch_plan.restype = ctypes.c_int
+    lib.qknorm_force_variant.argtypes = [i32, i64]
+    lib.qknorm_force_variant.restype = ctypes.c_int
+    lib.qknorm_version.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def qknorm_status_string(status: int) -> str:
+    return lib.qknorm_status_string(int(status)).decode()
+
+
+def qknorm_last_error() -> str:
+    return lib.qknorm_last_error().decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != QKNORM_OK:
+        raise QKNormError(fn, status, qknorm_last_error() if status == QKNORM_ERR_CUDA else "")
+
+
+def _stream_handle(device: torch.device, stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPE:
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.float32 or torch.bfloat16")
+    return _DTYPE[t.dtype]
+
+
+def _need_cuda_contig(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def qknorm_fwd(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+               P: int, eps: float, out_q: Optional[torch.Tensor] = None,
+               out_k: Optional[torch.Tensor] = None, stream=None):
+    """Fused layerwise QK-Norm of q [T, Dq] and k [T, Dk]; returns (out_q, out_k)."""
+    if q.dim() != 2 or k.dim() != 2 or q.shape[0] != k.shape[0]:
+        raise ValueError("q and k must be [T, Dq] and [T, Dk] with the same T")
+    if q.dtype != k.dtype:
+        raise TypeError("q and k must have the same dtype")
+    out_q = torch.empty_like(q) if out_q is None else out_q
+    out_k = torch.empty_like(k) if out_k is None else out_k
+    for name, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k),
+                    ("out_q", out_q), ("out_k", out_k)):
+        _need_cuda_contig(name, t)
+    if gamma_q.dtype != torch.float32 or gamma_k.dtype != torch.float32:
+        raise TypeError("gamma must be float32")
+    if out_q.shape != q.shape or out_k.shape != k.shape or out_q.dtype != q.dtype or out_k.dtype != k.dtype:
+        raise ValueError("outputs must match the inputs' shape and dtype")
+    if gamma_q.numel() != q.shape[1] or gamma_k.numel() != k.shape[1]:
+        raise ValueError("gamma_q/gamma_k must have Dq/Dk elements")
+    T, Dq = q.shape
+    Dk = k.shape[1]
+    st = lib.qknorm_fwd(q.data_ptr(), k.data_ptr(), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                        out_q.data_ptr(), out_k.data_ptr(), T, Dq, Dk, int(P), float(eps),
+                        _dtype_code(q), _stream_handle(q.device, stream))
+    _check("qknorm_fwd", st)
+    return out_q, out_k
+
+
+def qknorm_partial_sumsq(x: torch.Tensor, P: int, stats: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """stats[t, p] = fp32 sum of squares of shard p of row t; returns stats [T, P]."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T, D]")
+    T, D = x.shape
+    stats = torch.empty((T, int(P)), dtype=torch.float32, device=x.device) if stats is None else stats
+    _need_cuda_contig("x", x)
+    _need_cuda_contig("stats", stats)
+    if stats.dtype != torch.float32 or stats.numel() != T * int(P):
+        raise ValueError("stats must be float32 with T*P elements")
+    st = lib.qknorm_partial_sumsq(x.data_ptr(), stats.data_ptr(), T, D, int(P), _dtype_code(x),
+                                  _stream_handle(x.device, stream))
+    _check("qknorm_partial_sumsq", st)
+    return stats
+
+
+def qknorm_apply(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps: float,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out = (x * gamma) * rsqrt(sum_p stats[t, p] / D + eps); P = stats.shape[1]."""
+    if x.dim() != 2 or stats.dim() != 2 or stats.shape[0] != x.shape[0]:
+        raise ValueError("x must be [T, D] and stats [T, P]")
+    T, D = x.shape
+    P = stats.shape[1]
+    out = torch.empty_like(x) if out is None else out
+    for name, t in (("x", x), ("gamma", gamma), ("stats", stats), ("out", out)):
+        _need_cuda_contig(name, t)
+    if gamma.dtype != torch.float32 or stats.dtype != torch.float32:
+        raise TypeError("gamma and stats must be float32")
+    if out.shape != x.shape or out.dtype != x.dtype or gamma.numel() != D:
+        raise ValueError("out must match x; gamma must have D elements")
+    st = lib.qknorm_apply(x.data_ptr(), gamma.data_ptr(), stats.data_ptr(), out.data_ptr(), T, D,
+                          P, float(eps), _dtype_code(x), _stream_handle(x.device, stream))
+    _check("qknorm_apply", st)
+    return out
+
+
+def qknorm_plan_fwd(T: int, Dq: int, Dk: int, P: int, dtype: int, num_sms: int,
+                    blocks_per_sm: int = 0) -> dict:
+    """The selector's plan for a device with ``num_sms`` SMs (host logic only)."""
+    pl = QKNormPlan()
+    _check("qknorm_plan_fwd", lib.qknorm_plan_fwd(T, Dq, Dk, P, dtype, num_sms, blocks_per_sm,
+                                                  ctypes.byref(pl)))
+    return pl.as_dict()
+
+
+def qknorm_launch_plan(T: int, Dq: int, Dk: int, P: int, dtype: int) -> dict:
+    """The plan qknorm_fwd uses on the current device."""
+    pl = QKNormPlan()
+    _check("qknorm_launch_plan", lib.qknorm_launch_plan(T, Dq, Dk, P, dtype, ctypes.byref(pl)))
+    return pl.as_dict()
+
+
+def qknorm_force_variant(variant: int = VARIANT_AUTO, grid: int = 0) -> None:
+    """Override the selector process-wide (tests and benchmarks)."""
+    _check("qknorm_force_variant", lib.qknorm_force_variant(int(variant), int(grid)))
+
+
+def qknorm_version() -> int:
+    return lib.qknorm_version()

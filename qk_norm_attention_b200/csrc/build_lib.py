@@ -1,0 +1,75 @@
+"""Build libqknorm.so in-tree with nvcc for sm_100a (B200).
+
+Usage: ``python qk_norm_attention_b200/csrc/build_lib.py [--force] [--verbose]``.
+This script does not import the package (whose import loads the library).
+``--verbose`` passes ``-Xptxas -v`` (registers, spills, shared memory per kernel).
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import subprocess
+import sys
+
+CSRC = os.path.dirname(os.path.abspath(__file__))
+PKG = os.path.dirname(CSRC)
+ROOT = os.path.dirname(PKG)
+LIBRARY = os.path.join(PKG, "libqknorm.so")
+HEADER = os.path.join(ROOT, "include", "qknorm.h")
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+    "-shared", "-cudart", "static",
+]
+
+
+def sources():
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+
+
+def _inputs():
+    files = sources() + [os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                         if f.endswith((".cuh", ".h"))] + [HEADER, __file__]
+    return files
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIBRARY):
+        return False
+    t = os.path.getmtime(LIBRARY)
+    return all(os.path.getmtime(f) <= t for f in _inputs())
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
+        if cand and (os.path.sep not in cand or os.path.exists(cand)):
+            return cand
+    return "nvcc"
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu under csrc/ into libqknorm.so (skipped when up to date)."""
+    if not force and not verbose and up_to_date():
+        return LIBRARY
+    tmp = LIBRARY + ".tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
+    if verbose:
+        cmd += ["-Xptxas", "-v"]
+    cmd += ["-o", tmp, *sources()]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIBRARY)
+    return LIBRARY
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    args = ap.parse_args(argv)
+    print(build(force=args.force, verbose=args.verbose))
+
+
+if __name__ == "__main__":
+    sys.exit(main())

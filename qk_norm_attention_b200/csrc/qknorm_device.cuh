@@ -1,0 +1,136 @@
+// qknorm_device.cuh -- device building blocks shared by every kernel of
+// libqknorm: 16-byte vector loads and stores, the per-vector sum of squares,
+// the lane butterfly, the shard combine, the factor and the apply step.
+//
+// Every kernel builds its sums from these functions in the same order (the
+// order stated in include/qknorm.h), which is why qknorm_fwd and the split
+// path (qknorm_partial_sumsq + qknorm_apply) give bit-identical outputs.
+// All floating-point steps use explicitly rounded intrinsics so that the
+// compiler cannot contract or reorder them differently in different kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qkn {
+
+constexpr int kLanes = 32;
+constexpr int kVcap = 8;  // 16-byte vectors per lane per group; fixes K = ceil(nv / 256)
+constexpr unsigned kFull = 0xffffffffu;
+
+struct F32Tag {
+    static constexpr int kVec = 4;  // fp32 values per 16-byte vector
+    static constexpr int kBytes = 4;
+};
+struct BF16Tag {
+    static constexpr int kVec = 8;  // bf16 values per 16-byte vector
+    static constexpr int kBytes = 2;
+};
+
+// ---------------------------------------------------------------- widening
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ---------------------------------------------------------------- Phase A: x^2
+
+// Sum of squares of one vector: e0*e0, then e_i*e_i + q fused, i = 1..3.
+__device__ __forceinline__ float vsumsq(F32Tag, const uint4 &v) {
+    const float e0 = __uint_as_float(v.x), e1 = __uint_as_float(v.y);
+    const float e2 = __uint_as_float(v.z), e3 = __uint_as_float(v.w);
+    float q = __fmul_rn(e0, e0);
+    q = __fmaf_rn(e1, e1, q);
+    q = __fmaf_rn(e2, e2, q);
+    q = __fmaf_rn(e3, e3, q);
+    return q;
+}
+
+// Same for 8 bf16 values; element 0 is the low half of v.x.
+// (A bf16 square is exact in fp32, so each fma rounds only the running sum.)
+__device__ __forceinline__ float vsumsq(BF16Tag, const uint4 &v) {
+    float q = __fmul_rn(bf_lo(v.x), bf_lo(v.x));
+    q = __fmaf_rn(bf_hi(v.x), bf_hi(v.x), q);
+    q = __fmaf_rn(bf_lo(v.y), bf_lo(v.y), q);
+    q = __fmaf_rn(bf_hi(v.y), bf_hi(v.y), q);
+    q = __fmaf_rn(bf_lo(v.z), bf_lo(v.z), q);
+    q = __fmaf_rn(bf_hi(v.z), bf_hi(v.z), q);
+    q = __fmaf_rn(bf_lo(v.w), bf_lo(v.w), q);
+    q = __fmaf_rn(bf_hi(v.w), bf_hi(v.w), q);
+    return q;
+}
+
+// xor butterfly over the 32 lanes; every lane ends with the same bits
+// (fp32 addition is commutative, so both partners of a pair agree).
+__device__ __forceinline__ float butterfly(float c) {
+    c = __fadd_rn(c, __shfl_xor_sync(kFull, c, 16));
+    c = __fadd_rn(c, __shfl_xor_sync(kFull, c, 8));
+    c = __fadd_rn(c, __shfl_xor_sync(kFull, c, 4));
+    c = __fadd_rn(c, __shfl_xor_sync(kFull, c, 2));
+    c = __fadd_rn(c, __shfl_xor_sync(kFull, c, 1));
+    return c;
+}
+
+// ---------------------------------------------------------------- Phase B: combine, factor
+
+// S = sum over p (in order) of S_p, S_p = sum over k (in order) of B[p*K + k].
+__device__ __forceinline__ float combine(const float *B, int P, int K) {
+    float S = 0.f;
+    for (int p = 0; p < P; ++p) {
+        float Sp = 0.f;
+        for (int k = 0; k < K; ++k) Sp = __fadd_rn(Sp, B[p * K + k]);
+        S = __fadd_rn(S, Sp);
+    }
+    return S;
+}
+
+// r = rsqrt(S / D + eps): the global RMS factor with the full width D.
+__device__ __forceinline__ float factor(float S, float Df, float eps) {
+    return rsqrtf(__fadd_rn(__fdiv_rn(S, Df), eps));
+}
+
+// ---------------------------------------------------------------- Phase B weight, Phase C
+
+__device__ __forceinline__ float wmul(float x, float g, float r) {
+    return __fmul_rn(__fmul_rn(x, g), r);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// y = (x * gamma) * r for one vector; g points at the vector's gamma (fp32).
+__device__ __forceinline__ uint4 vapply(F32Tag, const uint4 &v, const float *g, float r) {
+    const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g));
+    uint4 o;
+    o.x = __float_as_uint(wmul(__uint_as_float(v.x), g4.x, r));
+    o.y = __float_as_uint(wmul(__uint_as_float(v.y), g4.y, r));
+    o.z = __float_as_uint(wmul(__uint_as_float(v.z), g4.z, r));
+    o.w = __float_as_uint(wmul(__uint_as_float(v.w), g4.w, r));
+    return o;
+}
+
+__device__ __forceinline__ uint4 vapply(BF16Tag, const uint4 &v, const float *g, float r) {
+    const float4 ga = __ldg(reinterpret_cast<const float4 *>(g));
+    const float4 gb = __ldg(reinterpret_cast<const float4 *>(g) + 1);
+    uint4 o;
+    o.x = pack_bf16x2(wmul(bf_lo(v.x), ga.x, r), wmul(bf_hi(v.x), ga.y, r));
+    o.y = pack_bf16x2(wmul(bf_lo(v.y), ga.z, r), wmul(bf_hi(v.y), ga.w, r));
+    o.z = pack_bf16x2(wmul(bf_lo(v.z), gb.x, r), wmul(bf_hi(v.z), gb.y, r));
+    o.w = pack_bf16x2(wmul(bf_lo(v.w), gb.z, r), wmul(bf_hi(v.w), gb.w, r));
+    return o;
+}
+
+// ---------------------------------------------------------------- memory
+
+// Streaming (read-once / write-once) 16-byte accesses: evict-first in L1/L2.
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
+
+// Number of vectors lane `first` of a group holds: v = first + stride*i < nv.
+__device__ __forceinline__ int slot_count(int first, int nv, int stride) {
+    return first < nv ? (nv - first + stride - 1) / stride : 0;
+}
+
+}  // namespace qkn

@@ -1,0 +1,217 @@
+// qknorm_fused.cu -- single-pass fused QK-Norm kernels for sm_100a.
+//
+// SwiftQK technical review, Section 3, Algorithm 1: per token, Phase A sums
+// the squares of each shard, Phase B adds the shard scalars and forms the
+// factor while x * gamma is formed independently, Phase C writes the
+// weighted row times the factor. Here the shards are slices of one row in
+// this GPU's memory, so the "exchange" of Phase B is a read of a few floats
+// from shared memory; one HBM read and one HBM write per element remain.
+//
+// fused_cta: one CTA per token (Q row and K row), one warp per (tensor,
+//   shard, group) task. Each lane keeps its <= VMAX vectors of the row in
+//   registers between the reduction and the apply, so every element is read
+//   once. The grid is persistent (a stride loop over tokens, Algorithm 1's
+//   "persistent block-level stride loop", sized by the occupancy calculator
+//   as B_res x N_SM); with PREFETCH a CTA issues the loads of its next token
+//   before reducing the current one, so HBM reads stay in flight across the
+//   CTA barrier.
+// fused_generic: any shape. A CTA per token whose warps loop over the tasks;
+//   the apply pass re-reads the row (an L1/L2 hit). With one warp per CTA it
+//   is the warp-per-token variant.
+#include "qknorm_device.cuh"
+#include "qknorm_internal.h"
+
+namespace qkn {
+
+// Task decode shared by both kernels: task j of a token -> (tensor z, shard p,
+// group kg). Tasks 0 .. P*K0-1 belong to Q, the rest to K.
+struct Task {
+    int z, p, kg, K, nv;
+};
+
+// Select element z (0 or 1) of a two-entry kernel-argument array without
+// indexing it at run time (which would copy the arguments to local memory).
+template <class T>
+__device__ __forceinline__ T sel(const T (&arr)[2], int z) {
+    return z ? arr[1] : arr[0];
+}
+
+__device__ __forceinline__ Task decode_task(const FusedArgs &a, int j) {
+    Task t;
+    const int nt0 = a.P * a.K[0];
+    t.z = j < nt0 ? 0 : 1;
+    const int jj = t.z ? j - nt0 : j;
+    t.K = sel(a.K, t.z);
+    t.p = jj / t.K;
+    t.kg = jj - t.p * t.K;
+    t.nv = sel(a.nv, t.z);
+    return t;
+}
+
+template <class Tag, int VMAX, bool PREFETCH, int MAXT>
+__global__ void __launch_bounds__(MAXT) fused_cta(const FusedArgs a) {
+    constexpr int VEC = Tag::kVec;
+    __shared__ float red[2][32];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const Task tk = decode_task(a, warp);
+    const int stride = kLanes * tk.K;            // vector stride between a lane's slots
+    const int first = tk.kg * kLanes + lane;     // slot 0, as a vector index in the shard
+    const int cnt = slot_count(first, tk.nv, stride);
+    const int64_t rowvec = sel(a.D, tk.z) / VEC;      // vectors per row
+    const int64_t col0 = (int64_t)tk.p * tk.nv + first;
+    const uint4 *xs = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + col0;
+    uint4 *ys = reinterpret_cast<uint4 *>(sel(a.y, tk.z)) + col0;
+    const float *gs = sel(a.g, tk.z) + col0 * VEC;
+    const float Df = sel(a.Df, tk.z);
+    const float eps = a.eps;
+    const int red_base = tk.z ? a.P * a.K[0] : 0;
+
+    int64_t t = blockIdx.x;
+    const int64_t T = a.T;
+    const int64_t G = gridDim.x;
+
+    uint4 cur[VMAX];
+    if (t < T) {
+        const uint4 *src = xs + t * rowvec;
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
+    }
+    int buf = 0;
+    for (; t < T; t += G) {
+        const int64_t tn = t + G;
+        uint4 nxt[VMAX];
+        if (PREFETCH && tn < T) {
+            const uint4 *src = xs + tn * rowvec;
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt) nxt[i] = ld_stream(src + (int64_t)i * stride);
+        }
+        // Phase A: this lane's chain, then the butterfly -> group sum.
+        float c = 0.f;
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, cur[i]));
+        c = butterfly(c);
+        if (lane == 0) red[buf][warp] = c;
+        __syncthreads();
+        // Phase B: shard sums in order, the factor.
+        const float r = factor(combine(&red[buf][red_base], a.P, tk.K), Df, eps);
+        // Phase B weight multiply and Phase C, straight from registers.
+        uint4 *dst = ys + t * rowvec;
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (i < cnt)
+                st_stream(dst + (int64_t)i * stride,
+                          vapply(Tag{}, cur[i], gs + (int64_t)i * stride * VEC, r));
+        if (PREFETCH) {
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i) cur[i] = nxt[i];
+        } else if (tn < T) {
+            const uint4 *src = xs + tn * rowvec;
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
+        }
+        buf ^= 1;
+    }
+}
+
+template <class Tag>
+__global__ void __launch_bounds__(256) fused_generic(const FusedArgs a) {
+    constexpr int VEC = Tag::kVec;
+    extern __shared__ float red[];  // one float per task
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    const int nt0 = a.P * a.K[0];
+    const int ntask = nt0 + a.P * a.K[1];
+    for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
+        for (int j = warp; j < ntask; j += nw) {
+            const Task tk = decode_task(a, j);
+            const int stride = kLanes * tk.K;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) +
+                               t * (int64_t)(sel(a.D, tk.z) / VEC) + (int64_t)tk.p * tk.nv;
+            float c = 0.f;
+#pragma unroll 4
+            for (int v = tk.kg * kLanes + lane; v < tk.nv; v += stride)
+                c = __fadd_rn(c, vsumsq(Tag{}, src[v]));
+            c = butterfly(c);
+            if (lane == 0) red[j] = c;
+        }
+        __syncthreads();
+        const float r0 = factor(combine(red, a.P, a.K[0]), a.Df[0], a.eps);
+        const float r1 = factor(combine(red + nt0, a.P, a.K[1]), a.Df[1], a.eps);
+        for (int j = warp; j < ntask; j += nw) {
+            const Task tk = decode_task(a, j);
+            const int stride = kLanes * tk.K;
+            const int64_t off = t * (int64_t)(sel(a.D, tk.z) / VEC) + (int64_t)tk.p * tk.nv;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + off;
+            uint4 *dst = reinterpret_cast<uint4 *>(sel(a.y, tk.z)) + off;
+            const float *g = sel(a.g, tk.z) + (int64_t)tk.p * tk.nv * VEC;
+            const float r = tk.z ? r1 : r0;
+#pragma unroll 4
+            for (int v = tk.kg * kLanes + lane; v < tk.nv; v += stride)
+                st_stream(dst + v, vapply(Tag{}, src[v], g + (int64_t)v * VEC, r));
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- instance tables
+
+template <class Tag, int VMAX, bool PF>
+constexpr int cta_max_threads() { return VMAX <= 2 ? 1024 : 512; }
+
+template <class Tag, int VMAX, bool PF>
+const void *cta_fn() {
+    return reinterpret_cast<const void *>(&fused_cta<Tag, VMAX, PF, cta_max_threads<Tag, VMAX, PF>()>);
+}
+
+template <class Tag, bool PF>
+const void *cta_table(int vmax) {
+    switch (vmax) {
+    case 1: return cta_fn<Tag, 1, PF>();
+    case 2: return cta_fn<Tag, 2, PF>();
+    case 3: return cta_fn<Tag, 3, PF>();
+    case 4: return cta_fn<Tag, 4, PF>();
+    case 5: return cta_fn<Tag, 5, PF>();
+    case 6: return cta_fn<Tag, 6, PF>();
+    case 7: return cta_fn<Tag, 7, PF>();
+    case 8: return cta_fn<Tag, 8, PF>();
+    default: return nullptr;
+    }
+}
+
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, int *max_threads) {
+    if (vmax < 1 || vmax > kVcap) return nullptr;
+    if (max_threads) *max_threads = vmax <= 2 ? 1024 : 512;
+    if (dtype == 0) return prefetch ? cta_table<F32Tag, true>(vmax) : cta_table<F32Tag, false>(vmax);
+    if (dtype == 1) return prefetch ? cta_table<BF16Tag, true>(vmax) : cta_table<BF16Tag, false>(vmax);
+    return nullptr;
+}
+
+const void *fused_generic_kernel(int dtype) {
+    if (dtype == 0) return reinterpret_cast<const void *>(&fused_generic<F32Tag>);
+    if (dtype == 1) return reinterpret_cast<const void *>(&fused_generic<BF16Tag>);
+    return nullptr;
+}
+
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, const FusedArgs &a, int block,
+                             int64_t grid, cudaStream_t s) {
+    const void *fn = fused_cta_kernel(dtype, vmax, prefetch, nullptr);
+    if (!fn) return cudaErrorInvalidValue;
+    void *args[] = {const_cast<FusedArgs *>(&a)};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+}
+
+cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
+                                 size_t smem, cudaStream_t s) {
+    const void *fn = fused_generic_kernel(dtype);
+    if (!fn) return cudaErrorInvalidValue;
+    void *args[] = {const_cast<FusedArgs *>(&a)};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, smem, s);
+}
+
+}  // namespace qkn

@@ -1,0 +1,56 @@
+// qknorm_internal.h -- host-side interfaces between the C ABI (qknorm_api.cu)
+// and the kernel launchers (qknorm_fused.cu, qknorm_split.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qkn {
+
+// Shape of one tensor (Q or K) as the kernels see it.
+struct TensorShape {
+    int32_t D;    // width
+    int32_t nv;   // 16-byte vectors per shard
+    int32_t K;    // groups per shard: ceil(nv / (32 * kVcap))
+    int32_t vmax; // vectors per lane per group: ceil(nv / (32 * K))
+};
+
+// Arguments of the fused kernels; index 0 is Q, index 1 is K.
+struct FusedArgs {
+    const void *x[2];
+    const float *g[2];
+    void *y[2];
+    int64_t T;
+    int32_t D[2];
+    int32_t nv[2];
+    int32_t K[2];
+    int32_t P;
+    float Df[2];
+    float eps;
+};
+
+TensorShape make_shape(int32_t D, int32_t P, int vec);
+
+// Kernel handles for occupancy queries and launches. Each returns nullptr if
+// the combination does not exist.
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, int *max_threads);
+const void *fused_generic_kernel(int dtype);
+const void *stats_kernel(int dtype, int vmax);
+const void *apply_kernel(int dtype);
+
+// Launchers: enqueue one kernel; return the cudaError_t of the launch.
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, const FusedArgs &a,
+                             int block, int64_t grid, cudaStream_t s);
+cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
+                                 size_t smem, cudaStream_t s);
+cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64_t T,
+                         const TensorShape &sh, int32_t P, int block, int64_t grid,
+                         cudaStream_t s);
+cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
+                         int64_t T, int32_t D, int32_t P, float eps, int block, int64_t grid,
+                         cudaStream_t s);
+
+// Largest dynamic shared memory the generic kernel is given (bytes).
+constexpr int kGenericMaxSmem = 200 * 1024;
+
+}  // namespace qkn

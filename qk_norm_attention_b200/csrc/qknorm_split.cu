@@ -1,0 +1,140 @@
+// qknorm_split.cu -- the split path: statistics, then apply.
+//
+// SwiftQK technical review, Section 3, Algorithm 1, and Section 4's
+// "MiniMax(eager)" ladder rung (scalar statistics first, normalisation
+// afterwards, not fused): qknorm_partial_sumsq is Phase A alone and writes
+// each shard's sum of squares to stats[T, P] (the scalar a rank would
+// publish to its IPC slot); qknorm_apply is Phases B and C given stats.
+//
+// stats: one warp per (token, shard) task, the same reduction order as the
+//   fused kernels (groups of 32 lane chains, butterfly, groups in order), so
+//   S[t,p] equals the fused kernel's shard sum bit for bit. No barriers; the
+//   grid is a stride loop over tasks.
+// apply: one CTA per row (stride loop over rows). Every thread adds the P
+//   shard sums of its row in order and forms the factor, then streams its
+//   vectors of the row through (x * gamma) * r. The row's first loads are
+//   issued before the factor so the statistic's latency overlaps them.
+#include "qknorm_device.cuh"
+#include "qknorm_internal.h"
+
+namespace qkn {
+
+template <class Tag, int VMAX>
+__global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int64_t T, int32_t D,
+                                               int32_t P, int32_t nv, int32_t K) {
+    constexpr int VEC = Tag::kVec;
+    const int lane = threadIdx.x & 31;
+    const int64_t rowvec = D / VEC;
+    const int64_t ntask = T * (int64_t)P;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int stride = kLanes * K;
+    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntask;
+         task += nwarps) {
+        const int64_t t = task / P;
+        const int p = (int)(task - t * P);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec + (int64_t)p * nv;
+        float S = 0.f;
+        for (int kg = 0; kg < K; ++kg) {
+            const int first = kg * kLanes + lane;
+            const int cnt = slot_count(first, nv, stride);
+            uint4 v[VMAX];
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt) v[i] = ld_stream(src + first + (int64_t)i * stride);
+            float c = 0.f;
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, v[i]));
+            S = __fadd_rn(S, butterfly(c));
+        }
+        if (lane == 0) stats[task] = S;
+    }
+}
+
+template <class Tag>
+__global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, const float *stats,
+                                               void *y, int64_t T, int32_t D, int32_t P,
+                                               float eps) {
+    constexpr int VEC = Tag::kVec;
+    constexpr int UNR = 4;
+    const int64_t rowvec = D / VEC;
+    const float Df = (float)D;
+    const int nthr = blockDim.x;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec;
+        uint4 *dst = reinterpret_cast<uint4 *>(y) + t * rowvec;
+        float r = 0.f;
+        for (int64_t v0 = 0; v0 < rowvec; v0 += (int64_t)nthr * UNR) {
+            uint4 xv[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t v = v0 + threadIdx.x + (int64_t)u * nthr;
+                if (v < rowvec) xv[u] = ld_stream(src + v);
+            }
+            if (v0 == 0) {
+                // Phase B: S = sum of the P shard sums, in order of p.
+                const float *st = stats + t * P;
+                float S = 0.f;
+#pragma unroll 8
+                for (int p = 0; p < P; ++p) S = __fadd_rn(S, __ldg(st + p));
+                r = factor(S, Df, eps);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int64_t v = v0 + threadIdx.x + (int64_t)u * nthr;
+                if (v < rowvec) st_stream(dst + v, vapply(Tag{}, xv[u], g + v * VEC, r));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- instance tables
+
+template <class Tag>
+const void *stats_table(int vmax) {
+    switch (vmax) {
+    case 1: return reinterpret_cast<const void *>(&stats_k<Tag, 1>);
+    case 2: return reinterpret_cast<const void *>(&stats_k<Tag, 2>);
+    case 3: return reinterpret_cast<const void *>(&stats_k<Tag, 3>);
+    case 4: return reinterpret_cast<const void *>(&stats_k<Tag, 4>);
+    case 5: return reinterpret_cast<const void *>(&stats_k<Tag, 5>);
+    case 6: return reinterpret_cast<const void *>(&stats_k<Tag, 6>);
+    case 7: return reinterpret_cast<const void *>(&stats_k<Tag, 7>);
+    case 8: return reinterpret_cast<const void *>(&stats_k<Tag, 8>);
+    default: return nullptr;
+    }
+}
+
+const void *stats_kernel(int dtype, int vmax) {
+    if (dtype == 0) return stats_table<F32Tag>(vmax);
+    if (dtype == 1) return stats_table<BF16Tag>(vmax);
+    return nullptr;
+}
+
+const void *apply_kernel(int dtype) {
+    if (dtype == 0) return reinterpret_cast<const void *>(&apply_k<F32Tag>);
+    if (dtype == 1) return reinterpret_cast<const void *>(&apply_k<BF16Tag>);
+    return nullptr;
+}
+
+cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64_t T,
+                         const TensorShape &sh, int32_t P, int block, int64_t grid,
+                         cudaStream_t s) {
+    const void *fn = stats_kernel(dtype, vmax);
+    if (!fn) return cudaErrorInvalidValue;
+    int32_t D = sh.D, nv = sh.nv, K = sh.K;
+    void *args[] = {const_cast<void **>(&x), &stats, &T, &D, &P, &nv, &K};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+}
+
+cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
+                         int64_t T, int32_t D, int32_t P, float eps, int block, int64_t grid,
+                         cudaStream_t s) {
+    const void *fn = apply_kernel(dtype);
+    if (!fn) return cudaErrorInvalidValue;
+    void *args[] = {const_cast<void **>(&x), const_cast<float **>(&g),
+                    const_cast<float **>(&stats), &y, &T, &D, &P, &eps};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+}
+
+}  // namespace qkn

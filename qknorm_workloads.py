@@ -107,9 +107,13 @@ def to_storage(x64: np.ndarray, dtype: str) -> np.ndarray:
         return f32
     if dtype != "bf16":
         raise ValueError(f"unknown dtype {dtype!r}")
-    bits = f32.view(np.uint32).astype(np.uint64)
-    rounded = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    # For finite values bits <= 0xFF7FFFFF, so bits + 0x8000 fits in 32 bits.
+    bits = f32.view(np.uint32)
+    odd = (bits >> 16) & 1
+    bits += 0x7FFF
+    bits += odd
+    bits >>= 16
+    return bits.astype(np.uint16)
 
 
 def storage_to_f64(s: np.ndarray, dtype: str) -> np.ndarray:
@@ -150,9 +154,10 @@ def gen_rows_f64(wl: Workload, tensor: str, rows: Sequence[int]) -> np.ndarray:
     rows = np.asarray(rows, dtype=np.int64)
     out = np.empty((len(rows), D))
     cols = outlier_channels(wl, tensor, D)
+    blk = np.empty((ROW_BLOCK, D))
     for b in np.unique(rows // ROW_BLOCK):
         sel = (rows // ROW_BLOCK) == b
-        blk = _rng(wl.seed, TENSOR_CODE[tensor], int(b)).standard_normal((ROW_BLOCK, D))
+        _rng(wl.seed, TENSOR_CODE[tensor], int(b)).standard_normal(out=blk)
         blk *= wl.x_sigma
         if cols.size:
             blk[:, cols] *= wl.outlier_factor
@@ -172,8 +177,8 @@ def gen_tensor(wl: Workload, tensor: str, T: int) -> np.ndarray:
     D = wl.Dq if tensor == "q" else wl.Dk
     dt = np.float32 if wl.dtype == "f32" else np.uint16
     out = np.empty((T, D), dtype=dt)
-    for start in range(0, T, ROW_BLOCK * 16):
-        stop = min(T, start + ROW_BLOCK * 16)
+    for start in range(0, T, ROW_BLOCK):
+        stop = min(T, start + ROW_BLOCK)
         out[start:stop] = gen_rows(wl, tensor, np.arange(start, stop))
     return out
 
@@ -212,3 +217,48 @@ def stats_bytes(T: int, D: int, P: int, elem_bytes: int) -> int:
 def apply_bytes(T: int, D: int, P: int, elem_bytes: int) -> int:
     """Bytes of the apply pass alone: x read, y written, stats read, gamma."""
     return 2 * T * D * elem_bytes + 4 * T * P + 4 * D
+
+
+def gen_device_normal(T: int, D: int, seed: int, dtype, device, sigma: float = 1.0):
+    """Large synthetic input drawn on the device with torch's seeded generator
+    (N(0, sigma) in fp32, then rounded to `dtype`); for sizes too large to draw
+    on the host in reasonable time. Rows needed by the oracle are copied back
+    from the returned tensor."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = torch.empty((T, D), dtype=dtype, device=device)
+    step = max(1, (1 << 28) // D)
+    for t0 in range(0, T, step):
+        t1 = min(T, t0 + step)
+        x[t0:t1] = (torch.randn((t1 - t0, D), generator=gen, device=device) * sigma).to(dtype)
+    return x
+
+
+def gen_device_workload(wl: Workload, tensor: str, T: int, device, row0: int = 0):
+    """The workload's recipe drawn on the device with torch's seeded generator:
+    N(0, sigma), the same outlier channels, a per-token log-uniform scale when
+    the workload has one, rounded to the storage dtype. The values differ from
+    gen_tensor's (another random stream) but follow the same distribution; it
+    serves timing runs, where drawing on the host would take too long."""
+    import torch
+    D = wl.Dq if tensor == "q" else wl.Dk
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=device)
+    gen.manual_seed(wl.seed * 1_000_003 + TENSOR_CODE[tensor] * 7919 + row0)
+    sgen = torch.Generator(device=device)
+    sgen.manual_seed(wl.seed * 1_000_003 + SCALE_KEY + row0)
+    cols = torch.from_numpy(outlier_channels(wl, tensor, D)).to(device)
+    x = torch.empty((T, D), dtype=tdt, device=device)
+    step = max(1, (1 << 26) // D)
+    for t0 in range(0, T, step):
+        t1 = min(T, t0 + step)
+        blk = torch.randn((t1 - t0, D), generator=gen, device=device) * wl.x_sigma
+        if cols.numel():
+            blk[:, cols] *= wl.outlier_factor
+        if wl.token_scale_log10 is not None:
+            lo, hi = wl.token_scale_log10
+            u = torch.rand((t1 - t0, 1), generator=sgen, device=device) * (hi - lo) + lo
+            blk *= torch.pow(10.0, u)
+        x[t0:t1] = blk.to(tdt)
+    return x

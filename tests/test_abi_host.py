@@ -1,0 +1,172 @@
+"""Host-side checks of libqknorm (CPU only, no kernel launches): the library
+loads, exports every function the header declares, validates arguments before
+touching CUDA, and the selector plans the expected launches.
+
+Argument checks use fake addresses that the validation must reject; no call
+here passes validation with a fake address, and the module skips itself on a
+machine with a GPU so that no such address could ever reach a kernel."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qknorm.h")
+
+
+@pytest.fixture(scope="module")
+def qk():
+    import runpy
+    runpy.run_path(os.path.join(ROOT, "qk_norm_attention_b200", "csrc", "build_lib.py"))["build"]()
+    import qk_norm_attention_b200 as qk
+    return qk
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"QKNORM_API\s+(?:int|const char \*)\s*(qknorm_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for want in ("qknorm_fwd", "qknorm_partial_sumsq", "qknorm_apply", "qknorm_status_string"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(qk):
+    lib = ctypes.CDLL(qk.LIBRARY)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in qknorm.h but not exported"
+
+
+def test_status_strings(qk):
+    assert qk.qknorm_status_string(0) == "ok"
+    for s in range(1, 5):
+        assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
+    assert qk.qknorm_status_string(99) == "unknown status"
+    assert qk.qknorm_version() == 100
+
+
+# ----------------------------------------------------------------- argument checks
+
+needs_cpu = pytest.mark.skipif(
+    __import__("torch").cuda.is_available(),
+    reason="fake-address checks run only on machines without a GPU")
+
+A = 0x10000          # fake, 16-byte aligned addresses far apart
+B = 0x20000000
+C = 0x40000000
+Dd = 0x60000000
+E = 0x80000000
+F = 0xA0000000
+
+
+def fwd(qk, q=A, k=B, gq=C, gk=Dd, oq=E, ok=F, T=4, Dq=256, Dk=256, P=2, eps=1e-6, dtype=1):
+    return qk.lib.qknorm_fwd(q, k, gq, gk, oq, ok, T, Dq, Dk, P, eps, dtype, None)
+
+
+@needs_cpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), 1), (dict(Dq=0), 1), (dict(Dk=-8), 1), (dict(P=0), 1), (dict(P=-2), 1),
+    (dict(Dq=250, P=4), 1),                    # D % P != 0
+    (dict(eps=-1e-6), 1), (dict(eps=math.nan), 1), (dict(eps=math.inf), 1),
+    (dict(q=0), 1), (dict(k=0), 1), (dict(gq=0), 1), (dict(gk=0), 1), (dict(oq=0), 1), (dict(ok=0), 1),
+    (dict(dtype=2), 3), (dict(dtype=-1), 3),
+    (dict(Dq=40, Dk=40, P=2, dtype=1), 3),     # 20-wide bf16 shards
+    (dict(Dq=24, Dk=24, P=4, dtype=0), 3),     # 6-wide fp32 shards
+    (dict(q=A + 2), 2), (dict(k=B + 8), 2), (dict(gq=C + 4), 2), (dict(gk=Dd + 12), 2),
+    (dict(oq=E + 2), 2), (dict(ok=F + 6), 2),
+    (dict(oq=A + 16), 1),                      # output overlaps its input partly
+    (dict(oq=B), 1),                           # output aliases the other input
+    (dict(ok=E), 1),                           # the two outputs coincide
+    (dict(oq=C), 1),                           # output on gamma
+    (dict(ok=A), 1),                           # K output on Q input
+])
+def test_fwd_rejects(qk, kw, status):
+    assert fwd(qk, **kw) == status
+
+
+@needs_cpu
+def test_fwd_T0_is_a_noop(qk):
+    assert fwd(qk, T=0, q=0, k=0, gq=0, gk=0, oq=0, ok=0) == 0
+
+
+@needs_cpu
+def test_split_rejects(qk):
+    L = qk.lib
+    assert L.qknorm_partial_sumsq(A, B, 4, 250, 4, 1, None) == 1
+    assert L.qknorm_partial_sumsq(A, B, 4, 256, 4, 5, None) == 3
+    assert L.qknorm_partial_sumsq(A, B, 4, 256, 64, 1, None) == 3      # 4-wide bf16 shards
+    assert L.qknorm_partial_sumsq(A + 2, B, 4, 256, 4, 1, None) == 2
+    assert L.qknorm_partial_sumsq(A, B + 4, 4, 256, 4, 1, None) == 2
+    assert L.qknorm_partial_sumsq(A, A + 16, 4, 256, 4, 1, None) == 1  # stats inside x
+    assert L.qknorm_partial_sumsq(0, B, 4, 256, 4, 1, None) == 1
+    assert L.qknorm_partial_sumsq(0, 0, 0, 256, 4, 1, None) == 0
+    assert L.qknorm_apply(A, B, C, Dd, 4, 256, 4, -1.0, 1, None) == 1
+    assert L.qknorm_apply(A, B, C, Dd, 4, 256, 3, 1e-6, 1, None) == 1
+    assert L.qknorm_apply(A, B, C, Dd + 2, 4, 256, 4, 1e-6, 1, None) == 2
+    assert L.qknorm_apply(A, B, C, B, 4, 256, 4, 1e-6, 1, None) == 1   # out on gamma
+    assert L.qknorm_apply(A, B, C, C, 4, 256, 4, 1e-6, 1, None) == 1   # out on stats
+    assert L.qknorm_apply(A, B, C, A + 32, 4, 256, 4, 1e-6, 1, None) == 1
+    assert L.qknorm_apply(A, B, C, Dd, 4, 256, 4, 1e-6, 9, None) == 3
+
+
+@needs_cpu
+def test_valid_call_without_gpu_reports_cuda_error(qk):
+    """All checks pass, then the runtime finds no device: QKNORM_ERR_CUDA with text."""
+    assert fwd(qk) == 4
+    assert qk.qknorm_last_error() != ""
+
+
+# ----------------------------------------------------------------- the selector
+
+def test_plan_for_each_workload(qk):
+    import qknorm_workloads as W
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    dt = {"bf16": qk.QKNORM_BF16, "f32": qk.QKNORM_F32}
+    want_block = {"tiny": 4 * 32, "decode": 8 * 32, "prefill13b": 8 * 32, "gqa": 16 * 32,
+                  "split_large": 16 * 32}
+    want_vmax = {"tiny": 1, "decode": 4, "prefill13b": 5, "gqa": 3, "split_large": 2}
+    for name, wl in W.WORKLOADS.items():
+        for T in wl.Ts:
+            pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
+            assert pl["variant"] == qk.VARIANT_CTA, name
+            assert pl["block"] == want_block[name], name
+            assert pl["vmax"] == want_vmax[name], name
+            assert pl["grid"] == min(T, 148 * 4)
+            assert pl["prefetch"] == int(T > 148 * 4)
+            assert pl["groups_q"] == pl["groups_k"] == 1
+
+
+def test_plan_groups_and_fallbacks(qk):
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    pl = qk.qknorm_plan_fwd(10, 4096, 4096, 1, qk.QKNORM_BF16, 148)      # nv = 512
+    assert (pl["groups_q"], pl["vmax"], pl["block"]) == (2, 8, 4 * 32)
+    pl = qk.qknorm_plan_fwd(10, 4096, 4096, 16, qk.QKNORM_BF16, 148)     # 32 tasks, 1 vector
+    assert (pl["variant"], pl["block"], pl["vmax"]) == (qk.VARIANT_CTA, 1024, 1)
+    pl = qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)     # 64 tasks
+    assert (pl["variant"], pl["block"]) == (qk.VARIANT_GENERIC, 256)
+    pl = qk.qknorm_plan_fwd(10, 32768, 1024, 4, qk.QKNORM_BF16, 148)     # 20 tasks, vmax 8
+    assert pl["variant"] == qk.VARIANT_GENERIC and pl["groups_q"] == 4
+    with pytest.raises(qk.QKNormError):
+        qk.qknorm_plan_fwd(10, 4096, 4096, 3, qk.QKNORM_BF16, 148)
+
+
+def test_forced_variants(qk):
+    try:
+        qk.qknorm_force_variant(qk.VARIANT_WARP, 0)
+        pl = qk.qknorm_plan_fwd(64, 4096, 4096, 4, qk.QKNORM_BF16, 148, 32)
+        assert (pl["variant"], pl["block"], pl["grid"]) == (qk.VARIANT_WARP, 32, 64)
+        qk.qknorm_force_variant(qk.VARIANT_CTA, 7)
+        pl = qk.qknorm_plan_fwd(100, 4096, 4096, 4, qk.QKNORM_BF16, 148, 4)
+        assert (pl["grid"], pl["prefetch"]) == (7, 1)
+        qk.qknorm_force_variant(qk.VARIANT_CTA, 0)
+        with pytest.raises(qk.QKNormError) as ei:
+            qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
+        assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_force_variant(5, 0)
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)

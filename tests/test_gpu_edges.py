@@ -1,0 +1,213 @@
+"""GPU edge cases through the C ABI: empty and ragged inputs, every kernel
+variant (bit-identical by construction), shard shapes that reach each code
+path, in-place calls, guard regions around the outputs, unchanged inputs,
+and tensors of more than 2^31 elements."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qknorm_workloads as W
+from gpu_util import bits, check_outputs, check_stats, to_device, to_host
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = ("cta", "warp", "generic")
+
+
+@pytest.fixture(scope="module")
+def qk():
+    import qk_norm_attention_b200 as qk
+    yield qk
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.get()
+
+
+def _inputs(wl, T):
+    q = W.gen_rows(wl, "q", range(T))
+    k = W.gen_rows(wl, "k", range(T))
+    gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
+    return q, k, gq, gk
+
+
+def _fwd(qk, wl, q, k, gq, gk, variant=None, grid=0):
+    vid = {"cta": qk.VARIANT_CTA, "warp": qk.VARIANT_WARP, "generic": qk.VARIANT_GENERIC,
+           None: qk.VARIANT_AUTO}[variant]
+    qk.qknorm_force_variant(vid, grid)
+    try:
+        oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk),
+                               wl.P, wl.eps)
+        torch.cuda.synchronize()
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    return oq, ok
+
+
+def _check_oracle(orc, wl, q, k, gq, gk, oq, ok):
+    eps = float(np.float32(wl.eps))
+    yq, yk, _, _ = orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=8)
+    check_outputs(to_host(oq), yq, wl.dtype, f"{wl.name} q")
+    check_outputs(to_host(ok), yk, wl.dtype, f"{wl.name} k")
+
+
+SHAPES = [
+    # name, T, Dq, Dk, P, dtype
+    ("decode_odd_T", 33, 4096, 4096, 4, "bf16"),
+    ("gqa_ragged_lanes", 77, 5120, 1024, 8, "bf16"),
+    ("p1_two_groups", 19, 4096, 4096, 1, "bf16"),       # nv = 512 -> K = 2
+    ("p16_block1024", 21, 4096, 4096, 16, "bf16"),      # 32 warps, 1 vector per lane
+    ("p32_generic", 9, 4096, 4096, 32, "bf16"),         # 64 tasks -> generic
+    ("wide_p1", 5, 65536, 8192, 1, "bf16"),             # K = 32 -> generic
+    ("k_one_vector_shard", 13, 1024, 64, 8, "bf16"),    # K shard = one vector
+    ("mixed_groups", 7, 32768, 1024, 4, "bf16"),        # K_q = 4, K_k = 1
+    ("fp32_d4096", 29, 4096, 4096, 4, "f32"),
+    ("fp32_p64", 6, 1024, 512, 64, "f32"),              # 4-wide shards, generic
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_shapes_and_variants(qk, orc, shape):
+    name, T, Dq, Dk, P, dtype = shape
+    wl = W.custom(name, T, Dq, Dk, P, dtype=dtype, seed=zlib.crc32(name.encode()) % 1000)
+    q, k, gq, gk = _inputs(wl, T)
+    outs = {}
+    for v in VARIANTS:
+        try:
+            outs[v] = _fwd(qk, wl, q, k, gq, gk, variant=v)
+        except qk.QKNormError as e:
+            # Only the register-resident CTA kernel has shape limits.
+            assert v == "cta" and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
+    base = outs["generic"]
+    for v, (oq, ok) in outs.items():
+        assert torch.equal(bits(oq), bits(base[0])), f"{v} Q differs from generic"
+        assert torch.equal(bits(ok), bits(base[1])), f"{v} K differs from generic"
+    auto = _fwd(qk, wl, q, k, gq, gk)
+    assert torch.equal(bits(auto[0]), bits(base[0])) and torch.equal(bits(auto[1]), bits(base[1]))
+    _check_oracle(orc, wl, q, k, gq, gk, *auto)
+    # The split path agrees bit for bit with the fused path on every shape.
+    for x, g, out in ((q, gq, auto[0]), (k, gk, auto[1])):
+        xd = to_device(x)
+        st = qk.qknorm_partial_sumsq(xd, P)
+        y = qk.qknorm_apply(xd, to_device(g), st, wl.eps)
+        torch.cuda.synchronize()
+        assert torch.equal(bits(y), bits(out))
+        S_or = orc.partial_sumsq(x, P, dtype)
+        check_stats(st.cpu().numpy(), S_or, x.shape[1], P, dtype, name)
+
+
+@pytest.mark.parametrize("grid", [1, 5, 148])
+def test_persistent_stride_and_ragged_tail(qk, orc, grid):
+    """Forced small grids: every CTA walks many tokens (prefetch path) and the
+    last wave is partial; the result is bit-identical to the automatic plan."""
+    wl = W.custom("stride", 3 * 148 + 7, 4096, 1024, 4, seed=31)
+    q, k, gq, gk = _inputs(wl, wl.Ts[0])
+    ref = _fwd(qk, wl, q, k, gq, gk)
+    got = _fwd(qk, wl, q, k, gq, gk, variant="cta", grid=grid)
+    assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
+    got_w = _fwd(qk, wl, q, k, gq, gk, variant="warp", grid=grid)
+    assert torch.equal(bits(got_w[0]), bits(ref[0]))
+    _check_oracle(orc, wl, q, k, gq, gk, *ref)
+
+
+def test_plan_grid_tail(qk, orc):
+    """T one past a multiple of the automatic persistent grid."""
+    plan = qk.qknorm_launch_plan(100000, 5120, 5120, 4, qk.QKNORM_BF16)
+    T = 2 * plan["grid"] + 1
+    wl = W.custom("tail", T, 5120, 5120, 4, seed=32, x_sigma=1.5)
+    q, k, gq, gk = _inputs(wl, T)
+    oq, ok = _fwd(qk, wl, q, k, gq, gk)
+    _check_oracle(orc, wl, q, k, gq, gk, oq, ok)
+
+
+def test_empty_T(qk):
+    e = torch.empty((0, 4096), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(4096, dtype=torch.float32, device="cuda")
+    oq, ok = qk.qknorm_fwd(e, e.clone(), g, g, 4, 1e-6)
+    st = qk.qknorm_partial_sumsq(e, 4)
+    y = qk.qknorm_apply(e, g, st, 1e-6)
+    torch.cuda.synchronize()
+    assert oq.shape == (0, 4096) and st.shape == (0, 4) and y.shape == (0, 4096)
+
+
+def test_in_place(qk):
+    wl = W.custom("inplace", 50, 2048, 1024, 4, seed=33)
+    q, k, gq, gk = _inputs(wl, 50)
+    ref = _fwd(qk, wl, q, k, gq, gk)
+    qd, kd = to_device(q), to_device(k)
+    qk.qknorm_fwd(qd, kd, to_device(gq), to_device(gk), 4, wl.eps, out_q=qd, out_k=kd)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(qd), bits(ref[0])) and torch.equal(bits(kd), bits(ref[1]))
+    xd = to_device(q)
+    st = qk.qknorm_partial_sumsq(xd, 4)
+    qk.qknorm_apply(xd, to_device(gq), st, wl.eps, out=xd)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(xd), bits(ref[0]))
+
+
+def test_guard_regions_and_const_inputs(qk):
+    """Outputs sit inside larger buffers filled with a canary pattern; after
+    the calls the canaries and the inputs are byte-identical to before."""
+    T, Dq, Dk, P = 37, 5120, 1024, 8
+    wl = W.custom("guard", T, Dq, Dk, P, seed=34)
+    q, k, gq, gk = _inputs(wl, T)
+    qd, kd, gqd, gkd = (to_device(a) for a in (q, k, gq, gk))
+    saved = [t.clone() for t in (qd, kd, gqd, gkd)]
+    pad = 4096  # elements of guard on each side (8 KiB, keeps 16-byte alignment)
+    bq = torch.full((T * Dq + 2 * pad,), -7777.0, dtype=torch.bfloat16, device="cuda")
+    bk = torch.full((T * Dk + 2 * pad,), -7777.0, dtype=torch.bfloat16, device="cuda")
+    bs = torch.full((T * P + 2 * pad,), -5.5, dtype=torch.float32, device="cuda")
+    bcopy = [b.clone() for b in (bq, bk, bs)]
+    oq = bq[pad:pad + T * Dq].view(T, Dq)
+    ok = bk[pad:pad + T * Dk].view(T, Dk)
+    st = bs[pad:pad + T * P].view(T, P)
+    qk.qknorm_fwd(qd, kd, gqd, gkd, P, wl.eps, out_q=oq, out_k=ok)
+    qk.qknorm_partial_sumsq(qd, P, stats=st)
+    torch.cuda.synchronize()
+    for b, c in zip((bq, bk, bs), bcopy):
+        assert torch.equal(bits(b[:pad]), bits(c[:pad])) and torch.equal(bits(b[-pad:]), bits(c[-pad:]))
+    for t, s in zip((qd, kd, gqd, gkd), saved):
+        assert torch.equal(bits(t), bits(s))
+    ref = _fwd(qk, wl, q, k, gq, gk)
+    assert torch.equal(bits(oq), bits(ref[0])) and torch.equal(bits(ok), bits(ref[1]))
+
+
+def test_rejected_call_launches_nothing(qk):
+    x = torch.randn(8, 1000, device="cuda").to(torch.bfloat16)
+    g = torch.ones(1000, device="cuda")
+    out = torch.full_like(x, 3.0)
+    with pytest.raises(qk.QKNormError) as ei:
+        qk.qknorm_fwd(x, x, g, g, 3, 1e-6, out_q=out, out_k=out.clone())   # D % P != 0
+    assert ei.value.status == qk.QKNORM_ERR_INVALID_ARG
+    with pytest.raises(qk.QKNormError) as ei:
+        qk.qknorm_fwd(x, x, g, g, 50, 1e-6, out_q=out, out_k=out.clone())  # 20-wide shards
+    assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert bool((out == 3.0).all())
+
+
+def test_more_than_2_31_elements(qk, orc):
+    """Row offsets beyond 2^31 elements: T = 2^19 + 5 rows of 4096 bf16 (input
+    drawn on the device); the oracle checks rows at both ends."""
+    T, D, P = (1 << 19) + 5, 4096, 8
+    q = W.gen_device_normal(T, D, seed=41, dtype=torch.bfloat16, device="cuda")
+    k = W.gen_device_normal(T, D, seed=42, dtype=torch.bfloat16, device="cuda")
+    g = torch.from_numpy(W.gen_gamma(W.custom("big", 1, D, D, P, seed=43), "q")).cuda()
+    oq, ok = qk.qknorm_fwd(q, k, g, g, P, 1e-6)
+    st = qk.qknorm_partial_sumsq(k, P)
+    ak = qk.qknorm_apply(k, g, st, 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(ak), bits(ok))
+    rows = torch.tensor(list(range(0, 4)) + list(range(T - 70, T)), device="cuda")
+    gh = g.cpu().numpy()
+    for x, y in ((q, oq), (k, ok)):
+        xs = to_host(x.index_select(0, rows))
+        y_or, _ = orc.rmsnorm(xs, gh, P, float(np.float32(1e-6)), "bf16")
+        check_outputs(to_host(y.index_select(0, rows)), y_or, "bf16", "2^31+ rows")
+    del q, k, oq, ok, ak, st
+    torch.cuda.empty_cache()

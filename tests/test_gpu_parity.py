@@ -1,0 +1,107 @@
+"""GPU parity: libqknorm (through its C ABI) against the float64 oracle on the
+five seeded workloads, in the launch configuration the selector picks (the
+one the benchmark times), plus fused == split bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qknorm_workloads as W
+from gpu_util import bits, check_outputs, check_stats, to_device, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qk():
+    import qk_norm_attention_b200 as qk
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    return qk
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.get()
+
+
+def _eps64(wl):
+    return float(np.float32(wl.eps))
+
+
+def _run_case(qk, orc, wl, T, rows=None, chunk=2048):
+    """Fused and split paths on all T rows; oracle on `rows` (all if None)."""
+    q = W.gen_tensor(wl, "q", T)
+    k = W.gen_tensor(wl, "k", T)
+    gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
+    qd, kd, gqd, gkd = to_device(q), to_device(k), to_device(gq), to_device(gk)
+    oq, ok = qk.qknorm_fwd(qd, kd, gqd, gkd, wl.P, wl.eps)
+    sq = qk.qknorm_partial_sumsq(qd, wl.P)
+    sk = qk.qknorm_partial_sumsq(kd, wl.P)
+    aq = qk.qknorm_apply(qd, gqd, sq, wl.eps)
+    ak = qk.qknorm_apply(kd, gkd, sk, wl.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(aq), bits(oq)), "split Q differs from fused Q"
+    assert torch.equal(bits(ak), bits(ok)), "split K differs from fused K"
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    stats = []
+    for name, x, g, D, out, st in (("q", q, gq, wl.Dq, oq, sq), ("k", k, gk, wl.Dk, ok, sk)):
+        for c0 in range(0, len(rows), chunk):
+            r = rows[c0:c0 + chunk]
+            rt = torch.from_numpy(r).to(out.device)
+            y_gpu = to_host(out.index_select(0, rt))
+            S_gpu = st.index_select(0, rt).cpu().numpy()
+            y_or, _ = orc.rmsnorm(x[r], g, wl.P, _eps64(wl), wl.dtype, nthreads=8)
+            S_or = orc.partial_sumsq(x[r], wl.P, wl.dtype, nthreads=8)
+            stats.append(check_outputs(y_gpu, y_or, wl.dtype, f"{wl.name} T={T} {name}"))
+            check_stats(S_gpu, S_or, D, wl.P, wl.dtype, f"{wl.name} T={T} {name}")
+    return stats
+
+
+def test_tiny_fp32(qk, orc):
+    _run_case(qk, orc, W.WORKLOADS["tiny"], 4)
+
+
+@pytest.mark.parametrize("T", W.WORKLOADS["decode"].Ts)
+def test_decode_olmo2_7b(qk, orc, T):
+    _run_case(qk, orc, W.WORKLOADS["decode"], T)
+
+
+def test_prefill_13b_full(qk, orc):
+    wl = W.WORKLOADS["prefill13b"]
+    _run_case(qk, orc, wl, wl.Ts[0])
+
+
+@pytest.mark.parametrize("T", W.WORKLOADS["gqa"].Ts)
+def test_gqa_mixed_widths(qk, orc, T):
+    _run_case(qk, orc, W.WORKLOADS["gqa"], T)
+
+
+def test_split_large_sampled(qk, orc):
+    """T = 65536: every row checked fused == split on the GPU; the oracle
+    checks 3000 sampled rows (both ends, every 1000th row, random rows)."""
+    wl = W.WORKLOADS["split_large"]
+    T = wl.Ts[0]
+    rng = np.random.default_rng(99)
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(T - 64, T),
+                                     np.arange(0, T, 1000), rng.choice(T, 2800, replace=False)]))
+    _run_case(qk, orc, wl, T, rows=rows)
+
+
+def test_worked_example_on_gpu(qk, orc):
+    """The review's worked example (Section 4b, Eqs. (2)-(8)) through the kernels:
+    fp32, D = 8 split into 2 shards of 4, gamma = 1, eps = 1e-6."""
+    import oracle_pins
+    g = oracle_pins.load_worked_example()
+    x = np.array([g["x"][1]], dtype=np.float32)
+    ones = np.ones(8, dtype=np.float32)
+    xd = to_device(x)
+    oq, ok = qk.qknorm_fwd(xd, xd.clone(), to_device(ones), to_device(ones), 2, 1e-6)
+    st = qk.qknorm_partial_sumsq(xd, 2)
+    torch.cuda.synchronize()
+    assert st.cpu().numpy().tolist() == [g["S_local"][1]]
+    y = oq.cpu().numpy()[0]
+    for j, (yj, pj) in enumerate(zip(y, g["y"][1])):
+        assert abs(yj - pj) <= 0.5e-3 + 0.5e-4 * abs(x[0, j]) + 1e-6, (j, yj, pj)
+    y_or, _ = orc.rmsnorm(x, ones, 2, float(np.float32(1e-6)), "f32")
+    check_outputs(y[None, :], y_or, "f32", "worked example")
+    assert torch.equal(bits(oq), bits(ok))
