@@ -139,8 +139,11 @@ typedef enum {
                                    prefetched when a CTA has more than one */
     QKNORM_VARIANT_WARP = 1,    /* warp per token: one warp walks all shards of a
                                    token, then re-reads the row to apply */
-    QKNORM_VARIANT_GENERIC = 2  /* CTA per token, any shape: warps loop over the
+    QKNORM_VARIANT_GENERIC = 2, /* CTA per token, any shape: warps loop over the
                                    shard groups, re-read the row to apply */
+    QKNORM_VARIANT_BULK = 3     /* as CTA, but rows arrive by bulk asynchronous
+                                   copies (TMA engine) into a ring of token stages
+                                   in shared memory, completed on mbarriers */
 } qknorm_variant;
 
 /* A launch plan chosen by the selector (host-side description). */
@@ -152,6 +155,10 @@ typedef struct {
     int32_t prefetch;    /* 1 if a CTA prefetches its next token */
     int32_t groups_q;    /* K for a Q shard */
     int32_t groups_k;    /* K for a K shard */
+    int32_t stages;      /* ring stages per CTA (bulk variant), else 0 */
+    int32_t tokens_per_stage; /* tokens a bulk stage holds (1, 2 or 4), else 0 */
+    int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
+    int64_t smem_bytes;  /* dynamic shared memory per CTA */
 } qknorm_plan;
 
 /*
@@ -181,6 +188,33 @@ QKNORM_API int qknorm_force_variant(int32_t variant, int64_t grid);
  */
 QKNORM_API int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
                        qknorm_plan *plan);
+
+/*
+ * qknorm_set_tuning -- process-wide tuning of the bulk variant for tests and
+ * benchmarks: ring stages per CTA (0 = automatic), tokens per stage (0 =
+ * automatic, else 1, 2 or 4), gamma in registers (-1 = automatic, 0 = no,
+ * 1 = yes), the bound of every wait in milliseconds (0 = the default of
+ * 2000 ms). A combination without a kernel instance makes qknorm_fwd return
+ * QKNORM_ERR_UNSUPPORTED. Not thread-safe with concurrent calls.
+ */
+QKNORM_API int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_regs,
+                                 int32_t wait_limit_ms);
+
+/*
+ * qknorm_device_errors -- read (and with clear != 0, reset) the library's
+ * device error word. Bit 1: a bounded wait of the bulk variant ran out of
+ * time (that launch's outputs are incomplete); bit 2: copies were still in
+ * flight when such a CTA left. Synchronises with the device (blocking copy).
+ */
+QKNORM_API int qknorm_device_errors(uint32_t *flags, int32_t clear);
+
+/*
+ * qknorm_selftest_bounded_wait -- launch one CTA that waits on an mbarrier
+ * nobody arrives on, with the bulk variant's bounded wait and the given limit
+ * (nanoseconds). It must time out and set bit 1 of the device error word.
+ * No copy is in flight, so nothing is left pending. Asynchronous on stream.
+ */
+QKNORM_API int qknorm_selftest_bounded_wait(uint64_t limit_ns, void *stream);
 
 /* ABI version of this header (major * 100 + minor). */
 QKNORM_API int qknorm_version(void);

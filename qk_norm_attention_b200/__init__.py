@@ -37,8 +37,9 @@ QKNORM_ERR_MISALIGNED = 2
 QKNORM_ERR_UNSUPPORTED = 3
 QKNORM_ERR_CUDA = 4
 
-VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC = -1, 0, 1, 2
-VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic"}
+VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK = -1, 0, 1, 2, 3
+VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic",
+                 VARIANT_BULK: "bulk"}
 
 _DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16}
 
@@ -58,7 +59,9 @@ class QKNormPlan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("vmax", ctypes.c_int32),
                 ("prefetch", ctypes.c_int32), ("groups_q", ctypes.c_int32),
-                ("groups_k", ctypes.c_int32)]
+                ("groups_k", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("tokens_per_stage", ctypes.c_int32), ("gamma_regs", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int64)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -87,6 +90,12 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_force_variant.argtypes = [i32, i64]
     lib.qknorm_force_variant.restype = ctypes.c_int
     lib.qknorm_version.restype = ctypes.c_int
+    lib.qknorm_set_tuning.argtypes = [i32, i32, i32, i32]
+    lib.qknorm_set_tuning.restype = ctypes.c_int
+    lib.qknorm_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+    lib.qknorm_device_errors.restype = ctypes.c_int
+    lib.qknorm_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+    lib.qknorm_selftest_bounded_wait.restype = ctypes.c_int
     return lib
 
 
@@ -213,3 +222,25 @@ def qknorm_force_variant(variant: int = VARIANT_AUTO, grid: int = 0) -> None:
 
 def qknorm_version() -> int:
     return lib.qknorm_version()
+
+
+def qknorm_set_tuning(stages: int = 0, tokens_per_stage: int = 0, gamma_regs: int = -1,
+                      wait_limit_ms: int = 0) -> None:
+    """Tune the bulk variant process-wide (the defaults restore automatic choice)."""
+    _check("qknorm_set_tuning", lib.qknorm_set_tuning(int(stages), int(tokens_per_stage),
+                                                      int(gamma_regs), int(wait_limit_ms)))
+
+
+def qknorm_device_errors(clear: bool = True) -> int:
+    """The device error word (bit 1: a bounded wait timed out; bit 2: copies
+    were in flight when a CTA left). Synchronises with the device."""
+    v = ctypes.c_uint32(0)
+    _check("qknorm_device_errors", lib.qknorm_device_errors(ctypes.byref(v), int(bool(clear))))
+    return v.value
+
+
+def qknorm_selftest_bounded_wait(limit_ns: int, stream=None, device=None) -> None:
+    """Launch the bounded-wait self-test kernel (it must time out and set bit 1)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check("qknorm_selftest_bounded_wait",
+           lib.qknorm_selftest_bounded_wait(int(limit_ns), _stream_handle(dev, stream)))

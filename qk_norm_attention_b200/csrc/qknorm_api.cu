@@ -126,28 +126,108 @@ cudaError_t resident_blocks(int dev, const void *fn, int block, size_t smem, int
 
 // ---------------------------------------------------------------- the selector
 
-// Static part of the plan: which kernel, block size and template width.
-int plan_static(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t variant,
-                qknorm_plan *pl) {
-    const TensorShape sq = make_shape(Dq, P, vec_of(dtype));
-    const TensorShape sk = make_shape(Dk, P, vec_of(dtype));
-    const int64_t ntask = (int64_t)P * (sq.K + sk.K);
-    const int vmax = sq.vmax > sk.vmax ? sq.vmax : sk.vmax;
+int32_t g_tune_stages = 0;           // bulk stages per CTA; 0 = automatic
+int32_t g_tune_tb = 0;               // tokens per bulk stage; 0 = automatic
+int32_t g_tune_gamma_regs = -1;      // -1 = automatic
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+constexpr int kSmemPerSm = 228 * 1024;      // shared memory of one SM
+constexpr int kSmemPerCta = 227 * 1024;     // largest opt-in dynamic shared memory of a CTA
+constexpr int kSmemReservedPerCta = 1024;   // the runtime's per-CTA reservation
+constexpr int kRegsPerSm = 65536;
+constexpr int kThreadsPerSm = 2048;
+constexpr int kMaxStagesAuto = 8;
+constexpr int kRegsHint = 64;               // register estimate when no device is queried
+
+struct Shapes {
+    TensorShape q, k;
+    int64_t ntask;
+    int vmax;
+};
+
+Shapes shapes_of(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype) {
+    Shapes s;
+    s.q = make_shape(Dq, P, vec_of(dtype));
+    s.k = make_shape(Dk, P, vec_of(dtype));
+    s.ntask = (int64_t)P * (s.q.K + s.k.K);
+    s.vmax = s.q.vmax > s.k.vmax ? s.q.vmax : s.k.vmax;
+    return s;
+}
+
+bool gamma_regs_for(int32_t dtype, int vmax) {
+    if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
+    return vmax * vec_of(dtype) <= 40;
+}
+
+// Tokens per bulk stage: 2 where an instance exists (VMAX x TB <= 12).
+int tokens_per_stage_for(int vmax) {
+    if (g_tune_tb > 0) return g_tune_tb;
+    return vmax * 2 <= 12 ? 2 : 1;
+}
+
+// Stage count of the bulk kernel: the most stages (up to kMaxStagesAuto) that
+// fit when as many CTAs share an SM as threads and registers allow; fewer
+// CTAs per SM if that leaves less than two stages each.
+void bulk_stages(uint32_t stride, int block, int regs, qknorm_plan *pl) {
+    int ctas = kThreadsPerSm / block;
+    const int by_regs = kRegsPerSm / (regs * block);
+    if (by_regs < ctas) ctas = by_regs;
+    if (ctas < 1) ctas = 1;
+    int S = 0;
+    for (; ctas >= 1; --ctas) {
+        const int per_cta = kSmemPerSm / ctas - kSmemReservedPerCta;
+        const int cap = per_cta < kSmemPerCta ? per_cta : kSmemPerCta;
+        S = 0;
+        while (S < kMaxStagesAuto && (int64_t)bulk_smem_bytes(S + 1, stride) <= cap) ++S;
+        if (S >= 2) break;
+    }
+    if (g_tune_stages > 0) S = g_tune_stages;
+    pl->stages = S;
+    pl->smem_bytes = (int64_t)bulk_smem_bytes(S, stride);
+}
+
+// Static part of the plan: which kernel, block size, template width, stages.
+int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t variant,
+                int num_sms, int regs, qknorm_plan *pl) {
+    const Shapes sh = shapes_of(Dq, Dk, P, dtype);
     std::memset(pl, 0, sizeof *pl);
-    pl->groups_q = sq.K;
-    pl->groups_k = sk.K;
+    pl->groups_q = sh.q.K;
+    pl->groups_k = sh.k.K;
     int cta_max = 0;
-    fused_cta_kernel(dtype, vmax, false, &cta_max);
-    const bool cta_ok = ntask * kLanes <= cta_max;
-    if (variant == QKNORM_VARIANT_AUTO) variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
-    if (variant == QKNORM_VARIANT_CTA) {
-        if (!cta_ok) return QKNORM_ERR_UNSUPPORTED;
-        pl->variant = QKNORM_VARIANT_CTA;
-        pl->block = (int32_t)(ntask * kLanes);
-        pl->vmax = vmax;
+    fused_cta_kernel(dtype, sh.vmax, false, &cta_max);
+    const bool cta_ok = sh.ntask * kLanes <= cta_max;
+    const int tb = tokens_per_stage_for(sh.vmax);
+    int bulk_max = 0;
+    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, true, tb, &bulk_max) != nullptr;
+    const uint32_t stride = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
+                                              (int64_t)Dk * elem_of(dtype), tb);
+    const bool bulk_ok = bulk_inst && sh.ntask * kLanes <= bulk_max &&
+                         (int64_t)bulk_smem_bytes(2, stride) <= kSmemPerCta;
+    if (variant == QKNORM_VARIANT_AUTO) {
+        if (!cta_ok)
+            variant = QKNORM_VARIANT_GENERIC;
+        else if (bulk_ok && T > 2 * (int64_t)num_sms)
+            variant = QKNORM_VARIANT_BULK;
+        else
+            variant = QKNORM_VARIANT_CTA;
+    }
+    if (variant == QKNORM_VARIANT_CTA || variant == QKNORM_VARIANT_BULK) {
+        if (variant == QKNORM_VARIANT_CTA ? !cta_ok : !bulk_ok) return QKNORM_ERR_UNSUPPORTED;
+        pl->variant = variant;
+        pl->block = (int32_t)(sh.ntask * kLanes);
+        pl->vmax = sh.vmax;
+        if (variant == QKNORM_VARIANT_BULK) {
+            pl->gamma_regs = gamma_regs_for(dtype, sh.vmax) ? 1 : 0;
+            pl->tokens_per_stage = tb;
+            bulk_stages(stride, pl->block, regs > 0 ? regs : kRegsHint, pl);
+            if (pl->stages < 1 || pl->stages > bulk_max_stages() ||
+                pl->smem_bytes > kSmemPerCta)
+                return QKNORM_ERR_UNSUPPORTED;
+        }
         return QKNORM_OK;
     }
-    if ((size_t)ntask * sizeof(float) > (size_t)kGenericMaxSmem) return QKNORM_ERR_UNSUPPORTED;
+    if ((size_t)sh.ntask * sizeof(float) > (size_t)kGenericMaxSmem) return QKNORM_ERR_UNSUPPORTED;
+    pl->smem_bytes = (int64_t)(sh.ntask * sizeof(float));
     if (variant == QKNORM_VARIANT_WARP) {
         pl->variant = QKNORM_VARIANT_WARP;
         pl->block = kLanes;
@@ -155,15 +235,15 @@ int plan_static(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t varian
     }
     if (variant == QKNORM_VARIANT_GENERIC) {
         pl->variant = QKNORM_VARIANT_GENERIC;
-        const int64_t b = ntask * kLanes;
+        const int64_t b = sh.ntask * kLanes;
         pl->block = (int32_t)(b < 256 ? b : 256);
         return QKNORM_OK;
     }
     return QKNORM_ERR_INVALID_ARG;
 }
 
-// Grid: T CTAs up to B_res x N_SM (or the forced grid), prefetch when a CTA
-// gets more than one token.
+// Grid: T CTAs up to B_res x N_SM (or the forced grid); the register variant
+// prefetches when a CTA gets more than one token.
 void plan_grid(int64_t T, int num_sms, int blocks_per_sm, qknorm_plan *pl) {
     int64_t cap = (int64_t)num_sms * blocks_per_sm;
     if (g_forced_grid > 0) cap = g_forced_grid;
@@ -173,50 +253,85 @@ void plan_grid(int64_t T, int num_sms, int blocks_per_sm, qknorm_plan *pl) {
     pl->prefetch = (pl->variant == QKNORM_VARIANT_CTA && T > pl->grid) ? 1 : 0;
 }
 
-const void *plan_kernel(const qknorm_plan &pl, int32_t dtype) {
-    if (pl.variant == QKNORM_VARIANT_CTA) return fused_cta_kernel(dtype, pl.vmax, pl.prefetch != 0, nullptr);
-    return fused_generic_kernel(dtype);
-}
-
-size_t plan_smem(const qknorm_plan &pl, int32_t P) {
-    if (pl.variant == QKNORM_VARIANT_CTA) return 0;
-    return (size_t)P * (pl.groups_q + pl.groups_k) * sizeof(float);
-}
-
-bool generic_smem_ready[kMaxDevices][2];
-
-cudaError_t prepare_generic(int dtype) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (!generic_smem_ready[dev][dtype]) {
-        e = cudaFuncSetAttribute(fused_generic_kernel(dtype),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kGenericMaxSmem);
-        if (e != cudaSuccess) return e;
-        generic_smem_ready[dev][dtype] = true;
+// The kernel a plan launches (for the occupancy query: the register variant
+// with prefetch, whose footprint is the larger).
+const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy) {
+    switch (pl.variant) {
+    case QKNORM_VARIANT_CTA:
+        return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0, nullptr);
+    case QKNORM_VARIANT_BULK:
+        return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, nullptr);
+    default:
+        return fused_generic_kernel(dtype);
     }
+}
+
+// Per-device, per-kernel one-time set-up: the dynamic shared memory opt-in.
+struct Prepared {
+    int device;
+    const void *fn;
+};
+constexpr int kPreparedSlots = 512;
+Prepared g_prepared[kPreparedSlots];
+int g_prepared_n = 0;
+std::mutex g_prepared_mu;
+
+cudaError_t prepare_kernel(int dev, const void *fn, int max_dynamic_smem) {
+    std::lock_guard<std::mutex> lock(g_prepared_mu);
+    for (int i = 0; i < g_prepared_n; ++i)
+        if (g_prepared[i].device == dev && g_prepared[i].fn == fn) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dynamic_smem);
+    if (e != cudaSuccess) return e;
+    if (g_prepared_n < kPreparedSlots) g_prepared[g_prepared_n++] = Prepared{dev, fn};
     return cudaSuccess;
 }
 
-// Full device plan: occupancy for the chosen kernel (with prefetch, which has
-// the larger register footprint, for the persistent case).
+struct RegEntry {
+    const void *fn;
+    int regs;
+};
+RegEntry g_regs[kPreparedSlots];
+int g_regs_n = 0;
+
+cudaError_t kernel_regs(const void *fn, int *regs) {
+    std::lock_guard<std::mutex> lock(g_prepared_mu);
+    for (int i = 0; i < g_regs_n; ++i)
+        if (g_regs[i].fn == fn) {
+            *regs = g_regs[i].regs;
+            return cudaSuccess;
+        }
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, fn);
+    if (e != cudaSuccess) return e;
+    *regs = attr.numRegs > 0 ? attr.numRegs : kRegsHint;
+    if (g_regs_n < kPreparedSlots) g_regs[g_regs_n++] = RegEntry{fn, *regs};
+    return cudaSuccess;
+}
+
+// Full device plan: the kernel's registers and the device's SM count, then
+// occupancy with the plan's shared memory gives B_res.
 cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
                         qknorm_plan *pl, int *status) {
-    *status = plan_static(Dq, Dk, P, dtype, g_forced_variant, pl);
-    if (*status != QKNORM_OK) return cudaSuccess;
     int dev = 0, sms = 0;
     cudaError_t e = device_sms(&dev, &sms);
     if (e != cudaSuccess) return e;
-    if (pl->variant != QKNORM_VARIANT_CTA) {
-        e = prepare_generic(dtype);
+    *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, kRegsHint, pl);
+    if (*status != QKNORM_OK) return cudaSuccess;
+    if (pl->variant == QKNORM_VARIANT_BULK) {
+        int regs = kRegsHint;
+        e = kernel_regs(plan_kernel(*pl, dtype, true), &regs);
+        if (e != cudaSuccess) return e;
+        *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, regs, pl);
+        if (*status != QKNORM_OK) return cudaSuccess;
+    }
+    const void *fn = plan_kernel(*pl, dtype, true);
+    if (pl->smem_bytes > 48 * 1024 || pl->variant == QKNORM_VARIANT_GENERIC ||
+        pl->variant == QKNORM_VARIANT_WARP) {
+        e = prepare_kernel(dev, fn, pl->variant == QKNORM_VARIANT_BULK ? kSmemPerCta : kGenericMaxSmem);
         if (e != cudaSuccess) return e;
     }
-    qknorm_plan probe = *pl;
-    probe.prefetch = 1;
-    const void *fn = plan_kernel(probe, dtype);
     int bres = 1;
-    e = resident_blocks(dev, fn, pl->block, plan_smem(probe, P), &bres);
+    e = resident_blocks(dev, fn, pl->block, (size_t)pl->smem_bytes, &bres);
     if (e != cudaSuccess) return e;
     plan_grid(T, sms, bres, pl);
     return cudaSuccess;
@@ -237,7 +352,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 100; }
+int qknorm_version(void) { return 102; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -253,7 +368,7 @@ const char *qknorm_status_string(int status) {
 const char *qknorm_last_error(void) { return g_last_error; }
 
 int qknorm_force_variant(int32_t variant, int64_t grid) {
-    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_GENERIC || grid < 0)
+    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_BULK || grid < 0)
         return QKNORM_ERR_INVALID_ARG;
     g_forced_variant = variant;
     g_forced_grid = grid;
@@ -266,10 +381,14 @@ int qknorm_plan_fwd(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
     int st = check_shape(T, Dq, P, dtype);
     if (st == QKNORM_OK) st = check_shape(T, Dk, P, dtype);
     if (st != QKNORM_OK) return st;
-    st = plan_static(Dq, Dk, P, dtype, g_forced_variant, plan);
+    st = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, num_sms, kRegsHint, plan);
     if (st != QKNORM_OK) return st;
     if (blocks_per_sm <= 0) {
-        blocks_per_sm = 2048 / plan->block;
+        blocks_per_sm = kThreadsPerSm / plan->block;
+        if (plan->smem_bytes > 0) {
+            const int by_smem = kSmemPerSm / (int)(plan->smem_bytes + kSmemReservedPerCta);
+            if (by_smem < blocks_per_sm) blocks_per_sm = by_smem;
+        }
         if (blocks_per_sm > 32) blocks_per_sm = 32;
         if (blocks_per_sm < 1) blocks_per_sm = 1;
     }
@@ -337,10 +456,40 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
         e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, a, pl.block, pl.grid, s);
+    } else if (pl.variant == QKNORM_VARIANT_BULK) {
+        e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, a, pl.stages,
+                              pl.block, pl.grid, g_wait_limit_ns, s);
     } else {
-        e = launch_fused_generic(dtype, a, pl.block, pl.grid, plan_smem(pl, P), s);
+        e = launch_fused_generic(dtype, a, pl.block, pl.grid, (size_t)pl.smem_bytes, s);
     }
     return finish(e);
+}
+
+int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_regs,
+                      int32_t wait_limit_ms) {
+    if (stages < 0 || stages > bulk_max_stages() || gamma_regs < -1 || gamma_regs > 1 ||
+        wait_limit_ms < 0 || !(tokens_per_stage == 0 || tokens_per_stage == 1 ||
+                               tokens_per_stage == 2 || tokens_per_stage == 4))
+        return QKNORM_ERR_INVALID_ARG;
+    g_tune_stages = stages;
+    g_tune_tb = tokens_per_stage;
+    g_tune_gamma_regs = gamma_regs;
+    g_wait_limit_ns = wait_limit_ms > 0 ? (uint64_t)wait_limit_ms * 1000000ull : 2000000000ull;
+    return QKNORM_OK;
+}
+
+int qknorm_device_errors(uint32_t *flags, int32_t clear) {
+    if (flags == nullptr) return QKNORM_ERR_INVALID_ARG;
+    unsigned v = 0;
+    cudaError_t e = read_device_errors(&v, clear != 0);
+    if (e != cudaSuccess) return finish(e);
+    *flags = v;
+    return QKNORM_OK;
+}
+
+int qknorm_selftest_bounded_wait(uint64_t limit_ns, void *stream) {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return QKNORM_ERR_INVALID_ARG;
+    return finish(launch_bounded_wait_probe(limit_ns, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int32_t P,

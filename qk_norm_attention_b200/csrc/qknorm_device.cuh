@@ -122,6 +122,26 @@ __device__ __forceinline__ uint4 vapply(BF16Tag, const uint4 &v, const float *g,
     return o;
 }
 
+// Same as vapply with gamma already in registers (g[0..vec-1], indexed with
+// compile-time constants after unrolling).
+__device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float *g, float r) {
+    uint4 o;
+    o.x = __float_as_uint(wmul(__uint_as_float(v.x), g[0], r));
+    o.y = __float_as_uint(wmul(__uint_as_float(v.y), g[1], r));
+    o.z = __float_as_uint(wmul(__uint_as_float(v.z), g[2], r));
+    o.w = __float_as_uint(wmul(__uint_as_float(v.w), g[3], r));
+    return o;
+}
+
+__device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r) {
+    uint4 o;
+    o.x = pack_bf16x2(wmul(bf_lo(v.x), g[0], r), wmul(bf_hi(v.x), g[1], r));
+    o.y = pack_bf16x2(wmul(bf_lo(v.y), g[2], r), wmul(bf_hi(v.y), g[3], r));
+    o.z = pack_bf16x2(wmul(bf_lo(v.z), g[4], r), wmul(bf_hi(v.z), g[5], r));
+    o.w = pack_bf16x2(wmul(bf_lo(v.w), g[6], r), wmul(bf_hi(v.w), g[7], r));
+    return o;
+}
+
 // ---------------------------------------------------------------- memory
 
 // Streaming (read-once / write-once) 16-byte accesses: evict-first in L1/L2.

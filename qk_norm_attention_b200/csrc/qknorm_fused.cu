@@ -49,7 +49,7 @@ __device__ __forceinline__ Task decode_task(const FusedArgs &a, int j) {
 }
 
 template <class Tag, int VMAX, bool PREFETCH, int MAXT>
-__global__ void __launch_bounds__(MAXT) fused_cta(const FusedArgs a) {
+__global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     __shared__ float red[2][32];
     const int warp = threadIdx.x >> 5;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(MAXT) fused_cta(const FusedArgs a) {
 }
 
 template <class Tag>
-__global__ void __launch_bounds__(256) fused_generic(const FusedArgs a) {
+__global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     extern __shared__ float red[];  // one float per task
     const int warp = threadIdx.x >> 5;

@@ -1,0 +1,310 @@
+// qknorm_fused_bulk.cu -- the fused QK-Norm kernel fed by bulk copies.
+//
+// Same computation and reduction order as fused_cta (SwiftQK technical
+// review, Section 3, Algorithm 1, Phases A-C; one warp per (tensor, shard,
+// group) task; persistent stride loop over tokens), but the rows reach the SM
+// through the TMA engine: one elected thread issues cp.async.bulk copies of
+// whole Q and K rows into a ring of S stages in shared memory, each stage
+// completed on its own mbarrier. Bytes in flight per SM are then set by
+// shared memory, not by registers.
+//
+// A stage holds TB tokens (those the CTA meets in TB consecutive turns of its
+// stride loop). One pass of the loop reduces all TB tokens with independent
+// chains and butterflies, crosses ONE CTA barrier for all of them, and streams
+// their outputs, so the serial per-token work (shared-memory reads, FMA chain,
+// butterfly, barrier, combine, divide, rsqrt) overlaps across TB tokens and
+// each lane's gamma registers serve TB tokens.
+//
+// Per pass: wait for the stage (bounded), copy this lane's vectors of the TB
+// tokens from shared memory to registers, chains, butterflies, group sums to
+// shared memory; one barrier; thread 0 refills the stage with the tokens S
+// passes ahead; every lane forms the TB factors and writes (x*gamma)*r.
+#include "qknorm_bulk.cuh"
+#include "qknorm_device.cuh"
+#include "qknorm_internal.h"
+
+namespace qkn {
+
+__device__ unsigned int g_device_errors;
+
+struct BulkArgs {
+    uint32_t stages;       // S
+    uint32_t qbytes;       // bytes of one Q row
+    uint32_t kbytes;       // bytes of one K row
+    uint32_t stage_stride; // bytes between stages (multiple of 128)
+    uint64_t timeout_ns;   // bound of every wait
+};
+
+// Shared memory: [S mbarriers | pad][red: 2 x TBMAX x 32 floats][S stages].
+constexpr uint32_t kBarBytes = 128;
+constexpr int kMaxTB = 4;
+constexpr uint32_t kRedBytes = 2 * kMaxTB * 32 * sizeof(float);
+constexpr uint32_t kStageBase = kBarBytes + kRedBytes;
+constexpr uint32_t kMaxStages = 16;
+
+template <class Tag, int VMAX, bool GREG, int TB, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const BulkArgs b) {
+    constexpr int VEC = Tag::kVec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    float(*red)[kMaxTB][32] = reinterpret_cast<float(*)[kMaxTB][32]>(smem + kBarBytes);
+    unsigned char *stages = smem + kStageBase;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int nt0 = a.P * a.K[0];
+    const int z = warp < nt0 ? 0 : 1;
+    const int jj = z ? warp - nt0 : warp;
+    const int K = z ? a.K[1] : a.K[0];
+    const int p = jj / K;
+    const int kg = jj - p * K;
+    const int nv = z ? a.nv[1] : a.nv[0];
+    const int stride = kLanes * K;
+    const int first = kg * kLanes + lane;
+    const int cnt = slot_count(first, nv, stride);
+    const int64_t rowvec = (z ? a.D[1] : a.D[0]) / VEC;
+    const int64_t col0 = (int64_t)p * nv + first;
+    uint4 *ys = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + col0;
+    const float *gs = (z ? a.g[1] : a.g[0]) + col0 * VEC;
+    const float Df = z ? a.Df[1] : a.Df[0];
+    const float eps = a.eps;
+    const int red_base = z ? nt0 : 0;
+    const uint32_t tok_bytes = b.qbytes + b.kbytes;
+    // This lane's first vector inside a token of a stage (Q row, then K row).
+    const uint32_t lane_off = (z ? b.qbytes : 0u) + (uint32_t)col0 * 16u;
+
+    const int64_t T = a.T;
+    const int64_t G = gridDim.x;
+    const int S = (int)b.stages;
+    const char *qsrc = static_cast<const char *>(a.x[0]);
+    const char *ksrc = static_cast<const char *>(a.x[1]);
+
+    // Tokens of pass n: blockIdx.x + (n*TB + j)*G, j < TB (those below T).
+    auto issue = [&](int s, int64_t n) {
+        unsigned char *st = stages + (size_t)s * b.stage_stride;
+        const int64_t t0 = blockIdx.x + n * TB * G;
+        int ntok = 0;
+#pragma unroll
+        for (int j = 0; j < TB; ++j) ntok += (t0 + j * G < T) ? 1 : 0;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)ntok * tok_bytes);
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            const int64_t tt = t0 + j * G;
+            if (tt < T) {
+                bulk_copy_g2s(st + j * tok_bytes, qsrc + tt * (int64_t)b.qbytes, b.qbytes, &full[s]);
+                bulk_copy_g2s(st + j * tok_bytes + b.qbytes, ksrc + tt * (int64_t)b.kbytes,
+                              b.kbytes, &full[s]);
+            }
+        }
+    };
+
+    const int64_t npass = (T - blockIdx.x + TB * G - 1) / (TB * G);  // >= 1 since blockIdx.x < T
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int s = 0; s < S && s < npass; ++s) issue(s, s);
+    }
+
+    float gam[GREG ? VMAX * VEC : 1];
+    if (GREG) {
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (i < cnt) {
+#pragma unroll
+                for (int e = 0; e < VEC; e += 4) {
+                    const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
+                        gs + (int64_t)i * stride * VEC + e));
+                    gam[i * VEC + e] = g4.x;
+                    gam[i * VEC + e + 1] = g4.y;
+                    gam[i * VEC + e + 2] = g4.z;
+                    gam[i * VEC + e + 3] = g4.w;
+                }
+            }
+    }
+
+    int s = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    for (int64_t n = 0; n < npass; ++n) {
+        const int64_t t0 = blockIdx.x + n * TB * G;
+        const bool ok = mbar_wait_bounded(&full[s], phase, b.timeout_ns);
+        const unsigned char *st = stages + (size_t)s * b.stage_stride + lane_off;
+        uint4 cur[TB][VMAX];
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(st + j * tok_bytes);
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt && t0 + j * G < T) cur[j][i] = src[i * stride];
+        }
+        // Phase A for TB tokens: independent chains and butterflies.
+        float c[TB];
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            c[j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (i < cnt && t0 + j * G < T) c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
+        }
+#pragma unroll
+        for (int j = 0; j < TB; ++j) c[j] = butterfly(c[j]);
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < TB; ++j) red[buf][j][warp] = c[j];
+        }
+        if (__syncthreads_or(!ok)) {
+            // A stage never arrived: record it, let copies in flight land, leave.
+            if (tid == 0) {
+                atomicOr(&g_device_errors, kErrWaitTimeout);
+                int ds = s;
+                uint32_t dp = phase;
+                for (int64_t m = n; m < npass && m < n + S; ++m) {
+                    if (!mbar_wait_bounded(&full[ds], dp, b.timeout_ns))
+                        atomicOr(&g_device_errors, kErrDrainTimeout);
+                    if (++ds == S) {
+                        ds = 0;
+                        dp ^= 1u;
+                    }
+                }
+            }
+            return;
+        }
+        // Every lane holds its vectors in registers now: refill this stage.
+        if (tid == 0 && n + S < npass) {
+            fence_proxy_async_smem();
+            issue(s, n + S);
+        }
+        // Phase B: shard sums in order and the factor; weight multiply, Phase C.
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            const int64_t t = t0 + j * G;
+            if (t < T) {
+                const float r = factor(combine(&red[buf][j][red_base], a.P, K), Df, eps);
+                uint4 *dst = ys + t * rowvec;
+#pragma unroll
+                for (int i = 0; i < VMAX; ++i)
+                    if (i < cnt) {
+                        uint4 y;
+                        if (GREG)
+                            y = vapply_regs(Tag{}, cur[j][i], &gam[i * VEC], r);
+                        else
+                            y = vapply(Tag{}, cur[j][i], gs + (int64_t)i * stride * VEC, r);
+                        st_stream(dst + (int64_t)i * stride, y);
+                    }
+            }
+        }
+        buf ^= 1;
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+// A kernel that waits on an mbarrier nobody arrives on, with the same bounded
+// wait as fused_bulk: it must time out, record kErrWaitTimeout and return.
+__global__ void bounded_wait_probe(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_bounded(&bar, 0, timeout_ns);
+    if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicOr(&g_device_errors, kErrWaitTimeout);
+}
+
+// ---------------------------------------------------------------- instances and launch
+
+// Combinations that exist: TB tokens x VMAX vectors per lane <= 12 (registers).
+constexpr bool bulk_exists(int vmax, int tb) {
+    return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2 || tb == 4) && vmax * tb <= 12;
+}
+constexpr int bulk_max_threads(int vmax, int tb) { return vmax * tb <= 2 ? 1024 : 512; }
+
+template <class Tag, bool GREG, int V, int TB>
+const void *bulk_fn() {
+    if constexpr (bulk_exists(V, TB))
+        return reinterpret_cast<const void *>(&fused_bulk<Tag, V, GREG, TB, bulk_max_threads(V, TB)>);
+    else
+        return nullptr;
+}
+
+template <class Tag, bool GREG, int TB>
+const void *bulk_table_tb(int vmax) {
+    switch (vmax) {
+    case 1: return bulk_fn<Tag, GREG, 1, TB>();
+    case 2: return bulk_fn<Tag, GREG, 2, TB>();
+    case 3: return bulk_fn<Tag, GREG, 3, TB>();
+    case 4: return bulk_fn<Tag, GREG, 4, TB>();
+    case 5: return bulk_fn<Tag, GREG, 5, TB>();
+    case 6: return bulk_fn<Tag, GREG, 6, TB>();
+    case 7: return bulk_fn<Tag, GREG, 7, TB>();
+    case 8: return bulk_fn<Tag, GREG, 8, TB>();
+    default: return nullptr;
+    }
+}
+
+template <class Tag, bool GREG>
+const void *bulk_table(int vmax, int tb) {
+    switch (tb) {
+    case 1: return bulk_table_tb<Tag, GREG, 1>(vmax);
+    case 2: return bulk_table_tb<Tag, GREG, 2>(vmax);
+    case 4: return bulk_table_tb<Tag, GREG, 4>(vmax);
+    default: return nullptr;
+    }
+}
+
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int *max_threads) {
+    if (!bulk_exists(vmax, tb)) return nullptr;
+    if (max_threads) *max_threads = bulk_max_threads(vmax, tb);
+    if (dtype == 0) return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb) : bulk_table<F32Tag, false>(vmax, tb);
+    if (dtype == 1) return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb) : bulk_table<BF16Tag, false>(vmax, tb);
+    return nullptr;
+}
+
+uint32_t bulk_stage_stride(int64_t qbytes, int64_t kbytes, int tb) {
+    return (uint32_t)((tb * (qbytes + kbytes) + 127) / 128 * 128);
+}
+
+size_t bulk_smem_bytes(int stages, uint32_t stage_stride) {
+    return (size_t)kStageBase + (size_t)stages * stage_stride;
+}
+
+int bulk_max_stages() { return (int)kMaxStages; }
+
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, const FusedArgs &a,
+                              int stages, int block, int64_t grid, uint64_t timeout_ns,
+                              cudaStream_t s) {
+    const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, nullptr);
+    if (!fn || stages < 1 || stages > (int)kMaxStages) return cudaErrorInvalidValue;
+    const int64_t es = dtype == 1 ? 2 : 4;
+    BulkArgs b;
+    b.stages = (uint32_t)stages;
+    b.qbytes = (uint32_t)(a.D[0] * es);
+    b.kbytes = (uint32_t)(a.D[1] * es);
+    b.stage_stride = bulk_stage_stride(b.qbytes, b.kbytes, tb);
+    b.timeout_ns = timeout_ns;
+    const size_t smem = bulk_smem_bytes(stages, b.stage_stride);
+    void *args[] = {const_cast<FusedArgs *>(&a), &b};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, smem, s);
+}
+
+cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s) {
+    void *args[] = {&timeout_ns};
+    return cudaLaunchKernel(reinterpret_cast<const void *>(&bounded_wait_probe), dim3(1), dim3(64),
+                            args, 0, s);
+}
+
+cudaError_t read_device_errors(unsigned *out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_errors, sizeof(unsigned));
+    if (e != cudaSuccess || !clear) return e;
+    const unsigned zero = 0;
+    return cudaMemcpyToSymbol(g_device_errors, &zero, sizeof(unsigned));
+}
+
+}  // namespace qkn

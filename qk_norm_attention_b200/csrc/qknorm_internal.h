@@ -50,6 +50,18 @@ cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *
                          int64_t T, int32_t D, int32_t P, float eps, int block, int64_t grid,
                          cudaStream_t s);
 
+// The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
+// tb = tokens per ring stage (1, 2 or 4); nullptr if (vmax, tb) has no instance.
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int *max_threads);
+uint32_t bulk_stage_stride(int64_t qbytes, int64_t kbytes, int tb);
+size_t bulk_smem_bytes(int stages, uint32_t stage_stride);
+int bulk_max_stages();
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, const FusedArgs &a,
+                              int stages, int block, int64_t grid, uint64_t timeout_ns,
+                              cudaStream_t s);
+cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
+cudaError_t read_device_errors(unsigned *out, bool clear);
+
 // Largest dynamic shared memory the generic kernel is given (bytes).
 constexpr int kGenericMaxSmem = 200 * 1024;
 

@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 100
+    assert qk.qknorm_version() == 102
 
 
 # ----------------------------------------------------------------- argument checks
@@ -132,12 +132,19 @@ def test_plan_for_each_workload(qk):
     for name, wl in W.WORKLOADS.items():
         for T in wl.Ts:
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
-            assert pl["variant"] == qk.VARIANT_CTA, name
+            # Several tokens per CTA: the bulk-copy ring; otherwise registers only.
+            want = qk.VARIANT_BULK if T > 2 * 148 else qk.VARIANT_CTA
+            assert pl["variant"] == want, (name, T)
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
             assert pl["grid"] == min(T, 148 * 4)
-            assert pl["prefetch"] == int(T > 148 * 4)
             assert pl["groups_q"] == pl["groups_k"] == 1
+            if want == qk.VARIANT_BULK:
+                assert pl["prefetch"] == 0 and 2 <= pl["stages"] <= 8
+                stage = (wl.Dq + wl.Dk) * wl.elem_bytes
+                assert pl["smem_bytes"] >= pl["stages"] * stage
+            else:
+                assert pl["prefetch"] == int(T > 148 * 4) and pl["stages"] == 0
 
 
 def test_plan_groups_and_fallbacks(qk):
@@ -168,5 +175,39 @@ def test_forced_variants(qk):
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         with pytest.raises(qk.QKNormError):
             qk.qknorm_force_variant(5, 0)
+        qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
+        qk.qknorm_set_tuning(stages=3, tokens_per_stage=4, gamma_regs=0)
+        pl = qk.qknorm_plan_fwd(10, 4096, 4096, 8, qk.QKNORM_BF16, 148)   # vmax 2
+        assert (pl["variant"], pl["stages"], pl["gamma_regs"], pl["tokens_per_stage"]) == \
+            (qk.VARIANT_BULK, 3, 0, 4)
+        assert pl["smem_bytes"] >= 3 * 4 * 2 * 4096 * 2
+        qk.qknorm_set_tuning(tokens_per_stage=4)            # vmax 8 x 4 tokens: no instance
+        with pytest.raises(qk.QKNormError) as ei:
+            qk.qknorm_plan_fwd(10, 4096, 4096, 2, qk.QKNORM_BF16, 148)
+        assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_tuning(tokens_per_stage=3)
+        with pytest.raises(qk.QKNormError) as ei:      # 64 tasks do not fit one CTA
+            qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
+        assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_tuning(stages=17)
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+        qk.qknorm_set_tuning()
+
+
+def test_bulk_stages_fill_shared_memory(qk):
+    """Stage count: as many token stages as fit in each CTA's share of the
+    SM's 228 KiB (1 KiB reserved per CTA), at most 8. The host-only plan
+    assumes 64 registers: 256 threads -> 4 CTAs per SM -> 56 KiB each ->
+    two 20 KiB stages of the 13B prefill shape after the 384-byte header."""
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    pl = qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_BF16, 148)
+    stage = pl["tokens_per_stage"] * 2 * 5120 * 2
+    assert pl["tokens_per_stage"] == 2
+    assert (pl["stages"], pl["smem_bytes"]) == (2, 1152 + 2 * stage)
+    # A 1024-thread CTA (P = 16) is alone on its SM: 7 stages of 2 x 16 KiB
+    # tokens fit in 227 KiB after the header.
+    pl = qk.qknorm_plan_fwd(8192, 4096, 4096, 16, qk.QKNORM_BF16, 148)
+    assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 7, 2)

@@ -14,7 +14,7 @@ from gpu_util import bits, check_outputs, check_stats, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ("cta", "warp", "generic")
+VARIANTS = ("cta", "bulk", "warp", "generic")
 
 
 @pytest.fixture(scope="module")
@@ -38,7 +38,7 @@ def _inputs(wl, T):
 
 def _fwd(qk, wl, q, k, gq, gk, variant=None, grid=0):
     vid = {"cta": qk.VARIANT_CTA, "warp": qk.VARIANT_WARP, "generic": qk.VARIANT_GENERIC,
-           None: qk.VARIANT_AUTO}[variant]
+           "bulk": qk.VARIANT_BULK, None: qk.VARIANT_AUTO}[variant]
     qk.qknorm_force_variant(vid, grid)
     try:
         oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk),
@@ -81,8 +81,8 @@ def test_shapes_and_variants(qk, orc, shape):
         try:
             outs[v] = _fwd(qk, wl, q, k, gq, gk, variant=v)
         except qk.QKNormError as e:
-            # Only the register-resident CTA kernel has shape limits.
-            assert v == "cta" and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
+            # Only the register-resident kernels (cta, bulk) have shape limits.
+            assert v in ("cta", "bulk") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
     base = outs["generic"]
     for v, (oq, ok) in outs.items():
         assert torch.equal(bits(oq), bits(base[0])), f"{v} Q differs from generic"
@@ -211,3 +211,37 @@ def test_more_than_2_31_elements(qk, orc):
         check_outputs(to_host(y.index_select(0, rows)), y_or, "bf16", "2^31+ rows")
     del q, k, oq, ok, ak, st
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("stages", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("tokens_per_stage", [1, 2, 4])
+@pytest.mark.parametrize("gamma_regs", [0, 1])
+def test_bulk_ring_depths(qk, stages, tokens_per_stage, gamma_regs):
+    """Every ring depth, token batch and gamma placement gives the same bits,
+    with grids that make CTAs wrap the ring several times and end mid-stage."""
+    wl = W.custom("ring", 2 * 148 + 37, 5120, 1024, 8, seed=35)
+    q, k, gq, gk = _inputs(wl, wl.Ts[0])
+    ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
+    try:
+        qk.qknorm_set_tuning(stages=stages, tokens_per_stage=tokens_per_stage, gamma_regs=gamma_regs)
+        for grid in (0, 7, 148):
+            got = _fwd(qk, wl, q, k, gq, gk, variant="bulk", grid=grid)
+            assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
+    finally:
+        qk.qknorm_set_tuning()
+    assert qk.qknorm_device_errors() == 0
+
+
+def test_bounded_wait_times_out_and_reports(qk):
+    """A wait on an mbarrier nobody arrives on gives up after its limit, sets
+    the error bit, and leaves the context usable."""
+    assert qk.qknorm_device_errors(clear=True) == 0
+    qk.qknorm_selftest_bounded_wait(20_000_000)        # 20 ms
+    torch.cuda.synchronize()
+    assert qk.qknorm_device_errors(clear=True) & 1
+    assert qk.qknorm_device_errors(clear=False) == 0
+    x = torch.ones(4, 256, device="cuda")               # the context still works
+    g = torch.ones(256, device="cuda")
+    oq, _ = qk.qknorm_fwd(x, x.clone(), g, g, 2, 0.0)
+    torch.cuda.synchronize()
+    assert bool((oq == 1.0).all())
