@@ -224,6 +224,12 @@ def test_bulk_ring_depths(qk, stages, tokens_per_stage, gamma_regs):
     ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
     try:
         qk.qknorm_set_tuning(stages=stages, tokens_per_stage=tokens_per_stage, gamma_regs=gamma_regs)
+        ring = stages * tokens_per_stage * (5120 + 1024) * 2
+        if ring > 220 * 1024:      # more than one CTA's shared memory: rejected before launch
+            with pytest.raises(qk.QKNormError) as ei:
+                _fwd(qk, wl, q, k, gq, gk, variant="bulk")
+            assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+            return
         for grid in (0, 7, 148):
             got = _fwd(qk, wl, q, k, gq, gk, variant="bulk", grid=grid)
             assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
