@@ -36,6 +36,9 @@ METRIC = "QK-Norm GB/s and % of B200 HBM peak (prefill); μs/call at decode T≤
 HEADLINE = "prefill13b"
 FALLBACK_HBM_GBS = 6650.0
 
+KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_generic",
+                     3: "fused_bulk", 4: "fused_rows"}
+
 # dram bytes per launch of the headline kernel from one ncu capture, and the
 # hash of the kernel sources it was taken with (None until captured).
 NCU_TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
@@ -548,7 +551,8 @@ def run_native(args, dist):
         "tokens_per_s": round(dist.world * T / step_ms * 1000, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "fused_cta (qknorm_fwd)", "peak_source": peak_src,
+                     "kernel": KERNEL_OF_VARIANT.get(plan["variant"], "?") + " (qknorm_fwd)",
+                     "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": nbytes,
                      "kernel_us": round(kern_ms * 1000, 3)},
         "e2e": {"value": round(dist.world * nbytes / e2e_ms / 1e6, 2), "unit": "GB/s",

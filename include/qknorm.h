@@ -141,9 +141,14 @@ typedef enum {
                                    token, then re-reads the row to apply */
     QKNORM_VARIANT_GENERIC = 2, /* CTA per token, any shape: warps loop over the
                                    shard groups, re-read the row to apply */
-    QKNORM_VARIANT_BULK = 3     /* as CTA, but rows arrive by bulk asynchronous
+    QKNORM_VARIANT_BULK = 3,    /* as CTA, but rows arrive by bulk asynchronous
                                    copies (TMA engine) into a ring of token stages
                                    in shared memory, completed on mbarriers */
+    QKNORM_VARIANT_ROWS = 4     /* warp per row: each warp has its own ring of
+                                   bulk-copied row stages, walks all P shards of
+                                   the row itself and applies from shared memory
+                                   with gamma staged once per CTA; no CTA barrier
+                                   per row */
 } qknorm_variant;
 
 /* A launch plan chosen by the selector (host-side description). */
@@ -155,7 +160,7 @@ typedef struct {
     int32_t prefetch;    /* 1 if a CTA prefetches its next token */
     int32_t groups_q;    /* K for a Q shard */
     int32_t groups_k;    /* K for a K shard */
-    int32_t stages;      /* ring stages per CTA (bulk variant), else 0 */
+    int32_t stages;      /* ring stages per CTA (bulk) or per warp (rows), else 0 */
     int32_t tokens_per_stage; /* tokens a bulk stage holds (1, 2 or 4), else 0 */
     int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
     int64_t smem_bytes;  /* dynamic shared memory per CTA */
@@ -199,6 +204,13 @@ QKNORM_API int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, 
  */
 QKNORM_API int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_regs,
                                  int32_t wait_limit_ms);
+
+/*
+ * qknorm_set_rows_tuning -- process-wide tuning of the warp-per-row variant:
+ * warps per CTA (0 = as many as shared memory allows, up to 16) and row
+ * stages per warp (0 = automatic). Not thread-safe with concurrent calls.
+ */
+QKNORM_API int qknorm_set_rows_tuning(int32_t warps, int32_t stages);
 
 /*
  * qknorm_device_errors -- read (and with clear != 0, reset) the library's

@@ -37,9 +37,10 @@ QKNORM_ERR_MISALIGNED = 2
 QKNORM_ERR_UNSUPPORTED = 3
 QKNORM_ERR_CUDA = 4
 
-VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK = -1, 0, 1, 2, 3
+VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_ROWS = \
+    -1, 0, 1, 2, 3, 4
 VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic",
-                 VARIANT_BULK: "bulk"}
+                 VARIANT_BULK: "bulk", VARIANT_ROWS: "rows"}
 
 _DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16}
 
@@ -92,6 +93,8 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_version.restype = ctypes.c_int
     lib.qknorm_set_tuning.argtypes = [i32, i32, i32, i32]
     lib.qknorm_set_tuning.restype = ctypes.c_int
+    lib.qknorm_set_rows_tuning.argtypes = [i32, i32]
+    lib.qknorm_set_rows_tuning.restype = ctypes.c_int
     lib.qknorm_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     lib.qknorm_device_errors.restype = ctypes.c_int
     lib.qknorm_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
@@ -229,6 +232,11 @@ def qknorm_set_tuning(stages: int = 0, tokens_per_stage: int = 0, gamma_regs: in
     """Tune the bulk variant process-wide (the defaults restore automatic choice)."""
     _check("qknorm_set_tuning", lib.qknorm_set_tuning(int(stages), int(tokens_per_stage),
                                                       int(gamma_regs), int(wait_limit_ms)))
+
+
+def qknorm_set_rows_tuning(warps: int = 0, stages: int = 0) -> None:
+    """Warps per CTA and row stages per warp of the rows variant (0 = automatic)."""
+    _check("qknorm_set_rows_tuning", lib.qknorm_set_rows_tuning(int(warps), int(stages)))
 
 
 def qknorm_device_errors(clear: bool = True) -> int:

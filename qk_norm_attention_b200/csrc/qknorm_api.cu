@@ -130,13 +130,17 @@ int32_t g_tune_stages = 0;           // bulk stages per CTA; 0 = automatic
 int32_t g_tune_tb = 0;               // tokens per bulk stage; 0 = automatic
 int32_t g_tune_gamma_regs = -1;      // -1 = automatic
 uint64_t g_wait_limit_ns = 2000000000ull;
+int32_t g_rows_warps = 0;            // warps per CTA of the rows variant; 0 = automatic
+int32_t g_rows_stages = 0;           // row stages per warp; 0 = automatic
+constexpr int kRowsStagesAuto = 1;
+constexpr int kRowsMaxWarps = 16;
 
 constexpr int kSmemPerSm = 228 * 1024;      // shared memory of one SM
 constexpr int kSmemPerCta = 227 * 1024;     // largest opt-in dynamic shared memory of a CTA
 constexpr int kSmemReservedPerCta = 1024;   // the runtime's per-CTA reservation
 constexpr int kRegsPerSm = 65536;
 constexpr int kThreadsPerSm = 2048;
-constexpr int kMaxStagesAuto = 8;
+constexpr int kMaxStagesAuto = 2;   // measured best on B200 (2 CTAs x 2 stages per SM)
 constexpr int kRegsHint = 64;               // register estimate when no device is queried
 
 struct Shapes {
@@ -159,10 +163,11 @@ bool gamma_regs_for(int32_t dtype, int vmax) {
     return vmax * vec_of(dtype) <= 40;
 }
 
-// Tokens per bulk stage: 2 where an instance exists (VMAX x TB <= 12).
+// Tokens per bulk stage: 1 (batching tokens measured no gain on B200 once
+// the stage ring keeps enough bytes in flight).
 int tokens_per_stage_for(int vmax) {
-    if (g_tune_tb > 0) return g_tune_tb;
-    return vmax * 2 <= 12 ? 2 : 1;
+    (void)vmax;
+    return g_tune_tb > 0 ? g_tune_tb : 1;
 }
 
 // Stage count of the bulk kernel: the most stages (up to kMaxStagesAuto) that
@@ -186,6 +191,30 @@ void bulk_stages(uint32_t stride, int block, int regs, qknorm_plan *pl) {
     pl->smem_bytes = (int64_t)bulk_smem_bytes(S, stride);
 }
 
+// Warps per CTA of the rows variant: the most resident warps per SM (up to
+// kRowsMaxWarps) that shared memory allows, preferring two CTAs per SM (each
+// CTA holds its own copy of gamma).
+int rows_auto_warps(int32_t Dq, int32_t Dk, int32_t dtype, int S) {
+    int best_w = 0, best_total = 0;
+    for (int ctas = 2; ctas >= 1; --ctas) {
+        for (int W = kRowsMaxWarps / ctas; W >= 1; --W) {
+            const size_t sm = rows_layout(Dq, Dk, (int)elem_of(dtype), W, S).smem_bytes;
+            if (sm <= (size_t)kSmemPerCta && (int64_t)ctas * (sm + kSmemReservedPerCta) <= kSmemPerSm) {
+                if (ctas * W > best_total) {
+                    best_total = ctas * W;
+                    best_w = W;
+                }
+                break;
+            }
+        }
+    }
+    return best_w;
+}
+
+bool rows_fit(int32_t Dq, int32_t Dk, int32_t dtype) {
+    return rows_layout(Dq, Dk, (int)elem_of(dtype), 1, 1).smem_bytes <= (size_t)kSmemPerCta;
+}
+
 // Static part of the plan: which kernel, block size, template width, stages.
 int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t variant,
                 int num_sms, int regs, qknorm_plan *pl) {
@@ -203,13 +232,20 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
                                               (int64_t)Dk * elem_of(dtype), tb);
     const bool bulk_ok = bulk_inst && sh.ntask * kLanes <= bulk_max &&
                          (int64_t)bulk_smem_bytes(2, stride) <= kSmemPerCta;
+    const bool rows_ok = rows_fit(Dq, Dk, dtype);
     if (variant == QKNORM_VARIANT_AUTO) {
-        if (!cta_ok)
-            variant = QKNORM_VARIANT_GENERIC;
-        else if (bulk_ok && T > 2 * (int64_t)num_sms)
+        // Measured on B200: a CTA per token with registers wins while a CTA
+        // sees one token (decode); with several tokens per CTA the token ring
+        // wins when a lane holds >= 4 vectors per shard (per-token overhead
+        // amortised), the warp-per-row kernel otherwise.
+        if (T <= 2 * (int64_t)num_sms)
+            variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
+        else if (bulk_ok && sh.vmax >= 4)
             variant = QKNORM_VARIANT_BULK;
+        else if (rows_ok)
+            variant = QKNORM_VARIANT_ROWS;
         else
-            variant = QKNORM_VARIANT_CTA;
+            variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
     }
     if (variant == QKNORM_VARIANT_CTA || variant == QKNORM_VARIANT_BULK) {
         if (variant == QKNORM_VARIANT_CTA ? !cta_ok : !bulk_ok) return QKNORM_ERR_UNSUPPORTED;
@@ -226,6 +262,18 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         }
         return QKNORM_OK;
     }
+    if (variant == QKNORM_VARIANT_ROWS) {
+        const int S = g_rows_stages > 0 ? g_rows_stages : kRowsStagesAuto;
+        int W = g_rows_warps > 0 ? g_rows_warps : rows_auto_warps(Dq, Dk, dtype, S);
+        if (W < 1 || W > kRowsMaxWarps) return QKNORM_ERR_UNSUPPORTED;
+        const RowsLayout L = rows_layout(Dq, Dk, (int)elem_of(dtype), W, S);
+        if (L.smem_bytes > (size_t)kSmemPerCta) return QKNORM_ERR_UNSUPPORTED;
+        pl->variant = QKNORM_VARIANT_ROWS;
+        pl->block = W * kLanes;
+        pl->stages = S;
+        pl->smem_bytes = (int64_t)L.smem_bytes;
+        return QKNORM_OK;
+    }
     if ((size_t)sh.ntask * sizeof(float) > (size_t)kGenericMaxSmem) return QKNORM_ERR_UNSUPPORTED;
     pl->smem_bytes = (int64_t)(sh.ntask * sizeof(float));
     if (variant == QKNORM_VARIANT_WARP) {
@@ -240,6 +288,14 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         return QKNORM_OK;
     }
     return QKNORM_ERR_INVALID_ARG;
+}
+
+// Units of work a CTA can take: tokens, or for the rows variant the 2T rows
+// spread over block/32 warps per CTA.
+int64_t plan_units(int64_t T, const qknorm_plan &pl) {
+    if (pl.variant != QKNORM_VARIANT_ROWS) return T;
+    const int64_t w = pl.block / kLanes;
+    return (2 * T + w - 1) / w;
 }
 
 // Grid: T CTAs up to B_res x N_SM (or the forced grid); the register variant
@@ -261,6 +317,8 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy
         return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0, nullptr);
     case QKNORM_VARIANT_BULK:
         return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, nullptr);
+    case QKNORM_VARIANT_ROWS:
+        return fused_rows_kernel(dtype);
     default:
         return fused_generic_kernel(dtype);
     }
@@ -327,13 +385,14 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     const void *fn = plan_kernel(*pl, dtype, true);
     if (pl->smem_bytes > 48 * 1024 || pl->variant == QKNORM_VARIANT_GENERIC ||
         pl->variant == QKNORM_VARIANT_WARP) {
-        e = prepare_kernel(dev, fn, pl->variant == QKNORM_VARIANT_BULK ? kSmemPerCta : kGenericMaxSmem);
+        e = prepare_kernel(dev, fn, (pl->variant == QKNORM_VARIANT_BULK ||
+                                     pl->variant == QKNORM_VARIANT_ROWS) ? kSmemPerCta : kGenericMaxSmem);
         if (e != cudaSuccess) return e;
     }
     int bres = 1;
     e = resident_blocks(dev, fn, pl->block, (size_t)pl->smem_bytes, &bres);
     if (e != cudaSuccess) return e;
-    plan_grid(T, sms, bres, pl);
+    plan_grid(plan_units(T, *pl), sms, bres, pl);
     return cudaSuccess;
 }
 
@@ -352,7 +411,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 102; }
+int qknorm_version(void) { return 103; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -368,7 +427,7 @@ const char *qknorm_status_string(int status) {
 const char *qknorm_last_error(void) { return g_last_error; }
 
 int qknorm_force_variant(int32_t variant, int64_t grid) {
-    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_BULK || grid < 0)
+    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_ROWS || grid < 0)
         return QKNORM_ERR_INVALID_ARG;
     g_forced_variant = variant;
     g_forced_grid = grid;
@@ -392,7 +451,7 @@ int qknorm_plan_fwd(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
         if (blocks_per_sm > 32) blocks_per_sm = 32;
         if (blocks_per_sm < 1) blocks_per_sm = 1;
     }
-    plan_grid(T, num_sms, blocks_per_sm, plan);
+    plan_grid(plan_units(T, *plan), num_sms, blocks_per_sm, plan);
     return QKNORM_OK;
 }
 
@@ -456,6 +515,8 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
         e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, a, pl.block, pl.grid, s);
+    } else if (pl.variant == QKNORM_VARIANT_ROWS) {
+        e = launch_fused_rows(dtype, a, pl.block / kLanes, pl.stages, pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
         e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, a, pl.stages,
                               pl.block, pl.grid, g_wait_limit_ns, s);
@@ -475,6 +536,14 @@ int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_re
     g_tune_tb = tokens_per_stage;
     g_tune_gamma_regs = gamma_regs;
     g_wait_limit_ns = wait_limit_ms > 0 ? (uint64_t)wait_limit_ms * 1000000ull : 2000000000ull;
+    return QKNORM_OK;
+}
+
+int qknorm_set_rows_tuning(int32_t warps, int32_t stages) {
+    if (warps < 0 || warps > kRowsMaxWarps || stages < 0 || stages > bulk_max_stages())
+        return QKNORM_ERR_INVALID_ARG;
+    g_rows_warps = warps;
+    g_rows_stages = stages;
     return QKNORM_OK;
 }
 

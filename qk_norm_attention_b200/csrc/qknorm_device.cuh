@@ -142,6 +142,21 @@ __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const floa
     return o;
 }
 
+// Same as vapply with gamma read through an arbitrary pointer (used with
+// gamma staged in shared memory); same arithmetic, bit for bit.
+__device__ __forceinline__ uint4 vapply_ptr(F32Tag, const uint4 &v, const float *g, float r) {
+    const float4 g4 = *reinterpret_cast<const float4 *>(g);
+    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+    return vapply_regs(F32Tag{}, v, gg, r);
+}
+
+__device__ __forceinline__ uint4 vapply_ptr(BF16Tag, const uint4 &v, const float *g, float r) {
+    const float4 ga = *reinterpret_cast<const float4 *>(g);
+    const float4 gb = *(reinterpret_cast<const float4 *>(g) + 1);
+    const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    return vapply_regs(BF16Tag{}, v, gg, r);
+}
+
 // ---------------------------------------------------------------- memory
 
 // Streaming (read-once / write-once) 16-byte accesses: evict-first in L1/L2.

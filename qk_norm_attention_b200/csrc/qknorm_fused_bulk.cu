@@ -205,6 +205,152 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     }
 }
 
+// ---------------------------------------------------------------- warp per row
+
+// Warp-per-row kernel. Each warp owns a ring of S row stages in shared memory
+// and processes whole rows (a Q row or a K row of a token) on its own: lane 0
+// issues the bulk copy of the warp's next rows, the warp walks the row's P
+// shards in the order of the reduction (per group: lane chains, butterfly;
+// groups in order; shards in order), forms the factor, and applies
+// (x*gamma)*r re-reading the row from shared memory, with gamma staged in
+// shared memory once per CTA. No CTA-wide barrier is crossed per row, so
+// warps never wait for one another and the per-row bookkeeping is amortised
+// over the whole row.
+struct RowsArgs {
+    uint32_t stages;      // S, per warp
+    uint32_t stage_bytes; // bytes of one row stage (multiple of 128)
+    uint32_t gq_off;      // shared-memory offset of gamma_q
+    uint32_t gk_off;      // shared-memory offset of gamma_k
+    uint32_t ring_off;    // shared-memory offset of the warps' rings
+    uint64_t timeout_ns;
+};
+
+template <class Tag>
+__global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const RowsArgs b) {
+    constexpr int VEC = Tag::kVec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int W = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int S = (int)b.stages;
+    uint64_t *gbar = reinterpret_cast<uint64_t *>(smem);      // gamma barrier
+    uint64_t *full = gbar + 1 + warp * S;                     // this warp's stage barriers
+    const float *gam_q = reinterpret_cast<const float *>(smem + b.gq_off);
+    const float *gam_k = reinterpret_cast<const float *>(smem + b.gk_off);
+    unsigned char *ring = smem + b.ring_off + (size_t)warp * S * b.stage_bytes;
+
+    const int64_t T = a.T;
+    const int64_t R = 2 * T;                                  // Q rows, then K rows
+    const int64_t NW = (int64_t)gridDim.x * W;
+    const int64_t gw = (int64_t)blockIdx.x * W + warp;
+    const uint32_t qbytes = (uint32_t)a.D[0] * (uint32_t)Tag::kBytes;
+    const uint32_t kbytes = (uint32_t)a.D[1] * (uint32_t)Tag::kBytes;
+
+    auto issue = [&](int s, int64_t r) {
+        const bool isk = r >= T;
+        const int64_t t = isk ? r - T : r;
+        const uint32_t nb = isk ? kbytes : qbytes;
+        const char *src = static_cast<const char *>(isk ? a.x[1] : a.x[0]) + t * (int64_t)nb;
+        mbar_arrive_expect_tx(&full[s], nb);
+        bulk_copy_g2s(ring + (size_t)s * b.stage_bytes, src, nb, &full[s]);
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_init(gbar, 1);
+        for (int i = 0; i < W * S; ++i) mbar_init(gbar + 1 + i, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t gqb = (uint32_t)a.D[0] * 4u, gkb = (uint32_t)a.D[1] * 4u;
+        mbar_arrive_expect_tx(gbar, gqb + gkb);
+        bulk_copy_g2s(smem + b.gq_off, a.g[0], gqb, gbar);
+        bulk_copy_g2s(smem + b.gk_off, a.g[1], gkb, gbar);
+    }
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) {
+            const int64_t r = gw + (int64_t)s * NW;
+            if (r < R) issue(s, r);
+        }
+    }
+    // Leave after recording an error, once this warp's copies in flight have
+    // landed (each wait bounded).
+    auto fail = [&](int64_t n_first, int s0, uint32_t ph0) {
+        if (lane == 0) {
+            atomicOr(&g_device_errors, kErrWaitTimeout);
+            int ds = s0;
+            uint32_t dp = ph0;
+            for (int64_t n = n_first; n < n_first + S && gw + n * NW < R; ++n) {
+                if (!mbar_wait_bounded(&full[ds], dp, b.timeout_ns))
+                    atomicOr(&g_device_errors, kErrDrainTimeout);
+                if (++ds == S) {
+                    ds = 0;
+                    dp ^= 1u;
+                }
+            }
+            if (warp == 0 && !mbar_wait_bounded(gbar, 0, b.timeout_ns))
+                atomicOr(&g_device_errors, kErrDrainTimeout);
+        }
+    };
+    if (!__all_sync(kFull, mbar_wait_bounded(gbar, 0, b.timeout_ns))) {
+        fail(0, 0, 0);
+        return;
+    }
+
+    int s = 0;
+    uint32_t phase = 0;
+    for (int64_t n = 0;; ++n) {
+        const int64_t r = gw + n * NW;
+        if (r >= R) break;
+        if (!__all_sync(kFull, mbar_wait_bounded(&full[s], phase, b.timeout_ns))) {
+            fail(n, s, phase);
+            return;
+        }
+        const int z = r >= T ? 1 : 0;
+        const int64_t t = z ? r - T : r;
+        const uint4 *row = reinterpret_cast<const uint4 *>(ring + (size_t)s * b.stage_bytes);
+        const int P = a.P;
+        const int K = z ? a.K[1] : a.K[0];
+        const int nv = z ? a.nv[1] : a.nv[0];
+        const int stride = kLanes * K;
+        // Phase A and the ordered sums of Phase B.
+        float Ssum = 0.f;
+        for (int p = 0; p < P; ++p) {
+            const uint4 *sh = row + (int64_t)p * nv;
+            float Sp = 0.f;
+            for (int kg = 0; kg < K; ++kg) {
+                float c = 0.f;
+#pragma unroll 4
+                for (int v = kg * kLanes + lane; v < nv; v += stride)
+                    c = __fadd_rn(c, vsumsq(Tag{}, sh[v]));
+                Sp = __fadd_rn(Sp, butterfly(c));
+            }
+            Ssum = __fadd_rn(Ssum, Sp);
+        }
+        const float rr = factor(Ssum, z ? a.Df[1] : a.Df[0], a.eps);
+        // Phase B weight multiply and Phase C, element-wise over the row.
+        const int rowvec = (z ? a.D[1] : a.D[0]) / VEC;
+        const float *g = z ? gam_k : gam_q;
+        uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (int64_t)rowvec;
+#pragma unroll 4
+        for (int v = lane; v < rowvec; v += kLanes)
+            st_stream(dst + v, vapply_ptr(Tag{}, row[v], g + (int64_t)v * VEC, rr));
+        __syncwarp();
+        // Every lane is done with this stage: refill it with the warp's row S ahead.
+        if (lane == 0) {
+            const int64_t rn = gw + (n + S) * NW;
+            if (rn < R) {
+                fence_proxy_async_smem();
+                issue(s, rn);
+            }
+        }
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
 // A kernel that waits on an mbarrier nobody arrives on, with the same bounded
 // wait as fused_bulk: it must time out, record kErrWaitTimeout and return.
 __global__ void bounded_wait_probe(uint64_t timeout_ns) {
@@ -292,6 +438,41 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, cons
     const size_t smem = bulk_smem_bytes(stages, b.stage_stride);
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
     return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, smem, s);
+}
+
+const void *fused_rows_kernel(int dtype) {
+    if (dtype == 0) return reinterpret_cast<const void *>(&fused_rows<F32Tag>);
+    if (dtype == 1) return reinterpret_cast<const void *>(&fused_rows<BF16Tag>);
+    return nullptr;
+}
+
+// Shared-memory layout of fused_rows: [gamma barrier + W*S stage barriers,
+// padded to 128][gamma_q][gamma_k][W rings of S stages].
+RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int warps, int stages) {
+    RowsLayout L;
+    auto up = [](int64_t x) { return (x + 127) / 128 * 128; };
+    L.stage_bytes = (uint32_t)up((Dq > Dk ? Dq : Dk) * es);
+    L.gq_off = (uint32_t)up(8 * (1 + (int64_t)warps * stages));
+    L.gk_off = L.gq_off + (uint32_t)up(Dq * 4);
+    L.ring_off = L.gk_off + (uint32_t)up(Dk * 4);
+    L.smem_bytes = (size_t)L.ring_off + (size_t)warps * stages * L.stage_bytes;
+    return L;
+}
+
+cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stages, int64_t grid,
+                              uint64_t timeout_ns, cudaStream_t s) {
+    const void *fn = fused_rows_kernel(dtype);
+    if (!fn || warps < 1 || warps > 16 || stages < 1) return cudaErrorInvalidValue;
+    const RowsLayout L = rows_layout(a.D[0], a.D[1], dtype == 1 ? 2 : 4, warps, stages);
+    RowsArgs b;
+    b.stages = (uint32_t)stages;
+    b.stage_bytes = L.stage_bytes;
+    b.gq_off = L.gq_off;
+    b.gk_off = L.gk_off;
+    b.ring_off = L.ring_off;
+    b.timeout_ns = timeout_ns;
+    void *args[] = {const_cast<FusedArgs *>(&a), &b};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(32 * warps), args, L.smem_bytes, s);
 }
 
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s) {

@@ -59,6 +59,15 @@ int bulk_max_stages();
 cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, const FusedArgs &a,
                               int stages, int block, int64_t grid, uint64_t timeout_ns,
                               cudaStream_t s);
+// The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
+struct RowsLayout {
+    uint32_t stage_bytes, gq_off, gk_off, ring_off;
+    size_t smem_bytes;
+};
+const void *fused_rows_kernel(int dtype);
+RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int warps, int stages);
+cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stages, int64_t grid,
+                              uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
 cudaError_t read_device_errors(unsigned *out, bool clear);
 

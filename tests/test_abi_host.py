@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 102
+    assert qk.qknorm_version() == 103
 
 
 # ----------------------------------------------------------------- argument checks
@@ -132,15 +132,23 @@ def test_plan_for_each_workload(qk):
     for name, wl in W.WORKLOADS.items():
         for T in wl.Ts:
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
-            # Several tokens per CTA: the bulk-copy ring; otherwise registers only.
-            want = qk.VARIANT_BULK if T > 2 * 148 else qk.VARIANT_CTA
+            # One token per CTA: registers only. Several: the token ring when a
+            # lane holds >= 4 vectors per shard, else warp per row.
+            if T <= 2 * 148:
+                want = qk.VARIANT_CTA
+            else:
+                want = qk.VARIANT_BULK if want_vmax[name] >= 4 else qk.VARIANT_ROWS
             assert pl["variant"] == want, (name, T)
+            assert pl["groups_q"] == pl["groups_k"] == 1
+            if want == qk.VARIANT_ROWS:
+                assert pl["stages"] == 1 and pl["block"] % 32 == 0
+                assert pl["smem_bytes"] <= 227 * 1024
+                continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
             assert pl["grid"] == min(T, 148 * 4)
-            assert pl["groups_q"] == pl["groups_k"] == 1
             if want == qk.VARIANT_BULK:
-                assert pl["prefetch"] == 0 and 2 <= pl["stages"] <= 8
+                assert pl["prefetch"] == 0 and pl["stages"] == 2 and pl["tokens_per_stage"] == 1
                 stage = (wl.Dq + wl.Dk) * wl.elem_bytes
                 assert pl["smem_bytes"] >= pl["stages"] * stage
             else:
@@ -204,10 +212,29 @@ def test_bulk_stages_fill_shared_memory(qk):
     two 20 KiB stages of the 13B prefill shape after the 384-byte header."""
     qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     pl = qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_BF16, 148)
-    stage = pl["tokens_per_stage"] * 2 * 5120 * 2
-    assert pl["tokens_per_stage"] == 2
+    stage = 2 * 5120 * 2
+    assert (pl["variant"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 1)
     assert (pl["stages"], pl["smem_bytes"]) == (2, 1152 + 2 * stage)
-    # A 1024-thread CTA (P = 16) is alone on its SM: 7 stages of 2 x 16 KiB
-    # tokens fit in 227 KiB after the header.
-    pl = qk.qknorm_plan_fwd(8192, 4096, 4096, 16, qk.QKNORM_BF16, 148)
-    assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 7, 2)
+    # A 1024-thread CTA (P = 16) is alone on its SM: with the automatic cap
+    # of two stages, two stages of 16 KiB tokens.
+    try:
+        qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
+        pl = qk.qknorm_plan_fwd(8192, 4096, 4096, 16, qk.QKNORM_BF16, 148)
+        assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 2, 1)
+        assert pl["smem_bytes"] == 1152 + 2 * 16384
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+
+
+def test_rows_warps_fill_shared_memory(qk):
+    """Warp-per-row plan: one row stage per warp, gamma once per CTA, the most
+    warps per SM (at most 16) that shared memory allows, two CTAs preferred."""
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    # 65536 x 4096 bf16, P = 8: 8 KiB rows, 32 KiB of gamma: 2 CTAs x 8 warps.
+    pl = qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_BF16, 148)
+    assert (pl["variant"], pl["block"], pl["stages"]) == (qk.VARIANT_ROWS, 256, 1)
+    assert 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
+    # GQA 5120 / 1024: 10 KiB stages (the wider row), 24 KiB of gamma.
+    pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
+    assert (pl["variant"], pl["block"]) == (qk.VARIANT_ROWS, 256)
+    assert pl["grid"] == min(148 * 2, (2 * 4096 + 7) // 8)

@@ -14,7 +14,7 @@ from gpu_util import bits, check_outputs, check_stats, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ("cta", "bulk", "warp", "generic")
+VARIANTS = ("cta", "bulk", "rows", "warp", "generic")
 
 
 @pytest.fixture(scope="module")
@@ -38,7 +38,7 @@ def _inputs(wl, T):
 
 def _fwd(qk, wl, q, k, gq, gk, variant=None, grid=0):
     vid = {"cta": qk.VARIANT_CTA, "warp": qk.VARIANT_WARP, "generic": qk.VARIANT_GENERIC,
-           "bulk": qk.VARIANT_BULK, None: qk.VARIANT_AUTO}[variant]
+           "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS, None: qk.VARIANT_AUTO}[variant]
     qk.qknorm_force_variant(vid, grid)
     try:
         oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk),
@@ -81,8 +81,9 @@ def test_shapes_and_variants(qk, orc, shape):
         try:
             outs[v] = _fwd(qk, wl, q, k, gq, gk, variant=v)
         except qk.QKNormError as e:
-            # Only the register-resident kernels (cta, bulk) have shape limits.
-            assert v in ("cta", "bulk") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
+            # Only the register-resident kernels (cta, bulk) and the shared-memory
+            # staged ones (bulk, rows) have shape limits.
+            assert v in ("cta", "bulk", "rows") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
     base = outs["generic"]
     for v, (oq, ok) in outs.items():
         assert torch.equal(bits(oq), bits(base[0])), f"{v} Q differs from generic"
@@ -251,3 +252,21 @@ def test_bounded_wait_times_out_and_reports(qk):
     oq, _ = qk.qknorm_fwd(x, x.clone(), g, g, 2, 0.0)
     torch.cuda.synchronize()
     assert bool((oq == 1.0).all())
+
+
+@pytest.mark.parametrize("warps,stages", [(1, 1), (1, 3), (3, 2), (8, 1), (0, 0), (0, 3)])
+@pytest.mark.parametrize("grid", [0, 1, 5])
+def test_rows_variant_rings(qk, warps, stages, grid):
+    """Warp-per-row kernel: any warps per CTA, ring depth and grid (rows wrap
+    the rings many times; Q and K rows of unequal width share the rings) gives
+    the same bits as the generic kernel."""
+    wl = W.custom("rows", 2 * 148 + 41, 5120, 1024, 8, seed=36)
+    q, k, gq, gk = _inputs(wl, wl.Ts[0])
+    ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
+    try:
+        qk.qknorm_set_rows_tuning(warps, stages)
+        got = _fwd(qk, wl, q, k, gq, gk, variant="rows", grid=grid)
+    finally:
+        qk.qknorm_set_rows_tuning(0, 0)
+    assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
+    assert qk.qknorm_device_errors() == 0
