@@ -161,8 +161,9 @@ typedef struct {
     int32_t groups_q;    /* K for a Q shard */
     int32_t groups_k;    /* K for a K shard */
     int32_t stages;      /* ring stages per CTA (bulk) or per warp (rows), else 0 */
-    int32_t tokens_per_stage; /* tokens a bulk stage holds (1, 2 or 4), else 0 */
+    int32_t tokens_per_stage; /* tokens a bulk stage holds (1 or 2), else 0 */
     int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
+    int32_t full_lanes;  /* 1 if every lane holds exactly vmax vectors per task */
     int64_t smem_bytes;  /* dynamic shared memory per CTA */
 } qknorm_plan;
 
@@ -197,7 +198,7 @@ QKNORM_API int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, 
 /*
  * qknorm_set_tuning -- process-wide tuning of the bulk variant for tests and
  * benchmarks: ring stages per CTA (0 = automatic), tokens per stage (0 =
- * automatic, else 1, 2 or 4), gamma in registers (-1 = automatic, 0 = no,
+ * automatic, else 1 or 2), gamma in registers (-1 = automatic, 0 = no,
  * 1 = yes), the bound of every wait in milliseconds (0 = the default of
  * 2000 ms). A combination without a kernel instance makes qknorm_fwd return
  * QKNORM_ERR_UNSUPPORTED. Not thread-safe with concurrent calls.

@@ -62,7 +62,7 @@ class QKNormPlan(ctypes.Structure):
                 ("prefetch", ctypes.c_int32), ("groups_q", ctypes.c_int32),
                 ("groups_k", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("tokens_per_stage", ctypes.c_int32), ("gamma_regs", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int64)]
+                ("full_lanes", ctypes.c_int32), ("smem_bytes", ctypes.c_int64)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

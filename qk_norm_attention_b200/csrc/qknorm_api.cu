@@ -158,6 +158,15 @@ Shapes shapes_of(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype) {
     return s;
 }
 
+// True when every lane of every (shard, group) task of both tensors holds
+// exactly vmax vectors, so the kernels need no per-lane guards.
+bool full_lanes(const Shapes &sh) {
+    auto full = [&](const TensorShape &t) {
+        return t.nv % (kLanes * t.K) == 0 && t.nv / (kLanes * t.K) == sh.vmax;
+    };
+    return full(sh.q) && full(sh.k);
+}
+
 bool gamma_regs_for(int32_t dtype, int vmax) {
     if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
     return vmax * vec_of(dtype) <= 40;
@@ -223,11 +232,12 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     pl->groups_q = sh.q.K;
     pl->groups_k = sh.k.K;
     int cta_max = 0;
-    fused_cta_kernel(dtype, sh.vmax, false, &cta_max);
+    fused_cta_kernel(dtype, sh.vmax, false, false, &cta_max);
+    pl->full_lanes = full_lanes(sh) ? 1 : 0;
     const bool cta_ok = sh.ntask * kLanes <= cta_max;
     const int tb = tokens_per_stage_for(sh.vmax);
     int bulk_max = 0;
-    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, true, tb, &bulk_max) != nullptr;
+    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, true, tb, false, &bulk_max) != nullptr;
     const uint32_t stride = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
                                               (int64_t)Dk * elem_of(dtype), tb);
     const bool bulk_ok = bulk_inst && sh.ntask * kLanes <= bulk_max &&
@@ -314,9 +324,11 @@ void plan_grid(int64_t T, int num_sms, int blocks_per_sm, qknorm_plan *pl) {
 const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy) {
     switch (pl.variant) {
     case QKNORM_VARIANT_CTA:
-        return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0, nullptr);
+        return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0,
+                                pl.full_lanes != 0, nullptr);
     case QKNORM_VARIANT_BULK:
-        return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, nullptr);
+        return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
+                                 pl.full_lanes != 0, nullptr);
     case QKNORM_VARIANT_ROWS:
         return fused_rows_kernel(dtype);
     default:
@@ -411,7 +423,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 103; }
+int qknorm_version(void) { return 104; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -514,12 +526,14 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
     a.eps = eps;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
-        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, a, pl.block, pl.grid, s);
+        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes != 0, a, pl.block,
+                             pl.grid, s);
     } else if (pl.variant == QKNORM_VARIANT_ROWS) {
         e = launch_fused_rows(dtype, a, pl.block / kLanes, pl.stages, pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
-        e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage, a, pl.stages,
-                              pl.block, pl.grid, g_wait_limit_ns, s);
+        e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
+                              pl.full_lanes != 0, a, pl.stages, pl.block, pl.grid,
+                              g_wait_limit_ns, s);
     } else {
         e = launch_fused_generic(dtype, a, pl.block, pl.grid, (size_t)pl.smem_bytes, s);
     }
@@ -530,7 +544,7 @@ int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_re
                       int32_t wait_limit_ms) {
     if (stages < 0 || stages > bulk_max_stages() || gamma_regs < -1 || gamma_regs > 1 ||
         wait_limit_ms < 0 || !(tokens_per_stage == 0 || tokens_per_stage == 1 ||
-                               tokens_per_stage == 2 || tokens_per_stage == 4))
+                               tokens_per_stage == 2))
         return QKNORM_ERR_INVALID_ARG;
     g_tune_stages = stages;
     g_tune_tb = tokens_per_stage;

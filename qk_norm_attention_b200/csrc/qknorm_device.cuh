@@ -84,6 +84,16 @@ __device__ __forceinline__ float combine(const float *B, int P, int K) {
     return S;
 }
 
+// combine() with the common single-group shards (K = 1) as one short loop:
+// the same additions in the same order (0 + B[p] is exact), fewer branches.
+__device__ __forceinline__ float combine_fast(const float *B, int P, int K) {
+    if (K != 1) return combine(B, P, K);
+    float S = 0.f;
+#pragma unroll 4
+    for (int p = 0; p < P; ++p) S = __fadd_rn(S, B[p]);
+    return S;
+}
+
 // r = rsqrt(S / D + eps): the global RMS factor with the full width D.
 __device__ __forceinline__ float factor(float S, float Df, float eps) {
     return rsqrtf(__fadd_rn(__fdiv_rn(S, Df), eps));

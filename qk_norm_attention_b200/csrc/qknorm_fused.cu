@@ -48,7 +48,7 @@ __device__ __forceinline__ Task decode_task(const FusedArgs &a, int j) {
     return t;
 }
 
-template <class Tag, int VMAX, bool PREFETCH, int MAXT>
+template <class Tag, int VMAX, bool PREFETCH, bool FULL, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     __shared__ float red[2][32];
@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     const Task tk = decode_task(a, warp);
     const int stride = kLanes * tk.K;            // vector stride between a lane's slots
     const int first = tk.kg * kLanes + lane;     // slot 0, as a vector index in the shard
-    const int cnt = slot_count(first, tk.nv, stride);
+    // FULL: every lane of every task holds exactly VMAX vectors (no guards).
+    const int cnt = FULL ? VMAX : slot_count(first, tk.nv, stride);
     const int64_t rowvec = sel(a.D, tk.z) / VEC;      // vectors per row
     const int64_t col0 = (int64_t)tk.p * tk.nv + first;
     const uint4 *xs = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + col0;
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
         const uint4 *src = xs + t * rowvec;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
-            if (i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
+            if (FULL || i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
     }
     int buf = 0;
     for (; t < T; t += G) {
@@ -86,23 +87,23 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
             const uint4 *src = xs + tn * rowvec;
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
-                if (i < cnt) nxt[i] = ld_stream(src + (int64_t)i * stride);
+                if (FULL || i < cnt) nxt[i] = ld_stream(src + (int64_t)i * stride);
         }
         // Phase A: this lane's chain, then the butterfly -> group sum.
         float c = 0.f;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
-            if (i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, cur[i]));
+            if (FULL || i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, cur[i]));
         c = butterfly(c);
         if (lane == 0) red[buf][warp] = c;
         __syncthreads();
         // Phase B: shard sums in order, the factor.
-        const float r = factor(combine(&red[buf][red_base], a.P, tk.K), Df, eps);
+        const float r = factor(combine_fast(&red[buf][red_base], a.P, tk.K), Df, eps);
         // Phase B weight multiply and Phase C, straight from registers.
         uint4 *dst = ys + t * rowvec;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
-            if (i < cnt)
+            if (FULL || i < cnt)
                 st_stream(dst + (int64_t)i * stride,
                           vapply(Tag{}, cur[i], gs + (int64_t)i * stride * VEC, r));
         if (PREFETCH) {
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
             const uint4 *src = xs + tn * rowvec;
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
-                if (i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
+                if (FULL || i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
         }
         buf ^= 1;
     }
@@ -161,34 +162,39 @@ __global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
 
 // ---------------------------------------------------------------- instance tables
 
-template <class Tag, int VMAX, bool PF>
-constexpr int cta_max_threads() { return VMAX <= 2 ? 1024 : 512; }
+constexpr int cta_max_threads(int vmax) { return vmax <= 2 ? 1024 : 512; }
 
-template <class Tag, int VMAX, bool PF>
+template <class Tag, int VMAX, bool PF, bool FULL>
 const void *cta_fn() {
-    return reinterpret_cast<const void *>(&fused_cta<Tag, VMAX, PF, cta_max_threads<Tag, VMAX, PF>()>);
+    return reinterpret_cast<const void *>(&fused_cta<Tag, VMAX, PF, FULL, cta_max_threads(VMAX)>);
 }
 
-template <class Tag, bool PF>
+template <class Tag, bool PF, bool FULL>
 const void *cta_table(int vmax) {
     switch (vmax) {
-    case 1: return cta_fn<Tag, 1, PF>();
-    case 2: return cta_fn<Tag, 2, PF>();
-    case 3: return cta_fn<Tag, 3, PF>();
-    case 4: return cta_fn<Tag, 4, PF>();
-    case 5: return cta_fn<Tag, 5, PF>();
-    case 6: return cta_fn<Tag, 6, PF>();
-    case 7: return cta_fn<Tag, 7, PF>();
-    case 8: return cta_fn<Tag, 8, PF>();
+    case 1: return cta_fn<Tag, 1, PF, FULL>();
+    case 2: return cta_fn<Tag, 2, PF, FULL>();
+    case 3: return cta_fn<Tag, 3, PF, FULL>();
+    case 4: return cta_fn<Tag, 4, PF, FULL>();
+    case 5: return cta_fn<Tag, 5, PF, FULL>();
+    case 6: return cta_fn<Tag, 6, PF, FULL>();
+    case 7: return cta_fn<Tag, 7, PF, FULL>();
+    case 8: return cta_fn<Tag, 8, PF, FULL>();
     default: return nullptr;
     }
 }
 
-const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, int *max_threads) {
+template <class Tag>
+const void *cta_pick(int vmax, bool prefetch, bool full) {
+    if (prefetch) return full ? cta_table<Tag, true, true>(vmax) : cta_table<Tag, true, false>(vmax);
+    return full ? cta_table<Tag, false, true>(vmax) : cta_table<Tag, false, false>(vmax);
+}
+
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads) {
     if (vmax < 1 || vmax > kVcap) return nullptr;
-    if (max_threads) *max_threads = vmax <= 2 ? 1024 : 512;
-    if (dtype == 0) return prefetch ? cta_table<F32Tag, true>(vmax) : cta_table<F32Tag, false>(vmax);
-    if (dtype == 1) return prefetch ? cta_table<BF16Tag, true>(vmax) : cta_table<BF16Tag, false>(vmax);
+    if (max_threads) *max_threads = cta_max_threads(vmax);
+    if (dtype == 0) return cta_pick<F32Tag>(vmax, prefetch, full);
+    if (dtype == 1) return cta_pick<BF16Tag>(vmax, prefetch, full);
     return nullptr;
 }
 
@@ -198,9 +204,9 @@ const void *fused_generic_kernel(int dtype) {
     return nullptr;
 }
 
-cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, const FusedArgs &a, int block,
-                             int64_t grid, cudaStream_t s) {
-    const void *fn = fused_cta_kernel(dtype, vmax, prefetch, nullptr);
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
+                             int block, int64_t grid, cudaStream_t s) {
+    const void *fn = fused_cta_kernel(dtype, vmax, prefetch, full, nullptr);
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<FusedArgs *>(&a)};
     return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);

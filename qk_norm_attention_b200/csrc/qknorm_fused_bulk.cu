@@ -42,7 +42,7 @@ constexpr uint32_t kRedBytes = 2 * kMaxTB * 32 * sizeof(float);
 constexpr uint32_t kStageBase = kBarBytes + kRedBytes;
 constexpr uint32_t kMaxStages = 16;
 
-template <class Tag, int VMAX, bool GREG, int TB, int MAXT>
+template <class Tag, int VMAX, bool GREG, int TB, bool FULL, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const BulkArgs b) {
     constexpr int VEC = Tag::kVec;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     const int nv = z ? a.nv[1] : a.nv[0];
     const int stride = kLanes * K;
     const int first = kg * kLanes + lane;
-    const int cnt = slot_count(first, nv, stride);
+    // FULL: every lane of every task holds exactly VMAX vectors (no guards).
+    const int cnt = FULL ? VMAX : slot_count(first, nv, stride);
     const int64_t rowvec = (z ? a.D[1] : a.D[0]) / VEC;
     const int64_t col0 = (int64_t)p * nv + first;
     uint4 *ys = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + col0;
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     if (GREG) {
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
-            if (i < cnt) {
+            if (FULL || i < cnt) {
 #pragma unroll
                 for (int e = 0; e < VEC; e += 4) {
                     const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
             const uint4 *src = reinterpret_cast<const uint4 *>(st + j * tok_bytes);
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
-                if (i < cnt && t0 + j * G < T) cur[j][i] = src[i * stride];
+                if ((FULL || i < cnt) && (j == 0 || t0 + j * G < T)) cur[j][i] = src[i * stride];
         }
         // Phase A for TB tokens: independent chains and butterflies.
         float c[TB];
@@ -148,7 +149,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
             c[j] = 0.f;
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
-                if (i < cnt && t0 + j * G < T) c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
+                if ((FULL || i < cnt) && (j == 0 || t0 + j * G < T))
+                    c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
         }
 #pragma unroll
         for (int j = 0; j < TB; ++j) c[j] = butterfly(c[j]);
@@ -182,12 +184,12 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
 #pragma unroll
         for (int j = 0; j < TB; ++j) {
             const int64_t t = t0 + j * G;
-            if (t < T) {
-                const float r = factor(combine(&red[buf][j][red_base], a.P, K), Df, eps);
+            if (j == 0 || t < T) {
+                const float r = factor(combine_fast(&red[buf][j][red_base], a.P, K), Df, eps);
                 uint4 *dst = ys + t * rowvec;
 #pragma unroll
                 for (int i = 0; i < VMAX; ++i)
-                    if (i < cnt) {
+                    if (FULL || i < cnt) {
                         uint4 y;
                         if (GREG)
                             y = vapply_regs(Tag{}, cur[j][i], &gam[i * VEC], r);
@@ -315,17 +317,29 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
         const int stride = kLanes * K;
         // Phase A and the ordered sums of Phase B.
         float Ssum = 0.f;
-        for (int p = 0; p < P; ++p) {
-            const uint4 *sh = row + (int64_t)p * nv;
-            float Sp = 0.f;
-            for (int kg = 0; kg < K; ++kg) {
+        if (K == 1) {
+            // One group per shard: chain, butterfly, add (0 + x is exact, so
+            // this is the general order below with the inner loop removed).
+            for (int p = 0; p < P; ++p) {
+                const uint4 *sh = row + (int64_t)p * nv;
                 float c = 0.f;
 #pragma unroll 4
-                for (int v = kg * kLanes + lane; v < nv; v += stride)
-                    c = __fadd_rn(c, vsumsq(Tag{}, sh[v]));
-                Sp = __fadd_rn(Sp, butterfly(c));
+                for (int v = lane; v < nv; v += kLanes) c = __fadd_rn(c, vsumsq(Tag{}, sh[v]));
+                Ssum = __fadd_rn(Ssum, butterfly(c));
             }
-            Ssum = __fadd_rn(Ssum, Sp);
+        } else {
+            for (int p = 0; p < P; ++p) {
+                const uint4 *sh = row + (int64_t)p * nv;
+                float Sp = 0.f;
+                for (int kg = 0; kg < K; ++kg) {
+                    float c = 0.f;
+#pragma unroll 4
+                    for (int v = kg * kLanes + lane; v < nv; v += stride)
+                        c = __fadd_rn(c, vsumsq(Tag{}, sh[v]));
+                    Sp = __fadd_rn(Sp, butterfly(c));
+                }
+                Ssum = __fadd_rn(Ssum, Sp);
+            }
         }
         const float rr = factor(Ssum, z ? a.Df[1] : a.Df[0], a.eps);
         // Phase B weight multiply and Phase C, element-wise over the row.
@@ -366,50 +380,51 @@ __global__ void bounded_wait_probe(uint64_t timeout_ns) {
 
 // ---------------------------------------------------------------- instances and launch
 
-// Combinations that exist: TB tokens x VMAX vectors per lane <= 12 (registers).
+// Combinations that exist: TB (1 or 2) tokens x VMAX vectors per lane <= 12.
 constexpr bool bulk_exists(int vmax, int tb) {
-    return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2 || tb == 4) && vmax * tb <= 12;
+    return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12;
 }
 constexpr int bulk_max_threads(int vmax, int tb) { return vmax * tb <= 2 ? 1024 : 512; }
 
-template <class Tag, bool GREG, int V, int TB>
+template <class Tag, bool GREG, int V, int TB, bool FULL>
 const void *bulk_fn() {
     if constexpr (bulk_exists(V, TB))
-        return reinterpret_cast<const void *>(&fused_bulk<Tag, V, GREG, TB, bulk_max_threads(V, TB)>);
+        return reinterpret_cast<const void *>(
+            &fused_bulk<Tag, V, GREG, TB, FULL, bulk_max_threads(V, TB)>);
     else
         return nullptr;
 }
 
-template <class Tag, bool GREG, int TB>
+template <class Tag, bool GREG, int TB, bool FULL>
 const void *bulk_table_tb(int vmax) {
     switch (vmax) {
-    case 1: return bulk_fn<Tag, GREG, 1, TB>();
-    case 2: return bulk_fn<Tag, GREG, 2, TB>();
-    case 3: return bulk_fn<Tag, GREG, 3, TB>();
-    case 4: return bulk_fn<Tag, GREG, 4, TB>();
-    case 5: return bulk_fn<Tag, GREG, 5, TB>();
-    case 6: return bulk_fn<Tag, GREG, 6, TB>();
-    case 7: return bulk_fn<Tag, GREG, 7, TB>();
-    case 8: return bulk_fn<Tag, GREG, 8, TB>();
+    case 1: return bulk_fn<Tag, GREG, 1, TB, FULL>();
+    case 2: return bulk_fn<Tag, GREG, 2, TB, FULL>();
+    case 3: return bulk_fn<Tag, GREG, 3, TB, FULL>();
+    case 4: return bulk_fn<Tag, GREG, 4, TB, FULL>();
+    case 5: return bulk_fn<Tag, GREG, 5, TB, FULL>();
+    case 6: return bulk_fn<Tag, GREG, 6, TB, FULL>();
+    case 7: return bulk_fn<Tag, GREG, 7, TB, FULL>();
+    case 8: return bulk_fn<Tag, GREG, 8, TB, FULL>();
     default: return nullptr;
     }
 }
 
 template <class Tag, bool GREG>
-const void *bulk_table(int vmax, int tb) {
-    switch (tb) {
-    case 1: return bulk_table_tb<Tag, GREG, 1>(vmax);
-    case 2: return bulk_table_tb<Tag, GREG, 2>(vmax);
-    case 4: return bulk_table_tb<Tag, GREG, 4>(vmax);
-    default: return nullptr;
-    }
+const void *bulk_table(int vmax, int tb, bool full) {
+    if (tb == 1) return full ? bulk_table_tb<Tag, GREG, 1, true>(vmax) : bulk_table_tb<Tag, GREG, 1, false>(vmax);
+    if (tb == 2) return full ? bulk_table_tb<Tag, GREG, 2, true>(vmax) : bulk_table_tb<Tag, GREG, 2, false>(vmax);
+    return nullptr;
 }
 
-const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int *max_threads) {
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+                              int *max_threads) {
     if (!bulk_exists(vmax, tb)) return nullptr;
     if (max_threads) *max_threads = bulk_max_threads(vmax, tb);
-    if (dtype == 0) return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb) : bulk_table<F32Tag, false>(vmax, tb);
-    if (dtype == 1) return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb) : bulk_table<BF16Tag, false>(vmax, tb);
+    if (dtype == 0)
+        return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb, full) : bulk_table<F32Tag, false>(vmax, tb, full);
+    if (dtype == 1)
+        return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb, full) : bulk_table<BF16Tag, false>(vmax, tb, full);
     return nullptr;
 }
 
@@ -423,10 +438,10 @@ size_t bulk_smem_bytes(int stages, uint32_t stage_stride) {
 
 int bulk_max_stages() { return (int)kMaxStages; }
 
-cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, const FusedArgs &a,
-                              int stages, int block, int64_t grid, uint64_t timeout_ns,
-                              cudaStream_t s) {
-    const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, nullptr);
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+                              const FusedArgs &a, int stages, int block, int64_t grid,
+                              uint64_t timeout_ns, cudaStream_t s) {
+    const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, full, nullptr);
     if (!fn || stages < 1 || stages > (int)kMaxStages) return cudaErrorInvalidValue;
     const int64_t es = dtype == 1 ? 2 : 4;
     BulkArgs b;

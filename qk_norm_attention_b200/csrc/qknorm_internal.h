@@ -33,13 +33,14 @@ TensorShape make_shape(int32_t D, int32_t P, int vec);
 
 // Kernel handles for occupancy queries and launches. Each returns nullptr if
 // the combination does not exist.
-const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, int *max_threads);
+// full: every lane holds exactly vmax vectors in every task (guard-free instance).
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads);
 const void *fused_generic_kernel(int dtype);
 const void *stats_kernel(int dtype, int vmax);
 const void *apply_kernel(int dtype);
 
 // Launchers: enqueue one kernel; return the cudaError_t of the launch.
-cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, const FusedArgs &a,
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
                              int block, int64_t grid, cudaStream_t s);
 cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
                                  size_t smem, cudaStream_t s);
@@ -52,13 +53,14 @@ cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // tb = tokens per ring stage (1, 2 or 4); nullptr if (vmax, tb) has no instance.
-const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int *max_threads);
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+                              int *max_threads);
 uint32_t bulk_stage_stride(int64_t qbytes, int64_t kbytes, int tb);
 size_t bulk_smem_bytes(int stages, uint32_t stage_stride);
 int bulk_max_stages();
-cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, const FusedArgs &a,
-                              int stages, int block, int64_t grid, uint64_t timeout_ns,
-                              cudaStream_t s);
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+                              const FusedArgs &a, int stages, int block, int64_t grid,
+                              uint64_t timeout_ns, cudaStream_t s);
 // The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 struct RowsLayout {
     uint32_t stage_bytes, gq_off, gk_off, ring_off;

@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 103
+    assert qk.qknorm_version() == 104
 
 
 # ----------------------------------------------------------------- argument checks
@@ -155,6 +155,17 @@ def test_plan_for_each_workload(qk):
                 assert pl["prefetch"] == int(T > 148 * 4) and pl["stages"] == 0
 
 
+def test_full_lanes_flag(qk):
+    """Guard-free kernels only where every lane holds exactly vmax vectors."""
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    full = lambda *a: qk.qknorm_plan_fwd(*a, qk.QKNORM_BF16, 148)["full_lanes"]
+    assert full(8, 4096, 4096, 4) == 1          # 128 vectors per shard: 4 per lane
+    assert full(8, 5120, 5120, 4) == 1          # 160: 5 per lane
+    assert full(8, 5120, 1024, 8) == 0          # 80 and 16: ragged
+    assert full(8, 4096, 1024, 4) == 0          # 4 per lane for Q, 1 for K
+    assert full(8, 4096, 4096, 1) == 1          # 512 = 2 groups x 32 lanes x 8
+
+
 def test_plan_groups_and_fallbacks(qk):
     qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     pl = qk.qknorm_plan_fwd(10, 4096, 4096, 1, qk.QKNORM_BF16, 148)      # nv = 512
@@ -184,17 +195,18 @@ def test_forced_variants(qk):
         with pytest.raises(qk.QKNormError):
             qk.qknorm_force_variant(5, 0)
         qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
-        qk.qknorm_set_tuning(stages=3, tokens_per_stage=4, gamma_regs=0)
+        qk.qknorm_set_tuning(stages=3, tokens_per_stage=2, gamma_regs=0)
         pl = qk.qknorm_plan_fwd(10, 4096, 4096, 8, qk.QKNORM_BF16, 148)   # vmax 2
         assert (pl["variant"], pl["stages"], pl["gamma_regs"], pl["tokens_per_stage"]) == \
-            (qk.VARIANT_BULK, 3, 0, 4)
-        assert pl["smem_bytes"] >= 3 * 4 * 2 * 4096 * 2
-        qk.qknorm_set_tuning(tokens_per_stage=4)            # vmax 8 x 4 tokens: no instance
+            (qk.VARIANT_BULK, 3, 0, 2)
+        assert pl["smem_bytes"] >= 3 * 2 * 2 * 4096 * 2
+        assert pl["full_lanes"] == 1                        # 64 vectors = 2 per lane
+        qk.qknorm_set_tuning(tokens_per_stage=2)            # vmax 8 x 2 tokens: no instance
         with pytest.raises(qk.QKNormError) as ei:
             qk.qknorm_plan_fwd(10, 4096, 4096, 2, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         with pytest.raises(qk.QKNormError):
-            qk.qknorm_set_tuning(tokens_per_stage=3)
+            qk.qknorm_set_tuning(tokens_per_stage=4)
         with pytest.raises(qk.QKNormError) as ei:      # 64 tasks do not fit one CTA
             qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
