@@ -167,16 +167,19 @@ bool full_lanes(const Shapes &sh) {
     return full(sh.q) && full(sh.k);
 }
 
+// Gamma in registers pays off while a lane holds few vectors (measured on
+// B200: +5 % at 2 vectors per lane, -7 % at 5, where the registers cost
+// occupancy and gamma hits L1 anyway).
 bool gamma_regs_for(int32_t dtype, int vmax) {
     if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
-    return vmax * vec_of(dtype) <= 40;
+    return vmax * vec_of(dtype) <= 24;
 }
 
-// Tokens per bulk stage: 1 (batching tokens measured no gain on B200 once
-// the stage ring keeps enough bytes in flight).
+// Tokens per bulk stage: two while a lane holds <= 3 vectors per shard (the
+// per-token chain is short, so two tokens overlap it), one otherwise.
 int tokens_per_stage_for(int vmax) {
-    (void)vmax;
-    return g_tune_tb > 0 ? g_tune_tb : 1;
+    if (g_tune_tb > 0) return g_tune_tb;
+    return vmax <= 3 ? 2 : 1;
 }
 
 // Stage count of the bulk kernel: the most stages (up to kMaxStagesAuto) that
@@ -246,11 +249,11 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     if (variant == QKNORM_VARIANT_AUTO) {
         // Measured on B200: a CTA per token with registers wins while a CTA
         // sees one token (decode); with several tokens per CTA the token ring
-        // wins when a lane holds >= 4 vectors per shard (per-token overhead
-        // amortised), the warp-per-row kernel otherwise.
+        // is best or level on every measured shape; the warp-per-row kernel
+        // covers shapes whose tasks do not fit one CTA.
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
-        else if (bulk_ok && sh.vmax >= 4)
+        else if (bulk_ok)
             variant = QKNORM_VARIANT_BULK;
         else if (rows_ok)
             variant = QKNORM_VARIANT_ROWS;

@@ -132,24 +132,20 @@ def test_plan_for_each_workload(qk):
     for name, wl in W.WORKLOADS.items():
         for T in wl.Ts:
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
-            # One token per CTA: registers only. Several: the token ring when a
-            # lane holds >= 4 vectors per shard, else warp per row.
-            if T <= 2 * 148:
-                want = qk.VARIANT_CTA
-            else:
-                want = qk.VARIANT_BULK if want_vmax[name] >= 4 else qk.VARIANT_ROWS
+            # One token per CTA: registers only. Several: the token ring, two
+            # tokens per stage and gamma in registers while vmax <= 3.
+            want = qk.VARIANT_CTA if T <= 2 * 148 else qk.VARIANT_BULK
             assert pl["variant"] == want, (name, T)
             assert pl["groups_q"] == pl["groups_k"] == 1
-            if want == qk.VARIANT_ROWS:
-                assert pl["stages"] == 1 and pl["block"] % 32 == 0
-                assert pl["smem_bytes"] <= 227 * 1024
-                continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
             assert pl["grid"] == min(T, 148 * 4)
             if want == qk.VARIANT_BULK:
-                assert pl["prefetch"] == 0 and pl["stages"] == 2 and pl["tokens_per_stage"] == 1
-                stage = (wl.Dq + wl.Dk) * wl.elem_bytes
+                small = want_vmax[name] <= 3
+                assert pl["prefetch"] == 0 and pl["stages"] == 2
+                assert pl["tokens_per_stage"] == (2 if small else 1)
+                assert pl["gamma_regs"] == (1 if small else 0)
+                stage = (wl.Dq + wl.Dk) * wl.elem_bytes * pl["tokens_per_stage"]
                 assert pl["smem_bytes"] >= pl["stages"] * stage
             else:
                 assert pl["prefetch"] == int(T > 148 * 4) and pl["stages"] == 0
@@ -241,12 +237,15 @@ def test_bulk_stages_fill_shared_memory(qk):
 def test_rows_warps_fill_shared_memory(qk):
     """Warp-per-row plan: one row stage per warp, gamma once per CTA, the most
     warps per SM (at most 16) that shared memory allows, two CTAs preferred."""
-    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
-    # 65536 x 4096 bf16, P = 8: 8 KiB rows, 32 KiB of gamma: 2 CTAs x 8 warps.
-    pl = qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_BF16, 148)
-    assert (pl["variant"], pl["block"], pl["stages"]) == (qk.VARIANT_ROWS, 256, 1)
-    assert 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
-    # GQA 5120 / 1024: 10 KiB stages (the wider row), 24 KiB of gamma.
-    pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
-    assert (pl["variant"], pl["block"]) == (qk.VARIANT_ROWS, 256)
-    assert pl["grid"] == min(148 * 2, (2 * 4096 + 7) // 8)
+    try:
+        qk.qknorm_force_variant(qk.VARIANT_ROWS, 0)
+        # 65536 x 4096 bf16, P = 8: 8 KiB rows, 32 KiB of gamma: 2 CTAs x 8 warps.
+        pl = qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_BF16, 148)
+        assert (pl["variant"], pl["block"], pl["stages"]) == (qk.VARIANT_ROWS, 256, 1)
+        assert 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
+        # GQA 5120 / 1024: 10 KiB stages (the wider row), 24 KiB of gamma.
+        pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
+        assert (pl["variant"], pl["block"]) == (qk.VARIANT_ROWS, 256)
+        assert pl["grid"] == min(148 * 2, (2 * 4096 + 7) // 8)
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
