@@ -223,13 +223,13 @@ def test_bulk_stages_fill_shared_memory(qk):
     stage = 2 * 5120 * 2
     assert (pl["variant"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 1)
     assert (pl["stages"], pl["smem_bytes"]) == (2, 1152 + 2 * stage)
-    # A 1024-thread CTA (P = 16) is alone on its SM: with the automatic cap
-    # of two stages, two stages of 16 KiB tokens.
+    # A 1024-thread CTA (P = 16, one vector per lane) is alone on its SM:
+    # two stages of two 16 KiB tokens (the automatic caps).
     try:
         qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
         pl = qk.qknorm_plan_fwd(8192, 4096, 4096, 16, qk.QKNORM_BF16, 148)
-        assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 2, 1)
-        assert pl["smem_bytes"] == 1152 + 2 * 16384
+        assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 2, 2)
+        assert pl["smem_bytes"] == 1152 + 2 * 2 * 16384
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
 
