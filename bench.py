@@ -41,7 +41,10 @@ KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_ge
 
 # dram bytes per launch of the headline kernel from one ncu capture, and the
 # hash of the kernel sources it was taken with (None until captured).
-NCU_TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
+# From profiles/fused_bulk_prefill13b_full.md: dram__bytes_read.sum 167,837,952
+# + dram__bytes_write.sum 111,811,840 for one launch (cold, serialised capture;
+# ~56 MB of the writes were still in L2 when the kernel ended).
+NCU_TRAFFIC = {"src_sha": "13562c5ad35e2c38", "bytes_per_launch": 279649792}
 
 
 def parse_args(argv=None):
