@@ -56,7 +56,15 @@ def parse_args(argv=None):
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the decode / GQA / split measurements after the timed region")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS),
+                    help="workload of the timed region (default: the 13B-shaped prefill); "
+                         "the largest T of the workload is used")
+    ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows"),
+                    help="force a kernel variant (for profiling; default: the selector's choice)")
     return ap.parse_args(argv)
+
+
+VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4}
 
 
 def kernel_src_sha() -> str:
@@ -420,11 +428,22 @@ def cpu_baseline(wl, T, target_s=10.0):
             "tokens_per_s": round(passes * n / el, 1)}
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def buffer_sets(set_bytes: int) -> int:
+    """Rotating buffer sets so that the sets together exceed L2 at least twice."""
+    return max(2, -(-2 * L2_BYTES // max(1, set_bytes)))
+
+
 def config_of(wl, T, world):
+    nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes)
+    n = buffer_sets(nbytes)
     return {"workload": wl.note, "T_per_gpu": T, "global_tokens": T * world, "Dq": wl.Dq,
             "Dk": wl.Dk, "P": wl.P, "eps": wl.eps, "storage": wl.dtype,
             "accumulation": "fp32", "parallelism": f"token-sharded dp{world} (no collective)",
-            "l2": "inputs larger than L2: two rotating buffer sets of 336 MB each"}
+            "l2": f"inputs larger than L2: {n} rotating buffer sets of {nbytes / 1e6:.0f} MB "
+                  f"(inputs + outputs) each, {n * nbytes / 1e6:.0f} MB in all vs 132 MB of L2"}
 
 
 def run_reference(args, dist):
@@ -476,20 +495,22 @@ def run_native(args, dist):
     device = torch.device("cuda", dist.local_rank)
     torch.cuda.set_device(device)
     dist.init("nccl")
-    wl = W.WORKLOADS[HEADLINE]
-    T = wl.Ts[0]                       # tokens per GPU (weak scaling)
+    wl = W.WORKLOADS[args.workload]
+    T = max(wl.Ts)                     # tokens per GPU (weak scaling)
     row0, _ = shard_tokens(T * dist.world, dist.world, dist.rank)
     stream = torch.cuda.current_stream(device)
     peak, peak_src = hbm_peak()
-    dt = qk.QKNORM_BF16
+    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    qk.qknorm_force_variant(VARIANT_IDS[args.variant], 0)
 
     q, k, gq, gk = device_inputs(torch, wl, T, device, row0)
-    sets = [(q, k), (q.clone(), k.clone())]
+    nsets = buffer_sets(W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes))
+    sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(nsets - 1)]
     calls = [Fused(qk, (a, b, gq, gk, torch.empty_like(a), torch.empty_like(b)), T, wl.Dq, wl.Dk,
                    wl.P, wl.eps, dt, stream.cuda_stream) for a, b in sets]
     plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, dt)
     for i in range(max(3, args.warmup)):
-        calls[i % 2]()
+        calls[i % len(calls)]()
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
@@ -539,6 +560,7 @@ def run_native(args, dist):
     del qh, kh, oqh, okh
 
     extras = {}
+    qk.qknorm_force_variant(-1, 0)
     if dist.rank == 0 and not args.no_extras:
         dec = W.WORKLOADS["decode"]
         extras["decode_us_per_call"] = {str(t): latency_us(torch, qk, dec, t, device) for t in dec.Ts}

@@ -175,11 +175,11 @@ bool gamma_regs_for(int32_t dtype, int vmax) {
     return vmax * vec_of(dtype) <= 24;
 }
 
-// Tokens per bulk stage: two while a lane holds <= 3 vectors per shard (the
-// per-token chain is short, so two tokens overlap it), one otherwise.
+// Tokens per bulk stage: one (two tokens per stage measured within noise of
+// one and less steady across boxes).
 int tokens_per_stage_for(int vmax) {
-    if (g_tune_tb > 0) return g_tune_tb;
-    return vmax <= 3 ? 2 : 1;
+    (void)vmax;
+    return g_tune_tb > 0 ? g_tune_tb : 1;
 }
 
 // Stage count of the bulk kernel: the most stages (up to kMaxStagesAuto) that
@@ -248,12 +248,15 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     const bool rows_ok = rows_fit(Dq, Dk, dtype);
     if (variant == QKNORM_VARIANT_AUTO) {
         // Measured on B200: a CTA per token with registers wins while a CTA
-        // sees one token (decode); with several tokens per CTA the token ring
-        // is best or level on every measured shape; the warp-per-row kernel
-        // covers shapes whose tasks do not fit one CTA.
+        // sees one token (decode). With several tokens per CTA the token ring
+        // wins when every lane holds the same number of vectors; with ragged
+        // lanes (e.g. GQA widths) its CTA carries idle lanes and unequal Q/K
+        // warps, and the warp-per-row kernel wins. Shapes whose tasks do not
+        // fit one CTA go to the rows kernel too.
+        const bool ragged = !pl->full_lanes;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
-        else if (bulk_ok)
+        else if (bulk_ok && !(ragged && rows_ok))
             variant = QKNORM_VARIANT_BULK;
         else if (rows_ok)
             variant = QKNORM_VARIANT_ROWS;

@@ -318,14 +318,25 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
         // Phase A and the ordered sums of Phase B.
         float Ssum = 0.f;
         if (K == 1) {
-            // One group per shard: chain, butterfly, add (0 + x is exact, so
-            // this is the general order below with the inner loop removed).
-            for (int p = 0; p < P; ++p) {
-                const uint4 *sh = row + (int64_t)p * nv;
-                float c = 0.f;
-#pragma unroll 4
-                for (int v = lane; v < nv; v += kLanes) c = __fadd_rn(c, vsumsq(Tag{}, sh[v]));
-                Ssum = __fadd_rn(Ssum, butterfly(c));
+            // One group per shard. Four shards at a time: their lane chains
+            // advance together (slot-major), then four independent
+            // butterflies, then the ordered adds. Each shard's own order is
+            // unchanged (0 + x is exact), so the bits equal the general order.
+            const int cnt = slot_count(lane, nv, kLanes);
+            for (int p0 = 0; p0 < P; p0 += 4) {
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint4 *sh = row + (int64_t)p0 * nv + lane;
+                for (int i = 0; i < cnt; ++i) {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b)
+                        if (p0 + b < P)
+                            c[b] = __fadd_rn(c[b], vsumsq(Tag{}, sh[(int64_t)b * nv + i * kLanes]));
+                }
+#pragma unroll
+                for (int b = 0; b < 4; ++b) c[b] = butterfly(c[b]);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (p0 + b < P) Ssum = __fadd_rn(Ssum, c[b]);
             }
         } else {
             for (int p = 0; p < P; ++p) {

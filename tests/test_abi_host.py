@@ -132,18 +132,25 @@ def test_plan_for_each_workload(qk):
     for name, wl in W.WORKLOADS.items():
         for T in wl.Ts:
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
-            # One token per CTA: registers only. Several: the token ring, two
-            # tokens per stage and gamma in registers while vmax <= 3.
-            want = qk.VARIANT_CTA if T <= 2 * 148 else qk.VARIANT_BULK
+            # One token per CTA: registers only. Several: the token ring (one
+            # token per stage, gamma in registers while vmax <= 3), or warp
+            # per row when lanes are ragged (GQA widths).
+            if T <= 2 * 148:
+                want = qk.VARIANT_CTA
+            else:
+                want = qk.VARIANT_ROWS if name == "gqa" else qk.VARIANT_BULK
             assert pl["variant"] == want, (name, T)
             assert pl["groups_q"] == pl["groups_k"] == 1
+            if want == qk.VARIANT_ROWS:
+                assert pl["stages"] == 1 and pl["full_lanes"] == 0
+                continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
             assert pl["grid"] == min(T, 148 * 4)
             if want == qk.VARIANT_BULK:
                 small = want_vmax[name] <= 3
                 assert pl["prefetch"] == 0 and pl["stages"] == 2
-                assert pl["tokens_per_stage"] == (2 if small else 1)
+                assert pl["tokens_per_stage"] == 1
                 assert pl["gamma_regs"] == (1 if small else 0)
                 stage = (wl.Dq + wl.Dk) * wl.elem_bytes * pl["tokens_per_stage"]
                 assert pl["smem_bytes"] >= pl["stages"] * stage
@@ -224,12 +231,12 @@ def test_bulk_stages_fill_shared_memory(qk):
     assert (pl["variant"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 1)
     assert (pl["stages"], pl["smem_bytes"]) == (2, 1152 + 2 * stage)
     # A 1024-thread CTA (P = 16, one vector per lane) is alone on its SM:
-    # two stages of two 16 KiB tokens (the automatic caps).
+    # two stages of one 16 KiB token (the automatic caps).
     try:
         qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
         pl = qk.qknorm_plan_fwd(8192, 4096, 4096, 16, qk.QKNORM_BF16, 148)
-        assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 2, 2)
-        assert pl["smem_bytes"] == 1152 + 2 * 2 * 16384
+        assert (pl["variant"], pl["stages"], pl["tokens_per_stage"]) == (qk.VARIANT_BULK, 2, 1)
+        assert pl["smem_bytes"] == 1152 + 2 * 16384
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
 
