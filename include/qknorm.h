@@ -214,6 +214,16 @@ QKNORM_API int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32
 QKNORM_API int qknorm_set_rows_tuning(int32_t warps, int32_t stages);
 
 /*
+ * qknorm_set_pdl -- programmatic dependent launch on (1, the default) or off
+ * (0), process-wide. When on, every kernel is launched with the programmatic
+ * stream serialization attribute: it may start while the previous kernel in
+ * the stream finishes, does only shared-memory set-up until that kernel has
+ * completed and its memory is visible (griddepcontrol.wait), and lets the
+ * next such kernel start early. Results are the same either way.
+ */
+QKNORM_API int qknorm_set_pdl(int32_t enable);
+
+/*
  * qknorm_device_errors -- read (and with clear != 0, reset) the library's
  * device error word. Bit 1: a bounded wait of the bulk variant ran out of
  * time (that launch's outputs are incomplete); bit 2: copies were still in

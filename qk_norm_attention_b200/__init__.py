@@ -93,6 +93,8 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_version.restype = ctypes.c_int
     lib.qknorm_set_tuning.argtypes = [i32, i32, i32, i32]
     lib.qknorm_set_tuning.restype = ctypes.c_int
+    lib.qknorm_set_pdl.argtypes = [i32]
+    lib.qknorm_set_pdl.restype = ctypes.c_int
     lib.qknorm_set_rows_tuning.argtypes = [i32, i32]
     lib.qknorm_set_rows_tuning.restype = ctypes.c_int
     lib.qknorm_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -232,6 +234,11 @@ def qknorm_set_tuning(stages: int = 0, tokens_per_stage: int = 0, gamma_regs: in
     """Tune the bulk variant process-wide (the defaults restore automatic choice)."""
     _check("qknorm_set_tuning", lib.qknorm_set_tuning(int(stages), int(tokens_per_stage),
                                                       int(gamma_regs), int(wait_limit_ms)))
+
+
+def qknorm_set_pdl(enable: bool = True) -> None:
+    """Programmatic dependent launch on (default) or off, process-wide."""
+    _check("qknorm_set_pdl", lib.qknorm_set_pdl(int(bool(enable))))
 
 
 def qknorm_set_rows_tuning(warps: int = 0, stages: int = 0) -> None:

@@ -18,6 +18,9 @@
 
 namespace qkn {
 
+bool g_pdl = true;  // programmatic dependent launch (qknorm_set_pdl)
+bool pdl_enabled() { return g_pdl; }
+
 TensorShape make_shape(int32_t D, int32_t P, int vec) {
     TensorShape s;
     s.D = D;
@@ -429,7 +432,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 104; }
+int qknorm_version(void) { return 105; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -564,6 +567,12 @@ int qknorm_set_rows_tuning(int32_t warps, int32_t stages) {
         return QKNORM_ERR_INVALID_ARG;
     g_rows_warps = warps;
     g_rows_stages = stages;
+    return QKNORM_OK;
+}
+
+int qknorm_set_pdl(int32_t enable) {
+    if (enable != 0 && enable != 1) return QKNORM_ERR_INVALID_ARG;
+    g_pdl = enable != 0;
     return QKNORM_OK;
 }
 

@@ -167,6 +167,18 @@ __device__ __forceinline__ uint4 vapply_ptr(BF16Tag, const uint4 &v, const float
     return vapply_regs(BF16Tag{}, v, gg, r);
 }
 
+// ---------------------------------------------------------------- launch order
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialization attribute may start while the previous kernel in the
+// stream is still running. pdl_wait() blocks until that kernel has completed
+// and its memory is visible; every kernel here calls it before its first
+// global-memory access (and it returns at once when there is nothing to wait
+// for). pdl_trigger() lets the next such kernel in the stream launch now; its
+// own pdl_wait() still orders its memory accesses after this kernel's.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::); }
+
 // ---------------------------------------------------------------- memory
 
 // Streaming (read-once / write-once) 16-byte accesses: evict-first in L1/L2.

@@ -52,6 +52,8 @@ template <class Tag, int VMAX, bool PREFETCH, bool FULL, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     __shared__ float red[2][32];
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const Task tk = decode_task(a, warp);
@@ -123,6 +125,8 @@ template <class Tag>
 __global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     extern __shared__ float red[];  // one float per task
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nw = blockDim.x >> 5;
@@ -209,7 +213,7 @@ cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, cons
     const void *fn = fused_cta_kernel(dtype, vmax, prefetch, full, nullptr);
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<FusedArgs *>(&a)};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+    return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 
 cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
@@ -217,7 +221,7 @@ cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64
     const void *fn = fused_generic_kernel(dtype);
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<FusedArgs *>(&a)};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, smem, s);
+    return launch(fn, dim3((unsigned)grid), dim3(block), smem, s, args);
 }
 
 }  // namespace qkn

@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
         fence_mbar_init();
     }
     __syncthreads();
+    // Shared memory only so far; global reads start after the previous grid.
+    pdl_wait();
+    pdl_trigger();
     if (tid == 0) {
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
@@ -263,6 +266,9 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
         fence_mbar_init();
     }
     __syncthreads();
+    // Shared memory only so far; global reads start after the previous grid.
+    pdl_wait();
+    pdl_trigger();
     if (threadIdx.x == 0) {
         const uint32_t gqb = (uint32_t)a.D[0] * 4u, gkb = (uint32_t)a.D[1] * 4u;
         mbar_arrive_expect_tx(gbar, gqb + gkb);
@@ -463,7 +469,7 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool
     b.timeout_ns = timeout_ns;
     const size_t smem = bulk_smem_bytes(stages, b.stage_stride);
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, smem, s);
+    return launch(fn, dim3((unsigned)grid), dim3(block), smem, s, args);
 }
 
 const void *fused_rows_kernel(int dtype) {
@@ -498,7 +504,7 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stag
     b.ring_off = L.ring_off;
     b.timeout_ns = timeout_ns;
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(32 * warps), args, L.smem_bytes, s);
+    return launch(fn, dim3((unsigned)grid), dim3(32 * warps), L.smem_bytes, s, args);
 }
 
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s) {

@@ -73,6 +73,23 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stag
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
 cudaError_t read_device_errors(unsigned *out, bool clear);
 
+// Launch with programmatic dependent launch when enabled (qknorm_set_pdl).
+bool pdl_enabled();
+inline cudaError_t launch(const void *fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          void **args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 // Largest dynamic shared memory the generic kernel is given (bytes).
 constexpr int kGenericMaxSmem = 200 * 1024;
 

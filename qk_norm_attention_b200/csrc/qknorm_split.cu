@@ -23,6 +23,8 @@ template <class Tag, int VMAX>
 __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int64_t T, int32_t D,
                                                int32_t P, int32_t nv, int32_t K) {
     constexpr int VEC = Tag::kVec;
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t rowvec = D / VEC;
     const int64_t ntask = T * (int64_t)P;
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, co
                                                float eps) {
     constexpr int VEC = Tag::kVec;
     constexpr int UNR = 4;
+    pdl_wait();
+    pdl_trigger();
     const int64_t rowvec = D / VEC;
     const float Df = (float)D;
     const int nthr = blockDim.x;
@@ -124,7 +128,7 @@ cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64
     if (!fn) return cudaErrorInvalidValue;
     int32_t D = sh.D, nv = sh.nv, K = sh.K;
     void *args[] = {const_cast<void **>(&x), &stats, &T, &D, &P, &nv, &K};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+    return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 
 cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
@@ -134,7 +138,7 @@ cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<void **>(&x), const_cast<float **>(&g),
                     const_cast<float **>(&stats), &y, &T, &D, &P, &eps};
-    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(block), args, 0, s);
+    return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 
 }  // namespace qkn

@@ -270,3 +270,38 @@ def test_rows_variant_rings(qk, warps, stages, grid):
         qk.qknorm_set_rows_tuning(0, 0)
     assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
     assert qk.qknorm_device_errors() == 0
+
+
+@pytest.mark.parametrize("variant", ["cta", "bulk", "rows", "generic"])
+def test_dependent_launches_with_pdl(qk, variant):
+    """Each call reads the previous call's output. With programmatic dependent
+    launch every kernel waits for the previous grid before reading memory, so
+    a chain launched back to back equals the same chain with a device
+    synchronisation after every call, and the chain with PDL off."""
+    wl = W.custom("chain", 3 * 148 + 5, 4096, 1024, 4, seed=37)
+    q, k, gq, gk = _inputs(wl, wl.Ts[0])
+    vid = {"cta": qk.VARIANT_CTA, "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS,
+           "generic": qk.VARIANT_GENERIC}[variant]
+    gqd, gkd = to_device(gq), to_device(gk)
+
+    def chain(pdl, sync):
+        qk.qknorm_set_pdl(pdl)
+        qk.qknorm_force_variant(vid, 0)
+        try:
+            a, b = to_device(q), to_device(k)
+            for _ in range(6):
+                a, b = qk.qknorm_fwd(a, b, gqd, gkd, wl.P, wl.eps)
+                st = qk.qknorm_partial_sumsq(a, wl.P)       # split kernels in the chain too
+                a = qk.qknorm_apply(a, gqd, st, wl.eps)
+                if sync:
+                    torch.cuda.synchronize()
+            torch.cuda.synchronize()
+            return a, b
+        finally:
+            qk.qknorm_set_pdl(True)
+            qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+
+    ref = chain(False, True)
+    for pdl in (True, False):
+        got = chain(pdl, False)
+        assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
