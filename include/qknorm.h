@@ -125,6 +125,36 @@ QKNORM_API int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int3
 QKNORM_API int qknorm_apply(const void *x, const float *gamma, const float *stats, void *out,
                  int64_t T, int32_t D, int32_t P, float eps, int32_t dtype, void *stream);
 
+/*
+ * qknorm_xgamma -- the weight multiply alone: out[t,j] = x[t,j] * gamma[j],
+ * rounded once to dtype, no normalisation.
+ *
+ * Algorithm 1's Phase B compute path on its own. It is also what a deferred
+ * normalisation stores when a later RMSNorm cancels the per-token factor
+ * (pull request "perf(dsv4 decode swa): deferred attention RMSNorm and dep
+ * cleanup", attn_norm_xgamma): since RMSNorm(s * z) = RMSNorm(z) for a
+ * per-token s > 0, the factor of an earlier norm need not be applied.
+ *   x [T, D] input, dtype; gamma [D] fp32; out [T, D] output, dtype.
+ * D must be a multiple of the 16-byte vector (8 bf16 / 4 fp32 elements).
+ * out may be x (exact in-place). Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_xgamma(const void *x, const float *gamma, void *out, int64_t T, int32_t D,
+                             int32_t dtype, void *stream);
+
+/*
+ * qknorm_inv_rms -- the per-token factor alone: inv_rms[t] = rsqrt(S[t]/D + eps),
+ * S[t] formed from P shard sums in the reduction order above, fp32.
+ *
+ * The one dynamic scalar per token that RMSNorm factors into besides the
+ * static weight (abstract "QK-Normed MLA: QK normalization without full key
+ * caching"); bit-identical to the factor qknorm_fwd applies to that row, so
+ * out = xgamma(x) * inv_rms reproduces Eq. (1) up to the rounding of xgamma.
+ *   x [T, D] input, dtype; inv_rms [T] fp32 output.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_inv_rms(const void *x, float *inv_rms, int64_t T, int32_t D, int32_t P,
+                              float eps, int32_t dtype, void *stream);
+
 /* Static text for a qknorm_status value ("unknown status" otherwise). */
 QKNORM_API const char *qknorm_status_string(int status);
 

@@ -49,6 +49,8 @@ class Oracle:
         lib.qko_rmsnorm.argtypes = [vp, ctypes.c_int, vp, i64, i64, i64, ctypes.c_double,
                                     dp, dp, ctypes.c_int]
         lib.qko_rmsnorm.restype = ctypes.c_int
+        lib.qko_xgamma.argtypes = [vp, ctypes.c_int, vp, i64, i64, dp, ctypes.c_int]
+        lib.qko_xgamma.restype = ctypes.c_int
         lib.qko_has_openmp.restype = ctypes.c_int
         self._lib = lib
 
@@ -94,6 +96,25 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle rejected the arguments")
         return y, r
+
+    def xgamma(self, x: np.ndarray, gamma: np.ndarray, dtype: str, nthreads: int = 1) -> np.ndarray:
+        """u[t, j] = x[t, j] * gamma[j] in float64 (the weight multiply alone)."""
+        x = self._prep(x, dtype)
+        T, D = x.shape
+        g = np.ascontiguousarray(gamma, dtype=np.float32)
+        if g.shape != (D,):
+            raise ValueError("gamma must have shape [D]")
+        u = np.empty((T, D), dtype=np.float64)
+        if self._lib.qko_xgamma(x.ctypes.data, _DTYPE_CODE[dtype], g.ctypes.data, T, D,
+                                u.ctypes.data, nthreads) != 0:
+            raise ValueError("oracle rejected the arguments")
+        return u
+
+    def inv_rms(self, x: np.ndarray, P: int, eps: float, dtype: str, nthreads: int = 1) -> np.ndarray:
+        """r[t] = 1/sqrt(S[t]/D + eps) alone (the per-token dynamic statistic)."""
+        D = x.shape[1]
+        _, r = self.rmsnorm(x, np.ones(D, dtype=np.float32), P, eps, dtype, nthreads, want_y=False)
+        return r
 
     def qknorm(self, q, k, gamma_q, gamma_k, P, eps, dtype, nthreads: int = 1):
         """Layerwise QK-Norm: the RMSNorm above applied to Q and, on its own, to K."""

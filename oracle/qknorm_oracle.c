@@ -140,6 +140,30 @@ int qko_rmsnorm(const void *x, int dtype, const float *gamma, int64_t T, int64_t
     return 0;
 }
 
+/*
+ * u[t*D + j] = x[t,j] * gamma[j] in double: the weight multiply on its own,
+ * with no normalisation. This is what a deferred normalisation stores when a
+ * later RMSNorm cancels the per-token factor ("perf(dsv4 decode swa):
+ * deferred attention RMSNorm" pull request, attn_norm_xgamma), and it is
+ * Algorithm 1's Phase B compute path by itself.
+ */
+int qko_xgamma(const void *x, int dtype, const float *gamma, int64_t T, int64_t D, double *u,
+               int nthreads)
+{
+    if (qko_check(x, dtype, T, D, 1) != 0 || gamma == NULL || (T > 0 && u == NULL))
+        return -1;
+    if (nthreads <= 0)
+        nthreads = 1;
+    const size_t es = qko_elem_size(dtype);
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const char *row = (const char *)x + (size_t)t * (size_t)D * es;
+        for (int64_t j = 0; j < D; ++j)
+            u[t * D + j] = qko_load(row, dtype, j) * (double)gamma[j];
+    }
+    return 0;
+}
+
 /* 1 if built with OpenMP (the thread count is honoured), else 0. */
 int qko_has_openmp(void)
 {

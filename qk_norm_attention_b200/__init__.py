@@ -80,6 +80,10 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_apply.argtypes = [vp, vp, vp, vp, i64, i32, i32, f32, i32, vp]
     for fn in (lib.qknorm_fwd, lib.qknorm_partial_sumsq, lib.qknorm_apply):
         fn.restype = ctypes.c_int
+    lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
+    lib.qknorm_xgamma.restype = ctypes.c_int
+    lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
+    lib.qknorm_inv_rms.restype = ctypes.c_int
     lib.qknorm_status_string.argtypes = [ctypes.c_int]
     lib.qknorm_status_string.restype = ctypes.c_char_p
     lib.qknorm_last_error.argtypes = []
@@ -201,6 +205,38 @@ def qknorm_apply(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps:
     st = lib.qknorm_apply(x.data_ptr(), gamma.data_ptr(), stats.data_ptr(), out.data_ptr(), T, D,
                           P, float(eps), _dtype_code(x), _stream_handle(x.device, stream))
     _check("qknorm_apply", st)
+    return out
+
+
+def qknorm_xgamma(x: torch.Tensor, gamma: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """out = x * gamma (the weight multiply alone, rounded to x's dtype)."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T, D]")
+    T, D = x.shape
+    out = torch.empty_like(x) if out is None else out
+    for name, t in (("x", x), ("gamma", gamma), ("out", out)):
+        _need_cuda_contig(name, t)
+    if gamma.dtype != torch.float32 or gamma.numel() != D or out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("gamma must be float32 [D]; out must match x")
+    _check("qknorm_xgamma", lib.qknorm_xgamma(x.data_ptr(), gamma.data_ptr(), out.data_ptr(), T, D,
+                                              _dtype_code(x), _stream_handle(x.device, stream)))
+    return out
+
+
+def qknorm_inv_rms(x: torch.Tensor, P: int, eps: float, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """inv_rms[t] = rsqrt(mean_j x[t, j]^2 + eps) (fp32, the per-token factor alone)."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T, D]")
+    T, D = x.shape
+    out = torch.empty(T, dtype=torch.float32, device=x.device) if out is None else out
+    _need_cuda_contig("x", x)
+    _need_cuda_contig("out", out)
+    if out.dtype != torch.float32 or out.numel() != T:
+        raise ValueError("out must be float32 [T]")
+    _check("qknorm_inv_rms", lib.qknorm_inv_rms(x.data_ptr(), out.data_ptr(), T, D, int(P), float(eps),
+                                                _dtype_code(x), _stream_handle(x.device, stream)))
     return out
 
 

@@ -432,7 +432,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 105; }
+int qknorm_version(void) { return 106; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -549,6 +549,55 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
     return finish(e);
 }
 
+int qknorm_xgamma(const void *x, const float *gamma, void *out, int64_t T, int32_t D,
+                  int32_t dtype, void *stream) {
+    int st = check_shape(T, D, 1, dtype);
+    if (st != QKNORM_OK) return st;
+    if (T == 0) return QKNORM_OK;
+    if (!x || !gamma || !out) return QKNORM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(out)) return QKNORM_ERR_MISALIGNED;
+    const int64_t es = elem_of(dtype);
+    const Range ro = rng(out, T * D * es);
+    if (bad_alias(ro, rng(x, T * D * es), true) || bad_alias(ro, rng(gamma, (int64_t)D * 4), false))
+        return QKNORM_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    cudaError_t e = device_sms(&dev, &sms);
+    if (e != cudaSuccess) return finish(e);
+    const int64_t rowvec = D / vec_of(dtype);
+    int block = (int)((rowvec + kLanes - 1) / kLanes * kLanes);
+    if (block > 256) block = 256;
+    int bres = 1;
+    e = resident_blocks(dev, xgamma_kernel(dtype), block, 0, &bres);
+    if (e != cudaSuccess) return finish(e);
+    int64_t grid = (int64_t)sms * bres;
+    if (grid > T) grid = T;
+    return finish(launch_xgamma(dtype, x, gamma, out, T, D, block, grid,
+                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qknorm_inv_rms(const void *x, float *inv_rms, int64_t T, int32_t D, int32_t P, float eps,
+                   int32_t dtype, void *stream) {
+    int st = check_shape(T, D, P, dtype);
+    if (st == QKNORM_OK) st = check_eps(eps);
+    if (st != QKNORM_OK) return st;
+    if (T == 0) return QKNORM_OK;
+    if (!x || !inv_rms) return QKNORM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(inv_rms)) return QKNORM_ERR_MISALIGNED;
+    if (overlap(rng(inv_rms, T * 4), rng(x, T * D * elem_of(dtype)))) return QKNORM_ERR_INVALID_ARG;
+    const TensorShape sh = make_shape(D, P, vec_of(dtype));
+    int dev = 0, sms = 0;
+    cudaError_t e = device_sms(&dev, &sms);
+    if (e != cudaSuccess) return finish(e);
+    const int block = 256;
+    int bres = 1;
+    e = resident_blocks(dev, inv_rms_kernel(dtype), block, 0, &bres);
+    if (e != cudaSuccess) return finish(e);
+    int64_t grid = (T + block / kLanes - 1) / (block / kLanes);
+    if (grid > (int64_t)sms * bres) grid = (int64_t)sms * bres;
+    return finish(launch_inv_rms(dtype, x, inv_rms, T, sh, P, eps, block, grid,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_regs,
                       int32_t wait_limit_ms) {
     if (stages < 0 || stages > bulk_max_stages() || gamma_regs < -1 || gamma_regs > 1 ||
@@ -608,7 +657,8 @@ int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int3
     e = resident_blocks(dev, stats_kernel(dtype, sh.vmax), block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
     const int64_t ntask = T * P;
-    int64_t grid = (ntask + block / kLanes - 1) / (block / kLanes);
+    const int64_t per_block = (block / kLanes) * (sh.vmax <= 2 ? 4 : (sh.vmax <= 4 ? 2 : 1));
+    int64_t grid = (ntask + per_block - 1) / per_block;
     const int64_t cap = (int64_t)sms * bres;
     if (grid > cap) grid = cap;
     return finish(launch_stats(dtype, sh.vmax, x, stats, T, sh, P, block, grid,

@@ -152,6 +152,28 @@ __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const floa
     return o;
 }
 
+// u = x * gamma for one vector, rounded to the storage type (no factor).
+__device__ __forceinline__ uint4 vxgamma(F32Tag, const uint4 &v, const float *g) {
+    const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g));
+    uint4 o;
+    o.x = __float_as_uint(__fmul_rn(__uint_as_float(v.x), g4.x));
+    o.y = __float_as_uint(__fmul_rn(__uint_as_float(v.y), g4.y));
+    o.z = __float_as_uint(__fmul_rn(__uint_as_float(v.z), g4.z));
+    o.w = __float_as_uint(__fmul_rn(__uint_as_float(v.w), g4.w));
+    return o;
+}
+
+__device__ __forceinline__ uint4 vxgamma(BF16Tag, const uint4 &v, const float *g) {
+    const float4 ga = __ldg(reinterpret_cast<const float4 *>(g));
+    const float4 gb = __ldg(reinterpret_cast<const float4 *>(g) + 1);
+    uint4 o;
+    o.x = pack_bf16x2(__fmul_rn(bf_lo(v.x), ga.x), __fmul_rn(bf_hi(v.x), ga.y));
+    o.y = pack_bf16x2(__fmul_rn(bf_lo(v.y), ga.z), __fmul_rn(bf_hi(v.y), ga.w));
+    o.z = pack_bf16x2(__fmul_rn(bf_lo(v.z), gb.x), __fmul_rn(bf_hi(v.z), gb.y));
+    o.w = pack_bf16x2(__fmul_rn(bf_lo(v.w), gb.z), __fmul_rn(bf_hi(v.w), gb.w));
+    return o;
+}
+
 // Same as vapply with gamma read through an arbitrary pointer (used with
 // gamma staged in shared memory); same arithmetic, bit for bit.
 __device__ __forceinline__ uint4 vapply_ptr(F32Tag, const uint4 &v, const float *g, float r) {

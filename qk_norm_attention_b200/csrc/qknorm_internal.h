@@ -73,6 +73,14 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stag
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
 cudaError_t read_device_errors(unsigned *out, bool clear);
 
+// The deferred-normalisation steps (qknorm_deferred.cu).
+const void *xgamma_kernel(int dtype);
+const void *inv_rms_kernel(int dtype);
+cudaError_t launch_xgamma(int dtype, const void *x, const float *g, void *y, int64_t T, int32_t D,
+                          int block, int64_t grid, cudaStream_t s);
+cudaError_t launch_inv_rms(int dtype, const void *x, float *r, int64_t T, const TensorShape &sh,
+                           int32_t P, float eps, int block, int64_t grid, cudaStream_t s);
+
 // Launch with programmatic dependent launch when enabled (qknorm_set_pdl).
 bool pdl_enabled();
 inline cudaError_t launch(const void *fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s,

@@ -9,7 +9,8 @@
 // stats: one warp per (token, shard) task, the same reduction order as the
 //   fused kernels (groups of 32 lane chains, butterfly, groups in order), so
 //   S[t,p] equals the fused kernel's shard sum bit for bit. No barriers; the
-//   grid is a stride loop over tasks.
+//   grid is a stride loop over tasks, R tasks per warp turn with all their
+//   loads issued first.
 // apply: one CTA per row (stride loop over rows). Every thread adds the P
 //   shard sums of its row in order and forms the factor, then streams its
 //   vectors of the row through (x * gamma) * r. The row's first loads are
@@ -19,7 +20,7 @@
 
 namespace qkn {
 
-template <class Tag, int VMAX>
+template <class Tag, int VMAX, int R>
 __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int64_t T, int32_t D,
                                                int32_t P, int32_t nv, int32_t K) {
     constexpr int VEC = Tag::kVec;
@@ -30,26 +31,42 @@ __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int6
     const int64_t ntask = T * (int64_t)P;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int stride = kLanes * K;
-    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntask;
-         task += nwarps) {
-        const int64_t t = task / P;
-        const int p = (int)(task - t * P);
-        const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec + (int64_t)p * nv;
-        float S = 0.f;
+    const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // A warp takes R tasks per turn (tasks w0 + (n*R + j)*nwarps) and issues
+    // all their loads before reducing any, to keep more bytes in flight.
+    for (int64_t base = w0; base < ntask; base += (int64_t)R * nwarps) {
+        float S[R];
         for (int kg = 0; kg < K; ++kg) {
             const int first = kg * kLanes + lane;
             const int cnt = slot_count(first, nv, stride);
-            uint4 v[VMAX];
+            uint4 v[R][VMAX];
 #pragma unroll
-            for (int i = 0; i < VMAX; ++i)
-                if (i < cnt) v[i] = ld_stream(src + first + (int64_t)i * stride);
-            float c = 0.f;
+            for (int j = 0; j < R; ++j) {
+                const int64_t task = base + (int64_t)j * nwarps;
+                const int64_t t = task / P;
+                const int p = (int)(task - t * P);
+                const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec + (int64_t)p * nv;
 #pragma unroll
-            for (int i = 0; i < VMAX; ++i)
-                if (i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, v[i]));
-            S = __fadd_rn(S, butterfly(c));
+                for (int i = 0; i < VMAX; ++i)
+                    if (task < ntask && i < cnt) v[j][i] = ld_stream(src + first + (int64_t)i * stride);
+            }
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                float c = 0.f;
+#pragma unroll
+                for (int i = 0; i < VMAX; ++i)
+                    if (base + (int64_t)j * nwarps < ntask && i < cnt) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
+                const float b = butterfly(c);
+                S[j] = kg == 0 ? b : __fadd_rn(S[j], b);
+            }
         }
-        if (lane == 0) stats[task] = S;
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                const int64_t task = base + (int64_t)j * nwarps;
+                if (task < ntask) stats[task] = S[j];
+            }
+        }
     }
 }
 
@@ -94,17 +111,25 @@ __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, co
 
 // ---------------------------------------------------------------- instance tables
 
+// Tasks per warp turn: as many as keep R x VMAX <= 8 vectors per lane.
+constexpr int stats_r(int vmax) { return vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1); }
+
+template <class Tag, int V>
+const void *stats_fn() {
+    return reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V)>);
+}
+
 template <class Tag>
 const void *stats_table(int vmax) {
     switch (vmax) {
-    case 1: return reinterpret_cast<const void *>(&stats_k<Tag, 1>);
-    case 2: return reinterpret_cast<const void *>(&stats_k<Tag, 2>);
-    case 3: return reinterpret_cast<const void *>(&stats_k<Tag, 3>);
-    case 4: return reinterpret_cast<const void *>(&stats_k<Tag, 4>);
-    case 5: return reinterpret_cast<const void *>(&stats_k<Tag, 5>);
-    case 6: return reinterpret_cast<const void *>(&stats_k<Tag, 6>);
-    case 7: return reinterpret_cast<const void *>(&stats_k<Tag, 7>);
-    case 8: return reinterpret_cast<const void *>(&stats_k<Tag, 8>);
+    case 1: return stats_fn<Tag, 1>();
+    case 2: return stats_fn<Tag, 2>();
+    case 3: return stats_fn<Tag, 3>();
+    case 4: return stats_fn<Tag, 4>();
+    case 5: return stats_fn<Tag, 5>();
+    case 6: return stats_fn<Tag, 6>();
+    case 7: return stats_fn<Tag, 7>();
+    case 8: return stats_fn<Tag, 8>();
     default: return nullptr;
     }
 }

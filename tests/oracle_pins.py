@@ -296,6 +296,22 @@ def pin_row_independence(orc):
         assert np.array_equal(y_t[0], y_all[t]) and r_t[0] == r_all[t], f"row {t}"
 
 
+def pin_xgamma(orc):
+    """The weight multiply alone: exact products of stored values (a double
+    product of a bf16 or fp32 value and an fp32 weight is exact); gamma = 1
+    returns x; y = xgamma * r where r is the factor (Eq. (1) factorises)."""
+    for dtype, (x, g) in (("f32", tiny_q(4)), ("bf16", bf16_inputs(5, 1280, seed=13))):
+        x64 = widen(x, dtype)
+        u = orc.xgamma(x, g, dtype)
+        for t in range(x.shape[0]):
+            for j in (0, 1, x.shape[1] // 2, x.shape[1] - 1):
+                assert Fraction(float(u[t, j])) == Fraction(float(x64[t, j])) * Fraction(float(g[j]))
+        assert np.array_equal(orc.xgamma(x, np.ones(x.shape[1], np.float32), dtype), x64)
+        y, r = orc.rmsnorm(x, g, 4, 1e-6, dtype)
+        assert np.array_equal(y, u * r[:, None])      # same two roundings: (x*g) then *r
+        assert np.array_equal(orc.inv_rms(x, 4, 1e-6, dtype), r)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_shard_sums_exact,
@@ -308,4 +324,5 @@ ALL_PINS = [
     pin_scale_law,
     pin_deferred_prescale,
     pin_row_independence,
+    pin_xgamma,
 ]

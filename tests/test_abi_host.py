@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 105
+    assert qk.qknorm_version() == 106
 
 
 # ----------------------------------------------------------------- argument checks
@@ -256,3 +256,19 @@ def test_rows_warps_fill_shared_memory(qk):
         assert pl["grid"] == min(148 * 2, (2 * 4096 + 7) // 8)
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+
+
+@needs_cpu
+def test_deferred_entry_points_reject(qk):
+    L = qk.lib
+    assert L.qknorm_xgamma(A + 2, B, C, 4, 256, 1, None) == 2
+    assert L.qknorm_xgamma(A, B, C, 4, 252, 1, None) == 3          # 252 not a multiple of 8
+    assert L.qknorm_xgamma(A, B, A + 16, 4, 256, 1, None) == 1     # partial overlap
+    assert L.qknorm_xgamma(A, B, B, 4, 256, 1, None) == 1          # out on gamma
+    assert L.qknorm_xgamma(0, B, C, 4, 256, 1, None) == 1
+    assert L.qknorm_xgamma(0, 0, 0, 0, 256, 1, None) == 0
+    assert L.qknorm_inv_rms(A, B, 4, 256, 3, 1e-6, 1, None) == 1   # D % P
+    assert L.qknorm_inv_rms(A, B, 4, 256, 4, -1.0, 1, None) == 1
+    assert L.qknorm_inv_rms(A, A + 64, 4, 256, 4, 1e-6, 1, None) == 1
+    assert L.qknorm_inv_rms(A, B + 4, 4, 256, 4, 1e-6, 1, None) == 2
+    assert L.qknorm_inv_rms(A, B, 4, 256, 4, 1e-6, 7, None) == 3
