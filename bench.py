@@ -332,6 +332,46 @@ def throughput(torch, qk, wl, T, device, sets, steps=50):
             "algorithmic_bytes": nbytes, "buffer_sets": sets}
 
 
+def deferred_steps(torch, qk, device, peak, steps=100):
+    """qknorm_xgamma and qknorm_inv_rms on the 13B-shaped Q tensor (T = 8192,
+    D = 5120, bf16, P = 4), three rotating inputs (> L2)."""
+    wl = W.WORKLOADS["prefill13b"]
+    T, D, P = wl.Ts[0], wl.Dq, wl.P
+    stream = torch.cuda.current_stream(device)
+    h = stream.cuda_stream
+    x = W.gen_device_workload(wl, "q", T, device)
+    xs = [x, x.clone(), x.clone()]
+    g = torch.from_numpy(W.gen_gamma(wl, "q")).to(device)
+    us = [torch.empty_like(x) for _ in xs]
+    rs = [torch.empty(T, dtype=torch.float32, device=device) for _ in xs]
+    L = qk.lib
+
+    def xg(i):
+        def f():
+            if L.qknorm_xgamma(xs[i].data_ptr(), g.data_ptr(), us[i].data_ptr(), T, D, 1, h) != 0:
+                raise RuntimeError("qknorm_xgamma failed")
+        return f
+
+    def ir(i):
+        def f():
+            if L.qknorm_inv_rms(xs[i].data_ptr(), rs[i].data_ptr(), T, D, P, wl.eps, 1, h) != 0:
+                raise RuntimeError("qknorm_inv_rms failed")
+        return f
+
+    out = {"workload": "13B-shaped Q tensor: T=8192, D=5120, bf16, P=4"}
+    for name, calls, nbytes in (("xgamma", [xg(i) for i in range(3)], 2 * T * D * 2 + 4 * D),
+                                ("inv_rms", [ir(i) for i in range(3)], T * D * 2 + 4 * T)):
+        for i in range(6):
+            calls[i % 3]()
+        torch.cuda.synchronize()
+        tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
+        ms = tot / steps
+        out[name] = {"us_per_call": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
+                     "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1),
+                     "algorithmic_bytes": nbytes}
+    return out
+
+
 def split_path(torch, qk, device, peak, steps=20):
     """The split path (stats + apply for Q and K: 4 launches) and the fused path
     on the large-prefill workload, T = 65536, D = 4096, P = 8, bf16."""
@@ -570,6 +610,7 @@ def run_native(args, dist):
                          "T4096": throughput(torch, qk, gqa, 4096, device, sets=4)}
         extras["gqa"]["T4096"]["pct_hbm_peak"] = round(100 * extras["gqa"]["T4096"]["GB_s"] / peak, 1)
         extras["split_large"] = split_path(torch, qk, device, peak)
+        extras["deferred"] = deferred_steps(torch, qk, device, peak)
     dist.barrier()
 
     traffic = None
