@@ -100,6 +100,24 @@ QKNORM_API int qknorm_fwd(const void *q, const void *k, const float *gamma_q, co
                float eps, int32_t dtype, void *stream);
 
 /*
+ * qknorm_fwd_strided -- qknorm_fwd on rows that are not dense: row t of q
+ * starts at q + t*ldq elements (likewise k, out_q, out_k with ldk, ldoq,
+ * ldok). The common use is Q and K as column slices of one fused QKV
+ * projection buffer (q = qkv, k = qkv + Dq, ldq = ldk = Dq + 2*Dk), normalised
+ * in place (out_q = q, out_k = k, same strides) or into dense outputs.
+ * Strides are in elements, >= the width, and multiples of the 16-byte vector
+ * (8 bf16 / 4 fp32). Tensors with the same stride may interleave (the slices
+ * of one buffer) as long as their rows do not touch; an output may be its
+ * own input with the same stride. qknorm_fwd is this call with ld = D.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q,
+                                  const float *gamma_k, void *out_q, void *out_k, int64_t T,
+                                  int32_t Dq, int32_t Dk, int32_t P, float eps, int32_t dtype,
+                                  int64_t ldq, int64_t ldk, int64_t ldoq, int64_t ldok,
+                                  void *stream);
+
+/*
  * qknorm_partial_sumsq -- the statistics half of the split path.
  *
  * Algorithm 1, Phase A for one tensor: stats[t*P + p] = fp32 sum of

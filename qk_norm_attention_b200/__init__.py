@@ -80,6 +80,9 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_apply.argtypes = [vp, vp, vp, vp, i64, i32, i32, f32, i32, vp]
     for fn in (lib.qknorm_fwd, lib.qknorm_partial_sumsq, lib.qknorm_apply):
         fn.restype = ctypes.c_int
+    lib.qknorm_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32,
+                                       i64, i64, i64, i64, vp]
+    lib.qknorm_fwd_strided.restype = ctypes.c_int
     lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     lib.qknorm_xgamma.restype = ctypes.c_int
     lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
@@ -168,6 +171,41 @@ def qknorm_fwd(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k:
                         out_q.data_ptr(), out_k.data_ptr(), T, Dq, Dk, int(P), float(eps),
                         _dtype_code(q), _stream_handle(q.device, stream))
     _check("qknorm_fwd", st)
+    return out_q, out_k
+
+
+def _rows_view(name: str, t: torch.Tensor):
+    """(T, D, row stride) of a 2-D CUDA tensor whose rows are dense (stride 1
+    along a row), e.g. a column slice of a fused QKV buffer."""
+    if not t.is_cuda or t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be a 2-D CUDA tensor with unit stride along rows")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def qknorm_fwd_strided(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor,
+                       gamma_k: torch.Tensor, P: int, eps: float,
+                       out_q: Optional[torch.Tensor] = None, out_k: Optional[torch.Tensor] = None,
+                       stream=None):
+    """qknorm_fwd on row-strided q and k (e.g. slices of a fused QKV buffer);
+    the outputs may be the inputs themselves (in place) or dense tensors."""
+    T, Dq, ldq = _rows_view("q", q)
+    Tk, Dk, ldk = _rows_view("k", k)
+    if T != Tk or q.dtype != k.dtype:
+        raise ValueError("q and k must share T and dtype")
+    out_q = torch.empty((T, Dq), dtype=q.dtype, device=q.device) if out_q is None else out_q
+    out_k = torch.empty((T, Dk), dtype=k.dtype, device=k.device) if out_k is None else out_k
+    _, Doq, ldoq = _rows_view("out_q", out_q)
+    _, Dok, ldok = _rows_view("out_k", out_k)
+    if (Doq, Dok) != (Dq, Dk) or out_q.dtype != q.dtype or out_k.dtype != k.dtype:
+        raise ValueError("outputs must match the inputs' widths and dtype")
+    for name, g, D in (("gamma_q", gamma_q, Dq), ("gamma_k", gamma_k, Dk)):
+        _need_cuda_contig(name, g)
+        if g.dtype != torch.float32 or g.numel() != D:
+            raise ValueError(f"{name} must be float32 with {D} elements")
+    st = lib.qknorm_fwd_strided(q.data_ptr(), k.data_ptr(), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                                out_q.data_ptr(), out_k.data_ptr(), T, Dq, Dk, int(P), float(eps),
+                                _dtype_code(q), ldq, ldk, ldoq, ldok, _stream_handle(q.device, stream))
+    _check("qknorm_fwd_strided", st)
     return out_q, out_k
 
 

@@ -64,6 +64,36 @@ bool bad_alias(Range out, Range in, bool may_alias) {
     return !(may_alias && out.lo == in.lo && out.hi == in.hi);
 }
 
+// A strided tensor: T rows of `row` bytes whose starts are `ld` bytes apart.
+struct Strided {
+    uintptr_t base;
+    int64_t row, ld, T;
+};
+Strided strided(const void *p, int64_t row, int64_t ld, int64_t T) {
+    return Strided{reinterpret_cast<uintptr_t>(p), row, ld, T};
+}
+// True if any byte of a may be a byte of b. Tensors with the same row period
+// interleave without touching when their row segments are disjoint modulo
+// the period (e.g. the Q, K and V slices of one fused QKV buffer); otherwise
+// the test falls back to the spans.
+bool strided_overlap(const Strided &a, const Strided &b) {
+    if (a.T <= 0 || b.T <= 0) return false;
+    const Range ra{a.base, a.base + (uintptr_t)((a.T - 1) * a.ld + a.row)};
+    const Range rb{b.base, b.base + (uintptr_t)((b.T - 1) * b.ld + b.row)};
+    if (!overlap(ra, rb)) return false;
+    if (a.ld == b.ld && a.ld > 0) {
+        const int64_t d = (int64_t)(b.base - a.base);
+        const int64_t r = ((d % a.ld) + a.ld) % a.ld;  // b's row start within a's period
+        if (r >= a.row && r + b.row <= a.ld) return false;
+    }
+    return true;
+}
+// An output may be exactly its own input (same base, row and stride).
+bool strided_bad_alias(const Strided &out, const Strided &in, bool may_alias) {
+    if (may_alias && out.base == in.base && out.row == in.row && out.ld == in.ld) return false;
+    return strided_overlap(out, in);
+}
+
 // Checks common to every entry point for one [T, D] tensor with P shards.
 int check_shape(int64_t T, int32_t D, int32_t P, int32_t dtype) {
     if (T < 0 || D <= 0 || P <= 0) return QKNORM_ERR_INVALID_ARG;
@@ -432,7 +462,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 106; }
+int qknorm_version(void) { return 107; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -487,25 +517,35 @@ int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dty
     return st;
 }
 
-int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
-               void *out_q, void *out_k, int64_t T, int32_t Dq, int32_t Dk, int32_t P,
-               float eps, int32_t dtype, void *stream) {
+int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+                       void *out_q, void *out_k, int64_t T, int32_t Dq, int32_t Dk, int32_t P,
+                       float eps, int32_t dtype, int64_t ldq, int64_t ldk, int64_t ldoq,
+                       int64_t ldok, void *stream) {
     int st = check_shape(T, Dq, P, dtype);
     if (st == QKNORM_OK) st = check_shape(T, Dk, P, dtype);
     if (st == QKNORM_OK) st = check_eps(eps);
     if (st != QKNORM_OK) return st;
+    if (ldq < Dq || ldk < Dk || ldoq < Dq || ldok < Dk) return QKNORM_ERR_INVALID_ARG;
+    const int vec = vec_of(dtype);
+    if (ldq % vec || ldk % vec || ldoq % vec || ldok % vec) return QKNORM_ERR_MISALIGNED;
+    const int64_t es = elem_of(dtype);
+    const int64_t ldmax = ldq > ldk ? (ldq > ldoq ? (ldq > ldok ? ldq : ldok) : (ldoq > ldok ? ldoq : ldok))
+                                    : (ldk > ldoq ? (ldk > ldok ? ldk : ldok) : (ldoq > ldok ? ldoq : ldok));
+    if (T > 0 && T > INT64_MAX / (ldmax * es)) return QKNORM_ERR_INVALID_ARG;
     if (T == 0) return QKNORM_OK;
     if (!q || !k || !gamma_q || !gamma_k || !out_q || !out_k) return QKNORM_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(gamma_q) || !aligned16(gamma_k) ||
         !aligned16(out_q) || !aligned16(out_k))
         return QKNORM_ERR_MISALIGNED;
-    const int64_t es = elem_of(dtype);
-    const Range rq = rng(q, T * Dq * es), rk = rng(k, T * Dk * es);
-    const Range rgq = rng(gamma_q, (int64_t)Dq * 4), rgk = rng(gamma_k, (int64_t)Dk * 4);
-    const Range roq = rng(out_q, T * Dq * es), rok = rng(out_k, T * Dk * es);
-    if (bad_alias(roq, rq, true) || bad_alias(roq, rk, false) || bad_alias(roq, rgq, false) ||
-        bad_alias(roq, rgk, false) || bad_alias(roq, rok, false) || bad_alias(rok, rk, true) ||
-        bad_alias(rok, rq, false) || bad_alias(rok, rgq, false) || bad_alias(rok, rgk, false))
+    const Strided mq = strided(q, Dq * es, ldq * es, T), mk = strided(k, Dk * es, ldk * es, T);
+    const Strided mgq = strided(gamma_q, (int64_t)Dq * 4, (int64_t)Dq * 4, 1);
+    const Strided mgk = strided(gamma_k, (int64_t)Dk * 4, (int64_t)Dk * 4, 1);
+    const Strided moq = strided(out_q, Dq * es, ldoq * es, T), mok = strided(out_k, Dk * es, ldok * es, T);
+    if (strided_bad_alias(moq, mq, true) || strided_bad_alias(moq, mk, false) ||
+        strided_bad_alias(moq, mgq, false) || strided_bad_alias(moq, mgk, false) ||
+        strided_bad_alias(moq, mok, false) || strided_bad_alias(mok, mk, true) ||
+        strided_bad_alias(mok, mq, false) || strided_bad_alias(mok, mgq, false) ||
+        strided_bad_alias(mok, mgk, false))
         return QKNORM_ERR_INVALID_ARG;
 
     qknorm_plan pl;
@@ -533,6 +573,10 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
     a.Df[0] = (float)Dq;
     a.Df[1] = (float)Dk;
     a.eps = eps;
+    a.ldx[0] = ldq / vec;
+    a.ldx[1] = ldk / vec;
+    a.ldy[0] = ldoq / vec;
+    a.ldy[1] = ldok / vec;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
         e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes != 0, a, pl.block,
@@ -547,6 +591,13 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
         e = launch_fused_generic(dtype, a, pl.block, pl.grid, (size_t)pl.smem_bytes, s);
     }
     return finish(e);
+}
+
+int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+               void *out_q, void *out_k, int64_t T, int32_t Dq, int32_t Dk, int32_t P,
+               float eps, int32_t dtype, void *stream) {
+    return qknorm_fwd_strided(q, k, gamma_q, gamma_k, out_q, out_k, T, Dq, Dk, P, eps, dtype, Dq, Dk,
+                              Dq, Dk, stream);
 }
 
 int qknorm_xgamma(const void *x, const float *gamma, void *out, int64_t T, int32_t D,

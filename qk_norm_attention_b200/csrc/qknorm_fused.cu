@@ -61,7 +61,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     const int first = tk.kg * kLanes + lane;     // slot 0, as a vector index in the shard
     // FULL: every lane of every task holds exactly VMAX vectors (no guards).
     const int cnt = FULL ? VMAX : slot_count(first, tk.nv, stride);
-    const int64_t rowvec = sel(a.D, tk.z) / VEC;      // vectors per row
+    const int64_t ldx = sel(a.ldx, tk.z);             // row strides, in vectors
+    const int64_t ldy = sel(a.ldy, tk.z);
     const int64_t col0 = (int64_t)tk.p * tk.nv + first;
     const uint4 *xs = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + col0;
     uint4 *ys = reinterpret_cast<uint4 *>(sel(a.y, tk.z)) + col0;
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
 
     uint4 cur[VMAX];
     if (t < T) {
-        const uint4 *src = xs + t * rowvec;
+        const uint4 *src = xs + t * ldx;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
             if (FULL || i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
         const int64_t tn = t + G;
         uint4 nxt[VMAX];
         if (PREFETCH && tn < T) {
-            const uint4 *src = xs + tn * rowvec;
+            const uint4 *src = xs + tn * ldx;
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
                 if (FULL || i < cnt) nxt[i] = ld_stream(src + (int64_t)i * stride);
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
         // Phase B: shard sums in order, the factor.
         const float r = factor(combine_fast(&red[buf][red_base], a.P, tk.K), Df, eps);
         // Phase B weight multiply and Phase C, straight from registers.
-        uint4 *dst = ys + t * rowvec;
+        uint4 *dst = ys + t * ldy;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
             if (FULL || i < cnt)
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
 #pragma unroll
             for (int i = 0; i < VMAX; ++i) cur[i] = nxt[i];
         } else if (tn < T) {
-            const uint4 *src = xs + tn * rowvec;
+            const uint4 *src = xs + tn * ldx;
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
                 if (FULL || i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
             const Task tk = decode_task(a, j);
             const int stride = kLanes * tk.K;
             const uint4 *src = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) +
-                               t * (int64_t)(sel(a.D, tk.z) / VEC) + (int64_t)tk.p * tk.nv;
+                               t * sel(a.ldx, tk.z) + (int64_t)tk.p * tk.nv;
             float c = 0.f;
 #pragma unroll 4
             for (int v = tk.kg * kLanes + lane; v < tk.nv; v += stride)
@@ -151,9 +152,9 @@ __global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
         for (int j = warp; j < ntask; j += nw) {
             const Task tk = decode_task(a, j);
             const int stride = kLanes * tk.K;
-            const int64_t off = t * (int64_t)(sel(a.D, tk.z) / VEC) + (int64_t)tk.p * tk.nv;
-            const uint4 *src = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + off;
-            uint4 *dst = reinterpret_cast<uint4 *>(sel(a.y, tk.z)) + off;
+            const int64_t col = (int64_t)tk.p * tk.nv;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sel(a.x, tk.z)) + t * sel(a.ldx, tk.z) + col;
+            uint4 *dst = reinterpret_cast<uint4 *>(sel(a.y, tk.z)) + t * sel(a.ldy, tk.z) + col;
             const float *g = sel(a.g, tk.z) + (int64_t)tk.p * tk.nv * VEC;
             const float r = tk.z ? r1 : r0;
 #pragma unroll 4

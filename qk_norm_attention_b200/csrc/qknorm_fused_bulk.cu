@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     const int first = kg * kLanes + lane;
     // FULL: every lane of every task holds exactly VMAX vectors (no guards).
     const int cnt = FULL ? VMAX : slot_count(first, nv, stride);
-    const int64_t rowvec = (z ? a.D[1] : a.D[0]) / VEC;
+    const int64_t ldy = z ? a.ldy[1] : a.ldy[0];     // output row stride, in vectors
     const int64_t col0 = (int64_t)p * nv + first;
     uint4 *ys = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + col0;
     const float *gs = (z ? a.g[1] : a.g[0]) + col0 * VEC;
@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     const int S = (int)b.stages;
     const char *qsrc = static_cast<const char *>(a.x[0]);
     const char *ksrc = static_cast<const char *>(a.x[1]);
+    const int64_t ldq_b = a.ldx[0] * 16, ldk_b = a.ldx[1] * 16;   // input row strides, bytes
 
     // Tokens of pass n: blockIdx.x + (n*TB + j)*G, j < TB (those below T).
     auto issue = [&](int s, int64_t n) {
@@ -93,9 +94,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
         for (int j = 0; j < TB; ++j) {
             const int64_t tt = t0 + j * G;
             if (tt < T) {
-                bulk_copy_g2s(st + j * tok_bytes, qsrc + tt * (int64_t)b.qbytes, b.qbytes, &full[s]);
-                bulk_copy_g2s(st + j * tok_bytes + b.qbytes, ksrc + tt * (int64_t)b.kbytes,
-                              b.kbytes, &full[s]);
+                bulk_copy_g2s(st + j * tok_bytes, qsrc + tt * ldq_b, b.qbytes, &full[s]);
+                bulk_copy_g2s(st + j * tok_bytes + b.qbytes, ksrc + tt * ldk_b, b.kbytes, &full[s]);
             }
         }
     };
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
             const int64_t t = t0 + j * G;
             if (j == 0 || t < T) {
                 const float r = factor(combine_fast(&red[buf][j][red_base], a.P, K), Df, eps);
-                uint4 *dst = ys + t * rowvec;
+                uint4 *dst = ys + t * ldy;
 #pragma unroll
                 for (int i = 0; i < VMAX; ++i)
                     if (FULL || i < cnt) {
@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
         const bool isk = r >= T;
         const int64_t t = isk ? r - T : r;
         const uint32_t nb = isk ? kbytes : qbytes;
-        const char *src = static_cast<const char *>(isk ? a.x[1] : a.x[0]) + t * (int64_t)nb;
+        const char *src = static_cast<const char *>(isk ? a.x[1] : a.x[0]) +
+                          t * (isk ? a.ldx[1] : a.ldx[0]) * 16;
         mbar_arrive_expect_tx(&full[s], nb);
         bulk_copy_g2s(ring + (size_t)s * b.stage_bytes, src, nb, &full[s]);
     };
@@ -362,7 +363,7 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
         // Phase B weight multiply and Phase C, element-wise over the row.
         const int rowvec = (z ? a.D[1] : a.D[0]) / VEC;
         const float *g = z ? gam_k : gam_q;
-        uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (int64_t)rowvec;
+        uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]);
 #pragma unroll 4
         for (int v = lane; v < rowvec; v += kLanes)
             st_stream(dst + v, vapply_ptr(Tag{}, row[v], g + (int64_t)v * VEC, rr));

@@ -27,6 +27,8 @@ struct FusedArgs {
     int32_t P;
     float Df[2];
     float eps;
+    int64_t ldx[2];  // row strides of the inputs, in 16-byte vectors
+    int64_t ldy[2];  // row strides of the outputs, in 16-byte vectors
 };
 
 TensorShape make_shape(int32_t D, int32_t P, int vec);

@@ -2,9 +2,9 @@
 loads, exports every function the header declares, validates arguments before
 touching CUDA, and the selector plans the expected launches.
 
-Argument checks use fake addresses that the validation must reject; no call
-here passes validation with a fake address, and the module skips itself on a
-machine with a GPU so that no such address could ever reach a kernel."""
+Argument checks use fake addresses. The few calls that pass validation reach
+the CUDA runtime, which finds no device; these tests skip themselves on a
+machine with a GPU, so no fake address can ever reach a kernel."""
 import ctypes
 import math
 import os
@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 106
+    assert qk.qknorm_version() == 107
 
 
 # ----------------------------------------------------------------- argument checks
@@ -272,3 +272,29 @@ def test_deferred_entry_points_reject(qk):
     assert L.qknorm_inv_rms(A, A + 64, 4, 256, 4, 1e-6, 1, None) == 1
     assert L.qknorm_inv_rms(A, B + 4, 4, 256, 4, 1e-6, 1, None) == 2
     assert L.qknorm_inv_rms(A, B, 4, 256, 4, 1e-6, 7, None) == 3
+
+
+@needs_cpu
+def test_strided_checks(qk):
+    """Row strides: >= the width, a multiple of the 16-byte vector; Q and K as
+    slices of one fused QKV buffer may be normalised in place; an output that
+    lands on another tensor's rows is rejected."""
+    L = qk.lib
+    Dq, Dk = 256, 128
+    ld = Dq + 2 * Dk                       # one QKV row, bf16 elements
+    qkv = 0x100000
+    q, k, v = qkv, qkv + 2 * Dq, qkv + 2 * (Dq + Dk)
+
+    def call(q_, k_, oq, ok, ldq=ld, ldk=ld, ldoq=ld, ldok=ld, T=16):
+        return L.qknorm_fwd_strided(q_, k_, C, Dd, oq, ok, T, Dq, Dk, 2, 1e-6, 1,
+                                    ldq, ldk, ldoq, ldok, None)
+
+    assert call(q, k, q, k) == 4                          # in place: valid, then no GPU
+    assert call(q, k, E, F, ldoq=Dq, ldok=Dk) == 4        # strided in, dense out: valid
+    assert call(q, k, q, k, ldq=Dq - 8) == 1              # stride below the width
+    assert call(q, k, q, k, ldq=ld + 4) == 2              # stride not a multiple of 8 bf16
+    assert call(q, k, k, q) == 1                          # outputs on each other's input
+    assert call(q, k, v, k) == 1                          # Dq-wide output from V's start reaches next Q
+    assert call(q, k, q, v) == 4                          # Dk-wide K output into the V slot: disjoint rows
+    assert call(q, k, q + 16, k) == 1                     # Q output shifted into its own input
+    assert call(q, k, E, F, ldoq=Dq, ldok=Dk, T=0) == 0

@@ -305,3 +305,41 @@ def test_dependent_launches_with_pdl(qk, variant):
     for pdl in (True, False):
         got = chain(pdl, False)
         assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
+
+
+@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "generic"])
+@pytest.mark.parametrize("T", [37, 3 * 148 + 5])
+def test_strided_qkv_in_place(qk, variant, T):
+    """Q and K normalised in place inside a fused QKV buffer [T, Dq + 2 Dk]
+    (row stride Dq + 2 Dk): the slices equal dense calls bit for bit, V and
+    the padding are untouched; also strided in, dense out and dense in,
+    strided out."""
+    Dq, Dk, P = 2048, 512, 4
+    wl = W.custom("qkv", T, Dq, Dk, P, seed=38)
+    q, k, gq, gk = _inputs(wl, T)
+    ref = _fwd(qk, wl, q, k, gq, gk, variant=None if variant == "auto" else variant)
+    qd, kd = to_device(q), to_device(k)
+    ld = Dq + 2 * Dk + 64                        # QKV row plus 64 elements of padding
+    buf = torch.full((T, ld), 5.0, dtype=torch.bfloat16, device="cuda")
+    buf[:, :Dq] = qd
+    buf[:, Dq:Dq + Dk] = kd
+    untouched = buf[:, Dq + Dk:].clone()
+    vid = {"auto": qk.VARIANT_AUTO, "cta": qk.VARIANT_CTA, "bulk": qk.VARIANT_BULK,
+           "rows": qk.VARIANT_ROWS, "generic": qk.VARIANT_GENERIC}[variant]
+    gqd, gkd = to_device(gq), to_device(gk)
+    qk.qknorm_force_variant(vid, 0)
+    try:
+        qs, ks = buf[:, :Dq], buf[:, Dq:Dq + Dk]
+        dq, dk = qk.qknorm_fwd_strided(qs, ks, gqd, gkd, P, wl.eps)           # strided in, dense out
+        qk.qknorm_fwd_strided(qs, ks, gqd, gkd, P, wl.eps, out_q=qs, out_k=ks)  # in place
+        buf2 = torch.zeros((T, ld), dtype=torch.bfloat16, device="cuda")
+        qk.qknorm_fwd_strided(qd, kd, gqd, gkd, P, wl.eps, out_q=buf2[:, :Dq],
+                              out_k=buf2[:, Dq:Dq + Dk])                      # dense in, strided out
+        torch.cuda.synchronize()
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    for got_q, got_k in ((dq, dk), (buf[:, :Dq], buf[:, Dq:Dq + Dk]), (buf2[:, :Dq], buf2[:, Dq:Dq + Dk])):
+        assert torch.equal(bits(got_q.contiguous()), bits(ref[0]))
+        assert torch.equal(bits(got_k.contiguous()), bits(ref[1]))
+    assert torch.equal(bits(buf[:, Dq + Dk:]), bits(untouched))
+    assert bool((buf2[:, Dq + Dk:] == 0).all())
