@@ -372,6 +372,42 @@ def deferred_steps(torch, qk, device, peak, steps=100):
     return out
 
 
+def headwise(torch, qk, device, peak, steps=100):
+    """Headwise QK-Norm: T = 8192 tokens, Hq = 32 and Hk = 8 heads of 128
+    (bf16), gamma [128] per tensor, three rotating buffer sets."""
+    T, Hq, Hk, hd = 8192, 32, 8, 128
+    wl = W.custom("headwise", T, Hq * hd, Hk * hd, Hq, seed=7)
+    stream = torch.cuda.current_stream(device)
+    h = stream.cuda_stream
+    q = W.gen_device_workload(wl, "q", T, device)
+    k = W.gen_device_workload(wl, "k", T, device)
+    g = torch.ones(hd, dtype=torch.float32, device=device)
+    sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(2)]
+    outs = [(torch.empty_like(a), torch.empty_like(b)) for a, b in sets]
+    L = qk.lib
+
+    def call(i):
+        (a, b), (oa, ob) = sets[i], outs[i]
+
+        def f():
+            if L.qknorm_headwise_fwd(a.data_ptr(), b.data_ptr(), g.data_ptr(), g.data_ptr(),
+                                     oa.data_ptr(), ob.data_ptr(), T, Hq, Hk, hd, 1e-6, 1,
+                                     Hq * hd, Hk * hd, Hq * hd, Hk * hd, h) != 0:
+                raise RuntimeError("qknorm_headwise_fwd failed")
+        return f
+
+    calls = [call(i) for i in range(3)]
+    for i in range(6):
+        calls[i % 3]()
+    torch.cuda.synchronize()
+    tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
+    ms = tot / steps
+    nbytes = W.fused_bytes(T, Hq * hd, Hk * hd, 2)
+    return {"workload": "T=8192, Hq=32, Hk=8, head_dim=128, bf16", "us_per_call": round(ms * 1000, 2),
+            "GB_s": round(nbytes / ms / 1e6, 1), "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1),
+            "algorithmic_bytes": nbytes}
+
+
 def split_path(torch, qk, device, peak, steps=20):
     """The split path (stats + apply for Q and K: 4 launches) and the fused path
     on the large-prefill workload, T = 65536, D = 4096, P = 8, bf16."""
@@ -611,6 +647,7 @@ def run_native(args, dist):
         extras["gqa"]["T4096"]["pct_hbm_peak"] = round(100 * extras["gqa"]["T4096"]["GB_s"] / peak, 1)
         extras["split_large"] = split_path(torch, qk, device, peak)
         extras["deferred"] = deferred_steps(torch, qk, device, peak)
+        extras["headwise"] = headwise(torch, qk, device, peak)
     dist.barrier()
 
     traffic = None

@@ -118,6 +118,27 @@ QKNORM_API int qknorm_fwd_strided(const void *q, const void *k, const float *gam
                                   void *stream);
 
 /*
+ * qknorm_headwise_fwd -- headwise QK-Norm of Q and K: one factor per head.
+ *
+ * SwiftQK technical review, "Prerequisites" (layerwise vs. headwise) and
+ * Section 4c: the reduction of Eq. (1) spans one head's head_dim elements;
+ * gamma has head_dim entries shared by all heads of its tensor. For head h
+ * of row t: S = sum of squares of the head in the reduction order above
+ * (the head as the only shard), r = rsqrt(S / head_dim + eps),
+ * y = (x * gamma) * r.
+ *   q [T, Hq*head_dim] with row stride ldq, k [T, Hk*head_dim] stride ldk;
+ *   gamma_q, gamma_k [head_dim] fp32; out_q, out_k strides ldoq, ldok.
+ * head_dim must be a multiple of the 16-byte vector and at most 256 vectors;
+ * strides as in qknorm_fwd_strided (pass ld = H*head_dim for dense rows).
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_headwise_fwd(const void *q, const void *k, const float *gamma_q,
+                                   const float *gamma_k, void *out_q, void *out_k, int64_t T,
+                                   int32_t Hq, int32_t Hk, int32_t head_dim, float eps,
+                                   int32_t dtype, int64_t ldq, int64_t ldk, int64_t ldoq,
+                                   int64_t ldok, void *stream);
+
+/*
  * qknorm_partial_sumsq -- the statistics half of the split path.
  *
  * Algorithm 1, Phase A for one tensor: stats[t*P + p] = fp32 sum of

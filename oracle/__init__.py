@@ -116,6 +116,19 @@ class Oracle:
         _, r = self.rmsnorm(x, np.ones(D, dtype=np.float32), P, eps, dtype, nthreads, want_y=False)
         return r
 
+    def headwise(self, x: np.ndarray, gamma: np.ndarray, head_dim: int, eps: float, dtype: str,
+                 nthreads: int = 1) -> np.ndarray:
+        """Headwise RMSNorm: each head's head_dim values normalised on their
+        own (the same RMSNorm on rows of length head_dim), gamma [head_dim]
+        shared by the heads. x [T, H*head_dim] -> y [T, H*head_dim], float64."""
+        x = self._prep(x, dtype)
+        T, D = x.shape
+        if D % head_dim:
+            raise ValueError("width must be a multiple of head_dim")
+        y, _ = self.rmsnorm(np.ascontiguousarray(x.reshape(T * (D // head_dim), head_dim)),
+                            gamma, 1, eps, dtype, nthreads)
+        return y.reshape(T, D)
+
     def qknorm(self, q, k, gamma_q, gamma_k, P, eps, dtype, nthreads: int = 1):
         """Layerwise QK-Norm: the RMSNorm above applied to Q and, on its own, to K."""
         yq, rq = self.rmsnorm(q, gamma_q, P, eps, dtype, nthreads)

@@ -83,6 +83,9 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32,
                                        i64, i64, i64, i64, vp]
     lib.qknorm_fwd_strided.restype = ctypes.c_int
+    lib.qknorm_headwise_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32,
+                                        i64, i64, i64, i64, vp]
+    lib.qknorm_headwise_fwd.restype = ctypes.c_int
     lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     lib.qknorm_xgamma.restype = ctypes.c_int
     lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
@@ -206,6 +209,34 @@ def qknorm_fwd_strided(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor,
                                 out_q.data_ptr(), out_k.data_ptr(), T, Dq, Dk, int(P), float(eps),
                                 _dtype_code(q), ldq, ldk, ldoq, ldok, _stream_handle(q.device, stream))
     _check("qknorm_fwd_strided", st)
+    return out_q, out_k
+
+
+def qknorm_headwise_fwd(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor,
+                        gamma_k: torch.Tensor, head_dim: int, eps: float,
+                        out_q: Optional[torch.Tensor] = None, out_k: Optional[torch.Tensor] = None,
+                        stream=None):
+    """Headwise QK-Norm: q [T, Hq*head_dim], k [T, Hk*head_dim] (rows may be
+    strided), gamma [head_dim] per tensor; one factor per head."""
+    T, Dq, ldq = _rows_view("q", q)
+    Tk, Dk, ldk = _rows_view("k", k)
+    if T != Tk or q.dtype != k.dtype or Dq % head_dim or Dk % head_dim:
+        raise ValueError("q and k must share T and dtype; widths must be multiples of head_dim")
+    out_q = torch.empty((T, Dq), dtype=q.dtype, device=q.device) if out_q is None else out_q
+    out_k = torch.empty((T, Dk), dtype=k.dtype, device=k.device) if out_k is None else out_k
+    _, Doq, ldoq = _rows_view("out_q", out_q)
+    _, Dok, ldok = _rows_view("out_k", out_k)
+    if (Doq, Dok) != (Dq, Dk) or out_q.dtype != q.dtype or out_k.dtype != k.dtype:
+        raise ValueError("outputs must match the inputs' widths and dtype")
+    for name, g in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        _need_cuda_contig(name, g)
+        if g.dtype != torch.float32 or g.numel() != head_dim:
+            raise ValueError(f"{name} must be float32 with head_dim elements")
+    st = lib.qknorm_headwise_fwd(q.data_ptr(), k.data_ptr(), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                                 out_q.data_ptr(), out_k.data_ptr(), T, Dq // head_dim,
+                                 Dk // head_dim, int(head_dim), float(eps), _dtype_code(q),
+                                 ldq, ldk, ldoq, ldok, _stream_handle(q.device, stream))
+    _check("qknorm_headwise_fwd", st)
     return out_q, out_k
 
 

@@ -462,7 +462,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 107; }
+int qknorm_version(void) { return 108; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -598,6 +598,74 @@ int qknorm_fwd(const void *q, const void *k, const float *gamma_q, const float *
                float eps, int32_t dtype, void *stream) {
     return qknorm_fwd_strided(q, k, gamma_q, gamma_k, out_q, out_k, T, Dq, Dk, P, eps, dtype, Dq, Dk,
                               Dq, Dk, stream);
+}
+
+int qknorm_headwise_fwd(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+                        void *out_q, void *out_k, int64_t T, int32_t Hq, int32_t Hk,
+                        int32_t head_dim, float eps, int32_t dtype, int64_t ldq, int64_t ldk,
+                        int64_t ldoq, int64_t ldok, void *stream) {
+    if (T < 0 || Hq <= 0 || Hk <= 0 || head_dim <= 0) return QKNORM_ERR_INVALID_ARG;
+    if (Hq > INT32_MAX / head_dim || Hk > INT32_MAX / head_dim) return QKNORM_ERR_INVALID_ARG;
+    const int32_t Dq = Hq * head_dim, Dk = Hk * head_dim;
+    int st = check_shape(T, Dq, Hq, dtype);
+    if (st == QKNORM_OK) st = check_shape(T, Dk, Hk, dtype);
+    if (st == QKNORM_OK) st = check_eps(eps);
+    if (st != QKNORM_OK) return st;
+    const int vec = vec_of(dtype);
+    const int nv = head_dim / vec;
+    if (nv > 256) return QKNORM_ERR_UNSUPPORTED;
+    if (ldq < Dq || ldk < Dk || ldoq < Dq || ldok < Dk) return QKNORM_ERR_INVALID_ARG;
+    if (ldq % vec || ldk % vec || ldoq % vec || ldok % vec) return QKNORM_ERR_MISALIGNED;
+    const int64_t es = elem_of(dtype);
+    int64_t ldmax = ldq;
+    if (ldk > ldmax) ldmax = ldk;
+    if (ldoq > ldmax) ldmax = ldoq;
+    if (ldok > ldmax) ldmax = ldok;
+    if (T > 0 && T > INT64_MAX / (ldmax * es)) return QKNORM_ERR_INVALID_ARG;
+    if (T == 0) return QKNORM_OK;
+    if (!q || !k || !gamma_q || !gamma_k || !out_q || !out_k) return QKNORM_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(gamma_q) || !aligned16(gamma_k) ||
+        !aligned16(out_q) || !aligned16(out_k))
+        return QKNORM_ERR_MISALIGNED;
+    const Strided mq = strided(q, Dq * es, ldq * es, T), mk = strided(k, Dk * es, ldk * es, T);
+    const Strided mgq = strided(gamma_q, (int64_t)head_dim * 4, (int64_t)head_dim * 4, 1);
+    const Strided mgk = strided(gamma_k, (int64_t)head_dim * 4, (int64_t)head_dim * 4, 1);
+    const Strided moq = strided(out_q, Dq * es, ldoq * es, T), mok = strided(out_k, Dk * es, ldok * es, T);
+    if (strided_bad_alias(moq, mq, true) || strided_bad_alias(moq, mk, false) ||
+        strided_bad_alias(moq, mgq, false) || strided_bad_alias(moq, mgk, false) ||
+        strided_bad_alias(moq, mok, false) || strided_bad_alias(mok, mk, true) ||
+        strided_bad_alias(mok, mq, false) || strided_bad_alias(mok, mgq, false) ||
+        strided_bad_alias(mok, mgk, false))
+        return QKNORM_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    cudaError_t e = device_sms(&dev, &sms);
+    if (e != cudaSuccess) return finish(e);
+    const void *fn = headwise_kernel(dtype, nv);
+    if (!fn) return QKNORM_ERR_UNSUPPORTED;
+    const int block = 256;
+    int bres = 1;
+    e = resident_blocks(dev, fn, block, 0, &bres);
+    if (e != cudaSuccess) return finish(e);
+    int64_t grid = (T + block / kLanes - 1) / (block / kLanes);
+    if (grid > (int64_t)sms * bres) grid = (int64_t)sms * bres;
+    HeadArgs a;
+    a.x[0] = q;
+    a.x[1] = k;
+    a.g[0] = gamma_q;
+    a.g[1] = gamma_k;
+    a.y[0] = out_q;
+    a.y[1] = out_k;
+    a.T = T;
+    a.H[0] = Hq;
+    a.H[1] = Hk;
+    a.nv = nv;
+    a.Df = (float)head_dim;
+    a.eps = eps;
+    a.ldx[0] = ldq / vec;
+    a.ldx[1] = ldk / vec;
+    a.ldy[0] = ldoq / vec;
+    a.ldy[1] = ldok / vec;
+    return finish(launch_headwise(dtype, a, block, grid, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qknorm_xgamma(const void *x, const float *gamma, void *out, int64_t T, int32_t D,

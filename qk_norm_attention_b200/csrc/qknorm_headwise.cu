@@ -1,0 +1,154 @@
+// qknorm_headwise.cu -- headwise QK-Norm: one factor per attention head.
+//
+// SwiftQK technical review, "Prerequisites" (layerwise vs. headwise QK-Norm)
+// and Section 4c's comparison table: headwise QK-Norm normalises each head
+// on its own, the reduction of Eq. (1) spanning one head's head_dim elements;
+// the weight gamma has head_dim entries shared by the heads.
+//
+// Per head: S = sum of squares in the library's reduction order with the
+// head as the only shard (lane chains over vectors lane + 32 i, butterfly),
+// r = rsqrt(S / head_dim + eps), y = (x * gamma) * r.
+//
+// One warp per token walks that token's Q heads, then its K heads, in units:
+// with head_dim <= 32 vectors a unit packs 32 / SEG heads into the warp, SEG
+// lanes per head (SEG the smallest power of two >= the head's vectors), and
+// the butterfly runs over each SEG-lane segment. That equals the 32-lane
+// butterfly bit for bit: the xor steps it skips would only add the exact
+// zeros of lanes past the head's last vector. Larger heads take a whole warp,
+// each lane holding VMAX vectors. R units' loads are issued before any is
+// reduced.
+#include "qknorm_device.cuh"
+#include "qknorm_internal.h"
+
+namespace qkn {
+
+template <int SEG>
+__device__ __forceinline__ float seg_butterfly(float c) {
+#pragma unroll
+    for (int off = SEG / 2; off >= 1; off /= 2) c = __fadd_rn(c, __shfl_xor_sync(kFull, c, off));
+    return c;
+}
+
+template <class Tag, int SEG, int VMAX, int R>
+__global__ void __launch_bounds__(256) headwise_k(const HeadArgs a) {
+    constexpr int VEC = Tag::kVec;
+    constexpr int HPW = 32 / SEG;  // heads per unit
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int slot = lane & (SEG - 1);
+    const int hsub = lane / SEG;
+    const int nv = a.nv;
+    const int64_t NW = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int Uq = (a.H[0] + HPW - 1) / HPW;
+    const int U = Uq + (a.H[1] + HPW - 1) / HPW;
+    // Small heads: this lane's gamma for both tensors stays in registers.
+    float gr[2][VMAX == 1 ? VEC : 1];
+    if (VMAX == 1 && slot < nv) {
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4) {
+                const float4 g4 = __ldg(reinterpret_cast<const float4 *>(a.g[z] + slot * VEC + e));
+                gr[z][e] = g4.x;
+                gr[z][e + 1] = g4.y;
+                gr[z][e + 2] = g4.z;
+                gr[z][e + 3] = g4.w;
+            }
+    }
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += NW) {
+        for (int u0 = 0; u0 < U; u0 += R) {
+            uint4 v[R][VMAX];
+            bool ok[R];
+            const uint4 *src[R];
+            uint4 *dst[R];
+            int zz[R];
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                const int u = u0 + j;
+                const int z = u < Uq ? 0 : 1;
+                const int head = (z ? u - Uq : u) * HPW + hsub;
+                ok[j] = u < U && head < (z ? a.H[1] : a.H[0]);
+                zz[j] = z;
+                const int64_t col = (int64_t)head * nv;
+                src[j] = reinterpret_cast<const uint4 *>(z ? a.x[1] : a.x[0]) + t * (z ? a.ldx[1] : a.ldx[0]) + col;
+                dst[j] = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) + col;
+#pragma unroll
+                for (int i = 0; i < VMAX; ++i) {
+                    const int vv = slot + 32 * i;
+                    if (ok[j] && vv < nv) v[j][i] = ld_stream(src[j] + vv);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                float c = 0.f;
+#pragma unroll
+                for (int i = 0; i < VMAX; ++i)
+                    if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
+                const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
+#pragma unroll
+                for (int i = 0; i < VMAX; ++i) {
+                    const int vv = slot + 32 * i;
+                    if (ok[j] && vv < nv) {
+                        uint4 y;
+                        if (VMAX == 1) {
+                            float gg[VEC];  // select, so the array stays in registers
+#pragma unroll
+                            for (int e = 0; e < VEC; ++e) gg[e] = zz[j] ? gr[1][e] : gr[0][e];
+                            y = vapply_regs(Tag{}, v[j][i], gg, r);
+                        } else
+                            y = vapply(Tag{}, v[j][i], (zz[j] ? a.g[1] : a.g[0]) + (int64_t)vv * VEC, r);
+                        st_stream(dst[j] + vv, y);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// Lanes per head for a head of nv vectors (nv <= 32), else 32.
+static int seg_of(int nv) {
+    int s = 1;
+    while (s < nv && s < 32) s *= 2;
+    return s;
+}
+
+template <class Tag>
+const void *headwise_table(int nv) {
+    if (nv <= 32) {
+        switch (seg_of(nv)) {
+        case 1: return reinterpret_cast<const void *>(&headwise_k<Tag, 1, 1, 4>);
+        case 2: return reinterpret_cast<const void *>(&headwise_k<Tag, 2, 1, 4>);
+        case 4: return reinterpret_cast<const void *>(&headwise_k<Tag, 4, 1, 4>);
+        case 8: return reinterpret_cast<const void *>(&headwise_k<Tag, 8, 1, 4>);
+        case 16: return reinterpret_cast<const void *>(&headwise_k<Tag, 16, 1, 4>);
+        default: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 1, 4>);
+        }
+    }
+    switch ((nv + 31) / 32) {
+    case 2: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 2, 4>);
+    case 3: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 3, 2>);
+    case 4: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 4, 2>);
+    case 5: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 5, 1>);
+    case 6: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 6, 1>);
+    case 7: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 7, 1>);
+    case 8: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 8, 1>);
+    default: return nullptr;
+    }
+}
+
+const void *headwise_kernel(int dtype, int nv) {
+    if (nv < 1 || nv > 256) return nullptr;
+    if (dtype == 0) return headwise_table<F32Tag>(nv);
+    if (dtype == 1) return headwise_table<BF16Tag>(nv);
+    return nullptr;
+}
+
+cudaError_t launch_headwise(int dtype, const HeadArgs &a, int block, int64_t grid, cudaStream_t s) {
+    const void *fn = headwise_kernel(dtype, a.nv);
+    if (!fn) return cudaErrorInvalidValue;
+    void *args[] = {const_cast<HeadArgs *>(&a)};
+    return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
+}
+
+}  // namespace qkn

@@ -75,6 +75,22 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stag
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
 cudaError_t read_device_errors(unsigned *out, bool clear);
 
+// Arguments of the headwise kernel; index 0 is Q, index 1 is K.
+struct HeadArgs {
+    const void *x[2];
+    const float *g[2];  // head_dim entries each, shared by the heads
+    void *y[2];
+    int64_t T;
+    int32_t H[2];       // heads
+    int32_t nv;         // 16-byte vectors per head
+    float Df;           // head_dim
+    float eps;
+    int64_t ldx[2];     // row strides, in 16-byte vectors
+    int64_t ldy[2];
+};
+const void *headwise_kernel(int dtype, int nv);
+cudaError_t launch_headwise(int dtype, const HeadArgs &a, int block, int64_t grid, cudaStream_t s);
+
 // The deferred-normalisation steps (qknorm_deferred.cu).
 const void *xgamma_kernel(int dtype);
 const void *inv_rms_kernel(int dtype);

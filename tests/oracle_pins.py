@@ -312,6 +312,37 @@ def pin_xgamma(orc):
         assert np.array_equal(orc.inv_rms(x, 4, 1e-6, dtype), r)
 
 
+def pin_headwise(orc):
+    """Headwise form (one factor per head, gamma of head_dim shared by the
+    heads): torch rms_norm over the last axis of [T, H, head_dim]; a one-hot
+    head; heads independent of one another; unit RMS per head at gamma = 1."""
+    import torch
+    T, H, hd = 3, 5, 64
+    x, _ = bf16_inputs(T, H * hd, seed=14)
+    g = W.gen_gamma(W.custom("hw", 1, hd, hd, 1, seed=15), "q")
+    x64 = widen(x, "bf16")
+    for eps in (1e-6, 0.5):
+        y = orc.headwise(x, g, hd, eps, "bf16")
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x64).view(T, H, hd), (hd,),
+                                           weight=torch.from_numpy(g.astype(np.float64)), eps=eps)
+        assert rel_err(y, ref.reshape(T, H * hd).numpy()) <= 4 * (hd + 8) * U53
+        ones = orc.headwise(x, np.ones(hd, np.float32), hd, eps, "bf16").reshape(T, H, hd)
+        m = (x64.reshape(T, H, hd) ** 2).mean(axis=2)
+        assert rel_err((ones ** 2).mean(axis=2), m / (m + eps)) <= 4 * (hd + 8) * U53
+    one = np.zeros((1, H * hd))
+    one[0, 2 * hd + 7] = 3.0
+    y = orc.headwise(W.to_storage(one, "bf16"), g, hd, 1e-6, "bf16")
+    want = np.zeros((1, H * hd))
+    want[0, 2 * hd + 7] = float(g[7]) * 3.0 / math.sqrt(9.0 / hd + 1e-6)
+    assert rel_err(y[0, 2 * hd + 7:2 * hd + 8], want[0, 2 * hd + 7:2 * hd + 8]) <= 8 * U53
+    assert np.count_nonzero(y) == 1
+    x2 = x.copy()
+    x2[:, 3 * hd:4 * hd] = W.to_storage(np.full((T, hd), 0.75), "bf16")
+    y1, y2 = orc.headwise(x, g, hd, 1e-6, "bf16"), orc.headwise(x2, g, hd, 1e-6, "bf16")
+    keep = np.r_[0:3 * hd, 4 * hd:H * hd]
+    assert np.array_equal(y1[:, keep], y2[:, keep])
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_shard_sums_exact,
@@ -325,4 +356,5 @@ ALL_PINS = [
     pin_deferred_prescale,
     pin_row_independence,
     pin_xgamma,
+    pin_headwise,
 ]

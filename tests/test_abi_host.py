@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 107
+    assert qk.qknorm_version() == 108
 
 
 # ----------------------------------------------------------------- argument checks
@@ -298,3 +298,25 @@ def test_strided_checks(qk):
     assert call(q, k, q, v) == 4                          # Dk-wide K output into the V slot: disjoint rows
     assert call(q, k, q + 16, k) == 1                     # Q output shifted into its own input
     assert call(q, k, E, F, ldoq=Dq, ldok=Dk, T=0) == 0
+
+
+@needs_cpu
+def test_headwise_checks(qk):
+    L = qk.lib
+
+    def call(Hq=8, Hk=2, hd=128, T=4, ldq=None, ldk=None, ldoq=None, ldok=None, q=A, k=B, oq=E, ok=F,
+             eps=1e-6, dtype=1):
+        ldq = ldq or Hq * hd
+        ldk = ldk or Hk * hd
+        return L.qknorm_headwise_fwd(q, k, C, Dd, oq, ok, T, Hq, Hk, hd, eps, dtype, ldq, ldk,
+                                     ldoq or Hq * hd, ldok or Hk * hd, None)
+
+    assert call() == 4                                  # valid: the runtime finds no device
+    assert call(Hq=0) == 1 and call(hd=0) == 1 and call(T=-1) == 1
+    assert call(hd=100) == 3                            # not a multiple of 8 bf16
+    assert call(hd=8 * 257) == 3                        # more than 256 vectors per head
+    assert call(ldq=8 * 128 - 8) == 1                   # stride below the width
+    assert call(ldq=8 * 128 + 4) == 2
+    assert call(eps=-1.0) == 1 and call(dtype=3) == 3
+    assert call(oq=B) == 1                              # output on the other input
+    assert call(T=0, q=0, k=0, oq=0, ok=0) == 0
