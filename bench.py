@@ -372,6 +372,34 @@ def deferred_steps(torch, qk, device, peak, steps=100):
     return out
 
 
+def fp8_prefill(torch, qk, device, peak, steps=200):
+    """The 13B-shaped prefill (T = 8192, Dq = Dk = 5120, P = 4) in FP8 E4M3:
+    E4M3 in and out, fp32 statistics; half the bytes of the bf16 step."""
+    wl = W.custom("fp8 prefill", 8192, 5120, 5120, 4, dtype="e4m3", seed=3, x_sigma=1.5)
+    T = 8192
+    stream = torch.cuda.current_stream(device)
+    q = W.gen_device_workload(wl, "q", T, device)
+    k = W.gen_device_workload(wl, "k", T, device)
+    gq = torch.from_numpy(W.gen_gamma(wl, "q")).to(device)
+    gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(device)
+    nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, 1)
+    n = buffer_sets(nbytes)
+    sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(n - 1)]
+    calls = [Fused(qk, (a, b, gq, gk, torch.empty_like(a), torch.empty_like(b)), T, wl.Dq, wl.Dk,
+                   wl.P, wl.eps, qk.QKNORM_E4M3, stream.cuda_stream) for a, b in sets]
+    for i in range(10):
+        calls[i % n]()
+    torch.cuda.synchronize()
+    tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
+    ms = tot / steps
+    plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, qk.QKNORM_E4M3)
+    return {"workload": "13B-shaped prefill in FP8 E4M3: T=8192, Dq=Dk=5120, P=4",
+            "us_per_call": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
+            "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1),
+            "tokens_per_s": round(T / ms * 1000, 1), "algorithmic_bytes": nbytes,
+            "kernel": KERNEL_OF_VARIANT.get(plan["variant"], "?")}
+
+
 def headwise(torch, qk, device, peak, steps=100):
     """Headwise QK-Norm: T = 8192 tokens, Hq = 32 and Hk = 8 heads of 128
     (bf16), gamma [128] per tensor, three rotating buffer sets."""
@@ -648,6 +676,7 @@ def run_native(args, dist):
         extras["split_large"] = split_path(torch, qk, device, peak)
         extras["deferred"] = deferred_steps(torch, qk, device, peak)
         extras["headwise"] = headwise(torch, qk, device, peak)
+        extras["fp8_prefill13b"] = fp8_prefill(torch, qk, device, peak)
     dist.barrier()
 
     traffic = None

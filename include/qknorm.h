@@ -24,14 +24,15 @@
  *   no state besides per-device caches of launch parameters.
  * - Tensors are dense row-major: x[T, D] (row t starts at x + t*D), gamma[D]
  *   fp32, stats[T, P] fp32 (row t holds S[t,0..P-1]).
- * - dtype selects the storage type of x and y: QKNORM_F32 or QKNORM_BF16.
- *   Accumulation and the factor are always fp32. y is rounded to nearest
- *   even from fp32, once.
+ * - dtype selects the storage type of x and y: QKNORM_F32, QKNORM_BF16 or
+ *   QKNORM_E4M3 (the FP8 activations of the review's Section 4 precision
+ *   study). Accumulation and the factor are always fp32. y is rounded to
+ *   nearest even from fp32, once.
  * - stream is a cudaStream_t (0 = legacy default stream). Calls only
  *   enqueue work; none synchronises the host.
  * - Every pointer must be 16-byte aligned, and the shard width D/P must be a
- *   multiple of 8 (bf16) or 4 (fp32) elements, so that every row and shard
- *   starts on a 16-byte vector.
+ *   multiple of 16 (E4M3), 8 (bf16) or 4 (fp32) elements, so that every row
+ *   and shard starts on a 16-byte vector.
  * - An output may be the same buffer as its own input (exact in-place); any
  *   other overlap between an output and any other buffer is rejected.
  * - T == 0 returns QKNORM_OK and launches nothing.
@@ -41,7 +42,7 @@
  *
  * Reduction order (identical in every kernel of this library, so the fused
  * path and the split path give bit-identical outputs): a shard of nv
- * 16-byte vectors (8 bf16 or 4 fp32 values) is covered by K = ceil(nv/256)
+ * 16-byte vectors (16 E4M3, 8 bf16 or 4 fp32 values) is covered by K = ceil(nv/256)
  * groups; group k, lane l (0..31) sums, in increasing i, the per-vector sums
  * of squares of vectors v = 32k + l + 32Ki; the 32 lane sums are combined by
  * an xor butterfly (16, 8, 4, 2, 1); the K group sums are added in order of
@@ -66,7 +67,9 @@ extern "C" {
 
 typedef enum {
     QKNORM_F32 = 0,
-    QKNORM_BF16 = 1
+    QKNORM_BF16 = 1,
+    QKNORM_E4M3 = 2   /* FP8 E4M3 (OCP "fn": max 448, no infinities); outputs are
+                         rounded to nearest even and saturate to +-448 */
 } qknorm_dtype;
 
 typedef enum {

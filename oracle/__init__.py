@@ -23,7 +23,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "qknorm_oracle.c")
 LIBRARY = os.path.join(_HERE, "liboracle.so")
 
-_DTYPE_CODE = {"f32": 0, "bf16": 1}
+_DTYPE_CODE = {"f32": 0, "bf16": 1, "e4m3": 2}
+_STORAGE = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8}
 
 
 def build(force: bool = False, source: str = SOURCE, output: str = LIBRARY) -> str:
@@ -60,7 +61,7 @@ class Oracle:
 
     @staticmethod
     def _prep(x: np.ndarray, dtype: str) -> np.ndarray:
-        want = np.float32 if dtype == "f32" else np.uint16
+        want = _STORAGE[dtype]
         if x.ndim != 2 or x.dtype != want:
             raise ValueError(f"x must be a 2-D {want.__name__} array for dtype {dtype}")
         return np.ascontiguousarray(x)

@@ -24,7 +24,8 @@
  *   S[t]   = sum_{p = 0}^{P-1} S[t,p]                  (in order of p)
  *   r[t]   = 1 / sqrt(S[t] / D + eps)
  *   y[t,j] = (x[t,j] * gamma[j]) * r[t]                (kept unrounded)
- * x is the stored input (fp32, or bf16 given as its 16-bit pattern), widened
+ * x is the stored input (fp32, bf16 given as its 16-bit pattern, or FP8 E4M3
+ * given as its 8-bit code), widened
  * exactly to double; gamma is fp32 widened exactly; eps is passed as the
  * double value the caller wants (the fp32 value the GPU receives, widened).
  *
@@ -38,12 +39,30 @@
 
 #define QKO_F32 0
 #define QKO_BF16 1
+#define QKO_E4M3 2
+
+/* Exact value of an FP8 E4M3 code (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits; no infinities; S.1111.111 is NaN). */
+static double qko_e4m3(uint8_t b)
+{
+    int sign = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);           /* subnormal: m/8 * 2^(1-7) */
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
 
 /* Exact widening of element i of a stored row to double. */
 static double qko_load(const void *x, int dtype, int64_t i)
 {
     if (dtype == QKO_F32)
         return (double)((const float *)x)[i];
+    if (dtype == QKO_E4M3)
+        return qko_e4m3(((const uint8_t *)x)[i]);
     uint32_t bits = (uint32_t)((const uint16_t *)x)[i] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -54,7 +73,7 @@ static int qko_check(const void *x, int dtype, int64_t T, int64_t D, int64_t P)
 {
     if (T < 0 || D <= 0 || P <= 0 || D % P != 0)
         return -1;
-    if (dtype != QKO_F32 && dtype != QKO_BF16)
+    if (dtype != QKO_F32 && dtype != QKO_BF16 && dtype != QKO_E4M3)
         return -1;
     if (T > 0 && x == NULL)
         return -1;
@@ -63,7 +82,7 @@ static int qko_check(const void *x, int dtype, int64_t T, int64_t D, int64_t P)
 
 static size_t qko_elem_size(int dtype)
 {
-    return dtype == QKO_F32 ? 4 : 2;
+    return dtype == QKO_F32 ? 4 : (dtype == QKO_BF16 ? 2 : 1);
 }
 
 /* Phase A: per-shard sums of squares of one row, S_row[p] for p < P. */

@@ -15,8 +15,8 @@ Entry points (same names as the C ABI):
 * ``qknorm_apply(x, gamma, stats, eps, out=None)``: the factor from stats and
   (x * gamma) * r.
 
-Tensors are CUDA tensors, row-major contiguous, fp32 or bf16 for x/y and fp32
-for gamma and stats. Calls are asynchronous on ``torch.cuda.current_stream()``
+Tensors are CUDA tensors, row-major contiguous, fp32, bf16 or FP8 E4M3
+(torch.float8_e4m3fn) for x/y and fp32 for gamma and stats. Calls are asynchronous on ``torch.cuda.current_stream()``
 (or the ``stream`` argument).
 """
 from __future__ import annotations
@@ -30,7 +30,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(_HERE, "libqknorm.so")
 
-QKNORM_F32, QKNORM_BF16 = 0, 1
+QKNORM_F32, QKNORM_BF16, QKNORM_E4M3 = 0, 1, 2
 QKNORM_OK = 0
 QKNORM_ERR_INVALID_ARG = 1
 QKNORM_ERR_MISALIGNED = 2
@@ -42,7 +42,8 @@ VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_
 VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic",
                  VARIANT_BULK: "bulk", VARIANT_ROWS: "rows"}
 
-_DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16}
+_DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16,
+          torch.float8_e4m3fn: QKNORM_E4M3}
 
 
 class QKNormError(RuntimeError):
@@ -138,7 +139,8 @@ def _stream_handle(device: torch.device, stream) -> int:
 
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype not in _DTYPE:
-        raise TypeError(f"unsupported dtype {t.dtype}; use torch.float32 or torch.bfloat16")
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.float32, torch.bfloat16 "
+                        "or torch.float8_e4m3fn")
     return _DTYPE[t.dtype]
 
 

@@ -45,8 +45,8 @@ void set_error(cudaError_t e) {
                   cudaGetErrorString(e));
 }
 
-int vec_of(int32_t dtype) { return dtype == QKNORM_BF16 ? 8 : 4; }
-int64_t elem_of(int32_t dtype) { return dtype == QKNORM_BF16 ? 2 : 4; }
+int vec_of(int32_t dtype) { return dtype == QKNORM_BF16 ? 8 : (dtype == QKNORM_E4M3 ? 16 : 4); }
+int64_t elem_of(int32_t dtype) { return dtype == QKNORM_BF16 ? 2 : (dtype == QKNORM_E4M3 ? 1 : 4); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -98,7 +98,7 @@ bool strided_bad_alias(const Strided &out, const Strided &in, bool may_alias) {
 int check_shape(int64_t T, int32_t D, int32_t P, int32_t dtype) {
     if (T < 0 || D <= 0 || P <= 0) return QKNORM_ERR_INVALID_ARG;
     if (D % P != 0) return QKNORM_ERR_INVALID_ARG;
-    if (dtype != QKNORM_F32 && dtype != QKNORM_BF16) return QKNORM_ERR_UNSUPPORTED;
+    if (dtype != QKNORM_F32 && dtype != QKNORM_BF16 && dtype != QKNORM_E4M3) return QKNORM_ERR_UNSUPPORTED;
     if ((D / P) % vec_of(dtype) != 0) return QKNORM_ERR_UNSUPPORTED;
     if (T > 0 && T > INT64_MAX / ((int64_t)D * elem_of(dtype))) return QKNORM_ERR_INVALID_ARG;
     return QKNORM_OK;
@@ -462,7 +462,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 108; }
+int qknorm_version(void) { return 109; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {

@@ -100,12 +100,14 @@ __global__ void __launch_bounds__(256) inv_rms_k(const void *x, float *r, int64_
 const void *xgamma_kernel(int dtype) {
     if (dtype == 0) return reinterpret_cast<const void *>(&xgamma_k<F32Tag>);
     if (dtype == 1) return reinterpret_cast<const void *>(&xgamma_k<BF16Tag>);
+    if (dtype == 2) return reinterpret_cast<const void *>(&xgamma_k<E4M3Tag>);
     return nullptr;
 }
 
 const void *inv_rms_kernel(int dtype) {
     if (dtype == 0) return reinterpret_cast<const void *>(&inv_rms_k<F32Tag>);
     if (dtype == 1) return reinterpret_cast<const void *>(&inv_rms_k<BF16Tag>);
+    if (dtype == 2) return reinterpret_cast<const void *>(&inv_rms_k<E4M3Tag>);
     return nullptr;
 }
 

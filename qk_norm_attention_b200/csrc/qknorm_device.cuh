@@ -10,6 +10,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,11 +28,41 @@ struct BF16Tag {
     static constexpr int kVec = 8;  // bf16 values per 16-byte vector
     static constexpr int kBytes = 2;
 };
+struct E4M3Tag {
+    static constexpr int kVec = 16;  // FP8 E4M3 values per 16-byte vector
+    static constexpr int kBytes = 1;
+};
 
 // ---------------------------------------------------------------- widening
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two FP8 E4M3 values (the low byte first) widened exactly to fp32.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+
+// The 16 values of a 16-byte FP8 vector as 8 float pairs, element 0 first.
+__device__ __forceinline__ void e4m3x16_to_float(const uint4 &v, float (&f)[16]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = e4m3x2_to_float2(w[i]);
+        const float2 b = e4m3x2_to_float2(w[i] >> 16);
+        f[4 * i] = a.x;
+        f[4 * i + 1] = a.y;
+        f[4 * i + 2] = b.x;
+        f[4 * i + 3] = b.y;
+    }
+}
+
+// Two fp32 values to FP8 E4M3 (round to nearest even, saturating to +-448),
+// the first in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
 
 // ---------------------------------------------------------------- Phase A: x^2
 
@@ -57,6 +88,16 @@ __device__ __forceinline__ float vsumsq(BF16Tag, const uint4 &v) {
     q = __fmaf_rn(bf_hi(v.z), bf_hi(v.z), q);
     q = __fmaf_rn(bf_lo(v.w), bf_lo(v.w), q);
     q = __fmaf_rn(bf_hi(v.w), bf_hi(v.w), q);
+    return q;
+}
+
+// Same for 16 FP8 values (an E4M3 square is exact in fp32).
+__device__ __forceinline__ float vsumsq(E4M3Tag, const uint4 &v) {
+    float f[16];
+    e4m3x16_to_float(v, f);
+    float q = __fmul_rn(f[0], f[0]);
+#pragma unroll
+    for (int i = 1; i < 16; ++i) q = __fmaf_rn(f[i], f[i], q);
     return q;
 }
 
@@ -132,6 +173,21 @@ __device__ __forceinline__ uint4 vapply(BF16Tag, const uint4 &v, const float *g,
     return o;
 }
 
+__device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r);
+
+__device__ __forceinline__ uint4 vapply(E4M3Tag, const uint4 &v, const float *g, float r) {
+    float gg[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g) + i);
+        gg[4 * i] = g4.x;
+        gg[4 * i + 1] = g4.y;
+        gg[4 * i + 2] = g4.z;
+        gg[4 * i + 3] = g4.w;
+    }
+    return vapply_regs(E4M3Tag{}, v, gg, r);
+}
+
 // Same as vapply with gamma already in registers (g[0..vec-1], indexed with
 // compile-time constants after unrolling).
 __device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float *g, float r) {
@@ -141,6 +197,17 @@ __device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float
     o.z = __float_as_uint(wmul(__uint_as_float(v.z), g[2], r));
     o.w = __float_as_uint(wmul(__uint_as_float(v.w), g[3], r));
     return o;
+}
+
+__device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r) {
+    float f[16];
+    e4m3x16_to_float(v, f);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = pack_e4m3x2(wmul(f[4 * i], g[4 * i], r), wmul(f[4 * i + 1], g[4 * i + 1], r)) |
+               (pack_e4m3x2(wmul(f[4 * i + 2], g[4 * i + 2], r), wmul(f[4 * i + 3], g[4 * i + 3], r)) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r) {
@@ -174,6 +241,25 @@ __device__ __forceinline__ uint4 vxgamma(BF16Tag, const uint4 &v, const float *g
     return o;
 }
 
+__device__ __forceinline__ uint4 vxgamma(E4M3Tag, const uint4 &v, const float *g) {
+    float f[16], gg[16];
+    e4m3x16_to_float(v, f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g) + i);
+        gg[4 * i] = g4.x;
+        gg[4 * i + 1] = g4.y;
+        gg[4 * i + 2] = g4.z;
+        gg[4 * i + 3] = g4.w;
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = pack_e4m3x2(__fmul_rn(f[4 * i], gg[4 * i]), __fmul_rn(f[4 * i + 1], gg[4 * i + 1])) |
+               (pack_e4m3x2(__fmul_rn(f[4 * i + 2], gg[4 * i + 2]), __fmul_rn(f[4 * i + 3], gg[4 * i + 3])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Same as vapply with gamma read through an arbitrary pointer (used with
 // gamma staged in shared memory); same arithmetic, bit for bit.
 __device__ __forceinline__ uint4 vapply_ptr(F32Tag, const uint4 &v, const float *g, float r) {
@@ -200,6 +286,19 @@ __device__ __forceinline__ uint4 vapply_ptr(BF16Tag, const uint4 &v, const float
 // own pdl_wait() still orders its memory accesses after this kernel's.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::); }
+
+__device__ __forceinline__ uint4 vapply_ptr(E4M3Tag, const uint4 &v, const float *g, float r) {
+    float gg[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 g4 = *(reinterpret_cast<const float4 *>(g) + i);
+        gg[4 * i] = g4.x;
+        gg[4 * i + 1] = g4.y;
+        gg[4 * i + 2] = g4.z;
+        gg[4 * i + 3] = g4.w;
+    }
+    return vapply_regs(E4M3Tag{}, v, gg, r);
+}
 
 // ---------------------------------------------------------------- memory
 

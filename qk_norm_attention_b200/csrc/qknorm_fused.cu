@@ -167,11 +167,19 @@ __global__ void __launch_bounds__(256, 1) fused_generic(const FusedArgs a) {
 
 // ---------------------------------------------------------------- instance tables
 
-constexpr int cta_max_threads(int vmax) { return vmax <= 2 ? 1024 : 512; }
+// 1024-thread instances only while a lane holds <= 16 values (64 registers).
+constexpr int cta_max_threads(int vmax, int vec) { return (vmax <= 2 && vmax * vec <= 16) ? 1024 : 512; }
+// Register-resident instances exist up to 8 vectors per lane (4 for FP8,
+// whose 16 values per vector take twice the registers of bf16 once widened).
+constexpr bool cta_exists(int vmax, int vec) { return vmax >= 1 && vmax <= (vec == 16 ? 4 : kVcap); }
 
 template <class Tag, int VMAX, bool PF, bool FULL>
 const void *cta_fn() {
-    return reinterpret_cast<const void *>(&fused_cta<Tag, VMAX, PF, FULL, cta_max_threads(VMAX)>);
+    if constexpr (cta_exists(VMAX, Tag::kVec))
+        return reinterpret_cast<const void *>(
+            &fused_cta<Tag, VMAX, PF, FULL, cta_max_threads(VMAX, Tag::kVec)>);
+    else
+        return nullptr;
 }
 
 template <class Tag, bool PF, bool FULL>
@@ -196,16 +204,19 @@ const void *cta_pick(int vmax, bool prefetch, bool full) {
 }
 
 const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads) {
-    if (vmax < 1 || vmax > kVcap) return nullptr;
-    if (max_threads) *max_threads = cta_max_threads(vmax);
+    const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
+    if (!cta_exists(vmax, vec)) return nullptr;
+    if (max_threads) *max_threads = cta_max_threads(vmax, vec);
     if (dtype == 0) return cta_pick<F32Tag>(vmax, prefetch, full);
     if (dtype == 1) return cta_pick<BF16Tag>(vmax, prefetch, full);
+    if (dtype == 2) return cta_pick<E4M3Tag>(vmax, prefetch, full);
     return nullptr;
 }
 
 const void *fused_generic_kernel(int dtype) {
     if (dtype == 0) return reinterpret_cast<const void *>(&fused_generic<F32Tag>);
     if (dtype == 1) return reinterpret_cast<const void *>(&fused_generic<BF16Tag>);
+    if (dtype == 2) return reinterpret_cast<const void *>(&fused_generic<E4M3Tag>);
     return nullptr;
 }
 

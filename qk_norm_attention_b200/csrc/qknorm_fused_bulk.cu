@@ -398,17 +398,22 @@ __global__ void bounded_wait_probe(uint64_t timeout_ns) {
 
 // ---------------------------------------------------------------- instances and launch
 
-// Combinations that exist: TB (1 or 2) tokens x VMAX vectors per lane <= 12.
-constexpr bool bulk_exists(int vmax, int tb) {
-    return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12;
+// Combinations that exist: TB (1 or 2) tokens x VMAX vectors per lane <= 12;
+// for FP8 (16 values per vector) one token, <= 4 vectors, gamma in registers
+// only up to 2 vectors, so that no instance spills.
+constexpr bool bulk_exists(int vmax, int tb, int vec, bool greg) {
+    return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12 &&
+           (vec != 16 || (tb == 1 && vmax <= 4 && (!greg || vmax <= 2)));
 }
-constexpr int bulk_max_threads(int vmax, int tb) { return vmax * tb <= 2 ? 1024 : 512; }
+constexpr int bulk_max_threads(int vmax, int tb, int vec) {
+    return (vmax * tb <= 2 && vmax * tb * vec <= 16) ? 1024 : 512;
+}
 
 template <class Tag, bool GREG, int V, int TB, bool FULL>
 const void *bulk_fn() {
-    if constexpr (bulk_exists(V, TB))
+    if constexpr (bulk_exists(V, TB, Tag::kVec, GREG))
         return reinterpret_cast<const void *>(
-            &fused_bulk<Tag, V, GREG, TB, FULL, bulk_max_threads(V, TB)>);
+            &fused_bulk<Tag, V, GREG, TB, FULL, bulk_max_threads(V, TB, Tag::kVec)>);
     else
         return nullptr;
 }
@@ -437,12 +442,15 @@ const void *bulk_table(int vmax, int tb, bool full) {
 
 const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, bool full,
                               int *max_threads) {
-    if (!bulk_exists(vmax, tb)) return nullptr;
-    if (max_threads) *max_threads = bulk_max_threads(vmax, tb);
+    const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
+    if (!bulk_exists(vmax, tb, vec, gamma_regs)) return nullptr;
+    if (max_threads) *max_threads = bulk_max_threads(vmax, tb, vec);
     if (dtype == 0)
         return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb, full) : bulk_table<F32Tag, false>(vmax, tb, full);
     if (dtype == 1)
         return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb, full) : bulk_table<BF16Tag, false>(vmax, tb, full);
+    if (dtype == 2)
+        return gamma_regs ? bulk_table<E4M3Tag, true>(vmax, tb, full) : bulk_table<E4M3Tag, false>(vmax, tb, full);
     return nullptr;
 }
 
@@ -461,7 +469,7 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool
                               uint64_t timeout_ns, cudaStream_t s) {
     const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, full, nullptr);
     if (!fn || stages < 1 || stages > (int)kMaxStages) return cudaErrorInvalidValue;
-    const int64_t es = dtype == 1 ? 2 : 4;
+    const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
     BulkArgs b;
     b.stages = (uint32_t)stages;
     b.qbytes = (uint32_t)(a.D[0] * es);
@@ -476,6 +484,7 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool
 const void *fused_rows_kernel(int dtype) {
     if (dtype == 0) return reinterpret_cast<const void *>(&fused_rows<F32Tag>);
     if (dtype == 1) return reinterpret_cast<const void *>(&fused_rows<BF16Tag>);
+    if (dtype == 2) return reinterpret_cast<const void *>(&fused_rows<E4M3Tag>);
     return nullptr;
 }
 
@@ -496,7 +505,7 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stag
                               uint64_t timeout_ns, cudaStream_t s) {
     const void *fn = fused_rows_kernel(dtype);
     if (!fn || warps < 1 || warps > 16 || stages < 1) return cudaErrorInvalidValue;
-    const RowsLayout L = rows_layout(a.D[0], a.D[1], dtype == 1 ? 2 : 4, warps, stages);
+    const RowsLayout L = rows_layout(a.D[0], a.D[1], dtype == 1 ? 2 : (dtype == 2 ? 1 : 4), warps, stages);
     RowsArgs b;
     b.stages = (uint32_t)stages;
     b.stage_bytes = L.stage_bytes;

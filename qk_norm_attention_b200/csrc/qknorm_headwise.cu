@@ -141,6 +141,7 @@ const void *headwise_kernel(int dtype, int nv) {
     if (nv < 1 || nv > 256) return nullptr;
     if (dtype == 0) return headwise_table<F32Tag>(nv);
     if (dtype == 1) return headwise_table<BF16Tag>(nv);
+    if (dtype == 2) return headwise_table<E4M3Tag>(nv);
     return nullptr;
 }
 

@@ -137,12 +137,14 @@ const void *stats_table(int vmax) {
 const void *stats_kernel(int dtype, int vmax) {
     if (dtype == 0) return stats_table<F32Tag>(vmax);
     if (dtype == 1) return stats_table<BF16Tag>(vmax);
+    if (dtype == 2) return stats_table<E4M3Tag>(vmax);
     return nullptr;
 }
 
 const void *apply_kernel(int dtype) {
     if (dtype == 0) return reinterpret_cast<const void *>(&apply_k<F32Tag>);
     if (dtype == 1) return reinterpret_cast<const void *>(&apply_k<BF16Tag>);
+    if (dtype == 2) return reinterpret_cast<const void *>(&apply_k<E4M3Tag>);
     return nullptr;
 }
 

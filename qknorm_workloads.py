@@ -38,7 +38,21 @@ SCALE_KEY = 1_000_033
 GAMMA_KEY = 1_000_037
 TENSOR_CODE = {"q": 11, "k": 13}
 
-DTYPE_BYTES = {"f32": 4, "bf16": 2}
+DTYPE_BYTES = {"f32": 4, "bf16": 2, "e4m3": 1}
+
+
+def _e4m3_table():
+    """The 253 distinct finite FP8 E4M3 values (+0 only), ascending, and their codes."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F and c != 0x80], dtype=np.uint8)
+    e = (codes.astype(np.int64) >> 3) & 15
+    m = codes.astype(np.int64) & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1 + m / 8.0) * 2.0 ** (e - 7))
+    vals = np.where(codes >> 7, -mag, mag)
+    order = np.argsort(vals, kind="stable")
+    return vals[order], codes[order]
+
+
+_E4M3_VALS, _E4M3_CODES = _e4m3_table()
 
 
 @dataclass(frozen=True)
@@ -102,6 +116,8 @@ def to_storage(x64: np.ndarray, dtype: str) -> np.ndarray:
     fp32: round-to-nearest-even. bf16: fp32 first, then round-to-nearest-even
     on the low 16 bits; the result is the uint16 bit pattern. Finite inputs only.
     """
+    if dtype == "e4m3":
+        return _to_e4m3(np.ascontiguousarray(x64, dtype=np.float64))
     f32 = np.ascontiguousarray(x64, dtype=np.float64).astype(np.float32)
     if dtype == "f32":
         return f32
@@ -116,10 +132,29 @@ def to_storage(x64: np.ndarray, dtype: str) -> np.ndarray:
     return bits.astype(np.uint16)
 
 
+def _to_e4m3(x: np.ndarray) -> np.ndarray:
+    """float64 -> FP8 E4M3 codes: round to nearest, ties to the even code
+    (mantissa LSB 0), saturating to +-448 (finite inputs only)."""
+    v, c = _E4M3_VALS, _E4M3_CODES
+    xc = np.clip(x, v[0], v[-1])
+    hi = np.clip(np.searchsorted(v, xc, side="left"), 1, len(v) - 1)
+    lo = hi - 1
+    dlo, dhi = xc - v[lo], v[hi] - xc
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & ((c[hi] & 1) == 0))
+    out = np.where(pick_hi, c[hi], c[lo]).astype(np.uint8)
+    out[x == 0] = 0
+    return out
+
+
 def storage_to_f64(s: np.ndarray, dtype: str) -> np.ndarray:
     """Exact widening of stored values to float64 (bf16 bits -> fp32 -> f64)."""
     if dtype == "f32":
         return s.astype(np.float64)
+    if dtype == "e4m3":
+        e = (s.astype(np.int64) >> 3) & 15
+        m = s.astype(np.int64) & 7
+        mag = np.where(e == 0, m * 2.0 ** -9, (1 + m / 8.0) * 2.0 ** (e - 7))
+        return np.where(s >> 7, -mag, mag)
     bits = s.astype(np.uint32) << 16
     return bits.view(np.float32).astype(np.float64)
 
@@ -175,7 +210,7 @@ def gen_rows(wl: Workload, tensor: str, rows: Sequence[int]) -> np.ndarray:
 def gen_tensor(wl: Workload, tensor: str, T: int) -> np.ndarray:
     """All T rows of Q or K in storage form, [T, D]."""
     D = wl.Dq if tensor == "q" else wl.Dk
-    dt = np.float32 if wl.dtype == "f32" else np.uint16
+    dt = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8}[wl.dtype]
     out = np.empty((T, D), dtype=dt)
     for start in range(0, T, ROW_BLOCK):
         stop = min(T, start + ROW_BLOCK)
@@ -243,7 +278,7 @@ def gen_device_workload(wl: Workload, tensor: str, T: int, device, row0: int = 0
     serves timing runs, where drawing on the host would take too long."""
     import torch
     D = wl.Dq if tensor == "q" else wl.Dk
-    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    tdt = {"bf16": torch.bfloat16, "f32": torch.float32, "e4m3": torch.float8_e4m3fn}[wl.dtype]
     gen = torch.Generator(device=device)
     gen.manual_seed(wl.seed * 1_000_003 + TENSOR_CODE[tensor] * 7919 + row0)
     sgen = torch.Generator(device=device)

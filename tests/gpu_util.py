@@ -9,6 +9,9 @@ Tolerances
   half an ulp, 2^-9 relative) and the fp32 work before it adds ~1e-6, so the
   bound has a 4x margin.
 * fp32 outputs: |y - y_oracle| <= 1e-5 |y_oracle|, and y_oracle = 0 gives 0.
+* FP8 E4M3 outputs: |y - y_oracle| <= 2^-3 |y_oracle| + 2^-9. Rounding to
+  nearest costs at most 2^-4 relative on normals (3 mantissa bits) and 2^-10
+  absolute on subnormals (quantum 2^-9), so the bound has a 2x margin.
 * fp32 shard sums: all terms are non-negative, so the relative error of a
   sum formed by a tree of depth n is at most n u / (1 - n u), u = 2^-24. A
   term passes through vec - 1 fma roundings, at most vmax chain additions,
@@ -23,7 +26,9 @@ U24 = 2.0 ** -24
 
 
 def to_device(a: np.ndarray, device="cuda") -> torch.Tensor:
-    """Stored values (fp32, or bf16 bits as uint16) -> CUDA tensor of that dtype."""
+    """Stored values (fp32, bf16 bits as uint16, E4M3 codes as uint8) -> CUDA tensor."""
+    if a.dtype == np.uint8:
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e4m3fn).to(device)
     if a.dtype == np.uint16:
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
@@ -32,6 +37,8 @@ def to_device(a: np.ndarray, device="cuda") -> torch.Tensor:
 def to_host(t: torch.Tensor) -> np.ndarray:
     """CUDA tensor -> stored values (fp32 array, or bf16 bits as uint16)."""
     t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
     return t.numpy()
@@ -39,17 +46,20 @@ def to_host(t: torch.Tensor) -> np.ndarray:
 
 def bits(t: torch.Tensor) -> torch.Tensor:
     """The raw bit patterns of a tensor (for bit-for-bit comparisons)."""
-    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+    return t.view({1: torch.uint8, 2: torch.int16, 4: torch.int32}[t.element_size()])
 
 
 def widen(a: np.ndarray) -> np.ndarray:
+    if a.dtype == np.uint8:
+        import qknorm_workloads
+        return qknorm_workloads.storage_to_f64(a, "e4m3")
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return a.astype(np.float64)
 
 
 def rtol_of(dtype: str) -> float:
-    return 2.0 ** -7 if dtype == "bf16" else 1e-5
+    return {"bf16": 2.0 ** -7, "e4m3": 2.0 ** -3}.get(dtype, 1e-5)
 
 
 def check_outputs(y_dev_stored: np.ndarray, y_oracle: np.ndarray, dtype: str, what: str = ""):
@@ -58,6 +68,11 @@ def check_outputs(y_dev_stored: np.ndarray, y_oracle: np.ndarray, dtype: str, wh
     diff = np.abs(y - y_oracle)
     if dtype == "bf16":
         bound = 2.0 ** -7 * np.abs(y_oracle) + 2.0 ** -133
+    elif dtype == "e4m3":
+        # One E4M3 ulp of relative error (3 mantissa bits), and the smallest
+        # subnormal 2^-9 as the absolute floor; outputs must be inside +-448.
+        assert np.abs(y_oracle).max() < 448, "outputs beyond the E4M3 range"
+        bound = 2.0 ** -3 * np.abs(y_oracle) + 2.0 ** -9
     else:
         bound = 1e-5 * np.abs(y_oracle)
     bad = diff > bound
@@ -83,7 +98,7 @@ def rne_bf16(y64: np.ndarray) -> np.ndarray:
 
 
 def stats_depth(D: int, P: int, dtype: str) -> int:
-    vec = 8 if dtype == "bf16" else 4
+    vec = {"bf16": 8, "e4m3": 16}.get(dtype, 4)
     nv = D // P // vec
     K = max(1, -(-nv // 256))
     vmax = -(-nv // (32 * K))

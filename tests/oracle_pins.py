@@ -54,6 +54,7 @@ def widen(x, dtype):
     return W.storage_to_f64(x, dtype)
 
 
+
 def exact_shard_sums(row64, P):
     """Exact Fraction sum of squares of each shard of one widened row."""
     D = len(row64)
@@ -343,6 +344,43 @@ def pin_headwise(orc):
     assert np.array_equal(y1[:, keep], y2[:, keep])
 
 
+def e4m3_inputs(T, D, seed, sigma=1.0):
+    wl = W.custom("pin8", T, D, D, 1, dtype="e4m3", seed=seed, x_sigma=sigma)
+    return W.gen_rows(wl, "q", range(T)), W.gen_gamma(wl, "q")
+
+
+def pin_e4m3(orc):
+    """FP8 E4M3 storage: codes fixed by the format (1.0 = 0x38, 448 = 0x7E,
+    2^-9 = 0x01 the smallest subnormal, 2^-6 = 0x08 the smallest normal,
+    -2 = 0xC0) widen exactly; torch's own float8_e4m3fn widening agrees on
+    every finite code; RMSNorm of FP8 rows matches torch rms_norm and exact
+    rational arithmetic."""
+    import torch
+    known = {0x38: 1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x08: 2.0 ** -6, 0xC0: -2.0, 0x00: 0.0}
+    for code, val in known.items():
+        x = np.zeros((1, 16), np.uint8)
+        x[0, 3] = code
+        S = orc.partial_sumsq(x, 1, "e4m3")[0, 0]
+        assert S == val * val, (hex(code), S)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    x = np.tile(codes[:, None], (1, 16))
+    g1 = np.ones(16, np.float32)
+    u = orc.xgamma(x, g1, "e4m3")
+    assert np.array_equal(u[:, 0], ref)
+    for xs, g in (e4m3_inputs(6, 512, seed=16), e4m3_inputs(4, 48, seed=17, sigma=40.0)):
+        x64 = widen(xs, "e4m3")
+        D = xs.shape[1]
+        for P in (1, 2, 4):
+            y, r = orc.rmsnorm(xs, g, P, 1e-6, "e4m3")
+            t = torch.nn.functional.rms_norm(torch.from_numpy(x64), (D,),
+                                             weight=torch.from_numpy(g.astype(np.float64)), eps=1e-6)
+            assert rel_err(y, t.numpy()) <= 4 * (D + 8) * U53
+        for t in range(xs.shape[0]):
+            ye, re = exact_y(x64[t], g, 1e-6)
+            assert rel_err(y[t], ye) <= (D + 8) * U53
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_shard_sums_exact,
@@ -357,4 +395,5 @@ ALL_PINS = [
     pin_row_independence,
     pin_xgamma,
     pin_headwise,
+    pin_e4m3,
 ]

@@ -46,7 +46,7 @@ def test_status_strings(qk):
     for s in range(1, 5):
         assert qk.qknorm_status_string(s) not in ("ok", "unknown status")
     assert qk.qknorm_status_string(99) == "unknown status"
-    assert qk.qknorm_version() == 108
+    assert qk.qknorm_version() // 100 == 1          # ABI major version
 
 
 # ----------------------------------------------------------------- argument checks
@@ -73,7 +73,8 @@ def fwd(qk, q=A, k=B, gq=C, gk=Dd, oq=E, ok=F, T=4, Dq=256, Dk=256, P=2, eps=1e-
     (dict(Dq=250, P=4), 1),                    # D % P != 0
     (dict(eps=-1e-6), 1), (dict(eps=math.nan), 1), (dict(eps=math.inf), 1),
     (dict(q=0), 1), (dict(k=0), 1), (dict(gq=0), 1), (dict(gk=0), 1), (dict(oq=0), 1), (dict(ok=0), 1),
-    (dict(dtype=2), 3), (dict(dtype=-1), 3),
+    (dict(dtype=3), 3), (dict(dtype=-1), 3),
+    (dict(Dq=48, Dk=48, P=2, dtype=2), 3),     # 24-wide FP8 shards (need multiples of 16)
     (dict(Dq=40, Dk=40, P=2, dtype=1), 3),     # 20-wide bf16 shards
     (dict(Dq=24, Dk=24, P=4, dtype=0), 3),     # 6-wide fp32 shards
     (dict(q=A + 2), 2), (dict(k=B + 8), 2), (dict(gq=C + 4), 2), (dict(gk=Dd + 12), 2),

@@ -46,6 +46,10 @@ MUTANTS = {
     # bf16 sign bit lost.
     "bf16_sign": [("(uint32_t)((const uint16_t *)x)[i] << 16;",
                    "((uint32_t)((const uint16_t *)x)[i] & 0x7fffu) << 16;")],
+    # FP8 exponent bias off by one.
+    "e4m3_bias": [("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)")],
+    # FP8 subnormals scaled like normals.
+    "e4m3_subnormal": [("ldexp((double)m, -9)", "ldexp((double)m, -10)")],
     # Outputs written to the first row only.
     "y_row_stride": [("y[t * D + j] = u * rt;", "y[j] = u * rt;")],
 }
