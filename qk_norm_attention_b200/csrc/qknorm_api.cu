@@ -205,6 +205,9 @@ bool full_lanes(const Shapes &sh) {
 // occupancy and gamma hits L1 anyway).
 bool gamma_regs_for(int32_t dtype, int vmax) {
     if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
+    // FP8 pays four 16-byte gamma loads per vector otherwise (measured: +80 %
+    // at 2 vectors per lane), so it keeps gamma in registers while it can.
+    if (dtype == QKNORM_E4M3) return vmax <= 3;
     return vmax * vec_of(dtype) <= 24;
 }
 
@@ -272,8 +275,9 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     pl->full_lanes = full_lanes(sh) ? 1 : 0;
     const bool cta_ok = sh.ntask * kLanes <= cta_max;
     const int tb = tokens_per_stage_for(sh.vmax);
+    const bool greg = gamma_regs_for(dtype, sh.vmax);
     int bulk_max = 0;
-    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, true, tb, false, &bulk_max) != nullptr;
+    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, greg, tb, false, &bulk_max) != nullptr;
     const uint32_t stride = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
                                               (int64_t)Dk * elem_of(dtype), tb);
     const bool bulk_ok = bulk_inst && sh.ntask * kLanes <= bulk_max &&
@@ -286,7 +290,9 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         // lanes (e.g. GQA widths) its CTA carries idle lanes and unequal Q/K
         // warps, and the warp-per-row kernel wins. Shapes whose tasks do not
         // fit one CTA go to the rows kernel too.
-        const bool ragged = !pl->full_lanes;
+        // FP8 is instruction-bound, and the token ring with gamma in registers
+        // wins for it even on ragged lanes (measured 63 % vs 46 % for rows).
+        const bool ragged = !pl->full_lanes && dtype != QKNORM_E4M3;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
         else if (bulk_ok && !(ragged && rows_ok))
@@ -302,7 +308,7 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         pl->block = (int32_t)(sh.ntask * kLanes);
         pl->vmax = sh.vmax;
         if (variant == QKNORM_VARIANT_BULK) {
-            pl->gamma_regs = gamma_regs_for(dtype, sh.vmax) ? 1 : 0;
+            pl->gamma_regs = greg ? 1 : 0;
             pl->tokens_per_stage = tb;
             bulk_stages(stride, pl->block, regs > 0 ? regs : kRegsHint, pl);
             if (pl->stages < 1 || pl->stages > bulk_max_stages() ||

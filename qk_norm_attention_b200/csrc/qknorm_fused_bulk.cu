@@ -400,10 +400,10 @@ __global__ void bounded_wait_probe(uint64_t timeout_ns) {
 
 // Combinations that exist: TB (1 or 2) tokens x VMAX vectors per lane <= 12;
 // for FP8 (16 values per vector) one token, <= 4 vectors, gamma in registers
-// only up to 2 vectors, so that no instance spills.
+// only up to 3 vectors, so that no instance spills.
 constexpr bool bulk_exists(int vmax, int tb, int vec, bool greg) {
     return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12 &&
-           (vec != 16 || (tb == 1 && vmax <= 4 && (!greg || vmax <= 2)));
+           (vec != 16 || (tb == 1 && vmax <= 4 && (!greg || vmax <= 3)));
 }
 constexpr int bulk_max_threads(int vmax, int tb, int vec) {
     return (vmax * tb <= 2 && vmax * tb * vec <= 16) ? 1024 : 512;
