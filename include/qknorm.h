@@ -197,6 +197,31 @@ QKNORM_API int qknorm_xgamma(const void *x, const float *gamma, void *out, int64
 QKNORM_API int qknorm_inv_rms(const void *x, float *inv_rms, int64_t T, int32_t D, int32_t P,
                               float eps, int32_t dtype, void *stream);
 
+/*
+ * qknorm_split_noalloc -- qknorm_partial_sumsq followed by qknorm_apply in one
+ * call, with the [T, P] statistics kept in a buffer inside the library, so
+ * that the caller allocates nothing (no counterpart in the paper; it is a
+ * convenience for callers who cannot allocate device memory, e.g. because all
+ * device memory belongs to a framework's pool, or because cudaMalloc's
+ * implicit synchronisation is unacceptable in their loop).
+ *
+ * Arguments, layouts, checks and results are those of the two calls it
+ * makes; out equals qknorm_fwd's output for that tensor bit for bit.
+ * The library holds one buffer of qknorm_split_noalloc_max_stats() floats
+ * (2^20, 4 MiB) on each device that loads it, until exit; T * P beyond that
+ * returns QKNORM_ERR_UNSUPPORTED without launching anything. The call itself
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * The first call on a device looks up the buffer's device address (with that
+ * device current); make that first call before any stream capture. All calls
+ * share the buffer: calls that overlap on the GPU race. Nothing in it needs
+ * clearing between calls.
+ */
+QKNORM_API int qknorm_split_noalloc(const void *x, const float *gamma, void *out, int64_t T,
+                                    int32_t D, int32_t P, float eps, int32_t dtype, void *stream);
+
+/* The buffer size of qknorm_split_noalloc, in floats (the largest T * P). */
+QKNORM_API int64_t qknorm_split_noalloc_max_stats(void);
+
 /* Static text for a qknorm_status value ("unknown status" otherwise). */
 QKNORM_API const char *qknorm_status_string(int status);
 

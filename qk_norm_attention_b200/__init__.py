@@ -91,6 +91,10 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_xgamma.restype = ctypes.c_int
     lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
     lib.qknorm_inv_rms.restype = ctypes.c_int
+    lib.qknorm_split_noalloc.argtypes = [vp, vp, vp, i64, i32, i32, f32, i32, vp]
+    lib.qknorm_split_noalloc.restype = ctypes.c_int
+    lib.qknorm_split_noalloc_max_stats.argtypes = []
+    lib.qknorm_split_noalloc_max_stats.restype = ctypes.c_int64
     lib.qknorm_status_string.argtypes = [ctypes.c_int]
     lib.qknorm_status_string.restype = ctypes.c_char_p
     lib.qknorm_last_error.argtypes = []
@@ -366,3 +370,20 @@ def qknorm_selftest_bounded_wait(limit_ns: int, stream=None, device=None) -> Non
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     _check("qknorm_selftest_bounded_wait",
            lib.qknorm_selftest_bounded_wait(int(limit_ns), _stream_handle(dev, stream)))
+
+
+def qknorm_split_noalloc(x: torch.Tensor, gamma: torch.Tensor, P: int, eps: float,
+                         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The split path (statistics, then apply) in one call, with the statistics
+    in the library's own device buffer: for callers that cannot allocate
+    device memory. T * P must not exceed qknorm_split_noalloc_max_stats()."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T, D]")
+    T, D = x.shape
+    out = torch.empty_like(x) if out is None else out
+    for name, t in (("x", x), ("gamma", gamma), ("out", out)):
+        _need_cuda_contig(name, t)
+    st = lib.qknorm_split_noalloc(x.data_ptr(), gamma.data_ptr(), out.data_ptr(), T, D, int(P),
+                                  float(eps), _dtype_code(x), _stream_handle(x.device, stream))
+    _check("qknorm_split_noalloc", st)
+    return out

@@ -26,7 +26,7 @@ def qk():
 
 def declared_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"QKNORM_API\s+(?:int|const char \*)\s*(qknorm_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"QKNORM_API\s+(?:int|int64_t|const char \*)\s*(qknorm_\w+)\s*\(", src)))
 
 
 def test_header_declares_the_api():
