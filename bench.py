@@ -67,13 +67,17 @@ def parse_args(argv=None):
 VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4}
 
 
+# The sources that define the headline kernel (fused_bulk) and the plan it runs with.
+HEADLINE_SOURCES = ("qknorm_fused_bulk.cu", "qknorm_bulk.cuh", "qknorm_device.cuh",
+                    "qknorm_internal.h", "qknorm_api.cu")
+
+
 def kernel_src_sha() -> str:
     csrc = os.path.join(ROOT, "qk_norm_attention_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in HEADLINE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -375,8 +379,8 @@ def deferred_steps(torch, qk, device, peak, steps=100):
 def fp8_prefill(torch, qk, device, peak, steps=200):
     """The 13B-shaped prefill (T = 8192, Dq = Dk = 5120, P = 4) in FP8 E4M3:
     E4M3 in and out, fp32 statistics; half the bytes of the bf16 step."""
-    wl = W.custom("fp8 prefill", 8192, 5120, 5120, 4, dtype="e4m3", seed=3, x_sigma=1.5)
-    T = 8192
+    wl = W.WORKLOADS["prefill13b_e4m3"]
+    T = wl.Ts[0]
     stream = torch.cuda.current_stream(device)
     q = W.gen_device_workload(wl, "q", T, device)
     k = W.gen_device_workload(wl, "k", T, device)
