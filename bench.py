@@ -286,7 +286,7 @@ def latency_us(torch, qk, wl, T, device, n_eager=400, n_graph=100, graph_reps=10
     stream = torch.cuda.current_stream(device)
     q, k, gq, gk = device_inputs(torch, wl, T, device)
     bufs = (q, k, gq, gk, torch.empty_like(q), torch.empty_like(k))
-    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    dt = {"bf16": qk.QKNORM_BF16, "f32": qk.QKNORM_F32, "e4m3": qk.QKNORM_E4M3}[wl.dtype]
     f = Fused(qk, bufs, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
     for _ in range(50):
         f()
@@ -319,7 +319,7 @@ def latency_us(torch, qk, wl, T, device, n_eager=400, n_graph=100, graph_reps=10
 def throughput(torch, qk, wl, T, device, sets, steps=50):
     """GB/s of the fused path on T tokens with `sets` rotating buffer sets."""
     stream = torch.cuda.current_stream(device)
-    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    dt = {"bf16": qk.QKNORM_BF16, "f32": qk.QKNORM_F32, "e4m3": qk.QKNORM_E4M3}[wl.dtype]
     q, k, gq, gk = device_inputs(torch, wl, T, device)
     calls = []
     for s in range(sets):
@@ -608,7 +608,7 @@ def run_native(args, dist):
     row0, _ = shard_tokens(T * dist.world, dist.world, dist.rank)
     stream = torch.cuda.current_stream(device)
     peak, peak_src = hbm_peak()
-    dt = qk.QKNORM_BF16 if wl.dtype == "bf16" else qk.QKNORM_F32
+    dt = {"bf16": qk.QKNORM_BF16, "f32": qk.QKNORM_F32, "e4m3": qk.QKNORM_E4M3}[wl.dtype]
     qk.qknorm_force_variant(VARIANT_IDS[args.variant], 0)
 
     q, k, gq, gk = device_inputs(torch, wl, T, device, row0)
@@ -691,7 +691,7 @@ def run_native(args, dist):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": config_of(wl, T, dist.world),
         "pct_hbm_peak": round(100 * value / dist.world / peak, 2),
         "tokens_per_s": round(dist.world * T / step_ms * 1000, 1),
