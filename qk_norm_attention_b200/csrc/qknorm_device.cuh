@@ -64,6 +64,10 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
 }
 
+// Two fp32 products rounded to nearest even, as one packed sm_100 f32x2
+// multiply (each lane is exactly __fmul_rn of its operands).
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
 // ---------------------------------------------------------------- Phase A: x^2
 
 // Sum of squares of one vector: e0*e0, then e_i*e_i + q fused, i = 1..3.
@@ -199,15 +203,21 @@ __device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float
     return o;
 }
 
+// FP8: the two multiplies of each pair of values as packed f32x2 multiplies
+// (the same roundings as wmul), which halves their issue slots.
 __device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r) {
-    float f[16];
-    e4m3x16_to_float(v, f);
-    uint32_t w[4];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const float2 rr = make_float2(r, r);
+    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        w[i] = pack_e4m3x2(wmul(f[4 * i], g[4 * i], r), wmul(f[4 * i + 1], g[4 * i + 1], r)) |
-               (pack_e4m3x2(wmul(f[4 * i + 2], g[4 * i + 2], r), wmul(f[4 * i + 3], g[4 * i + 3], r)) << 16);
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    for (int i = 0; i < 4; ++i) {
+        const float2 x01 = e4m3x2_to_float2(w[i]);
+        const float2 x23 = e4m3x2_to_float2(w[i] >> 16);
+        const float2 y01 = fmul2_rn(fmul2_rn(x01, make_float2(g[4 * i], g[4 * i + 1])), rr);
+        const float2 y23 = fmul2_rn(fmul2_rn(x23, make_float2(g[4 * i + 2], g[4 * i + 3])), rr);
+        o[i] = pack_e4m3x2(y01.x, y01.y) | (pack_e4m3x2(y23.x, y23.y) << 16);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r) {

@@ -143,17 +143,18 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
             const uint4 *src = reinterpret_cast<const uint4 *>(st + j * tok_bytes);
 #pragma unroll
             for (int i = 0; i < VMAX; ++i)
-                if ((FULL || i < cnt) && (j == 0 || t0 + j * G < T)) cur[j][i] = src[i * stride];
+                cur[j][i] = ((FULL || i < cnt) && (j == 0 || t0 + j * G < T)) ? src[i * stride]
+                                                                              : make_uint4(0, 0, 0, 0);
         }
-        // Phase A for TB tokens: independent chains and butterflies.
+        // Phase A for TB tokens: independent chains and butterflies. A lane's
+        // missing vectors are its last slots and read as zeros, whose sum of
+        // squares (+0) leaves the chain unchanged, so the chains need no branch.
         float c[TB];
 #pragma unroll
         for (int j = 0; j < TB; ++j) {
             c[j] = 0.f;
 #pragma unroll
-            for (int i = 0; i < VMAX; ++i)
-                if ((FULL || i < cnt) && (j == 0 || t0 + j * G < T))
-                    c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
+            for (int i = 0; i < VMAX; ++i) c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
         }
 #pragma unroll
         for (int j = 0; j < TB; ++j) c[j] = butterfly(c[j]);
@@ -399,11 +400,12 @@ __global__ void bounded_wait_probe(uint64_t timeout_ns) {
 // ---------------------------------------------------------------- instances and launch
 
 // Combinations that exist: TB (1 or 2) tokens x VMAX vectors per lane <= 12;
-// for FP8 (16 values per vector) one token, <= 4 vectors, gamma in registers
-// only up to 3 vectors, so that no instance spills.
+// for FP8 (16 values per vector) TB x VMAX <= 4, two tokens only with gamma
+// read per use, gamma in registers only up to 3 vectors, so that no instance
+// spills.
 constexpr bool bulk_exists(int vmax, int tb, int vec, bool greg) {
     return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12 &&
-           (vec != 16 || (tb == 1 && vmax <= 4 && (!greg || vmax <= 3)));
+           (vec != 16 || (vmax * tb <= 4 && (tb == 1 || !greg) && (!greg || vmax <= 3)));
 }
 constexpr int bulk_max_threads(int vmax, int tb, int vec) {
     return (vmax * tb <= 2 && vmax * tb * vec <= 16) ? 1024 : 512;

@@ -93,3 +93,95 @@ def test_fp8_deferred_and_headwise(qk, orc):
     assert (np.abs(r.cpu().numpy() - r_or) / r_or).max() < 1e-5
     check_outputs(to_host(hq), orc.headwise(q, gq[:128], 128, EPS, "e4m3"), "e4m3", "headwise q")
     check_outputs(to_host(hk), orc.headwise(k, gk[:128], 128, EPS, "e4m3"), "e4m3", "headwise k")
+
+
+def _code_rows(T, D, seed):
+    """Rows built from E4M3 codes: every finite code, subnormal-only rows and
+    rows at the largest magnitudes (NaN codes 0x7f and 0xff excluded)."""
+    rng = np.random.default_rng(seed)
+    finite = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    sub = np.array([c for c in range(256) if (c & 0x78) == 0 and c & 0x7], dtype=np.uint8)
+    big = np.array([c for c in range(256) if (c & 0x7F) >= 0x70 and c & 0x7F != 0x7F], dtype=np.uint8)
+    x = np.empty((T, D), dtype=np.uint8)
+    for t in range(T):
+        pool = (finite, sub, big)[t % 3]
+        x[t] = rng.choice(pool, size=D)
+    x[0, :finite.size] = finite                      # each finite code at least once
+    return x
+
+
+@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "generic"])
+def test_fp8_every_code(qk, orc, variant):
+    """Every finite E4M3 code in, subnormal-only rows (whose factor is large,
+    so their outputs are far from zero) and rows near +-448, with gamma of
+    both signs: each variant against the oracle."""
+    T, D, P = 3 * 37, 4096, 4
+    q, k = _code_rows(T, D, 11), _code_rows(T, D, 12)
+    rng = np.random.default_rng(13)
+    gq = rng.uniform(0.5, 1.5, D).astype(np.float32) * rng.choice([-1.0, 1.0], D).astype(np.float32)
+    gk = rng.uniform(0.5, 1.5, D).astype(np.float32)
+    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "generic": 2}[variant]
+    qk.qknorm_force_variant(vid, 0)
+    try:
+        oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk), P, 1e-6)
+        torch.cuda.synchronize()
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    yq, yk, _, _ = orc.qknorm(q, k, gq, gk, P, EPS, "e4m3", nthreads=8)
+    check_outputs(to_host(oq), yq, "e4m3", "every-code q")
+    check_outputs(to_host(ok), yk, "e4m3", "every-code k")
+
+
+@pytest.mark.parametrize("D,P", [(4096, 4), (5120, 4), (1024, 8), (4096, 1)])
+def test_fp8_variants_bit_identical(qk, D, P):
+    """Every fused variant and the split path give the same bytes (one
+    reduction order, one rounding of each output)."""
+    T = 2 * 148 + 3
+    q = _code_rows(T, D, 21 + D)
+    k = _code_rows(T, D, 22 + D)
+    g = torch.from_numpy(np.random.default_rng(23).uniform(-1.5, 1.5, D).astype(np.float32)).cuda()
+    qd, kd = to_device(q), to_device(k)
+    outs = {}
+    for name, vid in (("cta", 0), ("bulk", 3), ("rows", 4), ("generic", 2)):
+        qk.qknorm_force_variant(vid, 0)
+        try:
+            outs[name] = qk.qknorm_fwd(qd, kd, g, g, P, 1e-6)
+        except qk.QKNormError as e:
+            assert name in ("cta", "bulk") and e.status == qk.QKNORM_ERR_UNSUPPORTED
+        finally:
+            qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    outs["split"] = tuple(qk.qknorm_apply(x, g, qk.qknorm_partial_sumsq(x, P), 1e-6) for x in (qd, kd))
+    torch.cuda.synchronize()
+    ref = outs["generic"]
+    for name, (oq, ok) in outs.items():
+        assert torch.equal(bits(oq), bits(ref[0])), f"{name} q"
+        assert torch.equal(bits(ok), bits(ref[1])), f"{name} k"
+
+
+def test_fp8_saturation(qk, orc):
+    """Outputs beyond the E4M3 range saturate to +-448 with the sign of
+    x * gamma, on every variant; the rest stay within one E4M3 ulp."""
+    T, D, P = 150, 4096, 4
+    q, k = _code_rows(T, D, 31), _code_rows(T, D, 32)
+    rng = np.random.default_rng(33)
+    g = rng.uniform(0.5, 1.5, D).astype(np.float32)
+    g[::7] *= -300.0                                   # these channels overflow the format
+    for vid in (-1, 0, 2, 3, 4):
+        qk.qknorm_force_variant(vid, 0)
+        try:
+            oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(g), to_device(g), P, 1e-6)
+            torch.cuda.synchronize()
+        except qk.QKNormError as e:
+            assert vid in (0, 3) and e.status == qk.QKNORM_ERR_UNSUPPORTED
+            continue
+        finally:
+            qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+        for x, out in ((q, oq), (k, ok)):
+            y_or, _ = orc.rmsnorm(x, g, P, EPS, "e4m3", nthreads=8)
+            y = W.storage_to_f64(to_host(out), "e4m3")
+            over = np.abs(y_or) > 448 * (1 + 2.0 ** -4)
+            assert over.any()
+            assert np.array_equal(y[over], np.sign(y_or[over]) * 448.0)
+            inside = np.abs(y_or) < 448
+            diff = np.abs(y[inside] - y_or[inside])
+            assert (diff <= 2.0 ** -3 * np.abs(y_or[inside]) + 2.0 ** -9).all()
