@@ -241,11 +241,11 @@ typedef enum {
     QKNORM_VARIANT_BULK = 3,    /* as CTA, but rows arrive by bulk asynchronous
                                    copies (TMA engine) into a ring of token stages
                                    in shared memory, completed on mbarriers */
-    QKNORM_VARIANT_ROWS = 4     /* warp per row: each warp has its own ring of
-                                   bulk-copied row stages, walks all P shards of
-                                   the row itself and applies from shared memory
-                                   with gamma staged once per CTA; no CTA barrier
-                                   per row */
+    QKNORM_VARIANT_ROWS = 4     /* warp per row: a CTA has a pool of warps for
+                                   Q rows and one for K rows; each warp has its
+                                   own ring of bulk-copied row stages, walks all
+                                   P shards of the row itself and applies from
+                                   shared memory; no CTA barrier per row */
 } qknorm_variant;
 
 /* A launch plan chosen by the selector (host-side description). */
@@ -262,6 +262,8 @@ typedef struct {
     int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
     int32_t full_lanes;  /* 1 if every lane holds exactly vmax vectors per task */
     int64_t smem_bytes;  /* dynamic shared memory per CTA */
+    int32_t q_warps;     /* rows: warps per CTA that take Q rows (the rest take K rows) */
+    int32_t gamma_smem;  /* rows: 1 if gamma is staged in shared memory, 0 if read via L1 */
 } qknorm_plan;
 
 /*
@@ -305,10 +307,14 @@ QKNORM_API int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32
 
 /*
  * qknorm_set_rows_tuning -- process-wide tuning of the warp-per-row variant:
- * warps per CTA (0 = as many as shared memory allows, up to 16) and row
- * stages per warp (0 = automatic). Not thread-safe with concurrent calls.
+ * warps per CTA of the Q pool and of the K pool (both 0 = automatic: the
+ * split in proportion to Dq : Dk with the most resident warps per SM; else
+ * each >= 1 and their sum <= 16), row stages per warp (0 = automatic) and
+ * gamma staging (-1 = automatic, 0 = read through L1, 1 = staged in shared
+ * memory once per CTA). Not thread-safe with concurrent calls.
  */
-QKNORM_API int qknorm_set_rows_tuning(int32_t warps, int32_t stages);
+QKNORM_API int qknorm_set_rows_tuning(int32_t q_warps, int32_t k_warps, int32_t stages,
+                                      int32_t gamma_smem);
 
 /*
  * qknorm_set_pdl -- programmatic dependent launch on (1, the default) or off

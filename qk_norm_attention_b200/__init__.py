@@ -63,7 +63,8 @@ class QKNormPlan(ctypes.Structure):
                 ("prefetch", ctypes.c_int32), ("groups_q", ctypes.c_int32),
                 ("groups_k", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("tokens_per_stage", ctypes.c_int32), ("gamma_regs", ctypes.c_int32),
-                ("full_lanes", ctypes.c_int32), ("smem_bytes", ctypes.c_int64)]
+                ("full_lanes", ctypes.c_int32), ("smem_bytes", ctypes.c_int64),
+                ("q_warps", ctypes.c_int32), ("gamma_smem", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -110,7 +111,7 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_set_tuning.restype = ctypes.c_int
     lib.qknorm_set_pdl.argtypes = [i32]
     lib.qknorm_set_pdl.restype = ctypes.c_int
-    lib.qknorm_set_rows_tuning.argtypes = [i32, i32]
+    lib.qknorm_set_rows_tuning.argtypes = [i32, i32, i32, i32]
     lib.qknorm_set_rows_tuning.restype = ctypes.c_int
     lib.qknorm_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     lib.qknorm_device_errors.restype = ctypes.c_int
@@ -352,9 +353,12 @@ def qknorm_set_pdl(enable: bool = True) -> None:
     _check("qknorm_set_pdl", lib.qknorm_set_pdl(int(bool(enable))))
 
 
-def qknorm_set_rows_tuning(warps: int = 0, stages: int = 0) -> None:
-    """Warps per CTA and row stages per warp of the rows variant (0 = automatic)."""
-    _check("qknorm_set_rows_tuning", lib.qknorm_set_rows_tuning(int(warps), int(stages)))
+def qknorm_set_rows_tuning(q_warps: int = 0, k_warps: int = 0, stages: int = 0,
+                           gamma_smem: int = -1) -> None:
+    """Q-pool and K-pool warps per CTA, row stages per warp and gamma staging
+    of the rows variant (0, 0, 0, -1 = automatic)."""
+    _check("qknorm_set_rows_tuning", lib.qknorm_set_rows_tuning(int(q_warps), int(k_warps),
+                                                                int(stages), int(gamma_smem)))
 
 
 def qknorm_device_errors(clear: bool = True) -> int:

@@ -163,9 +163,11 @@ int32_t g_tune_stages = 0;           // bulk stages per CTA; 0 = automatic
 int32_t g_tune_tb = 0;               // tokens per bulk stage; 0 = automatic
 int32_t g_tune_gamma_regs = -1;      // -1 = automatic
 uint64_t g_wait_limit_ns = 2000000000ull;
-int32_t g_rows_warps = 0;            // warps per CTA of the rows variant; 0 = automatic
+int32_t g_rows_wq = 0;               // Q-pool warps per CTA of the rows variant; 0 = automatic
+int32_t g_rows_wk = 0;               // K-pool warps per CTA; 0 = automatic
 int32_t g_rows_stages = 0;           // row stages per warp; 0 = automatic
-constexpr int kRowsStagesAuto = 1;
+int32_t g_rows_gsm = -1;             // gamma staged in shared memory: -1 automatic, 0, 1
+constexpr int kRowsStagesAuto = 2;
 constexpr int kRowsMaxWarps = 16;
 
 constexpr int kSmemPerSm = 228 * 1024;      // shared memory of one SM
@@ -239,28 +241,52 @@ void bulk_stages(uint32_t stride, int block, int regs, qknorm_plan *pl) {
     pl->smem_bytes = (int64_t)bulk_smem_bytes(S, stride);
 }
 
-// Warps per CTA of the rows variant: the most resident warps per SM (up to
-// kRowsMaxWarps) that shared memory allows, preferring two CTAs per SM (each
-// CTA holds its own copy of gamma).
-int rows_auto_warps(int32_t Dq, int32_t Dk, int32_t dtype, int S) {
-    int best_w = 0, best_total = 0;
-    for (int ctas = 2; ctas >= 1; --ctas) {
-        for (int W = kRowsMaxWarps / ctas; W >= 1; --W) {
-            const size_t sm = rows_layout(Dq, Dk, (int)elem_of(dtype), W, S).smem_bytes;
-            if (sm <= (size_t)kSmemPerCta && (int64_t)ctas * (sm + kSmemReservedPerCta) <= kSmemPerSm) {
-                if (ctas * W > best_total) {
-                    best_total = ctas * W;
-                    best_w = W;
+// Warps of the rows variant. A Q warp moves Dq/wq of a CTA's row bytes per
+// round and a K warp Dk/wk; the CTA moves (Dq + Dk) per round in the time of
+// the busier pool, so it works like (Dq + Dk) / max(Dq/wq, Dk/wk) fully busy
+// warps. Among the CTA shapes (wq + wk <= kRowsMaxWarps, wq, wk >= 1) and
+// CTAs per SM (1 to 8) that threads, registers and shared memory allow, take
+// the most such warps per SM; ties go to fewer warps per CTA.
+struct RowsChoice {
+    int wq = 0, wk = 0;
+    bool gsm = false;
+};
+
+bool rows_fits(int32_t Dq, int32_t Dk, int32_t dtype, int wq, int wk, int S, bool gsm, int ctas) {
+    const size_t sm = rows_layout(Dq, Dk, (int)elem_of(dtype), wq, wk, S, gsm).smem_bytes;
+    return sm <= (size_t)kSmemPerCta && (int64_t)ctas * (sm + kSmemReservedPerCta) <= kSmemPerSm;
+}
+
+RowsChoice rows_auto(int32_t Dq, int32_t Dk, int32_t dtype, int S, int gsm_pref, int regs) {
+    RowsChoice best;
+    double best_score = 0.0;
+    const int warp_regs = (regs + 7) / 8 * 8 * kLanes;   // registers are granted 8 per thread at a time
+    for (int g = 0; g <= 1; ++g) {
+        if (gsm_pref >= 0 && g != gsm_pref) continue;
+        for (int W = 2; W <= kRowsMaxWarps; ++W) {
+            for (int wq = 1; wq < W; ++wq) {
+                const int wk = W - wq;
+                const double busy = (double)(Dq + Dk) /
+                                    ((double)Dq / wq > (double)Dk / wk ? (double)Dq / wq : (double)Dk / wk);
+                for (int ctas = 8; ctas >= 1; --ctas) {
+                    if (ctas * W * kLanes > kThreadsPerSm || ctas * W * warp_regs > kRegsPerSm) continue;
+                    if (!rows_fits(Dq, Dk, dtype, wq, wk, S, g != 0, ctas)) continue;
+                    if (ctas * busy > best_score + 1e-9) {
+                        best_score = ctas * busy;
+                        best.wq = wq;
+                        best.wk = wk;
+                        best.gsm = g != 0;
+                    }
+                    break;
                 }
-                break;
             }
         }
     }
-    return best_w;
+    return best;
 }
 
 bool rows_fit(int32_t Dq, int32_t Dk, int32_t dtype) {
-    return rows_layout(Dq, Dk, (int)elem_of(dtype), 1, 1).smem_bytes <= (size_t)kSmemPerCta;
+    return rows_fits(Dq, Dk, dtype, 1, 1, 1, false, 1);
 }
 
 // Static part of the plan: which kernel, block size, template width, stages.
@@ -319,13 +345,20 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     }
     if (variant == QKNORM_VARIANT_ROWS) {
         const int S = g_rows_stages > 0 ? g_rows_stages : kRowsStagesAuto;
-        int W = g_rows_warps > 0 ? g_rows_warps : rows_auto_warps(Dq, Dk, dtype, S);
-        if (W < 1 || W > kRowsMaxWarps) return QKNORM_ERR_UNSUPPORTED;
-        const RowsLayout L = rows_layout(Dq, Dk, (int)elem_of(dtype), W, S);
+        RowsChoice c = rows_auto(Dq, Dk, dtype, S, g_rows_gsm, regs > 0 ? regs : kRegsHint);
+        if (g_rows_wq > 0) {
+            c.wq = g_rows_wq;
+            c.wk = g_rows_wk;
+            if (g_rows_gsm >= 0) c.gsm = g_rows_gsm != 0;
+        }
+        if (c.wq < 1 || c.wk < 1 || c.wq + c.wk > kRowsMaxWarps) return QKNORM_ERR_UNSUPPORTED;
+        const RowsLayout L = rows_layout(Dq, Dk, (int)elem_of(dtype), c.wq, c.wk, S, c.gsm);
         if (L.smem_bytes > (size_t)kSmemPerCta) return QKNORM_ERR_UNSUPPORTED;
         pl->variant = QKNORM_VARIANT_ROWS;
-        pl->block = W * kLanes;
+        pl->block = (c.wq + c.wk) * kLanes;
         pl->stages = S;
+        pl->q_warps = c.wq;
+        pl->gamma_smem = c.gsm ? 1 : 0;
         pl->smem_bytes = (int64_t)L.smem_bytes;
         return QKNORM_OK;
     }
@@ -345,12 +378,14 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     return QKNORM_ERR_INVALID_ARG;
 }
 
-// Units of work a CTA can take: tokens, or for the rows variant the 2T rows
-// spread over block/32 warps per CTA.
+// Units of work a CTA can take: tokens, or for the rows variant the CTAs
+// that give every warp of the smaller pool a row (T Q rows over q_warps
+// warps per CTA, T K rows over the others).
 int64_t plan_units(int64_t T, const qknorm_plan &pl) {
     if (pl.variant != QKNORM_VARIANT_ROWS) return T;
-    const int64_t w = pl.block / kLanes;
-    return (2 * T + w - 1) / w;
+    const int64_t wq = pl.q_warps, wk = pl.block / kLanes - pl.q_warps;
+    const int64_t w = wq < wk ? wq : wk;
+    return (T + w - 1) / w;
 }
 
 // Grid: T CTAs up to B_res x N_SM (or the forced grid); the register variant
@@ -432,7 +467,7 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     if (e != cudaSuccess) return e;
     *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, kRegsHint, pl);
     if (*status != QKNORM_OK) return cudaSuccess;
-    if (pl->variant == QKNORM_VARIANT_BULK) {
+    if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS) {
         int regs = kRegsHint;
         e = kernel_regs(plan_kernel(*pl, dtype, true), &regs);
         if (e != cudaSuccess) return e;
@@ -468,7 +503,7 @@ using namespace qkn;
 
 extern "C" {
 
-int qknorm_version(void) { return 109; }
+int qknorm_version(void) { return 110; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -588,7 +623,8 @@ int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const
         e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes != 0, a, pl.block,
                              pl.grid, s);
     } else if (pl.variant == QKNORM_VARIANT_ROWS) {
-        e = launch_fused_rows(dtype, a, pl.block / kLanes, pl.stages, pl.grid, g_wait_limit_ns, s);
+        e = launch_fused_rows(dtype, a, pl.q_warps, pl.block / kLanes - pl.q_warps, pl.stages,
+                              pl.gamma_smem != 0, pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
         e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
                               pl.full_lanes != 0, a, pl.stages, pl.block, pl.grid,
@@ -736,11 +772,16 @@ int qknorm_set_tuning(int32_t stages, int32_t tokens_per_stage, int32_t gamma_re
     return QKNORM_OK;
 }
 
-int qknorm_set_rows_tuning(int32_t warps, int32_t stages) {
-    if (warps < 0 || warps > kRowsMaxWarps || stages < 0 || stages > bulk_max_stages())
+int qknorm_set_rows_tuning(int32_t q_warps, int32_t k_warps, int32_t stages, int32_t gamma_smem) {
+    const bool autow = q_warps == 0 && k_warps == 0;
+    if (!autow && (q_warps < 1 || k_warps < 1 || q_warps + k_warps > kRowsMaxWarps))
         return QKNORM_ERR_INVALID_ARG;
-    g_rows_warps = warps;
+    if (stages < 0 || stages > bulk_max_stages() || gamma_smem < -1 || gamma_smem > 1)
+        return QKNORM_ERR_INVALID_ARG;
+    g_rows_wq = q_warps;
+    g_rows_wk = k_warps;
     g_rows_stages = stages;
+    g_rows_gsm = gamma_smem;
     return QKNORM_OK;
 }
 

@@ -213,21 +213,27 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
 
 // ---------------------------------------------------------------- warp per row
 
-// Warp-per-row kernel. Each warp owns a ring of S row stages in shared memory
-// and processes whole rows (a Q row or a K row of a token) on its own: lane 0
-// issues the bulk copy of the warp's next rows, the warp walks the row's P
-// shards in the order of the reduction (per group: lane chains, butterfly;
-// groups in order; shards in order), forms the factor, and applies
-// (x*gamma)*r re-reading the row from shared memory, with gamma staged in
-// shared memory once per CTA. No CTA-wide barrier is crossed per row, so
-// warps never wait for one another and the per-row bookkeeping is amortised
-// over the whole row.
+// Warp-per-row kernel. A CTA holds two pools of warps: WQ warps that take Q
+// rows and W - WQ warps that take K rows, so that each pool's ring stages have
+// the size of its own rows and the pools can be sized in proportion to the
+// bytes of Q and K. Each warp owns a ring of S row stages in shared memory and
+// processes whole rows on its own: lane 0 issues the bulk copies of the
+// warp's next rows, the warp walks the row's P shards in the order of the
+// reduction (per group: lane chains, butterfly; groups in order; shards in
+// order), forms the factor, and applies (x*gamma)*r re-reading the row from
+// shared memory, with gamma read from shared memory (staged once per CTA) or
+// through the L1 cache. No CTA-wide barrier is crossed per row, so warps never
+// wait for one another and the per-row bookkeeping is amortised over the row.
 struct RowsArgs {
-    uint32_t stages;      // S, per warp
-    uint32_t stage_bytes; // bytes of one row stage (multiple of 128)
-    uint32_t gq_off;      // shared-memory offset of gamma_q
-    uint32_t gk_off;      // shared-memory offset of gamma_k
-    uint32_t ring_off;    // shared-memory offset of the warps' rings
+    uint32_t stages;       // S, per warp
+    uint32_t wq;           // warps of the Q pool (the others take K rows)
+    uint32_t qstage;       // bytes of one Q row stage (multiple of 128)
+    uint32_t kstage;       // bytes of one K row stage (multiple of 128)
+    uint32_t gq_off;       // shared-memory offset of gamma_q (when staged)
+    uint32_t gk_off;       // shared-memory offset of gamma_k (when staged)
+    uint32_t qring_off;    // shared-memory offset of the Q pool's rings
+    uint32_t kring_off;    // shared-memory offset of the K pool's rings
+    uint32_t gamma_smem;   // 1: gamma staged in shared memory, 0: read through L1
     uint64_t timeout_ns;
 };
 
@@ -239,27 +245,27 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int S = (int)b.stages;
+    const int WQ = (int)b.wq;
+    const int z = warp < WQ ? 0 : 1;                          // 0: Q pool, 1: K pool
+    const int wz = z ? warp - WQ : warp;                      // index in the pool
+    const int Wz = z ? W - WQ : WQ;                           // pool size
+    const bool gsm = b.gamma_smem != 0;
     uint64_t *gbar = reinterpret_cast<uint64_t *>(smem);      // gamma barrier
     uint64_t *full = gbar + 1 + warp * S;                     // this warp's stage barriers
-    const float *gam_q = reinterpret_cast<const float *>(smem + b.gq_off);
-    const float *gam_k = reinterpret_cast<const float *>(smem + b.gk_off);
-    unsigned char *ring = smem + b.ring_off + (size_t)warp * S * b.stage_bytes;
+    const uint32_t stage_bytes = z ? b.kstage : b.qstage;
+    unsigned char *ring = smem + (z ? b.kring_off : b.qring_off) + (size_t)wz * S * stage_bytes;
+    const float *g = gsm ? reinterpret_cast<const float *>(smem + (z ? b.gk_off : b.gq_off)) : (z ? a.g[1] : a.g[0]);
 
     const int64_t T = a.T;
-    const int64_t R = 2 * T;                                  // Q rows, then K rows
-    const int64_t NW = (int64_t)gridDim.x * W;
-    const int64_t gw = (int64_t)blockIdx.x * W + warp;
-    const uint32_t qbytes = (uint32_t)a.D[0] * (uint32_t)Tag::kBytes;
-    const uint32_t kbytes = (uint32_t)a.D[1] * (uint32_t)Tag::kBytes;
+    const int64_t NW = (int64_t)gridDim.x * Wz;               // warps of this pool in the grid
+    const int64_t gw = (int64_t)blockIdx.x * Wz + wz;
+    const uint32_t nb = (uint32_t)(z ? a.D[1] : a.D[0]) * (uint32_t)Tag::kBytes;
+    const char *xsrc = static_cast<const char *>((z ? a.x[1] : a.x[0]));
+    const int64_t ldx_b = (z ? a.ldx[1] : a.ldx[0]) * 16;
 
-    auto issue = [&](int s, int64_t r) {
-        const bool isk = r >= T;
-        const int64_t t = isk ? r - T : r;
-        const uint32_t nb = isk ? kbytes : qbytes;
-        const char *src = static_cast<const char *>(isk ? a.x[1] : a.x[0]) +
-                          t * (isk ? a.ldx[1] : a.ldx[0]) * 16;
+    auto issue = [&](int s, int64_t t) {
         mbar_arrive_expect_tx(&full[s], nb);
-        bulk_copy_g2s(ring + (size_t)s * b.stage_bytes, src, nb, &full[s]);
+        bulk_copy_g2s(ring + (size_t)s * stage_bytes, xsrc + t * ldx_b, nb, &full[s]);
     };
 
     if (threadIdx.x == 0) {
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
     // Shared memory only so far; global reads start after the previous grid.
     pdl_wait();
     pdl_trigger();
-    if (threadIdx.x == 0) {
+    if (gsm && threadIdx.x == 0) {
         const uint32_t gqb = (uint32_t)a.D[0] * 4u, gkb = (uint32_t)a.D[1] * 4u;
         mbar_arrive_expect_tx(gbar, gqb + gkb);
         bulk_copy_g2s(smem + b.gq_off, a.g[0], gqb, gbar);
@@ -279,8 +285,8 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
     }
     if (lane == 0) {
         for (int s = 0; s < S; ++s) {
-            const int64_t r = gw + (int64_t)s * NW;
-            if (r < R) issue(s, r);
+            const int64_t t = gw + (int64_t)s * NW;
+            if (t < T) issue(s, t);
         }
     }
     // Leave after recording an error, once this warp's copies in flight have
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
             atomicOr(&g_device_errors, kErrWaitTimeout);
             int ds = s0;
             uint32_t dp = ph0;
-            for (int64_t n = n_first; n < n_first + S && gw + n * NW < R; ++n) {
+            for (int64_t n = n_first; n < n_first + S && gw + n * NW < T; ++n) {
                 if (!mbar_wait_bounded(&full[ds], dp, b.timeout_ns))
                     atomicOr(&g_device_errors, kErrDrainTimeout);
                 if (++ds == S) {
@@ -298,31 +304,33 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
                     dp ^= 1u;
                 }
             }
-            if (warp == 0 && !mbar_wait_bounded(gbar, 0, b.timeout_ns))
+            if (gsm && warp == 0 && !mbar_wait_bounded(gbar, 0, b.timeout_ns))
                 atomicOr(&g_device_errors, kErrDrainTimeout);
         }
     };
-    if (!__all_sync(kFull, mbar_wait_bounded(gbar, 0, b.timeout_ns))) {
+    if (gsm && !__all_sync(kFull, mbar_wait_bounded(gbar, 0, b.timeout_ns))) {
         fail(0, 0, 0);
         return;
     }
 
+    const int P = a.P;
+    const int K = (z ? a.K[1] : a.K[0]);
+    const int nv = (z ? a.nv[1] : a.nv[0]);
+    const int stride = kLanes * K;
+    const float Df = (z ? a.Df[1] : a.Df[0]);
+    const int rowvec = (z ? a.D[1] : a.D[0]) / VEC;
+    const int64_t ldy = (z ? a.ldy[1] : a.ldy[0]);
+    uint4 *ybase = reinterpret_cast<uint4 *>((z ? a.y[1] : a.y[0]));
     int s = 0;
     uint32_t phase = 0;
     for (int64_t n = 0;; ++n) {
-        const int64_t r = gw + n * NW;
-        if (r >= R) break;
+        const int64_t t = gw + n * NW;
+        if (t >= T) break;
         if (!__all_sync(kFull, mbar_wait_bounded(&full[s], phase, b.timeout_ns))) {
             fail(n, s, phase);
             return;
         }
-        const int z = r >= T ? 1 : 0;
-        const int64_t t = z ? r - T : r;
-        const uint4 *row = reinterpret_cast<const uint4 *>(ring + (size_t)s * b.stage_bytes);
-        const int P = a.P;
-        const int K = z ? a.K[1] : a.K[0];
-        const int nv = z ? a.nv[1] : a.nv[0];
-        const int stride = kLanes * K;
+        const uint4 *row = reinterpret_cast<const uint4 *>(ring + (size_t)s * stage_bytes);
         // Phase A and the ordered sums of Phase B.
         float Ssum = 0.f;
         if (K == 1) {
@@ -336,15 +344,15 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
                 const uint4 *sh = row + (int64_t)p0 * nv + lane;
                 for (int i = 0; i < cnt; ++i) {
 #pragma unroll
-                    for (int b = 0; b < 4; ++b)
-                        if (p0 + b < P)
-                            c[b] = __fadd_rn(c[b], vsumsq(Tag{}, sh[(int64_t)b * nv + i * kLanes]));
+                    for (int q = 0; q < 4; ++q)
+                        if (p0 + q < P)
+                            c[q] = __fadd_rn(c[q], vsumsq(Tag{}, sh[(int64_t)q * nv + i * kLanes]));
                 }
 #pragma unroll
-                for (int b = 0; b < 4; ++b) c[b] = butterfly(c[b]);
+                for (int q = 0; q < 4; ++q) c[q] = butterfly(c[q]);
 #pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    if (p0 + b < P) Ssum = __fadd_rn(Ssum, c[b]);
+                for (int q = 0; q < 4; ++q)
+                    if (p0 + q < P) Ssum = __fadd_rn(Ssum, c[q]);
             }
         } else {
             for (int p = 0; p < P; ++p) {
@@ -360,21 +368,25 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
                 Ssum = __fadd_rn(Ssum, Sp);
             }
         }
-        const float rr = factor(Ssum, z ? a.Df[1] : a.Df[0], a.eps);
+        const float rr = factor(Ssum, Df, a.eps);
         // Phase B weight multiply and Phase C, element-wise over the row.
-        const int rowvec = (z ? a.D[1] : a.D[0]) / VEC;
-        const float *g = z ? gam_k : gam_q;
-        uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]);
+        uint4 *dst = ybase + t * ldy;
+        if (gsm) {
 #pragma unroll 4
-        for (int v = lane; v < rowvec; v += kLanes)
-            st_stream(dst + v, vapply_ptr(Tag{}, row[v], g + (int64_t)v * VEC, rr));
+            for (int v = lane; v < rowvec; v += kLanes)
+                st_stream(dst + v, vapply_ptr(Tag{}, row[v], g + (int64_t)v * VEC, rr));
+        } else {
+#pragma unroll 4
+            for (int v = lane; v < rowvec; v += kLanes)
+                st_stream(dst + v, vapply(Tag{}, row[v], g + (int64_t)v * VEC, rr));
+        }
         __syncwarp();
         // Every lane is done with this stage: refill it with the warp's row S ahead.
         if (lane == 0) {
-            const int64_t rn = gw + (n + S) * NW;
-            if (rn < R) {
+            const int64_t tn = gw + (n + S) * NW;
+            if (tn < T) {
                 fence_proxy_async_smem();
-                issue(s, rn);
+                issue(s, tn);
             }
         }
         if (++s == S) {
@@ -491,32 +503,40 @@ const void *fused_rows_kernel(int dtype) {
 }
 
 // Shared-memory layout of fused_rows: [gamma barrier + W*S stage barriers,
-// padded to 128][gamma_q][gamma_k][W rings of S stages].
-RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int warps, int stages) {
+// padded to 128][gamma_q][gamma_k (both only when staged)][WQ Q rings of S
+// stages][WK K rings of S stages].
+RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int wq, int wk, int stages, bool gamma_smem) {
     RowsLayout L;
     auto up = [](int64_t x) { return (x + 127) / 128 * 128; };
-    L.stage_bytes = (uint32_t)up((Dq > Dk ? Dq : Dk) * es);
-    L.gq_off = (uint32_t)up(8 * (1 + (int64_t)warps * stages));
-    L.gk_off = L.gq_off + (uint32_t)up(Dq * 4);
-    L.ring_off = L.gk_off + (uint32_t)up(Dk * 4);
-    L.smem_bytes = (size_t)L.ring_off + (size_t)warps * stages * L.stage_bytes;
+    L.qstage = (uint32_t)up(Dq * es);
+    L.kstage = (uint32_t)up(Dk * es);
+    L.gq_off = (uint32_t)up(8 * (1 + (int64_t)(wq + wk) * stages));
+    L.gk_off = L.gq_off + (gamma_smem ? (uint32_t)up(Dq * 4) : 0u);
+    L.qring_off = L.gk_off + (gamma_smem ? (uint32_t)up(Dk * 4) : 0u);
+    L.kring_off = L.qring_off + (uint32_t)((int64_t)wq * stages * L.qstage);
+    L.smem_bytes = (size_t)L.kring_off + (size_t)wk * stages * L.kstage;
     return L;
 }
 
-cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stages, int64_t grid,
-                              uint64_t timeout_ns, cudaStream_t s) {
+cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int wq, int wk, int stages,
+                              bool gamma_smem, int64_t grid, uint64_t timeout_ns, cudaStream_t s) {
     const void *fn = fused_rows_kernel(dtype);
-    if (!fn || warps < 1 || warps > 16 || stages < 1) return cudaErrorInvalidValue;
-    const RowsLayout L = rows_layout(a.D[0], a.D[1], dtype == 1 ? 2 : (dtype == 2 ? 1 : 4), warps, stages);
+    if (!fn || wq < 1 || wk < 1 || wq + wk > 16 || stages < 1) return cudaErrorInvalidValue;
+    const RowsLayout L = rows_layout(a.D[0], a.D[1], dtype == 1 ? 2 : (dtype == 2 ? 1 : 4), wq, wk,
+                                     stages, gamma_smem);
     RowsArgs b;
     b.stages = (uint32_t)stages;
-    b.stage_bytes = L.stage_bytes;
+    b.wq = (uint32_t)wq;
+    b.qstage = L.qstage;
+    b.kstage = L.kstage;
     b.gq_off = L.gq_off;
     b.gk_off = L.gk_off;
-    b.ring_off = L.ring_off;
+    b.qring_off = L.qring_off;
+    b.kring_off = L.kring_off;
+    b.gamma_smem = gamma_smem ? 1u : 0u;
     b.timeout_ns = timeout_ns;
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
-    return launch(fn, dim3((unsigned)grid), dim3(32 * warps), L.smem_bytes, s, args);
+    return launch(fn, dim3((unsigned)grid), dim3(32 * (wq + wk)), L.smem_bytes, s, args);
 }
 
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s) {

@@ -64,14 +64,15 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool
                               const FusedArgs &a, int stages, int block, int64_t grid,
                               uint64_t timeout_ns, cudaStream_t s);
 // The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
+// wq warps take Q rows and wk warps take K rows in each CTA.
 struct RowsLayout {
-    uint32_t stage_bytes, gq_off, gk_off, ring_off;
+    uint32_t qstage, kstage, gq_off, gk_off, qring_off, kring_off;
     size_t smem_bytes;
 };
 const void *fused_rows_kernel(int dtype);
-RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int warps, int stages);
-cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int warps, int stages, int64_t grid,
-                              uint64_t timeout_ns, cudaStream_t s);
+RowsLayout rows_layout(int64_t Dq, int64_t Dk, int es, int wq, int wk, int stages, bool gamma_smem);
+cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int wq, int wk, int stages,
+                              bool gamma_smem, int64_t grid, uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s);
 cudaError_t read_device_errors(unsigned *out, bool clear);
 

@@ -144,7 +144,7 @@ def test_plan_for_each_workload(qk):
             assert pl["variant"] == want, (name, T)
             assert pl["groups_q"] == pl["groups_k"] == 1
             if want == qk.VARIANT_ROWS:
-                assert pl["stages"] == 1 and pl["full_lanes"] == 0
+                assert pl["stages"] == 2 and pl["full_lanes"] == 0
                 continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
@@ -243,20 +243,38 @@ def test_bulk_stages_fill_shared_memory(qk):
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
 
 
-def test_rows_warps_fill_shared_memory(qk):
-    """Warp-per-row plan: one row stage per warp, gamma once per CTA, the most
-    warps per SM (at most 16) that shared memory allows, two CTAs preferred."""
+def test_rows_pools_plan(qk):
+    """Warp-per-row plan: a Q pool and a K pool of warps (at least one each,
+    at most 16 together), row stages per warp, CTAs that fit shared memory;
+    the pools follow the widths, and a forced tuning is honoured."""
     try:
         qk.qknorm_force_variant(qk.VARIANT_ROWS, 0)
-        # 65536 x 4096 bf16, P = 8: 8 KiB rows, 32 KiB of gamma: 2 CTAs x 8 warps.
-        pl = qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_BF16, 148)
-        assert (pl["variant"], pl["block"], pl["stages"]) == (qk.VARIANT_ROWS, 256, 1)
-        assert 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
-        # GQA 5120 / 1024: 10 KiB stages (the wider row), 24 KiB of gamma.
+        for T, Dq, Dk, P in ((4096, 5120, 1024, 8), (65536, 4096, 4096, 8), (300, 256, 4096, 2)):
+            pl = qk.qknorm_plan_fwd(T, Dq, Dk, P, qk.QKNORM_BF16, 148)
+            W = pl["block"] // 32
+            wq, wk = pl["q_warps"], W - pl["q_warps"]
+            assert pl["variant"] == qk.VARIANT_ROWS and wq >= 1 and wk >= 1 and W <= 16
+            assert pl["stages"] == 2 and pl["smem_bytes"] <= 227 * 1024
+            if Dq > Dk:
+                assert wq >= wk
+            elif Dq < Dk:
+                assert wq <= wk
+            # every warp of the smaller pool gets a row, the grid stays persistent
+            assert pl["grid"] <= -(-T // min(wq, wk))
+        qk.qknorm_set_rows_tuning(5, 1, 3, 1)
         pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
-        assert (pl["variant"], pl["block"]) == (qk.VARIANT_ROWS, 256)
-        assert pl["grid"] == min(148 * 2, (2 * 4096 + 7) // 8)
+        assert (pl["block"], pl["q_warps"], pl["stages"], pl["gamma_smem"]) == (192, 5, 3, 1)
+        # 19 barriers (padded to 256 B), 24 KiB of gamma, 3 stages of 5 x 10 KiB
+        # Q rows and of 1 x 2 KiB K rows
+        assert pl["smem_bytes"] == 256 + (5120 + 1024) * 4 + 3 * (5 * 10240 + 2048)
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_rows_tuning(0, 2, 0, -1)
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_rows_tuning(9, 8, 0, -1)
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_rows_tuning(1, 1, 0, 2)
     finally:
+        qk.qknorm_set_rows_tuning()
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
 
 

@@ -254,20 +254,21 @@ def test_bounded_wait_times_out_and_reports(qk):
     assert bool((oq == 1.0).all())
 
 
-@pytest.mark.parametrize("warps,stages", [(1, 1), (1, 3), (3, 2), (8, 1), (0, 0), (0, 3)])
+@pytest.mark.parametrize("wq,wk,stages,gsm", [(1, 1, 1, 0), (1, 1, 3, 1), (2, 1, 2, 0), (5, 1, 2, 1),
+                                               (3, 4, 1, 1), (7, 1, 3, 0), (0, 0, 0, -1), (0, 0, 3, 0)])
 @pytest.mark.parametrize("grid", [0, 1, 5])
-def test_rows_variant_rings(qk, warps, stages, grid):
-    """Warp-per-row kernel: any warps per CTA, ring depth and grid (rows wrap
-    the rings many times; Q and K rows of unequal width share the rings) gives
-    the same bits as the generic kernel."""
+def test_rows_variant_rings(qk, wq, wk, stages, gsm, grid):
+    """Warp-per-row kernel: any Q and K pool sizes, ring depth, gamma staging
+    and grid (rows wrap the rings many times; the two pools have rings of
+    their own row widths) gives the same bits as the generic kernel."""
     wl = W.custom("rows", 2 * 148 + 41, 5120, 1024, 8, seed=36)
     q, k, gq, gk = _inputs(wl, wl.Ts[0])
     ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
     try:
-        qk.qknorm_set_rows_tuning(warps, stages)
+        qk.qknorm_set_rows_tuning(wq, wk, stages, gsm)
         got = _fwd(qk, wl, q, k, gq, gk, variant="rows", grid=grid)
     finally:
-        qk.qknorm_set_rows_tuning(0, 0)
+        qk.qknorm_set_rows_tuning()
     assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
     assert qk.qknorm_device_errors() == 0
 
