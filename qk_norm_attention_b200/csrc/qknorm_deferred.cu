@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(256) inv_rms_k(const void *x, float *r, int64_
             for (int p0 = 0; p0 < P; p0 += 4) {
                 float c[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint4 *sh = row + (int64_t)p0 * nv + lane;
+                // Two slots' loads are issued before either is reduced.
+#pragma unroll 2
                 for (int i = 0; i < cnt; ++i) {
                     uint4 v[4];
 #pragma unroll

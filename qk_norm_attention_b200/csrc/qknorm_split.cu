@@ -32,10 +32,29 @@ __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int6
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int stride = kLanes * K;
     const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // Task = t * P + p. The (t, p) of a warp's tasks advance by a fixed step
+    // (nwarps tasks), so they are carried along instead of divided out.
+    const int64_t dt = nwarps / P;
+    const int dp = (int)(nwarps - dt * P);
+    int64_t tb = w0 / P;
+    int pb = (int)(w0 - tb * P);
     // A warp takes R tasks per turn (tasks w0 + (n*R + j)*nwarps) and issues
     // all their loads before reducing any, to keep more bytes in flight.
     for (int64_t base = w0; base < ntask; base += (int64_t)R * nwarps) {
         float S[R];
+        int64_t tj[R];
+        int pj[R];
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            tj[j] = tb;
+            pj[j] = pb;
+            tb += dt;
+            pb += dp;
+            if (pb >= P) {
+                pb -= P;
+                ++tb;
+            }
+        }
         for (int kg = 0; kg < K; ++kg) {
             const int first = kg * kLanes + lane;
             const int cnt = slot_count(first, nv, stride);
@@ -43,8 +62,8 @@ __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int6
 #pragma unroll
             for (int j = 0; j < R; ++j) {
                 const int64_t task = base + (int64_t)j * nwarps;
-                const int64_t t = task / P;
-                const int p = (int)(task - t * P);
+                const int64_t t = tj[j];
+                const int p = pj[j];
                 const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec + (int64_t)p * nv;
 #pragma unroll
                 for (int i = 0; i < VMAX; ++i)
