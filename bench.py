@@ -61,6 +61,12 @@ def parse_args(argv=None):
                          "the largest T of the workload is used")
     ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows"),
                     help="force a kernel variant (for profiling; default: the selector's choice)")
+    ap.add_argument("--path", default="fused", choices=("fused", "split"),
+                    help="what a step runs: qknorm_fwd (default), or the split path "
+                         "(qknorm_partial_sumsq then qknorm_apply, for Q and for K: 4 launches)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per GPU of the timed region (default: the workload's largest T); "
+                         "a smaller T gives a small case for profiling")
     return ap.parse_args(argv)
 
 
@@ -244,6 +250,32 @@ class Fused:
         if st != 0:
             raise RuntimeError(f"qknorm_fwd: {self.qk.qknorm_status_string(st)} "
                                f"{self.qk.qknorm_last_error()}")
+
+
+class Split:
+    """The split path for one buffer set through the raw C ABI: statistics of
+    Q and K (qknorm_partial_sumsq), then the apply step of each (qknorm_apply)."""
+
+    def __init__(self, qk, bufs, stats, T, Dq, Dk, P, eps, dtype_code, stream):
+        q, k, gq, gk, oq, ok = bufs
+        sq, sk = stats
+        L = qk.lib
+        self.calls = [
+            (L.qknorm_partial_sumsq, (q.data_ptr(), sq.data_ptr(), T, Dq, P, dtype_code, stream)),
+            (L.qknorm_partial_sumsq, (k.data_ptr(), sk.data_ptr(), T, Dk, P, dtype_code, stream)),
+            (L.qknorm_apply, (q.data_ptr(), gq.data_ptr(), sq.data_ptr(), oq.data_ptr(), T, Dq, P, eps,
+                              dtype_code, stream)),
+            (L.qknorm_apply, (k.data_ptr(), gk.data_ptr(), sk.data_ptr(), ok.data_ptr(), T, Dk, P, eps,
+                              dtype_code, stream)),
+        ]
+        self.qk = qk
+
+    def __call__(self):
+        for fn, a in self.calls:
+            st = fn(*a)
+            if st != 0:
+                raise RuntimeError(f"split path: {self.qk.qknorm_status_string(st)} "
+                                   f"{self.qk.qknorm_last_error()}")
 
 
 def device_inputs(torch, wl, T, device, row0=0):
@@ -604,7 +636,8 @@ def run_native(args, dist):
     torch.cuda.set_device(device)
     dist.init("nccl")
     wl = W.WORKLOADS[args.workload]
-    T = max(wl.Ts)                     # tokens per GPU (weak scaling)
+    T = args.tokens if args.tokens > 0 else max(wl.Ts)   # tokens per GPU (weak scaling)
+    split = args.path == "split"
     row0, _ = shard_tokens(T * dist.world, dist.world, dist.rank)
     stream = torch.cuda.current_stream(device)
     peak, peak_src = hbm_peak()
@@ -614,8 +647,14 @@ def run_native(args, dist):
     q, k, gq, gk = device_inputs(torch, wl, T, device, row0)
     nsets = buffer_sets(W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes))
     sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(nsets - 1)]
-    calls = [Fused(qk, (a, b, gq, gk, torch.empty_like(a), torch.empty_like(b)), T, wl.Dq, wl.Dk,
-                   wl.P, wl.eps, dt, stream.cuda_stream) for a, b in sets]
+    def step_of(bufs):
+        if split:
+            st = (torch.empty((T, wl.P), dtype=torch.float32, device=device),
+                  torch.empty((T, wl.P), dtype=torch.float32, device=device))
+            return Split(qk, bufs, st, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+        return Fused(qk, bufs, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+
+    calls = [step_of((a, b, gq, gk, torch.empty_like(a), torch.empty_like(b))) for a, b in sets]
     plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, dt)
     for i in range(max(3, args.warmup)):
         calls[i % len(calls)]()
@@ -628,11 +667,16 @@ def run_native(args, dist):
     dist.barrier()
     torch.cuda.synchronize()
     step_ms = dist.max(total_ms / args.steps, device)
-    nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes)
+    if split:
+        nbytes = (W.split_bytes(T, wl.Dq, wl.P, wl.elem_bytes) +
+                  W.split_bytes(T, wl.Dk, wl.P, wl.elem_bytes))
+    else:
+        nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes)
     value = dist.world * nbytes / step_ms / 1e6          # GB/s, all ranks
-    # Each step is one launch of the kernel, so its average duration over the
-    # timed region is the step time (launch gaps included).
-    achieved = nbytes / step_ms / 1e6                    # GB/s, one launch
+    # A fused step is one launch of the kernel, so its average duration over
+    # the timed region is the step time (launch gaps included). A split step is
+    # four launches; its figure is for the four together.
+    achieved = nbytes / step_ms / 1e6                    # GB/s
     # Reference only: the same launches with an event pair around each one.
     _, per = time_launches(torch, calls, min(args.steps, 200), stream, per_launch=True)
     kern_ms = dist.max(statistics.mean(per), device)
@@ -644,7 +688,7 @@ def run_native(args, dist):
     okh = torch.empty(k.shape, dtype=k.dtype).pin_memory()
     qd, kd = sets[1]
     oqd, okd = (torch.empty_like(q), torch.empty_like(k))
-    f = Fused(qk, (qd, kd, gq, gk, oqd, okd), T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+    f = step_of((qd, kd, gq, gk, oqd, okd))
 
     def e2e_step():
         qd.copy_(qh, non_blocking=True)
@@ -684,20 +728,23 @@ def run_native(args, dist):
     dist.barrier()
 
     traffic = None
-    if NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"]:
+    if (not split and args.workload == HEADLINE and T == max(wl.Ts) and
+            NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"]):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
+    kernel = ("stats_k + apply_k (split path, 4 launches per step)" if split
+              else KERNEL_OF_VARIANT.get(plan["variant"], "?") + " (qknorm_fwd)")
     line = {
         "impl": "native",
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": config_of(wl, T, dist.world),
+        "config": dict(config_of(wl, T, dist.world), path=args.path),
         "pct_hbm_peak": round(100 * value / dist.world / peak, 2),
         "tokens_per_s": round(dist.world * T / step_ms * 1000, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": KERNEL_OF_VARIANT.get(plan["variant"], "?") + " (qknorm_fwd)",
+                     "kernel": kernel,
                      "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": nbytes,
                      "launch_us": round(step_ms * 1000, 3),
@@ -707,8 +754,9 @@ def run_native(args, dist):
         "e2e": {"value": round(dist.world * nbytes / e2e_ms / 1e6, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
-                "path": "pinned host -> device copies, qknorm_fwd, device -> pinned host"},
-        "gpu_launches": args.steps,
+                "path": "pinned host -> device copies, " +
+                        ("the split path" if split else "qknorm_fwd") + ", device -> pinned host"},
+        "gpu_launches": args.steps * (4 if split else 1),
         "clocks": clk.summary(),
         "plan": plan,
     }
