@@ -260,7 +260,9 @@ typedef struct {
     int32_t stages;      /* ring stages per CTA (bulk) or per warp (rows), else 0 */
     int32_t tokens_per_stage; /* tokens a bulk stage holds (1 or 2), else 0 */
     int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
-    int32_t full_lanes;  /* 1 if every lane holds exactly vmax vectors per task */
+    int32_t full_lanes;  /* 1 if every lane holds exactly vmax vectors per task; 2 (FP8,
+                            bulk) if every lane holds vmax - 1 and the last slot's
+                            <= 16 vectors are split in halves over the 32 lanes */
     int64_t smem_bytes;  /* dynamic shared memory per CTA */
     int32_t q_warps;     /* rows: warps per CTA that take Q rows (the rest take K rows) */
     int32_t gamma_smem;  /* rows: 1 if gamma is staged in shared memory, 0 if read via L1 */

@@ -202,6 +202,18 @@ bool full_lanes(const Shapes &sh) {
     return full(sh.q) && full(sh.k);
 }
 
+// How the bulk kernel's lanes hold vectors: 1 full (as above); 2 when the
+// dtype is FP8 and each tensor's shards are one group whose last slot holds
+// at most 16 vectors (split in halves over the 32 lanes); else 0.
+int lane_mode(const Shapes &sh, int32_t dtype) {
+    if (full_lanes(sh)) return 1;
+    auto half = [&](const TensorShape &t) {
+        const int r = t.nv - kLanes * (sh.vmax - 1);
+        return t.K == 1 && r > 0 && r <= kLanes / 2;
+    };
+    return (dtype == QKNORM_E4M3 && half(sh.q) && half(sh.k)) ? 2 : 0;
+}
+
 // Gamma in registers pays off while a lane holds few vectors (measured on
 // B200: +5 % at 2 vectors per lane, -7 % at 5, where the registers cost
 // occupancy and gamma hits L1 anyway).
@@ -298,12 +310,13 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     pl->groups_k = sh.k.K;
     int cta_max = 0;
     fused_cta_kernel(dtype, sh.vmax, false, false, &cta_max);
-    pl->full_lanes = full_lanes(sh) ? 1 : 0;
+    pl->full_lanes = lane_mode(sh, dtype);
     const bool cta_ok = sh.ntask * kLanes <= cta_max;
     const int tb = tokens_per_stage_for(sh.vmax);
+    if (pl->full_lanes == 2 && tb != 1) pl->full_lanes = 0;   // the half-slot mode has one token per stage
     const bool greg = gamma_regs_for(dtype, sh.vmax);
     int bulk_max = 0;
-    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, greg, tb, false, &bulk_max) != nullptr;
+    const bool bulk_inst = fused_bulk_kernel(dtype, sh.vmax, greg, tb, 0, &bulk_max) != nullptr;
     const uint32_t stride = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
                                               (int64_t)Dk * elem_of(dtype), tb);
     const bool bulk_ok = bulk_inst && sh.ntask * kLanes <= bulk_max &&
@@ -405,10 +418,10 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy
     switch (pl.variant) {
     case QKNORM_VARIANT_CTA:
         return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0,
-                                pl.full_lanes != 0, nullptr);
+                                pl.full_lanes == 1, nullptr);
     case QKNORM_VARIANT_BULK:
         return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
-                                 pl.full_lanes != 0, nullptr);
+                                 pl.full_lanes, nullptr);
     case QKNORM_VARIANT_ROWS:
         return fused_rows_kernel(dtype);
     default:
@@ -620,14 +633,14 @@ int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const
     a.ldy[1] = ldok / vec;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
-        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes != 0, a, pl.block,
+        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes == 1, a, pl.block,
                              pl.grid, s);
     } else if (pl.variant == QKNORM_VARIANT_ROWS) {
         e = launch_fused_rows(dtype, a, pl.q_warps, pl.block / kLanes - pl.q_warps, pl.stages,
                               pl.gamma_smem != 0, pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
         e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
-                              pl.full_lanes != 0, a, pl.stages, pl.block, pl.grid,
+                              pl.full_lanes, a, pl.stages, pl.block, pl.grid,
                               g_wait_limit_ns, s);
     } else {
         e = launch_fused_generic(dtype, a, pl.block, pl.grid, (size_t)pl.smem_bytes, s);

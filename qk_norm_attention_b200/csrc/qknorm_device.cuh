@@ -95,14 +95,28 @@ __device__ __forceinline__ float vsumsq(BF16Tag, const uint4 &v) {
     return q;
 }
 
-// Same for 16 FP8 values (an E4M3 square is exact in fp32).
-__device__ __forceinline__ float vsumsq(E4M3Tag, const uint4 &v) {
-    float f[16];
-    e4m3x16_to_float(v, f);
-    float q = __fmul_rn(f[0], f[0]);
-#pragma unroll
-    for (int i = 1; i < 16; ++i) q = __fmaf_rn(f[i], f[i], q);
+// The 8 FP8 values of half a vector (w0, w1; element 0 in the low byte of
+// w0): e0*e0, then e_i*e_i + q fused, i = 1..7 (an E4M3 square is exact in
+// fp32, so each fma rounds only the running sum).
+__device__ __forceinline__ float e4m3x8_sumsq(uint32_t w0, uint32_t w1) {
+    const float2 a = e4m3x2_to_float2(w0), b = e4m3x2_to_float2(w0 >> 16);
+    const float2 c = e4m3x2_to_float2(w1), d = e4m3x2_to_float2(w1 >> 16);
+    float q = __fmul_rn(a.x, a.x);
+    q = __fmaf_rn(a.y, a.y, q);
+    q = __fmaf_rn(b.x, b.x, q);
+    q = __fmaf_rn(b.y, b.y, q);
+    q = __fmaf_rn(c.x, c.x, q);
+    q = __fmaf_rn(c.y, c.y, q);
+    q = __fmaf_rn(d.x, d.x, q);
+    q = __fmaf_rn(d.y, d.y, q);
     return q;
+}
+
+// Same for 16 FP8 values: the sums of the two halves (elements 0-7, 8-15),
+// each in order, then added. Two independent chains; and a half vector is a
+// unit the bulk kernel can hand to another lane.
+__device__ __forceinline__ float vsumsq(E4M3Tag, const uint4 &v) {
+    return __fadd_rn(e4m3x8_sumsq(v.x, v.y), e4m3x8_sumsq(v.z, v.w));
 }
 
 // xor butterfly over the 32 lanes; every lane ends with the same bits
@@ -203,21 +217,33 @@ __device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float
     return o;
 }
 
-// FP8: the two multiplies of each pair of values as packed f32x2 multiplies
-// (the same roundings as wmul), which halves their issue slots.
-__device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// FP8, half a vector (8 values, gamma g[0..7]): the two multiplies of each
+// pair of values as packed f32x2 multiplies (the same roundings as wmul),
+// which halves their issue slots.
+__device__ __forceinline__ uint2 vapply_half_regs(E4M3Tag, uint32_t w0, uint32_t w1, const float *g,
+                                                  float r) {
+    const uint32_t w[2] = {w0, w1};
     const float2 rr = make_float2(r, r);
-    uint32_t o[4];
+    uint32_t o[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         const float2 x01 = e4m3x2_to_float2(w[i]);
         const float2 x23 = e4m3x2_to_float2(w[i] >> 16);
         const float2 y01 = fmul2_rn(fmul2_rn(x01, make_float2(g[4 * i], g[4 * i + 1])), rr);
         const float2 y23 = fmul2_rn(fmul2_rn(x23, make_float2(g[4 * i + 2], g[4 * i + 3])), rr);
         o[i] = pack_e4m3x2(y01.x, y01.y) | (pack_e4m3x2(y23.x, y23.y) << 16);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    return make_uint2(o[0], o[1]);
+}
+
+__device__ __forceinline__ uint2 vapply_half(E4M3Tag, const uint2 &h, const float *g, float r) {
+    return vapply_half_regs(E4M3Tag{}, h.x, h.y, g, r);
+}
+
+__device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r) {
+    const uint2 lo = vapply_half_regs(E4M3Tag{}, v.x, v.y, g, r);
+    const uint2 hi = vapply_half_regs(E4M3Tag{}, v.z, v.w, g + 8, r);
+    return make_uint4(lo.x, lo.y, hi.x, hi.y);
 }
 
 __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r) {

@@ -42,9 +42,19 @@ constexpr uint32_t kRedBytes = 2 * kMaxTB * 32 * sizeof(float);
 constexpr uint32_t kStageBase = kBarBytes + kRedBytes;
 constexpr uint32_t kMaxStages = 16;
 
-template <class Tag, int VMAX, bool GREG, int TB, bool FULL, int MAXT>
+// MODE (how lanes hold vectors): 0 any shape (guards); 1 every lane of every
+// task holds exactly VMAX vectors (no guards); 2 (FP8) every lane holds
+// VMAX - 1 whole vectors and the last slot's r <= 16 vectors are split in
+// halves over the 32 lanes (lane l and l + 16 take the low and high 8 bytes
+// of vector l), so the last slot costs half a slot instead of running with
+// half the lanes idle. The vector sum of squares is defined as the sum of its
+// two halves' sums, so the split changes no bits.
+template <class Tag, int VMAX, bool GREG, int TB, int MODE, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const BulkArgs b) {
     constexpr int VEC = Tag::kVec;
+    constexpr bool FULL = MODE == 1;
+    constexpr bool HALF = MODE == 2;
+    constexpr int NW = HALF ? VMAX - 1 : VMAX;     // whole-vector slots
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     float(*red)[kMaxTB][32] = reinterpret_cast<float(*)[kMaxTB][32]>(smem + kBarBytes);
@@ -62,8 +72,12 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     const int nv = z ? a.nv[1] : a.nv[0];
     const int stride = kLanes * K;
     const int first = kg * kLanes + lane;
-    // FULL: every lane of every task holds exactly VMAX vectors (no guards).
-    const int cnt = FULL ? VMAX : slot_count(first, nv, stride);
+    const int cnt = (FULL || HALF) ? NW : slot_count(first, nv, stride);
+    // HALF: this lane's half of the last slot: vector hv of the slot, bytes
+    // 8*hh .. 8*hh + 7 of it; hok if that vector exists.
+    const int hv = lane & 15, hh = lane >> 4;
+    const bool hok = HALF && hv < nv - kLanes * NW;
+    const int64_t hcol = (int64_t)p * nv + kLanes * NW + hv;   // its vector index in the row
     const int64_t ldy = z ? a.ldy[1] : a.ldy[0];     // output row stride, in vectors
     const int64_t col0 = (int64_t)p * nv + first;
     uint4 *ys = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + col0;
@@ -74,6 +88,7 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     const uint32_t tok_bytes = b.qbytes + b.kbytes;
     // This lane's first vector inside a token of a stage (Q row, then K row).
     const uint32_t lane_off = (z ? b.qbytes : 0u) + (uint32_t)col0 * 16u;
+    const uint32_t half_off = (z ? b.qbytes : 0u) + (uint32_t)hcol * 16u + 8u * hh;
 
     const int64_t T = a.T;
     const int64_t G = gridDim.x;
@@ -116,8 +131,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
     float gam[GREG ? VMAX * VEC : 1];
     if (GREG) {
 #pragma unroll
-        for (int i = 0; i < VMAX; ++i)
-            if (FULL || i < cnt) {
+        for (int i = 0; i < NW; ++i)
+            if (FULL || HALF || i < cnt) {
 #pragma unroll
                 for (int e = 0; e < VEC; e += 4) {
                     const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
@@ -128,6 +143,17 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
                     gam[i * VEC + e + 3] = g4.w;
                 }
             }
+        if (HALF && hok) {
+#pragma unroll
+            for (int e = 0; e < VEC / 2; e += 4) {
+                const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
+                    (z ? a.g[1] : a.g[0]) + hcol * VEC + 8 * hh + e));
+                gam[NW * VEC + e] = g4.x;
+                gam[NW * VEC + e + 1] = g4.y;
+                gam[NW * VEC + e + 2] = g4.z;
+                gam[NW * VEC + e + 3] = g4.w;
+            }
+        }
     }
 
     int s = 0;
@@ -137,14 +163,20 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
         const int64_t t0 = blockIdx.x + n * TB * G;
         const bool ok = mbar_wait_bounded(&full[s], phase, b.timeout_ns);
         const unsigned char *st = stages + (size_t)s * b.stage_stride + lane_off;
-        uint4 cur[TB][VMAX];
+        uint4 cur[TB][NW > 0 ? NW : 1];
+        uint2 hlf[TB];
+        const unsigned char *sth = stages + (size_t)s * b.stage_stride + half_off;
 #pragma unroll
         for (int j = 0; j < TB; ++j) {
             const uint4 *src = reinterpret_cast<const uint4 *>(st + j * tok_bytes);
 #pragma unroll
-            for (int i = 0; i < VMAX; ++i)
-                cur[j][i] = ((FULL || i < cnt) && (j == 0 || t0 + j * G < T)) ? src[i * stride]
-                                                                              : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < NW; ++i)
+                cur[j][i] = ((FULL || HALF || i < cnt) && (j == 0 || t0 + j * G < T)) ? src[i * stride]
+                                                                                      : make_uint4(0, 0, 0, 0);
+            if constexpr (HALF)
+                hlf[j] = (hok && (j == 0 || t0 + j * G < T))
+                             ? *reinterpret_cast<const uint2 *>(sth + j * tok_bytes)
+                             : make_uint2(0, 0);
         }
         // Phase A for TB tokens: independent chains and butterflies. A lane's
         // missing vectors are its last slots and read as zeros, whose sum of
@@ -154,7 +186,15 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
         for (int j = 0; j < TB; ++j) {
             c[j] = 0.f;
 #pragma unroll
-            for (int i = 0; i < VMAX; ++i) c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
+            for (int i = 0; i < NW; ++i) c[j] = __fadd_rn(c[j], vsumsq(Tag{}, cur[j][i]));
+            if constexpr (HALF) {
+                // The last slot: this lane's half sum; lane l < 16 adds the
+                // high half's sum from lane l + 16 to its own low half (the
+                // vector's sum, by its definition), then to its chain.
+                const float h = e4m3x8_sumsq(hlf[j].x, hlf[j].y);
+                const float hi = __shfl_down_sync(kFull, h, 16);
+                if (lane < 16) c[j] = __fadd_rn(c[j], __fadd_rn(h, hi));
+            }
         }
 #pragma unroll
         for (int j = 0; j < TB; ++j) c[j] = butterfly(c[j]);
@@ -192,8 +232,8 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
                 const float r = factor(combine_fast(&red[buf][j][red_base], a.P, K), Df, eps);
                 uint4 *dst = ys + t * ldy;
 #pragma unroll
-                for (int i = 0; i < VMAX; ++i)
-                    if (FULL || i < cnt) {
+                for (int i = 0; i < NW; ++i)
+                    if (FULL || HALF || i < cnt) {
                         uint4 y;
                         if (GREG)
                             y = vapply_regs(Tag{}, cur[j][i], &gam[i * VEC], r);
@@ -201,6 +241,18 @@ __global__ void __launch_bounds__(MAXT, 1) fused_bulk(const FusedArgs a, const B
                             y = vapply(Tag{}, cur[j][i], gs + (int64_t)i * stride * VEC, r);
                         st_stream(dst + (int64_t)i * stride, y);
                     }
+                if constexpr (HALF) {
+                  if (hok) {
+                    float gh[VEC / 2];
+#pragma unroll
+                    for (int e = 0; e < VEC / 2; ++e)
+                        gh[e] = GREG ? gam[NW * VEC + e]
+                                     : __ldg((z ? a.g[1] : a.g[0]) + hcol * VEC + 8 * hh + e);
+                    const uint2 y = vapply_half(Tag{}, hlf[j], gh, r);
+                    unsigned char *yb = reinterpret_cast<unsigned char *>(z ? a.y[1] : a.y[0]);
+                    __stcs(reinterpret_cast<uint2 *>(yb + (t * ldy + hcol) * 16 + 8 * hh), y);
+                  }
+                }
             }
         }
         buf ^= 1;
@@ -419,52 +471,69 @@ constexpr bool bulk_exists(int vmax, int tb, int vec, bool greg) {
     return vmax >= 1 && vmax <= kVcap && (tb == 1 || tb == 2) && vmax * tb <= 12 &&
            (vec != 16 || (vmax * tb <= 4 && (tb == 1 || !greg) && (!greg || vmax <= 3)));
 }
+// The half-slot mode exists for FP8 with one token per stage.
+constexpr bool bulk_mode_exists(int vmax, int tb, int vec, bool greg, int mode) {
+    return bulk_exists(vmax, tb, vec, greg) && mode >= 0 && mode <= 2 &&
+           (mode != 2 || (vec == 16 && tb == 1));
+}
 constexpr int bulk_max_threads(int vmax, int tb, int vec) {
     return (vmax * tb <= 2 && vmax * tb * vec <= 16) ? 1024 : 512;
 }
 
-template <class Tag, bool GREG, int V, int TB, bool FULL>
+template <class Tag, bool GREG, int V, int TB, int MODE>
 const void *bulk_fn() {
-    if constexpr (bulk_exists(V, TB, Tag::kVec, GREG))
+    if constexpr (bulk_mode_exists(V, TB, Tag::kVec, GREG, MODE))
         return reinterpret_cast<const void *>(
-            &fused_bulk<Tag, V, GREG, TB, FULL, bulk_max_threads(V, TB, Tag::kVec)>);
+            &fused_bulk<Tag, V, GREG, TB, MODE, bulk_max_threads(V, TB, Tag::kVec)>);
     else
         return nullptr;
 }
 
-template <class Tag, bool GREG, int TB, bool FULL>
+template <class Tag, bool GREG, int TB, int MODE>
 const void *bulk_table_tb(int vmax) {
     switch (vmax) {
-    case 1: return bulk_fn<Tag, GREG, 1, TB, FULL>();
-    case 2: return bulk_fn<Tag, GREG, 2, TB, FULL>();
-    case 3: return bulk_fn<Tag, GREG, 3, TB, FULL>();
-    case 4: return bulk_fn<Tag, GREG, 4, TB, FULL>();
-    case 5: return bulk_fn<Tag, GREG, 5, TB, FULL>();
-    case 6: return bulk_fn<Tag, GREG, 6, TB, FULL>();
-    case 7: return bulk_fn<Tag, GREG, 7, TB, FULL>();
-    case 8: return bulk_fn<Tag, GREG, 8, TB, FULL>();
+    case 1: return bulk_fn<Tag, GREG, 1, TB, MODE>();
+    case 2: return bulk_fn<Tag, GREG, 2, TB, MODE>();
+    case 3: return bulk_fn<Tag, GREG, 3, TB, MODE>();
+    case 4: return bulk_fn<Tag, GREG, 4, TB, MODE>();
+    case 5: return bulk_fn<Tag, GREG, 5, TB, MODE>();
+    case 6: return bulk_fn<Tag, GREG, 6, TB, MODE>();
+    case 7: return bulk_fn<Tag, GREG, 7, TB, MODE>();
+    case 8: return bulk_fn<Tag, GREG, 8, TB, MODE>();
+    default: return nullptr;
+    }
+}
+
+template <class Tag, bool GREG, int TB>
+const void *bulk_table_mode(int vmax, int mode) {
+    switch (mode) {
+    case 0: return bulk_table_tb<Tag, GREG, TB, 0>(vmax);
+    case 1: return bulk_table_tb<Tag, GREG, TB, 1>(vmax);
+    case 2: return bulk_table_tb<Tag, GREG, TB, 2>(vmax);
     default: return nullptr;
     }
 }
 
 template <class Tag, bool GREG>
-const void *bulk_table(int vmax, int tb, bool full) {
-    if (tb == 1) return full ? bulk_table_tb<Tag, GREG, 1, true>(vmax) : bulk_table_tb<Tag, GREG, 1, false>(vmax);
-    if (tb == 2) return full ? bulk_table_tb<Tag, GREG, 2, true>(vmax) : bulk_table_tb<Tag, GREG, 2, false>(vmax);
+const void *bulk_table(int vmax, int tb, int mode) {
+    if (tb == 1) return bulk_table_mode<Tag, GREG, 1>(vmax, mode);
+    if (tb == 2) return bulk_table_mode<Tag, GREG, 2>(vmax, mode);
     return nullptr;
 }
 
-const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int mode,
                               int *max_threads) {
     const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
-    if (!bulk_exists(vmax, tb, vec, gamma_regs)) return nullptr;
+    if (!bulk_exists(vmax, tb, vec, gamma_regs) || mode < 0 || mode > 2 ||
+        (mode == 2 && (vec != 16 || tb != 1)))
+        return nullptr;
     if (max_threads) *max_threads = bulk_max_threads(vmax, tb, vec);
     if (dtype == 0)
-        return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb, full) : bulk_table<F32Tag, false>(vmax, tb, full);
+        return gamma_regs ? bulk_table<F32Tag, true>(vmax, tb, mode) : bulk_table<F32Tag, false>(vmax, tb, mode);
     if (dtype == 1)
-        return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb, full) : bulk_table<BF16Tag, false>(vmax, tb, full);
+        return gamma_regs ? bulk_table<BF16Tag, true>(vmax, tb, mode) : bulk_table<BF16Tag, false>(vmax, tb, mode);
     if (dtype == 2)
-        return gamma_regs ? bulk_table<E4M3Tag, true>(vmax, tb, full) : bulk_table<E4M3Tag, false>(vmax, tb, full);
+        return gamma_regs ? bulk_table<E4M3Tag, true>(vmax, tb, mode) : bulk_table<E4M3Tag, false>(vmax, tb, mode);
     return nullptr;
 }
 
@@ -478,10 +547,10 @@ size_t bulk_smem_bytes(int stages, uint32_t stage_stride) {
 
 int bulk_max_stages() { return (int)kMaxStages; }
 
-cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, int mode,
                               const FusedArgs &a, int stages, int block, int64_t grid,
                               uint64_t timeout_ns, cudaStream_t s) {
-    const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, full, nullptr);
+    const void *fn = fused_bulk_kernel(dtype, vmax, gamma_regs, tb, mode, nullptr);
     if (!fn || stages < 1 || stages > (int)kMaxStages) return cudaErrorInvalidValue;
     const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
     BulkArgs b;

@@ -54,13 +54,15 @@ cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *
                          cudaStream_t s);
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
-// tb = tokens per ring stage (1, 2 or 4); nullptr if (vmax, tb) has no instance.
-const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+// tb = tokens per ring stage (1 or 2); mode: 0 any shape, 1 every lane holds
+// vmax whole vectors, 2 (FP8) vmax - 1 whole vectors and half a vector of the
+// last slot (see the kernel); nullptr if the combination has no instance.
+const void *fused_bulk_kernel(int dtype, int vmax, bool gamma_regs, int tb, int mode,
                               int *max_threads);
 uint32_t bulk_stage_stride(int64_t qbytes, int64_t kbytes, int tb);
 size_t bulk_smem_bytes(int stages, uint32_t stage_stride);
 int bulk_max_stages();
-cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, bool full,
+cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, int mode,
                               const FusedArgs &a, int stages, int block, int64_t grid,
                               uint64_t timeout_ns, cudaStream_t s);
 // The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
