@@ -47,7 +47,8 @@
  * of squares of vectors v = 32k + l + 32Ki; the 32 lane sums are combined by
  * an xor butterfly (16, 8, 4, 2, 1); the K group sums are added in order of
  * k, giving S[t,p]; the P shard sums are added in order of p. A vector's sum
- * of squares is e0*e0 followed by fused multiply-adds of e1..e_last.
+ * of squares is e0*e0 followed by fused multiply-adds of e1..e_last; for FP8
+ * (16 values) it is that sum over e0..e7 plus that sum over e8..e15.
  * Then r = rsqrt(S / D + eps) and y = (x * gamma) * r, each step fp32.
  */
 #ifndef QKNORM_H
