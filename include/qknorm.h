@@ -161,12 +161,46 @@ QKNORM_API int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int3
  * S = stats[t,0] + ... + stats[t,P-1] (in order of p), r = rsqrt(S/D + eps),
  * out[t,j] = (x[t,j] * gamma[j]) * r. A caller that already holds combined
  * per-token sums passes them as stats [T, 1] with P = 1.
- *   x [T, D] input, dtype; gamma [D] fp32; stats [T, P] fp32; out [T, D].
+ *   x [T, D] input, dtype; gamma [D] fp32; stats [T, P] fp32 (4-byte
+ *   alignment suffices: it is read one value at a time); out [T, D].
  * With stats from qknorm_partial_sumsq, out equals qknorm_fwd's bit for bit.
  * Returns a qknorm_status.
  */
 QKNORM_API int qknorm_apply(const void *x, const float *gamma, const float *stats, void *out,
                  int64_t T, int32_t D, int32_t P, float eps, int32_t dtype, void *stream);
+
+/*
+ * qknorm_apply_tp -- the apply step of one rank of a tensor-parallel group.
+ *
+ * SwiftQK technical review, Section 3, Algorithm 1 in its tensor-parallel
+ * form: the hidden dimension is split across `ranks` GPUs; each rank holds
+ * the D_local-wide slice of every row (its P_local shards), forms its shard
+ * sums (Phase A, qknorm_partial_sumsq on its slice), the group exchanges
+ * them, and each rank finishes its own slice (Phases B and C) with the full
+ * width H_total = ranks * D_local as the divisor. This call is that last
+ * step, given the exchanged sums as an all-gather of every rank's [T, P_local]
+ * leaves them:
+ *   stats: ranks blocks of [T, P_local] fp32, block g (rank g's shard sums)
+ *   at stats + g * stats_block_stride floats (0 means T * P_local, the dense
+ *   [ranks, T, P_local]; a larger stride serves a gather of several tensors'
+ *   sums at once, e.g. [ranks, 2, T, P_local] for Q and K with stride
+ *   2 * T * P_local and stats offset by T * P_local for K; stats need only
+ *   4-byte alignment here and in qknorm_apply);
+ *   S = the ranks * P_local sums in order of the global shard index
+ *       (g * P_local + p), r = rsqrt(S / (ranks * D_local) + eps),
+ *   out[t,j] = (x[t,j] * gamma[j]) * r for the local slice.
+ *   x [T, D_local] input, dtype; gamma [D_local] fp32 (the rank's slice of
+ *   gamma); out [T, D_local] output, dtype.
+ * With rank g's stats from qknorm_partial_sumsq(x_g, ..., D_local, P_local),
+ * out on rank g equals columns [g * D_local, (g + 1) * D_local) of qknorm_fwd
+ * on the whole rows with P = ranks * P_local, bit for bit. ranks = 1 is
+ * qknorm_apply. Errors as qknorm_apply; also QKNORM_ERR_INVALID_ARG for
+ * ranks < 1 or a stride below T * P_local (overlapping blocks).
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_apply_tp(const void *x, const float *gamma, const float *stats,
+                               int64_t stats_block_stride, void *out, int64_t T, int32_t D_local,
+                               int32_t P_local, int32_t ranks, float eps, int32_t dtype, void *stream);
 
 /*
  * qknorm_xgamma -- the weight multiply alone: out[t,j] = x[t,j] * gamma[j],

@@ -88,6 +88,8 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_headwise_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32,
                                         i64, i64, i64, i64, vp]
     lib.qknorm_headwise_fwd.restype = ctypes.c_int
+    lib.qknorm_apply_tp.argtypes = [vp, vp, vp, i64, vp, i64, i32, i32, i32, f32, i32, vp]
+    lib.qknorm_apply_tp.restype = ctypes.c_int
     lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     lib.qknorm_xgamma.restype = ctypes.c_int
     lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
@@ -281,6 +283,32 @@ def qknorm_apply(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps:
     st = lib.qknorm_apply(x.data_ptr(), gamma.data_ptr(), stats.data_ptr(), out.data_ptr(), T, D,
                           P, float(eps), _dtype_code(x), _stream_handle(x.device, stream))
     _check("qknorm_apply", st)
+    return out
+
+
+def qknorm_apply_tp(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps: float,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One tensor-parallel rank's apply step: x [T, D_local] (this rank's
+    slice), gamma [D_local], stats [ranks, T, P_local] (every rank's shard
+    sums, rank-major, as an all-gather leaves them; a strided view with
+    contiguous [T, P_local] blocks is accepted). The divisor is ranks * D_local."""
+    if x.dim() != 2 or stats.dim() != 3 or stats.shape[1] != x.shape[0]:
+        raise ValueError("x must be [T, D_local] and stats [ranks, T, P_local]")
+    T, D = x.shape
+    ranks, _, P = stats.shape
+    out = torch.empty_like(x) if out is None else out
+    for name, t in (("x", x), ("gamma", gamma), ("out", out)):
+        _need_cuda_contig(name, t)
+    if not stats.is_cuda or stats.stride(2) != 1 or stats.stride(1) != P:
+        raise ValueError("stats blocks must be contiguous [T, P_local] on the GPU")
+    if gamma.dtype != torch.float32 or stats.dtype != torch.float32:
+        raise TypeError("gamma and stats must be float32")
+    if out.shape != x.shape or out.dtype != x.dtype or gamma.numel() != D:
+        raise ValueError("out must match x; gamma must have D_local elements")
+    st = lib.qknorm_apply_tp(x.data_ptr(), gamma.data_ptr(), stats.data_ptr(), stats.stride(0),
+                             out.data_ptr(), T, D, P, ranks, float(eps), _dtype_code(x),
+                             _stream_handle(x.device, stream))
+    _check("qknorm_apply_tp", st)
     return out
 
 

@@ -514,9 +514,51 @@ int finish(cudaError_t e) {
 
 using namespace qkn;
 
+// The apply step for stats laid out as nb blocks [nb, T, Pb] (nb = 1: the
+// split path's [T, P]; nb = ranks: an all-gather of each rank's [T, P_local]
+// in a tensor-parallel group, whose rows are the D-wide local slices of
+// nb * D-wide rows). The divisor is nb * D.
+static int apply_blocks(const void *x, const float *gamma, const float *stats, int64_t sg, void *out,
+                        int64_t T, int32_t D, int32_t Pb, int32_t nb, float eps, int32_t dtype,
+                        void *stream) {
+    int st = check_shape(T, D, Pb, dtype);
+    if (st == QKNORM_OK) st = check_eps(eps);
+    if (st != QKNORM_OK) return st;
+    if (nb < 1 || (int64_t)D * nb > INT32_MAX) return QKNORM_ERR_INVALID_ARG;
+    if (T == 0) return QKNORM_OK;
+    if (!x || !gamma || !stats || !out) return QKNORM_ERR_INVALID_ARG;
+    // The statistics are read one fp32 at a time: 4-byte alignment suffices
+    // (a gather of Q's and K's sums puts K's blocks T * P floats further on).
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(out) ||
+        reinterpret_cast<uintptr_t>(stats) % 4 != 0)
+        return QKNORM_ERR_MISALIGNED;
+    if (T > INT64_MAX / 4 / Pb / nb) return QKNORM_ERR_INVALID_ARG;
+    if (sg == 0) sg = T * Pb;
+    if (sg < T * Pb || sg > INT64_MAX / 4 / nb) return QKNORM_ERR_INVALID_ARG;   // blocks may not overlap
+    const int64_t es = elem_of(dtype);
+    const Range ro = rng(out, T * D * es);
+    if (bad_alias(ro, rng(x, T * D * es), true) || bad_alias(ro, rng(gamma, (int64_t)D * 4), false) ||
+        bad_alias(ro, rng(stats, ((int64_t)(nb - 1) * sg + T * Pb) * 4), false))
+        return QKNORM_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    cudaError_t e = device_sms(&dev, &sms);
+    if (e != cudaSuccess) return finish(e);
+    const int64_t rowvec = D / vec_of(dtype);
+    int block = (int)((rowvec + kLanes - 1) / kLanes * kLanes);
+    if (block > 256) block = 256;
+    int bres = 1;
+    e = resident_blocks(dev, apply_kernel(dtype), block, 0, &bres);
+    if (e != cudaSuccess) return finish(e);
+    int64_t grid = (int64_t)sms * bres;
+    if (grid > T) grid = T;
+    return finish(launch_apply(dtype, x, gamma, stats, out, T, D, Pb, nb, sg,
+                               (float)((int64_t)D * nb), eps, block, grid,
+                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 extern "C" {
 
-int qknorm_version(void) { return 110; }
+int qknorm_version(void) { return 111; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -846,32 +888,15 @@ int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int3
 
 int qknorm_apply(const void *x, const float *gamma, const float *stats, void *out, int64_t T,
                  int32_t D, int32_t P, float eps, int32_t dtype, void *stream) {
-    int st = check_shape(T, D, P, dtype);
-    if (st == QKNORM_OK) st = check_eps(eps);
-    if (st != QKNORM_OK) return st;
-    if (T == 0) return QKNORM_OK;
-    if (!x || !gamma || !stats || !out) return QKNORM_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(gamma) || !aligned16(stats) || !aligned16(out))
-        return QKNORM_ERR_MISALIGNED;
-    if (T > INT64_MAX / 4 / P) return QKNORM_ERR_INVALID_ARG;
-    const int64_t es = elem_of(dtype);
-    const Range ro = rng(out, T * D * es);
-    if (bad_alias(ro, rng(x, T * D * es), true) || bad_alias(ro, rng(gamma, (int64_t)D * 4), false) ||
-        bad_alias(ro, rng(stats, T * P * 4), false))
-        return QKNORM_ERR_INVALID_ARG;
-    int dev = 0, sms = 0;
-    cudaError_t e = device_sms(&dev, &sms);
-    if (e != cudaSuccess) return finish(e);
-    const int64_t rowvec = D / vec_of(dtype);
-    int block = (int)((rowvec + kLanes - 1) / kLanes * kLanes);
-    if (block > 256) block = 256;
-    int bres = 1;
-    e = resident_blocks(dev, apply_kernel(dtype), block, 0, &bres);
-    if (e != cudaSuccess) return finish(e);
-    int64_t grid = (int64_t)sms * bres;
-    if (grid > T) grid = T;
-    return finish(launch_apply(dtype, x, gamma, stats, out, T, D, P, eps, block, grid,
-                               reinterpret_cast<cudaStream_t>(stream)));
+    return apply_blocks(x, gamma, stats, 0, out, T, D, P, 1, eps, dtype, stream);
+}
+
+int qknorm_apply_tp(const void *x, const float *gamma, const float *stats, int64_t stats_block_stride,
+                    void *out, int64_t T, int32_t D_local, int32_t P_local, int32_t ranks, float eps,
+                    int32_t dtype, void *stream) {
+    if (stats_block_stride < 0) return QKNORM_ERR_INVALID_ARG;
+    return apply_blocks(x, gamma, stats, stats_block_stride, out, T, D_local, P_local, ranks, eps,
+                        dtype, stream);
 }
 
 }  // extern "C"

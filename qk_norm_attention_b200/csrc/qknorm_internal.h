@@ -49,9 +49,11 @@ cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64
 cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64_t T,
                          const TensorShape &sh, int32_t P, int block, int64_t grid,
                          cudaStream_t s);
+// stats of token t: nb blocks of Pb sums, block b at stats + b * sg + t * Pb;
+// Df the divisor (full width).
 cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
-                         int64_t T, int32_t D, int32_t P, float eps, int block, int64_t grid,
-                         cudaStream_t s);
+                         int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg, float Df,
+                         float eps, int block, int64_t grid, cudaStream_t s);
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // tb = tokens per ring stage (1 or 2); mode: 0 any shape, 1 every lane holds

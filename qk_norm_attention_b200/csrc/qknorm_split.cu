@@ -89,16 +89,22 @@ __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int6
     }
 }
 
+// The statistics of token t are nb blocks of Pb shard sums, block b at
+// stats[b * sg + t * Pb + 0 .. Pb-1]: one block [T, P] for the split path
+// (nb = 1, Pb = P), or one block per rank of a tensor-parallel group as an
+// all-gather lays them out ([ranks, T, P_local]). They are added block by
+// block, each in order, which is the order of the global shard index.
+// The divisor Df is the full width (the local row width D, or the width
+// summed over the group).
 template <class Tag>
 __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, const float *stats,
-                                               void *y, int64_t T, int32_t D, int32_t P,
-                                               float eps) {
+                                               void *y, int64_t T, int32_t D, int32_t Pb, int32_t nb,
+                                               int64_t sg, float Df, float eps) {
     constexpr int VEC = Tag::kVec;
     constexpr int UNR = 4;
     pdl_wait();
     pdl_trigger();
     const int64_t rowvec = D / VEC;
-    const float Df = (float)D;
     const int nthr = blockDim.x;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec;
@@ -112,11 +118,13 @@ __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, co
                 if (v < rowvec) xv[u] = ld_stream(src + v);
             }
             if (v0 == 0) {
-                // Phase B: S = sum of the P shard sums, in order of p.
-                const float *st = stats + t * P;
+                // Phase B: S = sum of the shard sums, in order of the shard.
                 float S = 0.f;
+                for (int b = 0; b < nb; ++b) {
+                    const float *st = stats + b * sg + t * Pb;
 #pragma unroll 8
-                for (int p = 0; p < P; ++p) S = __fadd_rn(S, __ldg(st + p));
+                    for (int p = 0; p < Pb; ++p) S = __fadd_rn(S, __ldg(st + p));
+                }
                 r = factor(S, Df, eps);
             }
 #pragma unroll
@@ -178,12 +186,12 @@ cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64
 }
 
 cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
-                         int64_t T, int32_t D, int32_t P, float eps, int block, int64_t grid,
-                         cudaStream_t s) {
+                         int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg, float Df,
+                         float eps, int block, int64_t grid, cudaStream_t s) {
     const void *fn = apply_kernel(dtype);
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<void **>(&x), const_cast<float **>(&g),
-                    const_cast<float **>(&stats), &y, &T, &D, &P, &eps};
+                    const_cast<float **>(&stats), &y, &T, &D, &Pb, &nb, &sg, &Df, &eps};
     return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 

@@ -112,6 +112,21 @@ def test_split_rejects(qk):
     assert L.qknorm_apply(A, B, C, C, 4, 256, 4, 1e-6, 1, None) == 1   # out on stats
     assert L.qknorm_apply(A, B, C, A + 32, 4, 256, 4, 1e-6, 1, None) == 1
     assert L.qknorm_apply(A, B, C, Dd, 4, 256, 4, 1e-6, 9, None) == 3
+    assert L.qknorm_apply(A, B, C + 2, Dd, 4, 256, 4, 1e-6, 1, None) == 2   # stats need 4-byte alignment
+
+
+@needs_cpu
+def test_apply_tp_rejects(qk):
+    L = qk.lib
+    # x, gamma, stats, block stride, out, T, D_local, P_local, ranks, eps, dtype, stream
+    assert L.qknorm_apply_tp(A, B, C, 0, Dd, 4, 256, 4, 0, 1e-6, 1, None) == 1    # ranks < 1
+    assert L.qknorm_apply_tp(A, B, C, -1, Dd, 4, 256, 4, 2, 1e-6, 1, None) == 1   # negative stride
+    assert L.qknorm_apply_tp(A, B, C, 15, Dd, 4, 256, 4, 2, 1e-6, 1, None) == 1   # blocks overlap
+    assert L.qknorm_apply_tp(A, B, C + 2, 0, Dd, 4, 256, 4, 2, 1e-6, 1, None) == 2
+    assert L.qknorm_apply_tp(A + 8, B, C, 0, Dd, 4, 256, 4, 2, 1e-6, 1, None) == 2
+    assert L.qknorm_apply_tp(A, B, C, 0, Dd, 4, 256, 3, 2, 1e-6, 1, None) == 1    # D_local % P_local
+    assert L.qknorm_apply_tp(A, B, C, 0, C + 16, 4, 256, 4, 2, 1e-6, 1, None) == 1  # out on stats
+    assert L.qknorm_apply_tp(0, 0, 0, 0, 0, 0, 256, 4, 2, 1e-6, 1, None) == 0     # T = 0
 
 
 @needs_cpu
