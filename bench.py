@@ -44,7 +44,7 @@ KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_ge
 # From profiles/fused_bulk_prefill13b_full.md: dram__bytes_read.sum 167,837,952
 # + dram__bytes_write.sum 111,811,840 for one launch (cold, serialised capture;
 # ~56 MB of the writes were still in L2 when the kernel ended).
-NCU_TRAFFIC = {"src_sha": "5e5e2838ead8b065", "bytes_per_launch": 279847936}
+NCU_TRAFFIC = {"src_sha": "99136614c8a992f2", "bytes_per_launch": 279488768}
 
 
 def parse_args(argv=None):

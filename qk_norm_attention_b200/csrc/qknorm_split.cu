@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, co
             if (v0 == 0) {
                 // Phase B: S = sum of the shard sums, in order of the shard.
                 float S = 0.f;
-                for (int b = 0; b < nb; ++b) {
-                    const float *st = stats + b * sg + t * Pb;
+                const float *st = stats + t * Pb;
+                for (int b = 0; b < nb; ++b, st += sg) {
 #pragma unroll 8
                     for (int p = 0; p < Pb; ++p) S = __fadd_rn(S, __ldg(st + p));
                 }
