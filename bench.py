@@ -44,7 +44,9 @@ KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_ge
 # From profiles/fused_bulk_prefill13b_full.md: dram__bytes_read.sum 167,837,952
 # + dram__bytes_write.sum 111,811,840 for one launch (cold, serialised capture;
 # ~56 MB of the writes were still in L2 when the kernel ended).
-NCU_TRAFFIC = {"src_sha": "99136614c8a992f2", "bytes_per_launch": 279488768}
+NCU_TRAFFIC = {"src_sha": "9fa4a41f266a8af8", "bytes_per_launch": 279488768,
+               "plan": {"variant": 3, "block": 256, "grid": 296, "vmax": 5, "stages": 2,
+                        "tokens_per_stage": 1, "gamma_regs": 0, "full_lanes": 1}}
 
 
 def parse_args(argv=None):
@@ -73,9 +75,11 @@ def parse_args(argv=None):
 VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4}
 
 
-# The sources that define the headline kernel (fused_bulk) and the plan it runs with.
+# The sources of the headline kernel (fused_bulk) and of its launch. The
+# traffic figure is valid while they are unchanged AND the launch plan equals
+# the one captured (the plan is the selector's, in qknorm_api.cu).
 HEADLINE_SOURCES = ("qknorm_fused_bulk.cu", "qknorm_bulk.cuh", "qknorm_device.cuh",
-                    "qknorm_internal.h", "qknorm_api.cu")
+                    "qknorm_internal.h")
 
 
 def kernel_src_sha() -> str:
@@ -689,13 +693,30 @@ def run_native(args, dist):
     qd, kd = sets[1]
     oqd, okd = (torch.empty_like(q), torch.empty_like(k))
     f = step_of((qd, kd, gq, gk, oqd, okd))
+    if split:
+        e2e_path = "pinned host -> device copies, the split path, device -> pinned host"
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        f()
-        oqh.copy_(oqd, non_blocking=True)
-        okh.copy_(okd, non_blocking=True)
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            f()
+            oqh.copy_(oqd, non_blocking=True)
+            okh.copy_(okd, non_blocking=True)
+    else:
+        # The library's host-buffer entry point: chunks of 512 tokens copied in,
+        # normalised and copied out, the two copy directions overlapping.
+        e2e_path = ("qknorm_fwd_host: pinned host rows in, 512-token chunks over 3 device "
+                    "workspace sets, host->device copy / kernel / device->host copy overlapped")
+        ws = torch.empty(qk.qknorm_fwd_host_workspace(wl.Dq, wl.Dk, q.dtype), dtype=torch.uint8,
+                         device=device)
+        hargs = (qh.data_ptr(), kh.data_ptr(), gq.data_ptr(), gk.data_ptr(), oqh.data_ptr(),
+                 okh.data_ptr(), T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, ws.data_ptr(), ws.numel(), 0,
+                 stream.cuda_stream)
+
+        def e2e_step():
+            st = qk.lib.qknorm_fwd_host(*hargs)
+            if st != 0:
+                raise RuntimeError(f"qknorm_fwd_host: {qk.qknorm_status_string(st)}")
 
     e2e_step()
     torch.cuda.synchronize()
@@ -709,6 +730,12 @@ def run_native(args, dist):
     e2e_ms = dist.max(e0.elapsed_time(e1) / e2e_steps, device)
     h2d = (qh.numel() + kh.numel()) * qh.element_size()
     d2h = (oqh.numel() + okh.numel()) * oqh.element_size()
+    e2e_ok = True
+    if not split:      # the host outputs of the last step equal the device path's
+        f()
+        torch.cuda.synchronize()
+        e2e_ok = bool(torch.equal(oqh.view(torch.uint8), oqd.cpu().view(torch.uint8)) and
+                      torch.equal(okh.view(torch.uint8), okd.cpu().view(torch.uint8)))
     del qh, kh, oqh, okh
 
     extras = {}
@@ -729,7 +756,8 @@ def run_native(args, dist):
 
     traffic = None
     if (not split and args.workload == HEADLINE and T == max(wl.Ts) and
-            NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"]):
+            NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"] and
+            all(plan.get(key) == val for key, val in NCU_TRAFFIC["plan"].items())):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     kernel = ("stats_k + apply_k (split path, 4 launches per step)" if split
               else KERNEL_OF_VARIANT.get(plan["variant"], "?") + " (qknorm_fwd)")
@@ -754,8 +782,7 @@ def run_native(args, dist):
         "e2e": {"value": round(dist.world * nbytes / e2e_ms / 1e6, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
-                "path": "pinned host -> device copies, " +
-                        ("the split path" if split else "qknorm_fwd") + ", device -> pinned host"},
+                "path": e2e_path, "outputs_equal_device_path": e2e_ok},
         "gpu_launches": args.steps * (4 if split else 1),
         "clocks": clk.summary(),
         "plan": plan,

@@ -203,6 +203,43 @@ QKNORM_API int qknorm_apply_tp(const void *x, const float *gamma, const float *s
                                int32_t P_local, int32_t ranks, float eps, int32_t dtype, void *stream);
 
 /*
+ * qknorm_fwd_host -- qknorm_fwd on rows in HOST memory, end to end: the rows
+ * go to the device, are normalised there and come back (no counterpart in
+ * the paper; it is the path a caller with host-resident activations takes).
+ *
+ * The T tokens are processed in chunks of chunk_tokens (0 = 512). Each chunk
+ * is copied host-to-device into one of three workspace sets, normalised in
+ * place by qknorm_fwd on `stream`, and copied back, with the copies on two
+ * streams of the library's own, so the host-to-device copy of one chunk, the
+ * kernel of the next and the device-to-host copy of a third overlap (the two
+ * copy directions use separate copy engines). Results equal qknorm_fwd's bit
+ * for bit.
+ *   q, k [T, Dq], [T, Dk] host input, dtype; out_q, out_k host outputs of
+ *   the same shapes (each may be its own input; no other overlap); gamma_q,
+ *   gamma_k fp32 on the DEVICE; workspace: device memory of at least
+ *   qknorm_fwd_host_workspace(chunk_tokens, Dq, Dk, dtype) bytes, 16-byte
+ *   aligned, owned by the caller and not used by anything else until the
+ *   call's work has completed.
+ * Ordering: all work is ordered after the work already on `stream`, and work
+ * enqueued on `stream` afterwards waits until the outputs are in host memory
+ * (synchronise `stream` before reading them). Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister); pageable memory works but its copies do
+ * not overlap. Enqueueing is serialised across host threads.
+ * Returns a qknorm_status (QKNORM_ERR_INVALID_ARG also for a workspace that
+ * is too small or a negative chunk_tokens).
+ */
+QKNORM_API int qknorm_fwd_host(const void *q, const void *k, const float *gamma_q,
+                               const float *gamma_k, void *out_q, void *out_k, int64_t T,
+                               int32_t Dq, int32_t Dk, int32_t P, float eps, int32_t dtype,
+                               void *workspace, int64_t workspace_bytes, int64_t chunk_tokens,
+                               void *stream);
+
+/* Workspace bytes qknorm_fwd_host needs for chunk_tokens (0 = the default),
+ * or -1 for invalid widths or dtype. */
+QKNORM_API int64_t qknorm_fwd_host_workspace(int64_t chunk_tokens, int32_t Dq, int32_t Dk,
+                                             int32_t dtype);
+
+/*
  * qknorm_xgamma -- the weight multiply alone: out[t,j] = x[t,j] * gamma[j],
  * rounded once to dtype, no normalisation.
  *

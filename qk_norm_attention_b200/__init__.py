@@ -23,7 +23,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -88,6 +88,11 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_headwise_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32,
                                         i64, i64, i64, i64, vp]
     lib.qknorm_headwise_fwd.restype = ctypes.c_int
+    lib.qknorm_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, f32, i32, vp, i64,
+                                    i64, vp]
+    lib.qknorm_fwd_host.restype = ctypes.c_int
+    lib.qknorm_fwd_host_workspace.argtypes = [i64, i32, i32, i32]
+    lib.qknorm_fwd_host_workspace.restype = ctypes.c_int64
     lib.qknorm_apply_tp.argtypes = [vp, vp, vp, i64, vp, i64, i32, i32, i32, f32, i32, vp]
     lib.qknorm_apply_tp.restype = ctypes.c_int
     lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
@@ -284,6 +289,43 @@ def qknorm_apply(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps:
                           P, float(eps), _dtype_code(x), _stream_handle(x.device, stream))
     _check("qknorm_apply", st)
     return out
+
+
+def qknorm_fwd_host_workspace(Dq: int, Dk: int, dtype: torch.dtype, chunk_tokens: int = 0) -> int:
+    """Device workspace bytes qknorm_fwd_host needs."""
+    n = lib.qknorm_fwd_host_workspace(int(chunk_tokens), int(Dq), int(Dk), _DTYPE[dtype])
+    if n < 0:
+        raise ValueError("invalid widths or dtype")
+    return n
+
+
+def qknorm_fwd_host(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                    P: int, eps: float, workspace: torch.Tensor,
+                    out_q: Optional[torch.Tensor] = None, out_k: Optional[torch.Tensor] = None,
+                    chunk_tokens: int = 0, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """qknorm_fwd on CPU tensors q [T, Dq], k [T, Dk] (pinned for overlap),
+    gamma on the GPU, `workspace` a uint8 CUDA tensor of at least
+    qknorm_fwd_host_workspace bytes. Returns CPU outputs; they are complete
+    once `stream` (default: the current stream of workspace's device) is
+    synchronised."""
+    if q.dim() != 2 or k.dim() != 2 or q.shape[0] != k.shape[0] or q.dtype != k.dtype:
+        raise ValueError("q [T, Dq] and k [T, Dk] of one dtype")
+    if q.is_cuda or k.is_cuda or not (q.is_contiguous() and k.is_contiguous()):
+        raise ValueError("q and k must be contiguous host (CPU) tensors")
+    T, Dq = q.shape
+    Dk = k.shape[1]
+    out_q = torch.empty_like(q, pin_memory=q.is_pinned()) if out_q is None else out_q
+    out_k = torch.empty_like(k, pin_memory=k.is_pinned()) if out_k is None else out_k
+    for name, t in (("gamma_q", gamma_q), ("gamma_k", gamma_k), ("workspace", workspace)):
+        _need_cuda_contig(name, t)
+    if out_q.shape != q.shape or out_k.shape != k.shape or out_q.is_cuda or out_k.is_cuda:
+        raise ValueError("outputs must be host tensors shaped like q and k")
+    st = lib.qknorm_fwd_host(q.data_ptr(), k.data_ptr(), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                             out_q.data_ptr(), out_k.data_ptr(), T, Dq, Dk, int(P), float(eps),
+                             _dtype_code(q), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             int(chunk_tokens), _stream_handle(workspace.device, stream))
+    _check("qknorm_fwd_host", st)
+    return out_q, out_k
 
 
 def qknorm_apply_tp(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, eps: float,

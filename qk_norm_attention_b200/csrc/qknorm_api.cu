@@ -509,6 +509,48 @@ int finish(cudaError_t e) {
     return QKNORM_OK;
 }
 
+// ---------------------------------------------------------------- host buffers
+
+// qknorm_fwd_host's pipeline: per device, a stream for host-to-device copies,
+// one for device-to-host copies (both non-blocking) and kHostSets workspace
+// sets with three events each, created once. The caller's stream runs the
+// kernels. Calls are serialised by a mutex while they enqueue.
+constexpr int kHostSets = 3;
+constexpr int64_t kHostChunkDefault = 512;   // tokens per chunk
+constexpr int kHostMaxDevices = 64;
+
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t in_done[kHostSets] = {}, k_done[kHostSets] = {}, out_done[kHostSets] = {};
+};
+HostPipe g_host_pipes[kHostMaxDevices];
+std::mutex g_host_mu;
+
+cudaError_t host_pipe(HostPipe **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kHostMaxDevices) return cudaErrorInvalidDevice;
+    HostPipe &hp = g_host_pipes[dev];
+    if (!hp.ready) {
+        if ((e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming)) != cudaSuccess) return e;
+        for (int i = 0; i < kHostSets; ++i) {
+            if ((e = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+            if ((e = cudaEventCreateWithFlags(&hp.k_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+            if ((e = cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+        }
+        hp.ready = true;
+    }
+    *out = &hp;
+    return cudaSuccess;
+}
+
+int64_t host_chunk(int64_t chunk_tokens) { return chunk_tokens > 0 ? chunk_tokens : kHostChunkDefault; }
+
 }  // namespace
 }  // namespace qkn
 
@@ -558,7 +600,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 111; }
+int qknorm_version(void) { return 112; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -897,6 +939,83 @@ int qknorm_apply_tp(const void *x, const float *gamma, const float *stats, int64
     if (stats_block_stride < 0) return QKNORM_ERR_INVALID_ARG;
     return apply_blocks(x, gamma, stats, stats_block_stride, out, T, D_local, P_local, ranks, eps,
                         dtype, stream);
+}
+
+int64_t qknorm_fwd_host_workspace(int64_t chunk_tokens, int32_t Dq, int32_t Dk, int32_t dtype) {
+    if (Dq <= 0 || Dk <= 0 || (dtype != QKNORM_F32 && dtype != QKNORM_BF16 && dtype != QKNORM_E4M3))
+        return -1;
+    const int64_t C = host_chunk(chunk_tokens);
+    const int64_t row = ((int64_t)Dq + Dk) * elem_of(dtype);
+    if (C > INT64_MAX / kHostSets / row) return -1;
+    return kHostSets * C * row;
+}
+
+int qknorm_fwd_host(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+                    void *out_q, void *out_k, int64_t T, int32_t Dq, int32_t Dk, int32_t P, float eps,
+                    int32_t dtype, void *workspace, int64_t workspace_bytes, int64_t chunk_tokens,
+                    void *stream) {
+    int st = check_shape(T, Dq, P, dtype);
+    if (st == QKNORM_OK) st = check_shape(T, Dk, P, dtype);
+    if (st == QKNORM_OK) st = check_eps(eps);
+    if (st != QKNORM_OK) return st;
+    if (chunk_tokens < 0) return QKNORM_ERR_INVALID_ARG;
+    if (T == 0) return QKNORM_OK;
+    if (!q || !k || !gamma_q || !gamma_k || !out_q || !out_k || !workspace) return QKNORM_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return QKNORM_ERR_MISALIGNED;
+    int64_t C = host_chunk(chunk_tokens);
+    if (C > T) C = T;
+    const int64_t es = elem_of(dtype);
+    const int64_t qrow = (int64_t)Dq * es, krow = (int64_t)Dk * es;
+    if (T > INT64_MAX / (qrow + krow)) return QKNORM_ERR_INVALID_ARG;
+    const int64_t need = qknorm_fwd_host_workspace(C, Dq, Dk, dtype);
+    if (need < 0 || workspace_bytes < need) return QKNORM_ERR_INVALID_ARG;
+    // Host ranges must not overlap the outputs (inputs and outputs are
+    // distinct host buffers; an output may be its own input).
+    const Range roq = rng(out_q, T * qrow), rok = rng(out_k, T * krow);
+    if (bad_alias(roq, rng(q, T * qrow), true) || bad_alias(roq, rng(k, T * krow), false) ||
+        bad_alias(rok, rng(k, T * krow), true) || bad_alias(rok, rng(q, T * qrow), false) ||
+        overlap(roq, rok))
+        return QKNORM_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    HostPipe *hp = nullptr;
+    cudaError_t e = host_pipe(&hp);
+    if (e != cudaSuccess) return finish(e);
+    // Everything is ordered after the work already on the caller's stream.
+    if ((e = cudaEventRecord(hp->start, s)) != cudaSuccess) return finish(e);
+    if ((e = cudaStreamWaitEvent(hp->h2d, hp->start, 0)) != cudaSuccess) return finish(e);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const unsigned char *qh = static_cast<const unsigned char *>(q);
+    const unsigned char *kh = static_cast<const unsigned char *>(k);
+    unsigned char *oqh = static_cast<unsigned char *>(out_q);
+    unsigned char *okh = static_cast<unsigned char *>(out_k);
+    int64_t c = 0;
+    for (int64_t t0 = 0; t0 < T; t0 += C, ++c) {
+        const int64_t n = (T - t0) < C ? (T - t0) : C;
+        const int i = (int)(c % kHostSets);
+        unsigned char *dq = ws + (int64_t)i * C * (qrow + krow);
+        unsigned char *dk = dq + C * qrow;
+        // Set i is free once its previous contents have left for the host.
+        if ((e = cudaStreamWaitEvent(hp->h2d, hp->out_done[i], 0)) != cudaSuccess) return finish(e);
+        if ((e = cudaMemcpyAsync(dq, qh + t0 * qrow, n * qrow, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(dk, kh + t0 * krow, n * krow, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess ||
+            (e = cudaEventRecord(hp->in_done[i], hp->h2d)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(s, hp->in_done[i], 0)) != cudaSuccess)
+            return finish(e);
+        // The chunk is normalised in place in the workspace.
+        st = qknorm_fwd(dq, dk, gamma_q, gamma_k, dq, dk, n, Dq, Dk, P, eps, dtype, stream);
+        if (st != QKNORM_OK) return st;
+        if ((e = cudaEventRecord(hp->k_done[i], s)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(hp->d2h, hp->k_done[i], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(oqh + t0 * qrow, dq, n * qrow, cudaMemcpyDeviceToHost, hp->d2h)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(okh + t0 * krow, dk, n * krow, cudaMemcpyDeviceToHost, hp->d2h)) != cudaSuccess ||
+            (e = cudaEventRecord(hp->out_done[i], hp->d2h)) != cudaSuccess)
+            return finish(e);
+    }
+    // Later work on the caller's stream waits for the outputs to reach the host.
+    for (int i = 0; i < kHostSets && i < c; ++i)
+        if ((e = cudaStreamWaitEvent(s, hp->out_done[i], 0)) != cudaSuccess) return finish(e);
+    return QKNORM_OK;
 }
 
 }  // extern "C"

@@ -115,6 +115,32 @@ def test_split_rejects(qk):
     assert L.qknorm_apply(A, B, C + 2, Dd, 4, 256, 4, 1e-6, 1, None) == 2   # stats need 4-byte alignment
 
 
+def test_host_workspace_size(qk):
+    L = qk.lib
+    assert L.qknorm_fwd_host_workspace(0, 5120, 5120, 1) == 3 * 512 * 10240 * 2
+    assert L.qknorm_fwd_host_workspace(7, 256, 128, 0) == 3 * 7 * 384 * 4
+    assert L.qknorm_fwd_host_workspace(7, 256, 128, 2) == 3 * 7 * 384
+    assert L.qknorm_fwd_host_workspace(7, 0, 128, 1) == -1
+    assert L.qknorm_fwd_host_workspace(7, 256, 128, 9) == -1
+
+
+@needs_cpu
+def test_fwd_host_rejects(qk):
+    L = qk.lib
+    ws = L.qknorm_fwd_host_workspace(4, 256, 256, 1)    # T = 4 tokens make one chunk of 4
+    # q, k, gamma_q, gamma_k, out_q, out_k, T, Dq, Dk, P, eps, dtype, ws, ws_bytes, chunk, stream
+    base = [A, A + 0x100000, B, B + 0x1000, C, C + 0x100000, 4, 256, 256, 4, 1e-6, 1, Dd, ws, 0, None]
+    call = lambda **kw: L.qknorm_fwd_host(*[kw.get(str(i), v) for i, v in enumerate(base)])
+    assert call(**{"13": ws - 16}) == 1          # workspace too small
+    assert call(**{"12": Dd + 8}) == 2           # workspace not 16-byte aligned
+    assert call(**{"14": -1}) == 1               # negative chunk
+    assert call(**{"4": A + 64}) == 1            # out_q partly over q
+    assert call(**{"5": C + 512}) == 1           # out_k over out_q
+    assert call(**{"6": 0}) == 0                 # T = 0
+    assert call(**{"9": 3}) == 1                 # D % P
+    assert call(**{"12": 0}) == 1                # no workspace
+
+
 @needs_cpu
 def test_apply_tp_rejects(qk):
     L = qk.lib
