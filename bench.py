@@ -37,14 +37,14 @@ HEADLINE = "prefill13b"
 FALLBACK_HBM_GBS = 6650.0
 
 KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_generic",
-                     3: "fused_bulk", 4: "fused_rows"}
+                     3: "fused_bulk", 4: "fused_rows", 5: "fused_pair"}
 
 # dram bytes per launch of the headline kernel from one ncu capture, and the
 # hash of the kernel sources it was taken with (None until captured).
 # From profiles/fused_bulk_prefill13b_full.md: dram__bytes_read.sum 167,837,952
 # + dram__bytes_write.sum 111,811,840 for one launch (cold, serialised capture;
 # ~56 MB of the writes were still in L2 when the kernel ended).
-NCU_TRAFFIC = {"src_sha": "9fa4a41f266a8af8", "bytes_per_launch": 279488768,
+NCU_TRAFFIC = {"src_sha": "aa4e7d5756db0513", "bytes_per_launch": 279488768,
                "plan": {"variant": 3, "block": 256, "grid": 296, "vmax": 5, "stages": 2,
                         "tokens_per_stage": 1, "gamma_regs": 0, "full_lanes": 1}}
 
@@ -61,7 +61,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS),
                     help="workload of the timed region (default: the 13B-shaped prefill); "
                          "the largest T of the workload is used")
-    ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows"),
+    ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows", "pair"),
                     help="force a kernel variant (for profiling; default: the selector's choice)")
     ap.add_argument("--path", default="fused", choices=("fused", "split"),
                     help="what a step runs: qknorm_fwd (default), or the split path "
@@ -72,22 +72,31 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4}
+VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4, "pair": 5}
 
 
-# The sources of the headline kernel (fused_bulk) and of its launch. The
-# traffic figure is valid while they are unchanged AND the launch plan equals
-# the one captured (the plan is the selector's, in qknorm_api.cu).
-HEADLINE_SOURCES = ("qknorm_fused_bulk.cu", "qknorm_bulk.cuh", "qknorm_device.cuh",
-                    "qknorm_internal.h")
+# The source of the headline kernel (the fused_bulk template, from its
+# declaration to the next section of its file) and of the device helpers it
+# uses. The traffic figure is valid while they are unchanged AND the launch
+# plan equals the one captured (the plan is the selector's, in qknorm_api.cu).
+HEADLINE_SOURCES = (
+    ("qknorm_fused_bulk.cu", "template <class Tag, int VMAX, bool GREG, int TB, int MODE, int MAXT>",
+     "// ---------------------------------------------------------------- warp per row"),
+    ("qknorm_bulk.cuh", None, None),
+    ("qknorm_device.cuh", None, None),
+)
 
 
 def kernel_src_sha() -> str:
     csrc = os.path.join(ROOT, "qk_norm_attention_b200", "csrc")
     h = hashlib.sha256()
-    for f in HEADLINE_SOURCES:
+    for f, start, end in HEADLINE_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+            text = fh.read()
+        if start is not None:
+            i = text.index(start.encode())
+            text = text[i:text.index(end.encode(), i)]
+        h.update(f.encode() + b"\0" + text)
     return h.hexdigest()[:16]
 
 

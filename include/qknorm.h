@@ -313,11 +313,15 @@ typedef enum {
     QKNORM_VARIANT_BULK = 3,    /* as CTA, but rows arrive by bulk asynchronous
                                    copies (TMA engine) into a ring of token stages
                                    in shared memory, completed on mbarriers */
-    QKNORM_VARIANT_ROWS = 4     /* warp per row: a CTA has a pool of warps for
+    QKNORM_VARIANT_ROWS = 4,    /* warp per row: a CTA has a pool of warps for
                                    Q rows and one for K rows; each warp has its
                                    own ring of bulk-copied row stages, walks all
                                    P shards of the row itself and applies from
                                    shared memory; no CTA barrier per row */
+    QKNORM_VARIANT_PAIR = 5     /* as BULK with P warps per token instead of 2P
+                                   (GQA-like shapes: P even, K shards of <= 16
+                                   vectors): a warp takes two Q shards, or two
+                                   K shards on its lane halves */
 } qknorm_variant;
 
 /* A launch plan chosen by the selector (host-side description). */

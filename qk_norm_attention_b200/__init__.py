@@ -37,10 +37,10 @@ QKNORM_ERR_MISALIGNED = 2
 QKNORM_ERR_UNSUPPORTED = 3
 QKNORM_ERR_CUDA = 4
 
-VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_ROWS = \
-    -1, 0, 1, 2, 3, 4
+VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_ROWS, VARIANT_PAIR = \
+    -1, 0, 1, 2, 3, 4, 5
 VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic",
-                 VARIANT_BULK: "bulk", VARIANT_ROWS: "rows"}
+                 VARIANT_BULK: "bulk", VARIANT_ROWS: "rows", VARIANT_PAIR: "pair"}
 
 _DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16,
           torch.float8_e4m3fn: QKNORM_E4M3}

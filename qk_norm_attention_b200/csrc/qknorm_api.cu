@@ -301,6 +301,20 @@ bool rows_fit(int32_t Dq, int32_t Dk, int32_t dtype) {
     return rows_fits(Dq, Dk, dtype, 1, 1, 1, false, 1);
 }
 
+// The shard-pair ring's conditions: P even and at most 16 (P warps), one
+// group per shard, K shards of at most 16 vectors (one per lane of a half
+// warp), Q shards of at most 3 vectors per lane, and an instance for the
+// gamma placement.
+bool pair_greg(const Shapes &sh, int32_t dtype) {
+    if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
+    return !(dtype == QKNORM_E4M3 && sh.q.vmax >= 3);
+}
+
+bool pair_fits(const Shapes &sh, int32_t P, int32_t dtype) {
+    return !(P & 1) && P <= 16 && sh.q.K == 1 && sh.k.K == 1 && sh.k.nv <= kLanes / 2 &&
+           sh.q.vmax <= 3 && fused_pair_kernel(dtype, sh.q.vmax, pair_greg(sh, dtype)) != nullptr;
+}
+
 // Static part of the plan: which kernel, block size, template width, stages.
 int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t variant,
                 int num_sms, int regs, qknorm_plan *pl) {
@@ -331,9 +345,15 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         // fit one CTA go to the rows kernel too.
         // FP8 is instruction-bound, and the token ring with gamma in registers
         // wins for it even on ragged lanes (measured 63 % vs 46 % for rows).
+        // GQA-like shapes (Q shards wider than a warp, K shards of at most 16
+        // vectors) take the shard-pair ring: P warps per token instead of 2P,
+        // two CTAs per SM (measured at T = 4096, 5120/1024, P = 8: 84.8 % vs
+        // 66.4 % for rows and 59.8 % for the ring with 2P warps).
         const bool ragged = !pl->full_lanes && dtype != QKNORM_E4M3;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
+        else if (pair_fits(sh, P, dtype) && sh.q.nv > kLanes)
+            variant = QKNORM_VARIANT_PAIR;
         else if (bulk_ok && !(ragged && rows_ok))
             variant = QKNORM_VARIANT_BULK;
         else if (rows_ok)
@@ -354,6 +374,29 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
                 pl->smem_bytes > kSmemPerCta)
                 return QKNORM_ERR_UNSUPPORTED;
         }
+        return QKNORM_OK;
+    }
+    if (variant == QKNORM_VARIANT_PAIR) {
+        // P warps: Q shards in pairs, K shards (<= 16 vectors) in pairs on lane halves.
+        if (!pair_fits(sh, P, dtype)) return QKNORM_ERR_UNSUPPORTED;
+        const bool greg_p = pair_greg(sh, dtype);
+        pl->variant = QKNORM_VARIANT_PAIR;
+        pl->block = P * kLanes;
+        pl->vmax = sh.q.vmax;
+        pl->gamma_regs = greg_p ? 1 : 0;
+        pl->tokens_per_stage = 1;
+        const uint32_t stride1 = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
+                                                   (int64_t)Dk * elem_of(dtype), 1);
+        bulk_stages(stride1, pl->block, regs > 0 ? regs : kRegsHint, pl);
+        // A third stage pays once a CTA meets about 20 tokens or more (measured:
+        // T = 8192, 86.1 -> 89.5 %; T = 16384, 90.9 -> 95.6 %; T = 4096, 84.8 -> 83.7 %).
+        if (g_tune_stages == 0 && pl->stages == 2 && T >= 40 * (int64_t)num_sms &&
+            2 * ((int64_t)bulk_smem_bytes(3, stride1) + kSmemReservedPerCta) <= kSmemPerSm) {
+            pl->stages = 3;
+            pl->smem_bytes = (int64_t)bulk_smem_bytes(3, stride1);
+        }
+        if (pl->stages < 1 || pl->stages > bulk_max_stages() || pl->smem_bytes > kSmemPerCta)
+            return QKNORM_ERR_UNSUPPORTED;
         return QKNORM_OK;
     }
     if (variant == QKNORM_VARIANT_ROWS) {
@@ -424,6 +467,8 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy
                                  pl.full_lanes, nullptr);
     case QKNORM_VARIANT_ROWS:
         return fused_rows_kernel(dtype);
+    case QKNORM_VARIANT_PAIR:
+        return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0);
     default:
         return fused_generic_kernel(dtype);
     }
@@ -480,7 +525,8 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     if (e != cudaSuccess) return e;
     *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, kRegsHint, pl);
     if (*status != QKNORM_OK) return cudaSuccess;
-    if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS) {
+    if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS ||
+        pl->variant == QKNORM_VARIANT_PAIR) {
         int regs = kRegsHint;
         e = kernel_regs(plan_kernel(*pl, dtype, true), &regs);
         if (e != cudaSuccess) return e;
@@ -491,7 +537,8 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     if (pl->smem_bytes > 48 * 1024 || pl->variant == QKNORM_VARIANT_GENERIC ||
         pl->variant == QKNORM_VARIANT_WARP) {
         e = prepare_kernel(dev, fn, (pl->variant == QKNORM_VARIANT_BULK ||
-                                     pl->variant == QKNORM_VARIANT_ROWS) ? kSmemPerCta : kGenericMaxSmem);
+                                     pl->variant == QKNORM_VARIANT_ROWS ||
+                                     pl->variant == QKNORM_VARIANT_PAIR) ? kSmemPerCta : kGenericMaxSmem);
         if (e != cudaSuccess) return e;
     }
     int bres = 1;
@@ -616,7 +663,7 @@ const char *qknorm_status_string(int status) {
 const char *qknorm_last_error(void) { return g_last_error; }
 
 int qknorm_force_variant(int32_t variant, int64_t grid) {
-    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_ROWS || grid < 0)
+    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_PAIR || grid < 0)
         return QKNORM_ERR_INVALID_ARG;
     g_forced_variant = variant;
     g_forced_grid = grid;
@@ -722,6 +769,9 @@ int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const
     } else if (pl.variant == QKNORM_VARIANT_ROWS) {
         e = launch_fused_rows(dtype, a, pl.q_warps, pl.block / kLanes - pl.q_warps, pl.stages,
                               pl.gamma_smem != 0, pl.grid, g_wait_limit_ns, s);
+    } else if (pl.variant == QKNORM_VARIANT_PAIR) {
+        e = launch_fused_pair(dtype, pl.vmax, pl.gamma_regs != 0, a, pl.stages, pl.grid,
+                              g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
         e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
                               pl.full_lanes, a, pl.stages, pl.block, pl.grid,

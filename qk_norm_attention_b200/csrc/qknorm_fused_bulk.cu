@@ -448,6 +448,197 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
     }
 }
 
+// ---------------------------------------------------------------- shard pairs
+
+// The token ring for GQA-like shapes (P even, K shards of at most 16 vectors):
+// a CTA of P warps per token instead of 2P. Warp w < P/2 takes Q shards 2w and
+// 2w + 1 (two independent lane chains and butterflies, each shard's order
+// unchanged); warp P/2 + w takes K shards 2w and 2w + 1 on its lane halves
+// (lanes 0-15 and 16-31, one vector per lane) and reduces each half with a
+// 16-lane butterfly. That equals the 32-lane butterfly bit for bit: the xor-16
+// step it skips adds the exact zeros of the lanes past a shard's 16 vectors.
+// With half the warps per token, two CTAs fit an SM and each warp carries
+// twice the work per token barrier. One token per stage.
+template <class Tag, int VQ, bool GREG>
+__global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const BulkArgs b) {
+    constexpr int VEC = Tag::kVec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    float(*red)[64] = reinterpret_cast<float(*)[64]>(smem + kBarBytes);   // [buf][Q: 0..31, K: 32..63]
+    unsigned char *stages = smem + kStageBase;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int half = a.P >> 1;
+    const int z = warp < half ? 0 : 1;
+    const int w = z ? warp - half : warp;
+    const int pa = 2 * w;                                // first shard of the pair
+    const int nvq = a.nv[0], nvk = a.nv[1];
+    // Q: this lane's vectors of shards pa, pa + 1: lane + 32 i, i < cnt.
+    const int cnt = z ? 0 : slot_count(lane, nvq, kLanes);
+    // K: lane half h takes shard pa + h, vector kv of it.
+    const int hk = lane >> 4, kv = lane & 15;
+    const bool kok = z && kv < nvk;
+    const int kshard = pa + hk;
+    const float Df = z ? a.Df[1] : a.Df[0];
+    const float eps = a.eps;
+    const uint32_t tok_bytes = b.qbytes + b.kbytes;
+    // Offsets inside a stage (bytes): Q vector (p, v) at (p*nvq + v)*16; K at
+    // qbytes + (p*nvk + v)*16.
+    const uint32_t qoff = (uint32_t)((pa * nvq + lane) * 16);
+    const uint32_t koff = b.qbytes + (uint32_t)((kshard * nvk + kv) * 16);
+
+    const int64_t T = a.T;
+    const int64_t G = gridDim.x;
+    const int S = (int)b.stages;
+    const char *qsrc = static_cast<const char *>(a.x[0]);
+    const char *ksrc = static_cast<const char *>(a.x[1]);
+    const int64_t ldq_b = a.ldx[0] * 16, ldk_b = a.ldx[1] * 16;
+
+    auto issue = [&](int s, int64_t n) {
+        unsigned char *st = stages + (size_t)s * b.stage_stride;
+        const int64_t tt = blockIdx.x + n * G;
+        mbar_arrive_expect_tx(&full[s], tok_bytes);
+        bulk_copy_g2s(st, qsrc + tt * ldq_b, b.qbytes, &full[s]);
+        bulk_copy_g2s(st + b.qbytes, ksrc + tt * ldk_b, b.kbytes, &full[s]);
+    };
+
+    const int64_t npass = (T - blockIdx.x + G - 1) / G;
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+    if (tid == 0) {
+        for (int s = 0; s < S && s < npass; ++s) issue(s, s);
+    }
+
+    // Gamma in registers: Q lanes 2 x VQ vectors, K lanes one vector.
+    float gam[GREG ? 2 * VQ * VEC : 1];
+    if (GREG) {
+        if (z == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < VQ; ++i)
+                    if (i < cnt)
+#pragma unroll
+                        for (int e = 0; e < VEC; e += 4) {
+                            const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
+                                a.g[0] + ((int64_t)(pa + h) * nvq + lane + 32 * i) * VEC + e));
+                            float *d = &gam[(h * VQ + i) * VEC + e];
+                            d[0] = g4.x;
+                            d[1] = g4.y;
+                            d[2] = g4.z;
+                            d[3] = g4.w;
+                        }
+        } else if (kok) {
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4) {
+                const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
+                    a.g[1] + ((int64_t)kshard * nvk + kv) * VEC + e));
+                gam[e] = g4.x;
+                gam[e + 1] = g4.y;
+                gam[e + 2] = g4.z;
+                gam[e + 3] = g4.w;
+            }
+        }
+    }
+
+    int s = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    for (int64_t n = 0; n < npass; ++n) {
+        const int64_t t = blockIdx.x + n * G;
+        const bool ok = mbar_wait_bounded(&full[s], phase, b.timeout_ns);
+        const unsigned char *st = stages + (size_t)s * b.stage_stride;
+        uint4 cur[2][VQ];
+        float c0 = 0.f, c1 = 0.f;
+        if (z == 0) {
+            const uint4 *src0 = reinterpret_cast<const uint4 *>(st + qoff);
+            const uint4 *src1 = src0 + nvq;
+#pragma unroll
+            for (int i = 0; i < VQ; ++i) {
+                cur[0][i] = i < cnt ? src0[32 * i] : make_uint4(0, 0, 0, 0);
+                cur[1][i] = i < cnt ? src1[32 * i] : make_uint4(0, 0, 0, 0);
+            }
+            // Missing vectors are a lane's last slots and add +0 (no change).
+#pragma unroll
+            for (int i = 0; i < VQ; ++i) {
+                c0 = __fadd_rn(c0, vsumsq(Tag{}, cur[0][i]));
+                c1 = __fadd_rn(c1, vsumsq(Tag{}, cur[1][i]));
+            }
+            c0 = butterfly(c0);
+            c1 = butterfly(c1);
+            if (lane == 0) {
+                red[buf][pa] = c0;
+                red[buf][pa + 1] = c1;
+            }
+        } else {
+            cur[0][0] = kok ? *reinterpret_cast<const uint4 *>(st + koff) : make_uint4(0, 0, 0, 0);
+            // One vector per lane: the lane chain is its vector's sum (0 + s).
+            c0 = vsumsq(Tag{}, cur[0][0]);
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) c0 = __fadd_rn(c0, __shfl_xor_sync(kFull, c0, off));
+            if (kv == 0) red[buf][32 + kshard] = c0;
+        }
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_device_errors, kErrWaitTimeout);
+                int ds = s;
+                uint32_t dp = phase;
+                for (int64_t m = n; m < npass && m < n + S; ++m) {
+                    if (!mbar_wait_bounded(&full[ds], dp, b.timeout_ns))
+                        atomicOr(&g_device_errors, kErrDrainTimeout);
+                    if (++ds == S) {
+                        ds = 0;
+                        dp ^= 1u;
+                    }
+                }
+            }
+            return;
+        }
+        if (tid == 0 && n + S < npass) {
+            fence_proxy_async_smem();
+            issue(s, n + S);
+        }
+        const float r = factor(combine_fast(&red[buf][z ? 32 : 0], a.P, 1), Df, eps);
+        if (z == 0) {
+            uint4 *dst = reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0] + (int64_t)pa * nvq + lane;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < VQ; ++i)
+                    if (i < cnt) {
+                        const int64_t col = (int64_t)h * nvq + 32 * i;
+                        uint4 y;
+                        if (GREG)
+                            y = vapply_regs(Tag{}, cur[h][i], &gam[(h * VQ + i) * VEC], r);
+                        else
+                            y = vapply(Tag{}, cur[h][i],
+                                       a.g[0] + ((int64_t)pa * nvq + lane + col) * VEC, r);
+                        st_stream(dst + col, y);
+                    }
+        } else if (kok) {
+            uint4 *dst = reinterpret_cast<uint4 *>(a.y[1]) + t * a.ldy[1] + (int64_t)kshard * nvk + kv;
+            uint4 y;
+            if (GREG)
+                y = vapply_regs(Tag{}, cur[0][0], gam, r);
+            else
+                y = vapply(Tag{}, cur[0][0], a.g[1] + ((int64_t)kshard * nvk + kv) * VEC, r);
+            st_stream(dst, y);
+        }
+        buf ^= 1;
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
 // A kernel that waits on an mbarrier nobody arrives on, with the same bounded
 // wait as fused_bulk: it must time out, record kErrWaitTimeout and return.
 __global__ void bounded_wait_probe(uint64_t timeout_ns) {
@@ -606,6 +797,45 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int wq, int wk, int
     b.timeout_ns = timeout_ns;
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
     return launch(fn, dim3((unsigned)grid), dim3(32 * (wq + wk)), L.smem_bytes, s, args);
+}
+
+// fused_pair instances: VQ 1..3 vectors per lane per Q shard, gamma in
+// registers or not.
+template <class Tag>
+const void *pair_table(int vq, bool greg) {
+    switch (vq) {
+    case 1: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 1, true>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 1, false>);
+    case 2: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 2, true>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 2, false>);
+    case 3: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 3, true>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 3, false>);
+    default: return nullptr;
+    }
+}
+
+const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs) {
+    if (dtype == 0) return pair_table<F32Tag>(vq, gamma_regs);
+    if (dtype == 1) return pair_table<BF16Tag>(vq, gamma_regs);
+    // FP8 with 3 vectors per lane and gamma in registers would spill: no instance.
+    if (dtype == 2) return (vq == 3 && gamma_regs) ? nullptr : pair_table<E4M3Tag>(vq, gamma_regs);
+    return nullptr;
+}
+
+cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, const FusedArgs &a, int stages,
+                              int64_t grid, uint64_t timeout_ns, cudaStream_t s) {
+    const void *fn = fused_pair_kernel(dtype, vq, gamma_regs);
+    if (!fn || stages < 1 || stages > (int)kMaxStages || (a.P & 1) || a.P > 16) return cudaErrorInvalidValue;
+    const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
+    BulkArgs b;
+    b.stages = (uint32_t)stages;
+    b.qbytes = (uint32_t)(a.D[0] * es);
+    b.kbytes = (uint32_t)(a.D[1] * es);
+    b.stage_stride = bulk_stage_stride(b.qbytes, b.kbytes, 1);
+    b.timeout_ns = timeout_ns;
+    const size_t smem = bulk_smem_bytes(stages, b.stage_stride);
+    void *args[] = {const_cast<FusedArgs *>(&a), &b};
+    return launch(fn, dim3((unsigned)grid), dim3(32 * a.P), smem, s, args);
 }
 
 cudaError_t launch_bounded_wait_probe(uint64_t timeout_ns, cudaStream_t s) {

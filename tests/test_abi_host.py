@@ -176,16 +176,17 @@ def test_plan_for_each_workload(qk):
         for T in wl.Ts:
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
             # One token per CTA: registers only. Several: the token ring (one
-            # token per stage, gamma in registers while vmax <= 3), or warp
-            # per row when lanes are ragged (GQA widths).
+            # token per stage, gamma in registers while vmax <= 3), or for the
+            # GQA widths the shard-pair ring (P warps per token).
             if T <= 2 * 148:
                 want = qk.VARIANT_CTA
             else:
-                want = qk.VARIANT_ROWS if name == "gqa" else qk.VARIANT_BULK
+                want = qk.VARIANT_PAIR if name == "gqa" else qk.VARIANT_BULK
             assert pl["variant"] == want, (name, T)
             assert pl["groups_q"] == pl["groups_k"] == 1
-            if want == qk.VARIANT_ROWS:
-                assert pl["stages"] == 2 and pl["full_lanes"] == 0
+            if want == qk.VARIANT_PAIR:
+                assert pl["block"] == wl.P * 32 and pl["vmax"] == 3 and pl["gamma_regs"] == 1
+                assert pl["stages"] == (3 if T >= 40 * 148 else 2) and pl["tokens_per_stage"] == 1
                 continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
@@ -239,7 +240,16 @@ def test_forced_variants(qk):
             qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         with pytest.raises(qk.QKNormError):
-            qk.qknorm_force_variant(5, 0)
+            qk.qknorm_force_variant(6, 0)
+        # The shard-pair ring: P warps, GQA-like shapes only.
+        qk.qknorm_force_variant(qk.VARIANT_PAIR, 0)
+        pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
+        assert (pl["variant"], pl["block"], pl["vmax"], pl["tokens_per_stage"]) == \
+            (qk.VARIANT_PAIR, 8 * 32, 3, 1)
+        for shape in ((4096, 5120, 5120, 4), (4096, 1280, 640, 5), (4096, 5120, 4096, 8), (64, 4096, 512, 32)):
+            with pytest.raises(qk.QKNormError) as ei:           # K shards wider than 16 vectors,
+                qk.qknorm_plan_fwd(*shape, qk.QKNORM_BF16, 148)  # P odd, or P > 16
+            assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         qk.qknorm_force_variant(qk.VARIANT_BULK, 0)
         qk.qknorm_set_tuning(stages=3, tokens_per_stage=2, gamma_regs=0)
         pl = qk.qknorm_plan_fwd(10, 4096, 4096, 8, qk.QKNORM_BF16, 148)   # vmax 2

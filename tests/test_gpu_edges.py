@@ -14,7 +14,7 @@ from gpu_util import bits, check_outputs, check_stats, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ("cta", "bulk", "rows", "warp", "generic")
+VARIANTS = ("cta", "bulk", "rows", "pair", "warp", "generic")
 
 
 @pytest.fixture(scope="module")
@@ -38,7 +38,8 @@ def _inputs(wl, T):
 
 def _fwd(qk, wl, q, k, gq, gk, variant=None, grid=0):
     vid = {"cta": qk.VARIANT_CTA, "warp": qk.VARIANT_WARP, "generic": qk.VARIANT_GENERIC,
-           "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS, None: qk.VARIANT_AUTO}[variant]
+           "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS, "pair": qk.VARIANT_PAIR,
+           None: qk.VARIANT_AUTO}[variant]
     qk.qknorm_force_variant(vid, grid)
     try:
         oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk),
@@ -81,9 +82,9 @@ def test_shapes_and_variants(qk, orc, shape):
         try:
             outs[v] = _fwd(qk, wl, q, k, gq, gk, variant=v)
         except qk.QKNormError as e:
-            # Only the register-resident kernels (cta, bulk) and the shared-memory
-            # staged ones (bulk, rows) have shape limits.
-            assert v in ("cta", "bulk", "rows") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
+            # Only the register-resident kernels (cta, bulk, pair) and the
+            # shared-memory staged ones (bulk, rows, pair) have shape limits.
+            assert v in ("cta", "bulk", "rows", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
     base = outs["generic"]
     for v, (oq, ok) in outs.items():
         assert torch.equal(bits(oq), bits(base[0])), f"{v} Q differs from generic"
@@ -273,16 +274,36 @@ def test_rows_variant_rings(qk, wq, wk, stages, gsm, grid):
     assert qk.qknorm_device_errors() == 0
 
 
-@pytest.mark.parametrize("variant", ["cta", "bulk", "rows", "generic"])
+@pytest.mark.parametrize("T,Dq,Dk,P", [(2 * 148 + 41, 5120, 1024, 8), (700, 4096, 1024, 8),
+                                        (301, 2048, 256, 4), (150, 1536, 256, 2)])
+@pytest.mark.parametrize("grid,stages", [(0, 0), (1, 1), (5, 3), (0, 1)])
+def test_pair_variant(qk, T, Dq, Dk, P, grid, stages):
+    """The shard-pair token ring (two Q shards per warp, two K shards on lane
+    halves): any grid (tokens wrap the ring many times) and ring depth gives
+    the same bits as the generic kernel."""
+    wl = W.custom("pair", T, Dq, Dk, P, seed=38 + P)
+    q, k, gq, gk = _inputs(wl, wl.Ts[0])
+    ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
+    try:
+        qk.qknorm_set_tuning(stages, 0, -1, 0)
+        got = _fwd(qk, wl, q, k, gq, gk, variant="pair", grid=grid)
+    finally:
+        qk.qknorm_set_tuning()
+    assert torch.equal(bits(got[0]), bits(ref[0])) and torch.equal(bits(got[1]), bits(ref[1]))
+    assert qk.qknorm_device_errors() == 0
+
+
+@pytest.mark.parametrize("variant", ["cta", "bulk", "rows", "pair", "generic"])
 def test_dependent_launches_with_pdl(qk, variant):
     """Each call reads the previous call's output. With programmatic dependent
     launch every kernel waits for the previous grid before reading memory, so
     a chain launched back to back equals the same chain with a device
     synchronisation after every call, and the chain with PDL off."""
-    wl = W.custom("chain", 3 * 148 + 5, 4096, 1024, 4, seed=37)
+    # (the shard-pair ring needs K shards of <= 16 vectors: P = 8 there)
+    wl = W.custom("chain", 3 * 148 + 5, 4096, 1024, 8 if variant == "pair" else 4, seed=37)
     q, k, gq, gk = _inputs(wl, wl.Ts[0])
     vid = {"cta": qk.VARIANT_CTA, "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS,
-           "generic": qk.VARIANT_GENERIC}[variant]
+           "pair": qk.VARIANT_PAIR, "generic": qk.VARIANT_GENERIC}[variant]
     gqd, gkd = to_device(gq), to_device(gk)
 
     def chain(pdl, sync):

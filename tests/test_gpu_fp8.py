@@ -55,17 +55,17 @@ SHAPES = [
 
 
 @pytest.mark.parametrize("name,T,Dq,Dk,P", SHAPES)
-@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "generic"])
+@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "pair", "generic"])
 def test_fp8_fused_and_split(qk, orc, name, T, Dq, Dk, P, variant):
     wl, q, k, gq, gk = _inputs(name, T, Dq, Dk, P, sigma=1.5)
-    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "generic": 2}[variant]
+    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "pair": 5, "generic": 2}[variant]
     qd, kd, gqd, gkd = to_device(q), to_device(k), to_device(gq), to_device(gk)
     qk.qknorm_force_variant(vid, 0)
     try:
         oq, ok = qk.qknorm_fwd(qd, kd, gqd, gkd, P, 1e-6)
         torch.cuda.synchronize()
     except qk.QKNormError as e:
-        assert variant in ("cta", "bulk") and e.status == qk.QKNORM_ERR_UNSUPPORTED
+        assert variant in ("cta", "bulk", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
         return
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
@@ -142,12 +142,12 @@ def test_fp8_variants_bit_identical(qk, D, P):
     g = torch.from_numpy(np.random.default_rng(23).uniform(-1.5, 1.5, D).astype(np.float32)).cuda()
     qd, kd = to_device(q), to_device(k)
     outs = {}
-    for name, vid in (("cta", 0), ("bulk", 3), ("rows", 4), ("generic", 2)):
+    for name, vid in (("cta", 0), ("bulk", 3), ("rows", 4), ("pair", 5), ("generic", 2)):
         qk.qknorm_force_variant(vid, 0)
         try:
             outs[name] = qk.qknorm_fwd(qd, kd, g, g, P, 1e-6)
         except qk.QKNormError as e:
-            assert name in ("cta", "bulk") and e.status == qk.QKNORM_ERR_UNSUPPORTED
+            assert name in ("cta", "bulk", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
         finally:
             qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     outs["split"] = tuple(qk.qknorm_apply(x, g, qk.qknorm_partial_sumsq(x, P), 1e-6) for x in (qd, kd))
@@ -166,13 +166,13 @@ def test_fp8_saturation(qk, orc):
     rng = np.random.default_rng(33)
     g = rng.uniform(0.5, 1.5, D).astype(np.float32)
     g[::7] *= -300.0                                   # these channels overflow the format
-    for vid in (-1, 0, 2, 3, 4):
+    for vid in (-1, 0, 2, 3, 4, 5):
         qk.qknorm_force_variant(vid, 0)
         try:
             oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(g), to_device(g), P, 1e-6)
             torch.cuda.synchronize()
         except qk.QKNormError as e:
-            assert vid in (0, 3) and e.status == qk.QKNORM_ERR_UNSUPPORTED
+            assert vid in (0, 3, 5) and e.status == qk.QKNORM_ERR_UNSUPPORTED
             continue
         finally:
             qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
