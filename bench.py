@@ -361,6 +361,22 @@ def latency_us(torch, qk, wl, T, device, n_eager=400, n_graph=100, graph_reps=10
     return {"eager_us": round(eager, 3), "graph_us": round(graph, 3)}
 
 
+def decode_c_abi(wl):
+    """The decode sizes timed by the C++ program built beside the library
+    (qknorm_fwd called from C, no Python): device us per call and host us
+    per call, back to back on one stream."""
+    exe = os.path.join(ROOT, "qk_norm_attention_b200", "decode_bench")
+    if not os.path.exists(exe):
+        return {"unavailable": "decode_bench not built"}
+    import subprocess
+    r = subprocess.run([exe, str(wl.Dq), str(wl.P), "2000"], capture_output=True, text=True, timeout=120)
+    if r.returncode != 0:
+        return {"unavailable": r.stderr.strip()[-200:]}
+    out = json.loads(r.stdout)
+    out["how"] = "C++ program through the C ABI: 2000 back-to-back calls per T, CUDA events (device) and steady_clock (host)"
+    return out
+
+
 def throughput(torch, qk, wl, T, device, sets, steps=50):
     """GB/s of the fused path on T tokens with `sets` rotating buffer sets."""
     stream = torch.cuda.current_stream(device)
@@ -752,6 +768,7 @@ def run_native(args, dist):
     if dist.rank == 0 and not args.no_extras:
         dec = W.WORKLOADS["decode"]
         extras["decode_us_per_call"] = {str(t): latency_us(torch, qk, dec, t, device) for t in dec.Ts}
+        extras["decode_c_abi"] = decode_c_abi(dec)
         gqa = W.WORKLOADS["gqa"]
         extras["gqa"] = {"us_per_call": {str(t): latency_us(torch, qk, gqa, t, device)
                                          for t in gqa.Ts if t <= 256},

@@ -49,17 +49,28 @@ def nvcc() -> str:
     return "nvcc"
 
 
+DECODE_BENCH = os.path.join(PKG, "decode_bench")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into libqknorm.so (skipped when up to date)."""
-    if not force and not verbose and up_to_date():
-        return LIBRARY
-    tmp = LIBRARY + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", tmp, *sources()]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIBRARY)
+    """Compile every .cu under csrc/ into libqknorm.so (skipped when up to date),
+    and the C++ decode timing program linked against it."""
+    if force or verbose or not up_to_date():
+        tmp = LIBRARY + ".tmp"
+        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+        cmd += ["-o", tmp, *sources()]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, LIBRARY)
+    src = os.path.join(CSRC, "decode_bench.cpp")
+    if (force or not os.path.exists(DECODE_BENCH) or
+            os.path.getmtime(DECODE_BENCH) < max(os.path.getmtime(src), os.path.getmtime(LIBRARY))):
+        tmp = DECODE_BENCH + ".tmp"
+        subprocess.run([nvcc(), "-O2", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-I", os.path.join(ROOT, "include"), "-o", tmp, src,
+                        "-L", PKG, "-lqknorm", "-Xlinker", "-rpath,$ORIGIN"], check=True)
+        os.replace(tmp, DECODE_BENCH)
     return LIBRARY
 
 
