@@ -152,31 +152,57 @@ def test_in_place(qk):
     assert torch.equal(bits(xd), bits(ref[0]))
 
 
-def test_guard_regions_and_const_inputs(qk):
+GUARD_CASES = [
+    # variant, T, Dq, Dk, P, dtype
+    (None, 37, 5120, 1024, 8, "bf16"),
+    ("cta", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
+    ("bulk", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
+    ("rows", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
+    ("pair", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
+    ("generic", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
+    ("bulk", 2 * 148 + 41, 5120, 5120, 4, "e4m3"),     # the FP8 half-slot mode
+    ("pair", 2 * 148 + 41, 5120, 1024, 8, "e4m3"),
+]
+
+
+@pytest.mark.parametrize("variant,T,Dq,Dk,P,dtype", GUARD_CASES)
+def test_guard_regions_and_const_inputs(qk, variant, T, Dq, Dk, P, dtype):
     """Outputs sit inside larger buffers filled with a canary pattern; after
-    the calls the canaries and the inputs are byte-identical to before."""
-    T, Dq, Dk, P = 37, 5120, 1024, 8
-    wl = W.custom("guard", T, Dq, Dk, P, seed=34)
+    the calls (every kernel variant, ragged lanes, tokens that wrap the
+    persistent grid) the canaries and the inputs are byte-identical to before."""
+    wl = W.custom("guard", T, Dq, Dk, P, dtype=dtype, seed=34)
     q, k, gq, gk = _inputs(wl, T)
     qd, kd, gqd, gkd = (to_device(a) for a in (q, k, gq, gk))
     saved = [t.clone() for t in (qd, kd, gqd, gkd)]
-    pad = 4096  # elements of guard on each side (8 KiB, keeps 16-byte alignment)
-    bq = torch.full((T * Dq + 2 * pad,), -7777.0, dtype=torch.bfloat16, device="cuda")
-    bk = torch.full((T * Dk + 2 * pad,), -7777.0, dtype=torch.bfloat16, device="cuda")
+    pad = 4096  # elements of guard on each side (keeps 16-byte alignment)
+    def canary(n):
+        if dtype == "e4m3":   # the code 0xd6 (-14.0)
+            return torch.full((n,), 0xD6, dtype=torch.uint8, device="cuda").view(torch.float8_e4m3fn)
+        return torch.full((n,), -77.0, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32,
+                          device="cuda")
+    bq = canary(T * Dq + 2 * pad)
+    bk = canary(T * Dk + 2 * pad)
     bs = torch.full((T * P + 2 * pad,), -5.5, dtype=torch.float32, device="cuda")
     bcopy = [b.clone() for b in (bq, bk, bs)]
     oq = bq[pad:pad + T * Dq].view(T, Dq)
     ok = bk[pad:pad + T * Dk].view(T, Dk)
     st = bs[pad:pad + T * P].view(T, P)
-    qk.qknorm_fwd(qd, kd, gqd, gkd, P, wl.eps, out_q=oq, out_k=ok)
+    vid = {None: qk.VARIANT_AUTO, "cta": qk.VARIANT_CTA, "bulk": qk.VARIANT_BULK,
+           "rows": qk.VARIANT_ROWS, "pair": qk.VARIANT_PAIR, "generic": qk.VARIANT_GENERIC}[variant]
+    qk.qknorm_force_variant(vid, 0)
+    try:
+        qk.qknorm_fwd(qd, kd, gqd, gkd, P, wl.eps, out_q=oq, out_k=ok)
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     qk.qknorm_partial_sumsq(qd, P, stats=st)
     torch.cuda.synchronize()
     for b, c in zip((bq, bk, bs), bcopy):
         assert torch.equal(bits(b[:pad]), bits(c[:pad])) and torch.equal(bits(b[-pad:]), bits(c[-pad:]))
-    for t, s in zip((qd, kd, gqd, gkd), saved):
-        assert torch.equal(bits(t), bits(s))
-    ref = _fwd(qk, wl, q, k, gq, gk)
+    for t, s_ in zip((qd, kd, gqd, gkd), saved):
+        assert torch.equal(bits(t), bits(s_))
+    ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
     assert torch.equal(bits(oq), bits(ref[0])) and torch.equal(bits(ok), bits(ref[1]))
+    assert qk.qknorm_device_errors() == 0
 
 
 def test_rejected_call_launches_nothing(qk):
