@@ -632,14 +632,16 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
     int dev = 0, sms = 0;
     cudaError_t e = device_sms(&dev, &sms);
     if (e != cudaSuccess) return finish(e);
-    const int64_t rowvec = D / vec_of(dtype);
-    int block = (int)((rowvec + kLanes - 1) / kLanes * kLanes);
-    if (block > 256) block = 256;
+    // apply_threads_per_row(D) threads per row, as many rows per 256-thread
+    // block as fit.
+    const int tpr = apply_threads_per_row(D, dtype);
+    const int rpb = 256 / tpr;
+    const int block = tpr * rpb;
     int bres = 1;
-    e = resident_blocks(dev, apply_kernel(dtype), block, 0, &bres);
+    e = resident_blocks(dev, apply_kernel(dtype, rpb > 1), block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
     int64_t grid = (int64_t)sms * bres;
-    if (grid > T) grid = T;
+    if (grid > (T + rpb - 1) / rpb) grid = (T + rpb - 1) / rpb;
     return finish(launch_apply(dtype, x, gamma, stats, out, T, D, Pb, nb, sg,
                                (float)((int64_t)D * nb), eps, block, grid,
                                reinterpret_cast<cudaStream_t>(stream)));

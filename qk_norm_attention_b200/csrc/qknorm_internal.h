@@ -39,7 +39,8 @@ TensorShape make_shape(int32_t D, int32_t P, int vec);
 const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads);
 const void *fused_generic_kernel(int dtype);
 const void *stats_kernel(int dtype, int vmax);
-const void *apply_kernel(int dtype);
+// multi: the several-rows-per-block instance of apply_k (block != tpr).
+const void *apply_kernel(int dtype, bool multi);
 
 // Launchers: enqueue one kernel; return the cudaError_t of the launch.
 cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
@@ -50,7 +51,9 @@ cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64
                          const TensorShape &sh, int32_t P, int block, int64_t grid,
                          cudaStream_t s);
 // stats of token t: nb blocks of Pb sums, block b at stats + b * sg + t * Pb;
-// Df the divisor (full width).
+// Df the divisor (full width). block must be a multiple of
+// apply_threads_per_row(D, dtype).
+int apply_threads_per_row(int32_t D, int dtype);
 cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
                          int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg, float Df,
                          float eps, int block, int64_t grid, cudaStream_t s);
