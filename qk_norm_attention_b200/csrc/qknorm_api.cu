@@ -837,7 +837,8 @@ int qknorm_headwise_fwd(const void *q, const void *k, const float *gamma_q, cons
     int bres = 1;
     e = resident_blocks(dev, fn, block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
-    int64_t grid = (T + block / kLanes - 1) / (block / kLanes);
+    // One warp per work group, up to a resident grid.
+    int64_t grid = (headwise_groups(T, Hq, Hk, nv) + block / kLanes - 1) / (block / kLanes);
     if (grid > (int64_t)sms * bres) grid = (int64_t)sms * bres;
     HeadArgs a;
     a.x[0] = q;

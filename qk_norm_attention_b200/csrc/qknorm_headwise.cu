@@ -17,6 +17,12 @@
 // zeros of lanes past the head's last vector. Larger heads take a whole warp,
 // each lane holding VMAX vectors. R units' loads are issued before any is
 // reduced.
+//
+// Work is dealt in groups of R consecutive units of one token, not in whole
+// tokens: at T = 8192 a resident grid of ~4700 warps would otherwise hold one
+// or two tokens each, and the second half of the launch would run with the
+// one-token warps already gone. Groups are ~5x finer, so every warp ends
+// within one group of the others.
 #include "qknorm_device.cuh"
 #include "qknorm_internal.h"
 
@@ -29,8 +35,13 @@ __device__ __forceinline__ float seg_butterfly(float c) {
     return c;
 }
 
+// Four 256-thread CTAs per SM (64 registers) where that costs no spills: the
+// bf16 and fp32 instances up to 4 vectors per lane. FP8 keeps 2 x 16 gamma
+// values per lane in registers and needs more.
+constexpr int headwise_min_blocks(int vec, int vmax) { return vec <= 8 && vmax <= 4 ? 4 : 1; }
+
 template <class Tag, int SEG, int VMAX, int R>
-__global__ void __launch_bounds__(256) headwise_k(const HeadArgs a) {
+__global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) headwise_k(const HeadArgs a) {
     constexpr int VEC = Tag::kVec;
     constexpr int HPW = 32 / SEG;  // heads per unit
     pdl_wait();
@@ -56,52 +67,65 @@ __global__ void __launch_bounds__(256) headwise_k(const HeadArgs a) {
                 gr[z][e + 3] = g4.w;
             }
     }
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < a.T; t += NW) {
-        for (int u0 = 0; u0 < U; u0 += R) {
-            uint4 v[R][VMAX];
-            bool ok[R];
-            const uint4 *src[R];
-            uint4 *dst[R];
-            int zz[R];
+    const int G = (U + R - 1) / R;  // groups per token
+    // Group gi = t * G + gsub; a warp's groups advance by NW, so (t, gsub) are
+    // carried along instead of divided out.
+    const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t dt = NW / G;
+    const int dg = (int)(NW - dt * G);
+    int64_t t = w0 / G;
+    int gsub = (int)(w0 - t * G);
+    while (t < a.T) {
+        const int u0 = gsub * R;
+        uint4 v[R][VMAX];
+        bool ok[R];
+        const uint4 *src[R];
+        uint4 *dst[R];
+        int zz[R];
 #pragma unroll
-            for (int j = 0; j < R; ++j) {
-                const int u = u0 + j;
-                const int z = u < Uq ? 0 : 1;
-                const int head = (z ? u - Uq : u) * HPW + hsub;
-                ok[j] = u < U && head < (z ? a.H[1] : a.H[0]);
-                zz[j] = z;
-                const int64_t col = (int64_t)head * nv;
-                src[j] = reinterpret_cast<const uint4 *>(z ? a.x[1] : a.x[0]) + t * (z ? a.ldx[1] : a.ldx[0]) + col;
-                dst[j] = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) + col;
+        for (int j = 0; j < R; ++j) {
+            const int u = u0 + j;
+            const int z = u < Uq ? 0 : 1;
+            const int head = (z ? u - Uq : u) * HPW + hsub;
+            ok[j] = u < U && head < (z ? a.H[1] : a.H[0]);
+            zz[j] = z;
+            const int64_t col = (int64_t)head * nv;
+            src[j] = reinterpret_cast<const uint4 *>(z ? a.x[1] : a.x[0]) + t * (z ? a.ldx[1] : a.ldx[0]) + col;
+            dst[j] = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) + col;
 #pragma unroll
-                for (int i = 0; i < VMAX; ++i) {
-                    const int vv = slot + 32 * i;
-                    if (ok[j] && vv < nv) v[j][i] = ld_stream(src[j] + vv);
+            for (int i = 0; i < VMAX; ++i) {
+                const int vv = slot + 32 * i;
+                if (ok[j] && vv < nv) v[j][i] = ld_stream(src[j] + vv);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            float c = 0.f;
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i)
+                if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
+            const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
+#pragma unroll
+            for (int i = 0; i < VMAX; ++i) {
+                const int vv = slot + 32 * i;
+                if (ok[j] && vv < nv) {
+                    uint4 y;
+                    if (VMAX == 1) {
+                        float gg[VEC];  // select, so the array stays in registers
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) gg[e] = zz[j] ? gr[1][e] : gr[0][e];
+                        y = vapply_regs(Tag{}, v[j][i], gg, r);
+                    } else
+                        y = vapply(Tag{}, v[j][i], (zz[j] ? a.g[1] : a.g[0]) + (int64_t)vv * VEC, r);
+                    st_stream(dst[j] + vv, y);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < R; ++j) {
-                float c = 0.f;
-#pragma unroll
-                for (int i = 0; i < VMAX; ++i)
-                    if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
-                const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
-#pragma unroll
-                for (int i = 0; i < VMAX; ++i) {
-                    const int vv = slot + 32 * i;
-                    if (ok[j] && vv < nv) {
-                        uint4 y;
-                        if (VMAX == 1) {
-                            float gg[VEC];  // select, so the array stays in registers
-#pragma unroll
-                            for (int e = 0; e < VEC; ++e) gg[e] = zz[j] ? gr[1][e] : gr[0][e];
-                            y = vapply_regs(Tag{}, v[j][i], gg, r);
-                        } else
-                            y = vapply(Tag{}, v[j][i], (zz[j] ? a.g[1] : a.g[0]) + (int64_t)vv * VEC, r);
-                        st_stream(dst[j] + vv, y);
-                    }
-                }
-            }
+        }
+        t += dt;
+        gsub += dg;
+        if (gsub >= G) {
+            gsub -= G;
+            ++t;
         }
     }
 }
@@ -113,28 +137,44 @@ static int seg_of(int nv) {
     return s;
 }
 
+// Units per group (R) for heads of up to 32 * VMAX vectors: as many as keep
+// R x VMAX <= 8 vectors per lane.
+constexpr int units_per_group(int vmax) { return vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1); }
+
+template <class Tag, int SEG, int VMAX>
+const void *headwise_fn() {
+    return reinterpret_cast<const void *>(&headwise_k<Tag, SEG, VMAX, units_per_group(VMAX)>);
+}
+
 template <class Tag>
 const void *headwise_table(int nv) {
     if (nv <= 32) {
         switch (seg_of(nv)) {
-        case 1: return reinterpret_cast<const void *>(&headwise_k<Tag, 1, 1, 4>);
-        case 2: return reinterpret_cast<const void *>(&headwise_k<Tag, 2, 1, 4>);
-        case 4: return reinterpret_cast<const void *>(&headwise_k<Tag, 4, 1, 4>);
-        case 8: return reinterpret_cast<const void *>(&headwise_k<Tag, 8, 1, 4>);
-        case 16: return reinterpret_cast<const void *>(&headwise_k<Tag, 16, 1, 4>);
-        default: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 1, 4>);
+        case 1: return headwise_fn<Tag, 1, 1>();
+        case 2: return headwise_fn<Tag, 2, 1>();
+        case 4: return headwise_fn<Tag, 4, 1>();
+        case 8: return headwise_fn<Tag, 8, 1>();
+        case 16: return headwise_fn<Tag, 16, 1>();
+        default: return headwise_fn<Tag, 32, 1>();
         }
     }
     switch ((nv + 31) / 32) {
-    case 2: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 2, 4>);
-    case 3: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 3, 2>);
-    case 4: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 4, 2>);
-    case 5: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 5, 1>);
-    case 6: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 6, 1>);
-    case 7: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 7, 1>);
-    case 8: return reinterpret_cast<const void *>(&headwise_k<Tag, 32, 8, 1>);
+    case 2: return headwise_fn<Tag, 32, 2>();
+    case 3: return headwise_fn<Tag, 32, 3>();
+    case 4: return headwise_fn<Tag, 32, 4>();
+    case 5: return headwise_fn<Tag, 32, 5>();
+    case 6: return headwise_fn<Tag, 32, 6>();
+    case 7: return headwise_fn<Tag, 32, 7>();
+    case 8: return headwise_fn<Tag, 32, 8>();
     default: return nullptr;
     }
+}
+
+int64_t headwise_groups(int64_t T, int32_t Hq, int32_t Hk, int32_t nv) {
+    const int hpw = nv <= kLanes ? kLanes / seg_of(nv) : 1;
+    const int64_t units = (Hq + hpw - 1) / hpw + (Hk + hpw - 1) / hpw;
+    const int r = units_per_group((nv + kLanes - 1) / kLanes);
+    return T * ((units + r - 1) / r);
 }
 
 const void *headwise_kernel(int dtype, int nv) {

@@ -102,6 +102,8 @@ struct HeadArgs {
     int64_t ldy[2];
 };
 const void *headwise_kernel(int dtype, int nv);
+// Work groups of the headwise kernel for nv (one warp each): T * ceil(units / R).
+int64_t headwise_groups(int64_t T, int32_t Hq, int32_t Hk, int32_t nv);
 cudaError_t launch_headwise(int dtype, const HeadArgs &a, int block, int64_t grid, cudaStream_t s);
 
 // The deferred-normalisation steps (qknorm_deferred.cu).
