@@ -437,16 +437,12 @@ def deferred_steps(torch, qk, device, peak, steps=100):
     return out
 
 
-def fp8_prefill(torch, qk, device, peak, steps=200):
-    """The 13B-shaped prefill (T = 8192, Dq = Dk = 5120, P = 4) in FP8 E4M3:
-    E4M3 in and out, fp32 statistics; half the bytes of the bf16 step."""
-    wl = W.WORKLOADS["prefill13b_e4m3"]
+def _fp8_case(torch, qk, device, peak, wl, gq, gk, steps):
+    """Time qknorm_fwd in FP8 E4M3 on wl's first T over rotating buffer sets."""
     T = wl.Ts[0]
     stream = torch.cuda.current_stream(device)
     q = W.gen_device_workload(wl, "q", T, device)
     k = W.gen_device_workload(wl, "k", T, device)
-    gq = torch.from_numpy(W.gen_gamma(wl, "q")).to(device)
-    gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(device)
     nbytes = W.fused_bytes(T, wl.Dq, wl.Dk, 1)
     n = buffer_sets(nbytes)
     sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(n - 1)]
@@ -458,11 +454,28 @@ def fp8_prefill(torch, qk, device, peak, steps=200):
     tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
     ms = tot / steps
     plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, qk.QKNORM_E4M3)
-    return {"workload": "13B-shaped prefill in FP8 E4M3: T=8192, Dq=Dk=5120, P=4",
-            "us_per_call": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
+    return {"us_per_call": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
             "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1),
             "tokens_per_s": round(T / ms * 1000, 1), "algorithmic_bytes": nbytes,
             "kernel": KERNEL_OF_VARIANT.get(plan["variant"], "?")}
+
+
+def fp8_prefill(torch, qk, device, peak, steps=200):
+    """The 13B-shaped prefill (T = 8192, Dq = Dk = 5120, P = 4) in FP8 E4M3:
+    E4M3 in and out, fp32 statistics; half the bytes of the bf16 step. Also
+    the large split shape in FP8 (T = 65536, D = 4096, P = 8: one vector per
+    lane, where the shard-pair ring takes Q and K)."""
+    wl = W.WORKLOADS["prefill13b_e4m3"]
+    gq = torch.from_numpy(W.gen_gamma(wl, "q")).to(device)
+    gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(device)
+    out = {"workload": "13B-shaped prefill in FP8 E4M3: T=8192, Dq=Dk=5120, P=4"}
+    out.update(_fp8_case(torch, qk, device, peak, wl, gq, gk, steps))
+    wl8 = W.custom("split_large_e4m3", 65536, 4096, 4096, 8, dtype="e4m3", seed=12)
+    g8 = torch.rand(4096, device=device) + 0.5
+    r = {"workload": "T=65536, Dq=Dk=4096, P=8 in FP8 E4M3"}
+    r.update(_fp8_case(torch, qk, device, peak, wl8, g8, g8, steps // 4))
+    out["split_large_e4m3"] = r
+    return out
 
 
 def tp_rank_step(torch, qk, device, peak, steps=100):

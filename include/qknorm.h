@@ -342,6 +342,8 @@ typedef struct {
     int64_t smem_bytes;  /* dynamic shared memory per CTA */
     int32_t q_warps;     /* rows: warps per CTA that take Q rows (the rest take K rows) */
     int32_t gamma_smem;  /* rows: 1 if gamma is staged in shared memory, 0 if read via L1 */
+    int32_t k_pairs;     /* pair: 1 if each K warp takes two K shards like a Q warp, 0 if
+                            two K shards of <= 16 vectors share a warp's lane halves */
 } qknorm_plan;
 
 /*

@@ -64,7 +64,8 @@ class QKNormPlan(ctypes.Structure):
                 ("groups_k", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("tokens_per_stage", ctypes.c_int32), ("gamma_regs", ctypes.c_int32),
                 ("full_lanes", ctypes.c_int32), ("smem_bytes", ctypes.c_int64),
-                ("q_warps", ctypes.c_int32), ("gamma_smem", ctypes.c_int32)]
+                ("q_warps", ctypes.c_int32), ("gamma_smem", ctypes.c_int32),
+                ("k_pairs", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -302,17 +302,21 @@ bool rows_fit(int32_t Dq, int32_t Dk, int32_t dtype) {
 }
 
 // The shard-pair ring's conditions: P even and at most 16 (P warps), one
-// group per shard, K shards of at most 16 vectors (one per lane of a half
-// warp), Q shards of at most 3 vectors per lane, and an instance for the
-// gamma placement.
+// group per shard, shards of at most 3 vectors per lane, and an instance for
+// the gamma placement. K shards of at most 16 vectors share a warp's lane
+// halves; wider K shards go in pairs like Q's (pair_kw).
+bool pair_kw(const Shapes &sh) { return sh.k.nv > kLanes / 2; }
+
+int pair_vq(const Shapes &sh) { return pair_kw(sh) ? sh.vmax : sh.q.vmax; }
+
 bool pair_greg(const Shapes &sh, int32_t dtype) {
     if (g_tune_gamma_regs >= 0) return g_tune_gamma_regs != 0;
-    return !(dtype == QKNORM_E4M3 && sh.q.vmax >= 3);
+    return !(dtype == QKNORM_E4M3 && pair_vq(sh) >= (pair_kw(sh) ? 2 : 3));
 }
 
 bool pair_fits(const Shapes &sh, int32_t P, int32_t dtype) {
-    return !(P & 1) && P <= 16 && sh.q.K == 1 && sh.k.K == 1 && sh.k.nv <= kLanes / 2 &&
-           sh.q.vmax <= 3 && fused_pair_kernel(dtype, sh.q.vmax, pair_greg(sh, dtype)) != nullptr;
+    return !(P & 1) && P <= 16 && sh.q.K == 1 && sh.k.K == 1 && pair_vq(sh) <= 3 &&
+           fused_pair_kernel(dtype, pair_vq(sh), pair_greg(sh, dtype), pair_kw(sh)) != nullptr;
 }
 
 // Static part of the plan: which kernel, block size, template width, stages.
@@ -349,10 +353,22 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         // vectors) take the shard-pair ring: P warps per token instead of 2P,
         // two CTAs per SM (measured at T = 4096, 5120/1024, P = 8: 84.8 % vs
         // 66.4 % for rows and 59.8 % for the ring with 2P warps).
+        // K shards as wide as Q's go in pairs too (P warps per token) where a
+        // warp's fixed work per token weighs most: FP8 at one vector per lane
+        // (measured 60.4 -> 82.3 % at T = 65536, D = 4096, P = 8; 58.9 ->
+        // 76.4 % at D = 2048, P = 4) and ragged bf16/fp32 lanes (5120/4096,
+        // P = 8: 83.4 % vs 76.1 % for rows). Not on full bf16 lanes (99.1 %
+        // for the ring with 2P warps vs 89.9 %), nor for FP8 at two or more
+        // vectors per lane, whose gamma no longer fits registers (77.7 % vs
+        // 44.9 %).
         const bool ragged = !pl->full_lanes && dtype != QKNORM_E4M3;
+        const bool kpairs = pair_fits(sh, P, dtype) && pair_kw(sh) && pair_greg(sh, dtype) &&
+                            (dtype == QKNORM_E4M3 ? pair_vq(sh) == 1 : ragged);
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
-        else if (pair_fits(sh, P, dtype) && sh.q.nv > kLanes)
+        else if (pair_fits(sh, P, dtype) && !pair_kw(sh) && sh.q.nv > kLanes)
+            variant = QKNORM_VARIANT_PAIR;
+        else if (kpairs)
             variant = QKNORM_VARIANT_PAIR;
         else if (bulk_ok && !(ragged && rows_ok))
             variant = QKNORM_VARIANT_BULK;
@@ -377,12 +393,13 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         return QKNORM_OK;
     }
     if (variant == QKNORM_VARIANT_PAIR) {
-        // P warps: Q shards in pairs, K shards (<= 16 vectors) in pairs on lane halves.
+        // P warps: Q shards in pairs; K shards in pairs, on lane halves if <= 16 vectors.
         if (!pair_fits(sh, P, dtype)) return QKNORM_ERR_UNSUPPORTED;
         const bool greg_p = pair_greg(sh, dtype);
         pl->variant = QKNORM_VARIANT_PAIR;
         pl->block = P * kLanes;
-        pl->vmax = sh.q.vmax;
+        pl->vmax = pair_vq(sh);
+        pl->k_pairs = pair_kw(sh) ? 1 : 0;
         pl->gamma_regs = greg_p ? 1 : 0;
         pl->tokens_per_stage = 1;
         const uint32_t stride1 = bulk_stage_stride((int64_t)Dq * elem_of(dtype),
@@ -468,7 +485,7 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy
     case QKNORM_VARIANT_ROWS:
         return fused_rows_kernel(dtype);
     case QKNORM_VARIANT_PAIR:
-        return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0);
+        return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0);
     default:
         return fused_generic_kernel(dtype);
     }
@@ -649,7 +666,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 112; }
+int qknorm_version(void) { return 113; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -772,8 +789,8 @@ int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const
         e = launch_fused_rows(dtype, a, pl.q_warps, pl.block / kLanes - pl.q_warps, pl.stages,
                               pl.gamma_smem != 0, pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_PAIR) {
-        e = launch_fused_pair(dtype, pl.vmax, pl.gamma_regs != 0, a, pl.stages, pl.grid,
-                              g_wait_limit_ns, s);
+        e = launch_fused_pair(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0, a, pl.stages,
+                              pl.grid, g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_BULK) {
         e = launch_fused_bulk(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
                               pl.full_lanes, a, pl.stages, pl.block, pl.grid,

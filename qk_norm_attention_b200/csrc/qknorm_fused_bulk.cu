@@ -459,7 +459,13 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
 // step it skips adds the exact zeros of the lanes past a shard's 16 vectors.
 // With half the warps per token, two CTAs fit an SM and each warp carries
 // twice the work per token barrier. One token per stage.
-template <class Tag, int VQ, bool GREG>
+//
+// KW: K shards as wide as Q's (more than 16 vectors) are taken like Q's,
+// warp P/2 + w holding K shards 2w and 2w + 1 with its own two chains and
+// butterflies. This halves the warps per token of the ring for equal-width
+// tensors, which pays where a warp's fixed work per token (wait, butterfly,
+// barrier, factor) weighs most: one or two vectors per lane, FP8.
+template <class Tag, int VQ, bool GREG, bool KW>
 __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const BulkArgs b) {
     constexpr int VEC = Tag::kVec;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -475,18 +481,22 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
     const int w = z ? warp - half : warp;
     const int pa = 2 * w;                                // first shard of the pair
     const int nvq = a.nv[0], nvk = a.nv[1];
-    // Q: this lane's vectors of shards pa, pa + 1: lane + 32 i, i < cnt.
-    const int cnt = z ? 0 : slot_count(lane, nvq, kLanes);
+    // Shard pairs (Q warps; K warps too with KW): this lane's vectors of
+    // shards pa, pa + 1 of tensor z: lane + 32 i, i < cnt.
+    const bool pairs = KW || z == 0;
+    const int nvz = z ? nvk : nvq;
+    const int cnt = pairs ? slot_count(lane, nvz, kLanes) : 0;
     // K: lane half h takes shard pa + h, vector kv of it.
     const int hk = lane >> 4, kv = lane & 15;
-    const bool kok = z && kv < nvk;
+    const bool kok = !pairs && kv < nvk;
     const int kshard = pa + hk;
     const float Df = z ? a.Df[1] : a.Df[0];
     const float eps = a.eps;
     const uint32_t tok_bytes = b.qbytes + b.kbytes;
     // Offsets inside a stage (bytes): Q vector (p, v) at (p*nvq + v)*16; K at
     // qbytes + (p*nvk + v)*16.
-    const uint32_t qoff = (uint32_t)((pa * nvq + lane) * 16);
+    const uint32_t qoff = (z ? b.qbytes : 0u) + (uint32_t)((pa * nvz + lane) * 16);
+    const float *gz = z ? a.g[1] : a.g[0];
     const uint32_t koff = b.qbytes + (uint32_t)((kshard * nvk + kv) * 16);
 
     const int64_t T = a.T;
@@ -516,10 +526,10 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
 
-    // Gamma in registers: Q lanes 2 x VQ vectors, K lanes one vector.
+    // Gamma in registers: shard-pair lanes 2 x VQ vectors, K half lanes one vector.
     float gam[GREG ? 2 * VQ * VEC : 1];
     if (GREG) {
-        if (z == 0) {
+        if (pairs) {
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
 #pragma unroll
                         for (int e = 0; e < VEC; e += 4) {
                             const float4 g4 = __ldg(reinterpret_cast<const float4 *>(
-                                a.g[0] + ((int64_t)(pa + h) * nvq + lane + 32 * i) * VEC + e));
+                                gz + ((int64_t)(pa + h) * nvz + lane + 32 * i) * VEC + e));
                             float *d = &gam[(h * VQ + i) * VEC + e];
                             d[0] = g4.x;
                             d[1] = g4.y;
@@ -557,9 +567,9 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
         const unsigned char *st = stages + (size_t)s * b.stage_stride;
         uint4 cur[2][VQ];
         float c0 = 0.f, c1 = 0.f;
-        if (z == 0) {
+        if (pairs) {
             const uint4 *src0 = reinterpret_cast<const uint4 *>(st + qoff);
-            const uint4 *src1 = src0 + nvq;
+            const uint4 *src1 = src0 + nvz;
 #pragma unroll
             for (int i = 0; i < VQ; ++i) {
                 cur[0][i] = i < cnt ? src0[32 * i] : make_uint4(0, 0, 0, 0);
@@ -574,8 +584,8 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
             c0 = butterfly(c0);
             c1 = butterfly(c1);
             if (lane == 0) {
-                red[buf][pa] = c0;
-                red[buf][pa + 1] = c1;
+                red[buf][32 * z + pa] = c0;
+                red[buf][32 * z + pa + 1] = c1;
             }
         } else {
             cur[0][0] = kok ? *reinterpret_cast<const uint4 *>(st + koff) : make_uint4(0, 0, 0, 0);
@@ -606,20 +616,20 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
             issue(s, n + S);
         }
         const float r = factor(combine_fast(&red[buf][z ? 32 : 0], a.P, 1), Df, eps);
-        if (z == 0) {
-            uint4 *dst = reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0] + (int64_t)pa * nvq + lane;
+        if (pairs) {
+            uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) +
+                         (int64_t)pa * nvz + lane;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int i = 0; i < VQ; ++i)
                     if (i < cnt) {
-                        const int64_t col = (int64_t)h * nvq + 32 * i;
+                        const int64_t col = (int64_t)h * nvz + 32 * i;
                         uint4 y;
                         if (GREG)
                             y = vapply_regs(Tag{}, cur[h][i], &gam[(h * VQ + i) * VEC], r);
                         else
-                            y = vapply(Tag{}, cur[h][i],
-                                       a.g[0] + ((int64_t)pa * nvq + lane + col) * VEC, r);
+                            y = vapply(Tag{}, cur[h][i], gz + ((int64_t)pa * nvz + lane + col) * VEC, r);
                         st_stream(dst + col, y);
                     }
         } else if (kok) {
@@ -799,33 +809,43 @@ cudaError_t launch_fused_rows(int dtype, const FusedArgs &a, int wq, int wk, int
     return launch(fn, dim3((unsigned)grid), dim3(32 * (wq + wk)), L.smem_bytes, s, args);
 }
 
-// fused_pair instances: VQ 1..3 vectors per lane per Q shard, gamma in
-// registers or not.
-template <class Tag>
-const void *pair_table(int vq, bool greg) {
+// fused_pair instances: VQ 1..3 vectors per lane per shard, gamma in
+// registers or not, K shards on lane halves or in pairs (kw).
+template <class Tag, bool KW>
+const void *pair_fn(int vq, bool greg) {
     switch (vq) {
-    case 1: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 1, true>)
-                        : reinterpret_cast<const void *>(&fused_pair<Tag, 1, false>);
-    case 2: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 2, true>)
-                        : reinterpret_cast<const void *>(&fused_pair<Tag, 2, false>);
-    case 3: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 3, true>)
-                        : reinterpret_cast<const void *>(&fused_pair<Tag, 3, false>);
+    case 1: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 1, true, KW>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 1, false, KW>);
+    case 2: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 2, true, KW>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 2, false, KW>);
+    case 3: return greg ? reinterpret_cast<const void *>(&fused_pair<Tag, 3, true, KW>)
+                        : reinterpret_cast<const void *>(&fused_pair<Tag, 3, false, KW>);
     default: return nullptr;
     }
 }
 
-const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs) {
-    if (dtype == 0) return pair_table<F32Tag>(vq, gamma_regs);
-    if (dtype == 1) return pair_table<BF16Tag>(vq, gamma_regs);
-    // FP8 with 3 vectors per lane and gamma in registers would spill: no instance.
-    if (dtype == 2) return (vq == 3 && gamma_regs) ? nullptr : pair_table<E4M3Tag>(vq, gamma_regs);
+template <class Tag>
+const void *pair_table(int vq, bool greg, bool kw) {
+    return kw ? pair_fn<Tag, true>(vq, greg) : pair_fn<Tag, false>(vq, greg);
+}
+
+const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs, bool kw) {
+    if (dtype == 0) return pair_table<F32Tag>(vq, gamma_regs, kw);
+    if (dtype == 1) return pair_table<BF16Tag>(vq, gamma_regs, kw);
+    // FP8 with gamma in registers for 3 vectors per lane (2 with K in pairs too)
+    // would spill: no instance.
+    if (dtype == 2)
+        return (gamma_regs && vq >= (kw ? 2 : 3)) ? nullptr : pair_table<E4M3Tag>(vq, gamma_regs, kw);
     return nullptr;
 }
 
-cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, const FusedArgs &a, int stages,
-                              int64_t grid, uint64_t timeout_ns, cudaStream_t s) {
-    const void *fn = fused_pair_kernel(dtype, vq, gamma_regs);
+cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const FusedArgs &a,
+                              int stages, int64_t grid, uint64_t timeout_ns, cudaStream_t s) {
+    const void *fn = fused_pair_kernel(dtype, vq, gamma_regs, kw);
     if (!fn || stages < 1 || stages > (int)kMaxStages || (a.P & 1) || a.P > 16) return cudaErrorInvalidValue;
+    // Each lane's slots must cover its shards: lane halves take at most 16 K vectors.
+    if (a.K[0] != 1 || a.K[1] != 1 || a.nv[0] > kLanes * vq || a.nv[1] > (kw ? kLanes * vq : kLanes / 2))
+        return cudaErrorInvalidValue;
     const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
     BulkArgs b;
     b.stages = (uint32_t)stages;

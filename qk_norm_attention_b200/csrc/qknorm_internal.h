@@ -70,11 +70,13 @@ int bulk_max_stages();
 cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, int mode,
                               const FusedArgs &a, int stages, int block, int64_t grid,
                               uint64_t timeout_ns, cudaStream_t s);
-// The shard-pair token ring for GQA-like shapes (qknorm_fused_bulk.cu): P even,
-// K shards of <= 16 vectors, Q shards of <= 32 * vq vectors, P <= 16; P warps per CTA.
-const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs);
-cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, const FusedArgs &a, int stages,
-                              int64_t grid, uint64_t timeout_ns, cudaStream_t s);
+// The shard-pair token ring (qknorm_fused_bulk.cu): P even, P <= 16, one group
+// per shard, P warps per CTA; Q shards of <= 32 * vq vectors, in pairs. K
+// shards of <= 16 vectors on lane halves (kw false, GQA-like shapes), or of
+// <= 32 * vq vectors in pairs like Q's (kw true).
+const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs, bool kw);
+cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const FusedArgs &a,
+                              int stages, int64_t grid, uint64_t timeout_ns, cudaStream_t s);
 // The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // wq warps take Q rows and wk warps take K rows in each CTA.
 struct RowsLayout {

@@ -164,6 +164,24 @@ def test_valid_call_without_gpu_reports_cuda_error(qk):
 
 # ----------------------------------------------------------------- the selector
 
+def test_auto_k_pairs(qk):
+    """The selector puts K shards in pairs (P warps per token) for FP8 at one
+    vector per lane and for ragged bf16 lanes, and keeps the ring with 2P
+    warps for full bf16 lanes and for FP8 at two or more vectors per lane."""
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    cases = [((65536, 4096, 4096, 8, qk.QKNORM_E4M3), (qk.VARIANT_PAIR, 1)),
+             ((16384, 2048, 2048, 4, qk.QKNORM_E4M3), (qk.VARIANT_PAIR, 1)),
+             ((8192, 5120, 4096, 8, qk.QKNORM_BF16), (qk.VARIANT_PAIR, 1)),
+             ((16384, 4096, 4096, 4, qk.QKNORM_E4M3), (qk.VARIANT_BULK, 0)),
+             ((65536, 4096, 4096, 8, qk.QKNORM_BF16), (qk.VARIANT_BULK, 0)),
+             ((8192, 5120, 5120, 4, qk.QKNORM_E4M3), (qk.VARIANT_BULK, 0))]
+    for shape, (variant, kp) in cases:
+        pl = qk.qknorm_plan_fwd(*shape, 148, 2)
+        assert (pl["variant"], pl["k_pairs"]) == (variant, kp), shape
+        if variant == qk.VARIANT_PAIR:
+            assert pl["block"] == shape[3] * 32 and pl["gamma_regs"] == 1
+
+
 def test_plan_for_each_workload(qk):
     import qknorm_workloads as W
     qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
@@ -244,10 +262,17 @@ def test_forced_variants(qk):
         # The shard-pair ring: P warps, GQA-like shapes only.
         qk.qknorm_force_variant(qk.VARIANT_PAIR, 0)
         pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
-        assert (pl["variant"], pl["block"], pl["vmax"], pl["tokens_per_stage"]) == \
-            (qk.VARIANT_PAIR, 8 * 32, 3, 1)
-        for shape in ((4096, 5120, 5120, 4), (4096, 1280, 640, 5), (4096, 5120, 4096, 8), (64, 4096, 512, 32)):
-            with pytest.raises(qk.QKNormError) as ei:           # K shards wider than 16 vectors,
+        assert (pl["variant"], pl["block"], pl["vmax"], pl["tokens_per_stage"], pl["k_pairs"]) == \
+            (qk.VARIANT_PAIR, 8 * 32, 3, 1, 0)
+        # K shards wider than 16 vectors go in pairs like Q's (vmax covers both tensors).
+        pl = qk.qknorm_plan_fwd(4096, 5120, 4096, 8, qk.QKNORM_BF16, 148)
+        assert (pl["variant"], pl["block"], pl["vmax"], pl["k_pairs"]) == (qk.VARIANT_PAIR, 8 * 32, 3, 1)
+        pl = qk.qknorm_plan_fwd(4096, 4096, 4096, 8, qk.QKNORM_E4M3, 148)
+        assert (pl["vmax"], pl["k_pairs"], pl["gamma_regs"]) == (1, 1, 1)
+        pl = qk.qknorm_plan_fwd(4096, 4096, 4096, 4, qk.QKNORM_E4M3, 148)
+        assert (pl["vmax"], pl["k_pairs"], pl["gamma_regs"]) == (2, 1, 0)   # 2 x 2 FP8 vectors: gamma via L1
+        for shape in ((4096, 5120, 5120, 4), (4096, 5120, 5120, 2), (4096, 1280, 640, 5), (64, 4096, 512, 32)):
+            with pytest.raises(qk.QKNormError) as ei:           # shards over 3 vectors per lane,
                 qk.qknorm_plan_fwd(*shape, qk.QKNORM_BF16, 148)  # P odd, or P > 16
             assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         qk.qknorm_force_variant(qk.VARIANT_BULK, 0)

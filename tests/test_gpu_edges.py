@@ -301,12 +301,16 @@ def test_rows_variant_rings(qk, wq, wk, stages, gsm, grid):
 
 
 @pytest.mark.parametrize("T,Dq,Dk,P", [(2 * 148 + 41, 5120, 1024, 8), (700, 4096, 1024, 8),
-                                        (301, 2048, 256, 4), (150, 1536, 256, 2)])
+                                        (301, 2048, 256, 4), (150, 1536, 256, 2),
+                                        # K shards wider than 16 vectors: K in pairs too
+                                        (2 * 148 + 41, 4096, 4096, 8), (301, 5120, 4096, 8),
+                                        (150, 2048, 2048, 4), (77, 1024, 1536, 2)])
 @pytest.mark.parametrize("grid,stages", [(0, 0), (1, 1), (5, 3), (0, 1)])
 def test_pair_variant(qk, T, Dq, Dk, P, grid, stages):
-    """The shard-pair token ring (two Q shards per warp, two K shards on lane
-    halves): any grid (tokens wrap the ring many times) and ring depth gives
-    the same bits as the generic kernel."""
+    """The shard-pair token ring (two Q shards per warp; two K shards on lane
+    halves, or in pairs like Q's when wider than 16 vectors): any grid (tokens
+    wrap the ring many times) and ring depth gives the same bits as the
+    generic kernel."""
     wl = W.custom("pair", T, Dq, Dk, P, seed=38 + P)
     q, k, gq, gk = _inputs(wl, wl.Ts[0])
     ref = _fwd(qk, wl, q, k, gq, gk, variant="generic")
