@@ -63,9 +63,10 @@ def parse_args(argv=None):
                          "the largest T of the workload is used")
     ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows", "pair"),
                     help="force a kernel variant (for profiling; default: the selector's choice)")
-    ap.add_argument("--path", default="fused", choices=("fused", "split"),
-                    help="what a step runs: qknorm_fwd (default), or the split path "
-                         "(qknorm_partial_sumsq then qknorm_apply, for Q and for K: 4 launches)")
+    ap.add_argument("--path", default="fused", choices=("fused", "split", "headwise"),
+                    help="what a step runs: qknorm_fwd (default), the split path "
+                         "(qknorm_partial_sumsq then qknorm_apply, for Q and for K: 4 launches), "
+                         "or headwise QK-Norm over heads of 128 (qknorm_headwise_fwd)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per GPU of the timed region (default: the workload's largest T); "
                          "a smaller T gives a small case for profiling")
@@ -291,6 +292,27 @@ class Split:
                                    f"{self.qk.qknorm_last_error()}")
 
 
+HEAD_DIM = 128
+
+
+class Headwise:
+    """Headwise QK-Norm for one buffer set through the raw C ABI: Q and K rows
+    as heads of HEAD_DIM values, gamma [HEAD_DIM] per tensor."""
+
+    def __init__(self, qk, bufs, T, Dq, Dk, eps, dtype_code, stream):
+        q, k, gq, gk, oq, ok = bufs
+        self.fn = qk.lib.qknorm_headwise_fwd
+        self.args = (q.data_ptr(), k.data_ptr(), gq.data_ptr(), gk.data_ptr(), oq.data_ptr(),
+                     ok.data_ptr(), T, Dq // HEAD_DIM, Dk // HEAD_DIM, HEAD_DIM, eps, dtype_code,
+                     Dq, Dk, Dq, Dk, stream)
+        self.qk = qk
+
+    def __call__(self):
+        st = self.fn(*self.args)
+        if st != 0:
+            raise RuntimeError(f"headwise: {self.qk.qknorm_status_string(st)} {self.qk.qknorm_last_error()}")
+
+
 def device_inputs(torch, wl, T, device, row0=0):
     """q, k (bf16 or fp32) drawn on the device with the workload's recipe, and
     gamma; rows start at row0."""
@@ -470,10 +492,11 @@ def fp8_prefill(torch, qk, device, peak, steps=200):
     gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(device)
     out = {"workload": "13B-shaped prefill in FP8 E4M3: T=8192, Dq=Dk=5120, P=4"}
     out.update(_fp8_case(torch, qk, device, peak, wl, gq, gk, steps))
-    wl8 = W.custom("split_large_e4m3", 65536, 4096, 4096, 8, dtype="e4m3", seed=12)
-    g8 = torch.rand(4096, device=device) + 0.5
+    wl8 = W.WORKLOADS["split_large_e4m3"]
+    g8q = torch.from_numpy(W.gen_gamma(wl8, "q")).to(device)
+    g8k = torch.from_numpy(W.gen_gamma(wl8, "k")).to(device)
     r = {"workload": "T=65536, Dq=Dk=4096, P=8 in FP8 E4M3"}
-    r.update(_fp8_case(torch, qk, device, peak, wl8, g8, g8, steps // 4))
+    r.update(_fp8_case(torch, qk, device, peak, wl8, g8q, g8k, steps // 4))
     out["split_large_e4m3"] = r
     return out
 
@@ -635,9 +658,10 @@ def split_path(torch, qk, device, peak, steps=20):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_rows_rate(wl, n_rows, nthreads, target_s):
-    """Run the float64 oracle on n_rows tokens of Q and K until target_s has
-    passed; returns (passes, seconds)."""
+def oracle_rows_rate(wl, n_rows, nthreads, target_s, headwise=False):
+    """Run the float64 oracle on n_rows tokens of Q and K (layerwise, or
+    headwise over heads of HEAD_DIM) until target_s has passed; returns
+    (passes, seconds)."""
     import oracle
     orc = oracle.get()
     rows = np.arange(n_rows)
@@ -646,20 +670,25 @@ def oracle_rows_rate(wl, n_rows, nthreads, target_s):
     eps = float(np.float32(wl.eps))
     passes, t0 = 0, time.perf_counter()
     while True:
-        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=nthreads)
+        if headwise:
+            orc.headwise(q, gq[:HEAD_DIM], HEAD_DIM, eps, wl.dtype, nthreads=nthreads)
+            orc.headwise(k, gk[:HEAD_DIM], HEAD_DIM, eps, wl.dtype, nthreads=nthreads)
+        else:
+            orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=nthreads)
         passes += 1
         el = time.perf_counter() - t0
         if el >= target_s:
             return passes, el
 
 
-def cpu_baseline(wl, T, target_s=10.0):
+def cpu_baseline(wl, T, target_s=10.0, headwise=False):
     cores = host_cores()
     n = min(T, 2048)
-    passes, el = oracle_rows_rate(wl, n, cores, target_s)
+    passes, el = oracle_rows_rate(wl, n, cores, target_s, headwise)
     nbytes = passes * W.fused_bytes(n, wl.Dq, wl.Dk, wl.elem_bytes)
+    what = f", headwise over heads of {HEAD_DIM}" if headwise else ""
     return {"value": round(nbytes / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} of the {T} tokens (Q and K rows), {passes} passes in {el:.1f} s, "
+            "sample": f"{n} of the {T} tokens (Q and K rows{what}), {passes} passes in {el:.1f} s, "
                       f"float64 C oracle with OpenMP over tokens on {cores} threads ({cpu_model()})",
             "tokens_per_s": round(passes * n / el, 1)}
 
@@ -734,6 +763,9 @@ def run_native(args, dist):
     wl = W.WORKLOADS[args.workload]
     T = args.tokens if args.tokens > 0 else max(wl.Ts)   # tokens per GPU (weak scaling)
     split = args.path == "split"
+    hw = args.path == "headwise"
+    if hw and (wl.Dq % HEAD_DIM or wl.Dk % HEAD_DIM):
+        raise SystemExit(f"--path headwise needs widths that are multiples of {HEAD_DIM}")
     row0, _ = shard_tokens(T * dist.world, dist.world, dist.rank)
     stream = torch.cuda.current_stream(device)
     peak, peak_src = hbm_peak()
@@ -741,6 +773,8 @@ def run_native(args, dist):
     qk.qknorm_force_variant(VARIANT_IDS[args.variant], 0)
 
     q, k, gq, gk = device_inputs(torch, wl, T, device, row0)
+    if hw:      # one gamma of head_dim per tensor
+        gq, gk = gq[:HEAD_DIM].contiguous(), gk[:HEAD_DIM].contiguous()
     nsets = buffer_sets(W.fused_bytes(T, wl.Dq, wl.Dk, wl.elem_bytes))
     sets = [(q, k)] + [(q.clone(), k.clone()) for _ in range(nsets - 1)]
     def step_of(bufs):
@@ -748,10 +782,14 @@ def run_native(args, dist):
             st = (torch.empty((T, wl.P), dtype=torch.float32, device=device),
                   torch.empty((T, wl.P), dtype=torch.float32, device=device))
             return Split(qk, bufs, st, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
+        if hw:
+            return Headwise(qk, bufs, T, wl.Dq, wl.Dk, wl.eps, dt, stream.cuda_stream)
         return Fused(qk, bufs, T, wl.Dq, wl.Dk, wl.P, wl.eps, dt, stream.cuda_stream)
 
     calls = [step_of((a, b, gq, gk, torch.empty_like(a), torch.empty_like(b))) for a, b in sets]
-    plan = qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, dt)
+    plan = (qk.qknorm_launch_plan(T, wl.Dq, wl.Dk, wl.P, dt) if not hw else
+            {"kernel": "headwise_k", "head_dim": HEAD_DIM, "heads_q": wl.Dq // HEAD_DIM,
+             "heads_k": wl.Dk // HEAD_DIM})
     for i in range(max(3, args.warmup)):
         calls[i % len(calls)]()
     torch.cuda.synchronize()
@@ -785,8 +823,8 @@ def run_native(args, dist):
     qd, kd = sets[1]
     oqd, okd = (torch.empty_like(q), torch.empty_like(k))
     f = step_of((qd, kd, gq, gk, oqd, okd))
-    if split:
-        e2e_path = "pinned host -> device copies, the split path, device -> pinned host"
+    if split or hw:
+        e2e_path = f"pinned host -> device copies, the {args.path} path, device -> pinned host"
 
         def e2e_step():
             qd.copy_(qh, non_blocking=True)
@@ -823,7 +861,7 @@ def run_native(args, dist):
     h2d = (qh.numel() + kh.numel()) * qh.element_size()
     d2h = (oqh.numel() + okh.numel()) * oqh.element_size()
     e2e_ok = True
-    if not split:      # the host outputs of the last step equal the device path's
+    if not split and not hw:      # the host outputs of the last step equal the device path's
         f()
         torch.cuda.synchronize()
         e2e_ok = bool(torch.equal(oqh.view(torch.uint8), oqd.cpu().view(torch.uint8)) and
@@ -849,11 +887,12 @@ def run_native(args, dist):
     dist.barrier()
 
     traffic = None
-    if (not split and args.workload == HEADLINE and T == max(wl.Ts) and
+    if (not split and not hw and args.workload == HEADLINE and T == max(wl.Ts) and
             NCU_TRAFFIC["src_sha"] == kernel_src_sha() and NCU_TRAFFIC["bytes_per_launch"] and
             all(plan.get(key) == val for key, val in NCU_TRAFFIC["plan"].items())):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     kernel = ("stats_k + apply_k (split path, 4 launches per step)" if split
+              else "headwise_k (qknorm_headwise_fwd)" if hw
               else KERNEL_OF_VARIANT.get(plan["variant"], "?") + " (qknorm_fwd)")
     line = {
         "impl": "native",
@@ -883,7 +922,7 @@ def run_native(args, dist):
     }
     line.update(extras)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, T)
+        line["cpu_baseline"] = cpu_baseline(wl, T, headwise=hw)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

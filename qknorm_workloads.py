@@ -107,6 +107,10 @@ WORKLOADS = {
         dtype="bf16", seed=5, token_scale_log10=(-2.0, 2.0),
         note="large prefill, split path: T=65536, D=4096, bf16, P=8, "
              "per-token scale log-uniform in [0.01, 100]"),
+    "split_large_e4m3": Workload(
+        "split_large_e4m3", Ts=(65536,), Dq=4096, Dk=4096, P=8, eps=1e-6,
+        dtype="e4m3", seed=12, x_sigma=1.5,
+        note="large prefill in FP8 E4M3: T=65536, D=4096, P=8 (one 16-byte vector per lane per shard)"),
 }
 
 
