@@ -18,8 +18,8 @@
 // each lane holding VMAX vectors. R units' loads are issued before any is
 // reduced.
 //
-// Work is dealt in groups of R consecutive units of one token, not in whole
-// tokens: at T = 8192 a resident grid of ~4700 warps would otherwise hold one
+// Work is dealt in groups of up to R consecutive units of one tensor of one
+// token, not in whole tokens: at T = 8192 a resident grid of ~4700 warps would otherwise hold one
 // or two tokens each, and the second half of the launch would run with the
 // one-token warps already gone. Groups are ~5x finer, so every warp ends
 // within one group of the others.
@@ -35,10 +35,58 @@ __device__ __forceinline__ float seg_butterfly(float c) {
     return c;
 }
 
-// Four 256-thread CTAs per SM (64 registers) where that costs no spills: the
-// bf16 and fp32 instances up to 4 vectors per lane. FP8 keeps 2 x 16 gamma
-// values per lane in registers and needs more.
-constexpr int headwise_min_blocks(int vec, int vmax) { return vec <= 8 && vmax <= 4 ? 4 : 1; }
+// CTAs per SM the register budget is sized for. bf16/fp32 heads of up to 32
+// vectors: four (64 registers; a 16-byte spill, measured faster than three
+// CTAs at 80 registers: 86.3 against 85.4 % at 32 + 8 heads of 128); up to 4
+// vectors per lane: two. FP8 keeps 2 x 16 gamma values per lane in registers
+// and needs more.
+constexpr int headwise_min_blocks(int vec, int vmax) {
+    return vec <= 8 && vmax <= 4 ? (vmax == 1 ? 4 : 2) : 1;
+}
+
+// One group: units u0 .. u0 + R - 1 of tensor Z (< Uz) of token t. The
+// tensor is a template argument, so its row pointers are formed once per
+// group and its gamma registers are used without a select.
+template <class Tag, int SEG, int VMAX, int R, int Z>
+__device__ __forceinline__ void headwise_group(const HeadArgs &a, int64_t t, int u0, int Uz, int slot,
+                                               int hsub, const float *gz) {
+    constexpr int VEC = Tag::kVec;
+    constexpr int HPW = 32 / SEG;
+    const int nv = a.nv;
+    const uint4 *xrow = reinterpret_cast<const uint4 *>(a.x[Z]) + t * a.ldx[Z];
+    uint4 *yrow = reinterpret_cast<uint4 *>(a.y[Z]) + t * a.ldy[Z];
+    uint4 v[R][VMAX];
+    bool ok[R];
+    int col[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        const int head = (u0 + j) * HPW + hsub;
+        ok[j] = u0 + j < Uz && head < a.H[Z];
+        col[j] = head * nv;
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i) {
+            const int vv = slot + 32 * i;
+            if (ok[j] && vv < nv) v[j][i] = ld_stream(xrow + col[j] + vv);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        float c = 0.f;
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
+        const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i) {
+            const int vv = slot + 32 * i;
+            if (ok[j] && vv < nv) {
+                const uint4 y = VMAX == 1 ? vapply_regs(Tag{}, v[j][i], gz, r)
+                                          : vapply(Tag{}, v[j][i], a.g[Z] + (int64_t)vv * VEC, r);
+                st_stream(yrow + col[j] + vv, y);
+            }
+        }
+    }
+}
 
 template <class Tag, int SEG, int VMAX, int R>
 __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) headwise_k(const HeadArgs a) {
@@ -52,7 +100,7 @@ __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) hea
     const int nv = a.nv;
     const int64_t NW = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int Uq = (a.H[0] + HPW - 1) / HPW;
-    const int U = Uq + (a.H[1] + HPW - 1) / HPW;
+    const int Uk = (a.H[1] + HPW - 1) / HPW;
     // Small heads: this lane's gamma for both tensors stays in registers.
     float gr[2][VMAX == 1 ? VEC : 1];
     if (VMAX == 1 && slot < nv) {
@@ -67,7 +115,9 @@ __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) hea
                 gr[z][e + 3] = g4.w;
             }
     }
-    const int G = (U + R - 1) / R;  // groups per token
+    // A token's groups: Gq of Q units, then Gk of K units (no group spans both).
+    const int Gq = (Uq + R - 1) / R;
+    const int G = Gq + (Uk + R - 1) / R;
     // Group gi = t * G + gsub; a warp's groups advance by NW, so (t, gsub) are
     // carried along instead of divided out.
     const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -76,51 +126,10 @@ __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) hea
     int64_t t = w0 / G;
     int gsub = (int)(w0 - t * G);
     while (t < a.T) {
-        const int u0 = gsub * R;
-        uint4 v[R][VMAX];
-        bool ok[R];
-        const uint4 *src[R];
-        uint4 *dst[R];
-        int zz[R];
-#pragma unroll
-        for (int j = 0; j < R; ++j) {
-            const int u = u0 + j;
-            const int z = u < Uq ? 0 : 1;
-            const int head = (z ? u - Uq : u) * HPW + hsub;
-            ok[j] = u < U && head < (z ? a.H[1] : a.H[0]);
-            zz[j] = z;
-            const int64_t col = (int64_t)head * nv;
-            src[j] = reinterpret_cast<const uint4 *>(z ? a.x[1] : a.x[0]) + t * (z ? a.ldx[1] : a.ldx[0]) + col;
-            dst[j] = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) + col;
-#pragma unroll
-            for (int i = 0; i < VMAX; ++i) {
-                const int vv = slot + 32 * i;
-                if (ok[j] && vv < nv) v[j][i] = ld_stream(src[j] + vv);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < R; ++j) {
-            float c = 0.f;
-#pragma unroll
-            for (int i = 0; i < VMAX; ++i)
-                if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
-            const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
-#pragma unroll
-            for (int i = 0; i < VMAX; ++i) {
-                const int vv = slot + 32 * i;
-                if (ok[j] && vv < nv) {
-                    uint4 y;
-                    if (VMAX == 1) {
-                        float gg[VEC];  // select, so the array stays in registers
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e) gg[e] = zz[j] ? gr[1][e] : gr[0][e];
-                        y = vapply_regs(Tag{}, v[j][i], gg, r);
-                    } else
-                        y = vapply(Tag{}, v[j][i], (zz[j] ? a.g[1] : a.g[0]) + (int64_t)vv * VEC, r);
-                    st_stream(dst[j] + vv, y);
-                }
-            }
-        }
+        if (gsub < Gq)
+            headwise_group<Tag, SEG, VMAX, R, 0>(a, t, gsub * R, Uq, slot, hsub, gr[0]);
+        else
+            headwise_group<Tag, SEG, VMAX, R, 1>(a, t, (gsub - Gq) * R, Uk, slot, hsub, gr[1]);
         t += dt;
         gsub += dg;
         if (gsub >= G) {
@@ -172,9 +181,9 @@ const void *headwise_table(int nv) {
 
 int64_t headwise_groups(int64_t T, int32_t Hq, int32_t Hk, int32_t nv) {
     const int hpw = nv <= kLanes ? kLanes / seg_of(nv) : 1;
-    const int64_t units = (Hq + hpw - 1) / hpw + (Hk + hpw - 1) / hpw;
+    const int64_t uq = (Hq + hpw - 1) / hpw, uk = (Hk + hpw - 1) / hpw;
     const int r = units_per_group((nv + kLanes - 1) / kLanes);
-    return T * ((units + r - 1) / r);
+    return T * ((uq + r - 1) / r + (uk + r - 1) / r);
 }
 
 const void *headwise_kernel(int dtype, int nv) {

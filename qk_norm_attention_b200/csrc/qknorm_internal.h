@@ -104,7 +104,8 @@ struct HeadArgs {
     int64_t ldy[2];
 };
 const void *headwise_kernel(int dtype, int nv);
-// Work groups of the headwise kernel for nv (one warp each): T * ceil(units / R).
+// Work groups of the headwise kernel for nv (one warp each): T * (ceil(Q units / R) +
+// ceil(K units / R)).
 int64_t headwise_groups(int64_t T, int32_t Hq, int32_t Hk, int32_t nv);
 cudaError_t launch_headwise(int dtype, const HeadArgs &a, int block, int64_t grid, cudaStream_t s);
 
