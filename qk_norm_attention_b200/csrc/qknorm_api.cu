@@ -869,6 +869,7 @@ int qknorm_headwise_fwd(const void *q, const void *k, const float *gamma_q, cons
     a.H[1] = Hk;
     a.nv = nv;
     a.Df = (float)head_dim;
+    a.inv_df = (head_dim & (head_dim - 1)) == 0 ? 1.0f / (float)head_dim : 0.f;
     a.eps = eps;
     a.ldx[0] = ldq / vec;
     a.ldx[1] = ldk / vec;

@@ -75,7 +75,13 @@ __device__ __forceinline__ void headwise_group(const HeadArgs &a, int64_t t, int
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
             if (ok[j] && slot + 32 * i < nv) c = __fadd_rn(c, vsumsq(Tag{}, v[j][i]));
-        const float r = factor(seg_butterfly<SEG>(c), a.Df, a.eps);
+        // rsqrt(S / head_dim + eps) as factor() forms it. For a power-of-two
+        // head_dim, S * (1 / head_dim) is the same correctly rounded number
+        // as the division (the quotient is S scaled by a power of two), so
+        // the multiply replaces it bit for bit.
+        const float S = seg_butterfly<SEG>(c);
+        const float r = a.inv_df != 0.f ? rsqrtf(__fadd_rn(__fmul_rn(S, a.inv_df), a.eps))
+                                        : factor(S, a.Df, a.eps);
 #pragma unroll
         for (int i = 0; i < VMAX; ++i) {
             const int vv = slot + 32 * i;

@@ -99,6 +99,7 @@ struct HeadArgs {
     int32_t H[2];       // heads
     int32_t nv;         // 16-byte vectors per head
     float Df;           // head_dim
+    float inv_df;       // 1 / head_dim when head_dim is a power of two (exact), else 0
     float eps;
     int64_t ldx[2];     // row strides, in 16-byte vectors
     int64_t ldy[2];
