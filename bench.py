@@ -504,9 +504,11 @@ def fp8_prefill(torch, qk, device, peak, steps=200):
 def tp_rank_step(torch, qk, device, peak, steps=100):
     """One rank's kernels of the tensor-parallel form at the 13B shape (T =
     8192, Dq = Dk = 5120, P = 8) for a group of `ranks` GPUs: the statistics
-    of its Q and K slices, then qknorm_apply_tp on each (4 launches). The
-    all-gather between them needs several GPUs and is not timed here; the
-    gathered sums are those of the emulated group, computed beforehand."""
+    of its Q and K slices, then the apply step of each, as two launches
+    (qknorm_partial_sumsq_qk, qknorm_apply_tp_qk: what qknorm_tp_fwd runs) and
+    as four one-tensor launches. The all-gather between them needs several
+    GPUs and is not timed here; the gathered sums are those of the emulated
+    group, computed beforehand."""
     T, D, P = 8192, 5120, 8
     stream = torch.cuda.current_stream(device)
     h = stream.cuda_stream
@@ -516,42 +518,58 @@ def tp_rank_step(torch, qk, device, peak, steps=100):
     k = W.gen_device_workload(wl, "k", T, device)
     g = torch.rand(D, device=device) + 0.5
     out = {}
+
+    def ok(rc):
+        if rc != 0:
+            raise RuntimeError(qk.qknorm_status_string(rc))
+
     for ranks in (2, 4, 8):
         Dl, Pl = D // ranks, P // ranks
         qs = [q[:, r * Dl:(r + 1) * Dl].contiguous() for r in range(ranks)]
         ks = [k[:, r * Dl:(r + 1) * Dl].contiguous() for r in range(ranks)]
-        gathered = torch.stack([torch.stack((qk.qknorm_partial_sumsq(a, Pl), qk.qknorm_partial_sumsq(b, Pl)))
-                                for a, b in zip(qs, ks)])            # [ranks, 2, T, P_local]
+        gathered = torch.stack([qk.qknorm_partial_sumsq_qk(a, b, Pl) for a, b in zip(qs, ks)])
         gl = g[:Dl].contiguous()
         sets = [(qs[r], ks[r], torch.empty_like(qs[r]), torch.empty_like(ks[r]),
                  torch.empty((2, T, Pl), dtype=torch.float32, device=device)) for r in range(ranks)]
         stride = gathered.stride(0)
+        gq_, gk_ = gathered[:, 0].data_ptr(), gathered[:, 1].data_ptr()
 
-        def step_of(a, b, oa, ob, st):
+        def step_two(a, b, oa, ob, st):
             def step():
-                for rc in (L.qknorm_partial_sumsq(a.data_ptr(), st[0].data_ptr(), T, Dl, Pl, 1, h),
-                           L.qknorm_partial_sumsq(b.data_ptr(), st[1].data_ptr(), T, Dl, Pl, 1, h),
-                           L.qknorm_apply_tp(a.data_ptr(), gl.data_ptr(), gathered[:, 0].data_ptr(), stride,
-                                             oa.data_ptr(), T, Dl, Pl, ranks, 1e-6, 1, h),
-                           L.qknorm_apply_tp(b.data_ptr(), gl.data_ptr(), gathered[:, 1].data_ptr(), stride,
-                                             ob.data_ptr(), T, Dl, Pl, ranks, 1e-6, 1, h)):
-                    if rc != 0:
-                        raise RuntimeError(qk.qknorm_status_string(rc))
+                ok(L.qknorm_partial_sumsq_qk(a.data_ptr(), b.data_ptr(), st[0].data_ptr(), st[1].data_ptr(),
+                                             T, Dl, Dl, Pl, 1, h))
+                ok(L.qknorm_apply_tp_qk(a.data_ptr(), b.data_ptr(), gl.data_ptr(), gl.data_ptr(), gq_, gk_,
+                                        stride, oa.data_ptr(), ob.data_ptr(), T, Dl, Dl, Pl, ranks, 1e-6,
+                                        1, h))
             return step
 
-        calls = [step_of(*st) for st in sets]        # the ranks' slices rotate (inputs beyond L2)
-        for i in range(10):
-            calls[i % ranks]()
-        torch.cuda.synchronize()
-        tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
-        ms = tot / steps
+        def step_four(a, b, oa, ob, st):
+            def step():
+                ok(L.qknorm_partial_sumsq(a.data_ptr(), st[0].data_ptr(), T, Dl, Pl, 1, h))
+                ok(L.qknorm_partial_sumsq(b.data_ptr(), st[1].data_ptr(), T, Dl, Pl, 1, h))
+                ok(L.qknorm_apply_tp(a.data_ptr(), gl.data_ptr(), gq_, stride, oa.data_ptr(), T, Dl, Pl,
+                                     ranks, 1e-6, 1, h))
+                ok(L.qknorm_apply_tp(b.data_ptr(), gl.data_ptr(), gk_, stride, ob.data_ptr(), T, Dl, Pl,
+                                     ranks, 1e-6, 1, h))
+            return step
+
         nbytes = 2 * (3 * T * Dl * 2 + 4 * T * Pl + 4 * ranks * T * Pl + 4 * Dl)
-        out[str(ranks)] = {"us_per_step": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
-                           "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1),
-                           "algorithmic_bytes": nbytes, "exchange_bytes_per_rank": 2 * 4 * T * Pl}
-        del qs, ks, gathered, sets, calls
+        res = {}
+        for label, mk in (("two_launches", step_two), ("four_launches", step_four)):
+            calls = [mk(*st) for st in sets]        # the ranks' slices rotate (inputs beyond L2)
+            for i in range(10):
+                calls[i % ranks]()
+            torch.cuda.synchronize()
+            tot, _ = time_launches(torch, calls, steps, stream, per_launch=False)
+            ms = tot / steps
+            res[label] = {"us_per_step": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
+                          "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1)}
+        out[str(ranks)] = dict(res["two_launches"], four_launches=res["four_launches"],
+                               algorithmic_bytes=nbytes, exchange_bytes_per_rank=2 * 4 * T * Pl)
+        del qs, ks, gathered, sets
     return {"workload": "13B-shaped Q and K (T=8192, D=5120, P=8) split over a tensor-parallel group; "
-                        "one rank's statistics + apply_tp kernels, the all-gather not timed",
+                        "one rank's statistics + apply kernels (Q and K in one launch each), "
+                        "the all-gather not timed",
             "ranks": out}
 
 

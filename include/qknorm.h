@@ -148,7 +148,8 @@ QKNORM_API int qknorm_headwise_fwd(const void *q, const void *k, const float *ga
  * Algorithm 1, Phase A for one tensor: stats[t*P + p] = fp32 sum of
  * squares of shard p of row t (the scalar each rank publishes to its IPC
  * slot in the review's multi-GPU form), in the reduction order above.
- *   x [T, D] input, dtype; stats [T, P] fp32 output.
+ *   x [T, D] input, dtype (16-byte aligned); stats [T, P] fp32 output
+ *   (4-byte alignment suffices: it is written one value at a time).
  * Returns a qknorm_status.
  */
 QKNORM_API int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int32_t P,
@@ -201,6 +202,43 @@ QKNORM_API int qknorm_apply(const void *x, const float *gamma, const float *stat
 QKNORM_API int qknorm_apply_tp(const void *x, const float *gamma, const float *stats,
                                int64_t stats_block_stride, void *out, int64_t T, int32_t D_local,
                                int32_t P_local, int32_t ranks, float eps, int32_t dtype, void *stream);
+
+/*
+ * qknorm_partial_sumsq_qk -- qknorm_partial_sumsq of Q and of K in one launch.
+ *
+ * Algorithm 1, Phase A for both tensors of a layer (e.g. one rank's Q and K
+ * slices in the tensor-parallel form): stats_q [T, P] from q [T, Dq] and
+ * stats_k [T, P] from k [T, Dk], each exactly as qknorm_partial_sumsq
+ * writes it (bit for bit). The launch's blocks are shared between the two in
+ * proportion to their widths, so the pair costs one launch's fixed start and
+ * drain instead of two. Same requirements as qknorm_partial_sumsq for each
+ * tensor; QKNORM_ERR_INVALID_ARG also when a statistics array overlaps the
+ * other statistics array or the other tensor.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_partial_sumsq_qk(const void *q, const void *k, float *stats_q, float *stats_k,
+                                       int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype,
+                                       void *stream);
+
+/*
+ * qknorm_apply_tp_qk -- qknorm_apply_tp of Q and of K in one launch.
+ *
+ * Phases B and C of Algorithm 1's tensor-parallel form for both tensors of
+ * one rank: out_q from q [T, Dq_local], gamma_q and stats_q, and out_k from
+ * k [T, Dk_local], gamma_k and stats_k, each exactly as qknorm_apply_tp
+ * computes it (bit for bit), with one stats_block_stride for both (an
+ * all-gather of [2, T, P_local] per rank gives [ranks, 2, T, P_local]:
+ * stats_q = its base, stats_k = base + T * P_local, stride 2 * T * P_local).
+ * ranks = 1 with stride 0 is qknorm_apply of both tensors. Same requirements
+ * as qknorm_apply_tp for each tensor; QKNORM_ERR_INVALID_ARG also when an
+ * output overlaps the other output or any input of the other tensor.
+ * Returns a qknorm_status.
+ */
+QKNORM_API int qknorm_apply_tp_qk(const void *q, const void *k, const float *gamma_q,
+                                  const float *gamma_k, const float *stats_q, const float *stats_k,
+                                  int64_t stats_block_stride, void *out_q, void *out_k, int64_t T,
+                                  int32_t Dq_local, int32_t Dk_local, int32_t P_local, int32_t ranks,
+                                  float eps, int32_t dtype, void *stream);
 
 /*
  * qknorm_fwd_host -- qknorm_fwd on rows in HOST memory, end to end: the rows

@@ -96,6 +96,11 @@ def _load() -> ctypes.CDLL:
     lib.qknorm_fwd_host_workspace.restype = ctypes.c_int64
     lib.qknorm_apply_tp.argtypes = [vp, vp, vp, i64, vp, i64, i32, i32, i32, f32, i32, vp]
     lib.qknorm_apply_tp.restype = ctypes.c_int
+    lib.qknorm_partial_sumsq_qk.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, vp]
+    lib.qknorm_partial_sumsq_qk.restype = ctypes.c_int
+    lib.qknorm_apply_tp_qk.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32,
+                                       f32, i32, vp]
+    lib.qknorm_apply_tp_qk.restype = ctypes.c_int
     lib.qknorm_xgamma.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     lib.qknorm_xgamma.restype = ctypes.c_int
     lib.qknorm_inv_rms.argtypes = [vp, vp, i64, i32, i32, f32, i32, vp]
@@ -353,6 +358,58 @@ def qknorm_apply_tp(x: torch.Tensor, gamma: torch.Tensor, stats: torch.Tensor, e
                              _stream_handle(x.device, stream))
     _check("qknorm_apply_tp", st)
     return out
+
+
+def qknorm_partial_sumsq_qk(q: torch.Tensor, k: torch.Tensor, P: int,
+                            stats: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The shard sums of q [T, Dq] and k [T, Dk] in one launch: returns
+    stats [2, T, P] (stats[0] Q's, stats[1] K's), each as qknorm_partial_sumsq."""
+    if q.dim() != 2 or k.dim() != 2 or q.shape[0] != k.shape[0]:
+        raise ValueError("q and k must be [T, Dq] and [T, Dk]")
+    T, P = q.shape[0], int(P)
+    stats = torch.empty((2, T, P), dtype=torch.float32, device=q.device) if stats is None else stats
+    for name, t in (("q", q), ("k", k), ("stats", stats)):
+        _need_cuda_contig(name, t)
+    if stats.dtype != torch.float32 or tuple(stats.shape) != (2, T, P) or q.dtype != k.dtype:
+        raise ValueError("stats must be float32 [2, T, P]; q and k of one dtype")
+    st = lib.qknorm_partial_sumsq_qk(q.data_ptr(), k.data_ptr(), stats[0].data_ptr(), stats[1].data_ptr(),
+                                     T, q.shape[1], k.shape[1], P, _dtype_code(q),
+                                     _stream_handle(q.device, stream))
+    _check("qknorm_partial_sumsq_qk", st)
+    return stats
+
+
+def qknorm_apply_tp_qk(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                       stats: torch.Tensor, eps: float, out_q: Optional[torch.Tensor] = None,
+                       out_k: Optional[torch.Tensor] = None,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """qknorm_apply_tp of one rank's q [T, Dq_local] and k [T, Dk_local] in one
+    launch, from stats [ranks, 2, T, P_local] (every rank's Q and K shard sums,
+    as an all-gather of each rank's [2, T, P_local] leaves them)."""
+    if q.dim() != 2 or k.dim() != 2 or stats.dim() != 4 or stats.shape[1] != 2 or \
+            stats.shape[2] != q.shape[0] or k.shape[0] != q.shape[0]:
+        raise ValueError("q, k must be [T, D_local] and stats [ranks, 2, T, P_local]")
+    T = q.shape[0]
+    ranks, _, _, P = stats.shape
+    out_q = torch.empty_like(q) if out_q is None else out_q
+    out_k = torch.empty_like(k) if out_k is None else out_k
+    for name, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("out_q", out_q),
+                    ("out_k", out_k)):
+        _need_cuda_contig(name, t)
+    if not stats.is_cuda or stats.stride(3) != 1 or stats.stride(2) != P or stats.stride(1) != T * P:
+        raise ValueError("stats must hold contiguous [2, T, P_local] blocks on the GPU")
+    if gamma_q.dtype != torch.float32 or gamma_k.dtype != torch.float32 or stats.dtype != torch.float32:
+        raise TypeError("gamma and stats must be float32")
+    if out_q.shape != q.shape or out_k.shape != k.shape or out_q.dtype != q.dtype or \
+            out_k.dtype != k.dtype or q.dtype != k.dtype or gamma_q.numel() != q.shape[1] or \
+            gamma_k.numel() != k.shape[1]:
+        raise ValueError("outputs must match their inputs; gamma_q, gamma_k of the local widths")
+    st = lib.qknorm_apply_tp_qk(q.data_ptr(), k.data_ptr(), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                                stats[:, 0].data_ptr(), stats[:, 1].data_ptr(), stats.stride(0),
+                                out_q.data_ptr(), out_k.data_ptr(), T, q.shape[1], k.shape[1], P, ranks,
+                                float(eps), _dtype_code(q), _stream_handle(q.device, stream))
+    _check("qknorm_apply_tp_qk", st)
+    return out_q, out_k
 
 
 def qknorm_xgamma(x: torch.Tensor, gamma: torch.Tensor, out: Optional[torch.Tensor] = None,

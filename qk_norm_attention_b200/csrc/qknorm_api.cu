@@ -620,13 +620,84 @@ int64_t host_chunk(int64_t chunk_tokens) { return chunk_tokens > 0 ? chunk_token
 
 using namespace qkn;
 
-// The apply step for stats laid out as nb blocks [nb, T, Pb] (nb = 1: the
-// split path's [T, P]; nb = ranks: an all-gather of each rank's [T, P_local]
-// in a tensor-parallel group, whose rows are the D-wide local slices of
-// nb * D-wide rows). The divisor is nb * D.
-static int apply_blocks(const void *x, const float *gamma, const float *stats, int64_t sg, void *out,
-                        int64_t T, int32_t D, int32_t Pb, int32_t nb, float eps, int32_t dtype,
-                        void *stream) {
+// Grid shares of a launch over n (1 or 2) tensors: at most cap blocks in
+// all, side z at most need[z] (its work) and at least 1, the rest in
+// proportion to the sides' bytes. Returns side 0's share; *total the grid.
+static int64_t split_grid(int n, const int64_t *need, const int64_t *bytes, int64_t cap,
+                          int64_t *total) {
+    if (n == 1) {
+        *total = need[0] < cap ? need[0] : cap;
+        return *total;
+    }
+    int64_t all = need[0] + need[1];
+    if (all > cap) all = cap;
+    if (all < 2) all = 2;
+    int64_t g0 = (int64_t)((double)all * (double)bytes[0] / (double)(bytes[0] + bytes[1]) + 0.5);
+    if (g0 > need[0]) g0 = need[0];
+    if (g0 > all - 1) g0 = all - 1;
+    if (g0 < 1) g0 = 1;
+    int64_t g1 = all - g0;
+    if (g1 > need[1]) g1 = need[1];
+    *total = g0 + g1;
+    return g0;
+}
+
+// Argument checks of the statistics pass for one tensor.
+static int check_stats_side(const void *x, const float *stats, int64_t T, int32_t D, int32_t P,
+                            int32_t dtype) {
+    int st = check_shape(T, D, P, dtype);
+    if (st != QKNORM_OK || T == 0) return st;
+    if (!x || !stats) return QKNORM_ERR_INVALID_ARG;
+    // The sums are written one fp32 at a time: 4-byte alignment suffices (the
+    // K half of a [2, T, P] array starts T * P floats in).
+    if (!aligned16(x) || reinterpret_cast<uintptr_t>(stats) % 4 != 0) return QKNORM_ERR_MISALIGNED;
+    if (T > INT64_MAX / 4 / P) return QKNORM_ERR_INVALID_ARG;
+    if (overlap(rng(stats, T * P * 4), rng(x, T * D * elem_of(dtype)))) return QKNORM_ERR_INVALID_ARG;
+    return QKNORM_OK;
+}
+
+// The statistics pass over n (1 or 2) checked tensors of T > 0 rows: one launch.
+static int stats_launch(int n, const void *const *x, float *const *stats, const int32_t *D,
+                        int64_t T, int32_t P, int32_t dtype, void *stream) {
+    TensorShape sh[2];
+    int vmax = 0;
+    for (int z = 0; z < n; ++z) {
+        sh[z] = make_shape(D[z], P, vec_of(dtype));
+        if (sh[z].vmax > vmax) vmax = sh[z].vmax;
+    }
+    int dev = 0, sms = 0;
+    cudaError_t e = device_sms(&dev, &sms);
+    if (e != cudaSuccess) return finish(e);
+    const int block = 256;
+    int bres = 1;
+    e = resident_blocks(dev, stats_kernel(dtype, vmax, n == 2), block, 0, &bres);
+    if (e != cudaSuccess) return finish(e);
+    // A block takes (block / 32) warps x R tasks per turn.
+    const int64_t per_block = (block / kLanes) * (vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1));
+    int64_t need[2], bytes[2], grid = 0;
+    for (int z = 0; z < n; ++z) {
+        need[z] = (T * P + per_block - 1) / per_block;
+        bytes[z] = (int64_t)D[z];
+    }
+    StatsArgs a;
+    for (int z = 0; z < 2; ++z) {
+        const int w = z < n ? z : 0;
+        a.side[z] = StatsSide{x[w], stats[w], D[w], sh[w].nv, sh[w].K};
+    }
+    a.T = T;
+    a.P = P;
+    a.split = (int32_t)split_grid(n, need, bytes, (int64_t)sms * bres, &grid);
+    return finish(launch_stats(dtype, vmax, a, block, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// Argument checks of the apply step for one tensor, stats laid out as nb
+// blocks [nb, T, Pb] (nb = 1: the split path's [T, P]; nb = ranks: an
+// all-gather of each rank's [T, P_local] in a tensor-parallel group, whose
+// rows are the D-wide local slices of nb * D-wide rows). *sg is set to the
+// block stride in use.
+static int check_apply_side(const void *x, const float *gamma, const float *stats, int64_t *sg,
+                            const void *out, int64_t T, int32_t D, int32_t Pb, int32_t nb, float eps,
+                            int32_t dtype) {
     int st = check_shape(T, D, Pb, dtype);
     if (st == QKNORM_OK) st = check_eps(eps);
     if (st != QKNORM_OK) return st;
@@ -639,34 +710,69 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
         reinterpret_cast<uintptr_t>(stats) % 4 != 0)
         return QKNORM_ERR_MISALIGNED;
     if (T > INT64_MAX / 4 / Pb / nb) return QKNORM_ERR_INVALID_ARG;
-    if (sg == 0) sg = T * Pb;
-    if (sg < T * Pb || sg > INT64_MAX / 4 / nb) return QKNORM_ERR_INVALID_ARG;   // blocks may not overlap
+    if (*sg == 0) *sg = T * Pb;
+    if (*sg < T * Pb || *sg > INT64_MAX / 4 / nb) return QKNORM_ERR_INVALID_ARG;   // blocks may not overlap
     const int64_t es = elem_of(dtype);
     const Range ro = rng(out, T * D * es);
     if (bad_alias(ro, rng(x, T * D * es), true) || bad_alias(ro, rng(gamma, (int64_t)D * 4), false) ||
-        bad_alias(ro, rng(stats, ((int64_t)(nb - 1) * sg + T * Pb) * 4), false))
+        bad_alias(ro, rng(stats, ((int64_t)(nb - 1) * *sg + T * Pb) * 4), false))
         return QKNORM_ERR_INVALID_ARG;
+    return QKNORM_OK;
+}
+
+// The apply step over n (1 or 2) checked tensors of T > 0 rows: one launch.
+// The divisor of side z is nb * D[z].
+static int apply_launch(int n, const void *const *x, const float *const *gamma,
+                        const float *const *stats, void *const *out, const int32_t *D, int64_t sg,
+                        int64_t T, int32_t Pb, int32_t nb, float eps, int32_t dtype, void *stream) {
     int dev = 0, sms = 0;
     cudaError_t e = device_sms(&dev, &sms);
     if (e != cudaSuccess) return finish(e);
-    // apply_threads_per_row(D) threads per row, as many rows per 256-thread
-    // block as fit.
-    const int tpr = apply_threads_per_row(D, dtype);
-    const int rpb = 256 / tpr;
-    const int block = tpr * rpb;
+    // apply_threads_per_row(D) threads per row. One tensor: as many rows per
+    // 256-thread block as fit. Two: a block size both sides' row groups
+    // divide (192 for 96-thread rows, else 256; a side's spare threads idle).
+    int tpr[2] = {0, 0};
+    bool multi = false, has96 = false, wide = false;
+    for (int z = 0; z < n; ++z) {
+        tpr[z] = apply_threads_per_row(D[z], dtype);
+        multi = multi || tpr[z] != 256;
+        has96 = has96 || tpr[z] == 96;
+        wide = wide || tpr[z] == 256;
+    }
+    const int block = n == 1 ? tpr[0] * (256 / tpr[0]) : (has96 && !wide ? 192 : 256);
     int bres = 1;
-    e = resident_blocks(dev, apply_kernel(dtype, rpb > 1), block, 0, &bres);
+    e = resident_blocks(dev, apply_kernel(dtype, multi, n == 2), block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
-    int64_t grid = (int64_t)sms * bres;
-    if (grid > (T + rpb - 1) / rpb) grid = (T + rpb - 1) / rpb;
-    return finish(launch_apply(dtype, x, gamma, stats, out, T, D, Pb, nb, sg,
-                               (float)((int64_t)D * nb), eps, block, grid,
-                               reinterpret_cast<cudaStream_t>(stream)));
+    int64_t need[2], bytes[2], grid = 0;
+    ApplyArgs a;
+    for (int z = 0; z < 2; ++z) {
+        const int w = z < n ? z : 0;
+        const int rpb = block / tpr[w];
+        need[z] = (T + rpb - 1) / rpb;
+        bytes[z] = (int64_t)D[w];
+        a.side[z] = ApplySide{x[w], gamma[w], stats[w], out[w], D[w], tpr[w],
+                              (float)((int64_t)D[w] * nb)};
+    }
+    a.T = T;
+    a.sg = sg;
+    a.Pb = Pb;
+    a.nb = nb;
+    a.eps = eps;
+    a.split = (int32_t)split_grid(n, need, bytes, (int64_t)sms * bres, &grid);
+    return finish(launch_apply(dtype, multi, a, block, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int apply_blocks(const void *x, const float *gamma, const float *stats, int64_t sg, void *out,
+                        int64_t T, int32_t D, int32_t Pb, int32_t nb, float eps, int32_t dtype,
+                        void *stream) {
+    int st = check_apply_side(x, gamma, stats, &sg, out, T, D, Pb, nb, eps, dtype);
+    if (st != QKNORM_OK || T == 0) return st;
+    return apply_launch(1, &x, &gamma, &stats, &out, &D, sg, T, Pb, nb, eps, dtype, stream);
 }
 
 extern "C" {
 
-int qknorm_version(void) { return 113; }
+int qknorm_version(void) { return 114; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -975,28 +1081,24 @@ int qknorm_selftest_bounded_wait(uint64_t limit_ns, void *stream) {
 
 int qknorm_partial_sumsq(const void *x, float *stats, int64_t T, int32_t D, int32_t P,
                          int32_t dtype, void *stream) {
-    int st = check_shape(T, D, P, dtype);
-    if (st != QKNORM_OK) return st;
-    if (T == 0) return QKNORM_OK;
-    if (!x || !stats) return QKNORM_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(stats)) return QKNORM_ERR_MISALIGNED;
-    if (T > INT64_MAX / 4 / P) return QKNORM_ERR_INVALID_ARG;
-    if (overlap(rng(stats, T * P * 4), rng(x, T * D * elem_of(dtype)))) return QKNORM_ERR_INVALID_ARG;
-    const TensorShape sh = make_shape(D, P, vec_of(dtype));
-    int dev = 0, sms = 0;
-    cudaError_t e = device_sms(&dev, &sms);
-    if (e != cudaSuccess) return finish(e);
-    const int block = 256;
-    int bres = 1;
-    e = resident_blocks(dev, stats_kernel(dtype, sh.vmax), block, 0, &bres);
-    if (e != cudaSuccess) return finish(e);
-    const int64_t ntask = T * P;
-    const int64_t per_block = (block / kLanes) * (sh.vmax <= 2 ? 4 : (sh.vmax <= 4 ? 2 : 1));
-    int64_t grid = (ntask + per_block - 1) / per_block;
-    const int64_t cap = (int64_t)sms * bres;
-    if (grid > cap) grid = cap;
-    return finish(launch_stats(dtype, sh.vmax, x, stats, T, sh, P, block, grid,
-                               reinterpret_cast<cudaStream_t>(stream)));
+    const int st = check_stats_side(x, stats, T, D, P, dtype);
+    if (st != QKNORM_OK || T == 0) return st;
+    return stats_launch(1, &x, &stats, &D, T, P, dtype, stream);
+}
+
+int qknorm_partial_sumsq_qk(const void *q, const void *k, float *stats_q, float *stats_k, int64_t T,
+                            int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, void *stream) {
+    int st = check_stats_side(q, stats_q, T, Dq, P, dtype);
+    if (st == QKNORM_OK) st = check_stats_side(k, stats_k, T, Dk, P, dtype);
+    if (st != QKNORM_OK || T == 0) return st;
+    const Range sq = rng(stats_q, T * P * 4), sk = rng(stats_k, T * P * 4);
+    if (overlap(sq, sk) || overlap(sq, rng(k, T * Dk * elem_of(dtype))) ||
+        overlap(sk, rng(q, T * Dq * elem_of(dtype))))
+        return QKNORM_ERR_INVALID_ARG;
+    const void *x[2] = {q, k};
+    float *stats[2] = {stats_q, stats_k};
+    const int32_t D[2] = {Dq, Dk};
+    return stats_launch(2, x, stats, D, T, P, dtype, stream);
 }
 
 int qknorm_apply(const void *x, const float *gamma, const float *stats, void *out, int64_t T,
@@ -1010,6 +1112,33 @@ int qknorm_apply_tp(const void *x, const float *gamma, const float *stats, int64
     if (stats_block_stride < 0) return QKNORM_ERR_INVALID_ARG;
     return apply_blocks(x, gamma, stats, stats_block_stride, out, T, D_local, P_local, ranks, eps,
                         dtype, stream);
+}
+
+int qknorm_apply_tp_qk(const void *q, const void *k, const float *gamma_q, const float *gamma_k,
+                       const float *stats_q, const float *stats_k, int64_t stats_block_stride,
+                       void *out_q, void *out_k, int64_t T, int32_t Dq_local, int32_t Dk_local,
+                       int32_t P_local, int32_t ranks, float eps, int32_t dtype, void *stream) {
+    if (stats_block_stride < 0) return QKNORM_ERR_INVALID_ARG;
+    int64_t sgq = stats_block_stride, sgk = stats_block_stride;
+    int st = check_apply_side(q, gamma_q, stats_q, &sgq, out_q, T, Dq_local, P_local, ranks, eps, dtype);
+    if (st == QKNORM_OK)
+        st = check_apply_side(k, gamma_k, stats_k, &sgk, out_k, T, Dk_local, P_local, ranks, eps, dtype);
+    if (st != QKNORM_OK || T == 0) return st;
+    // Across the two tensors nothing an output overlaps may be read or written.
+    const int64_t es = elem_of(dtype);
+    const int64_t sbytes = ((int64_t)(ranks - 1) * sgq + T * P_local) * 4;
+    const Range oq = rng(out_q, T * Dq_local * es), ok = rng(out_k, T * Dk_local * es);
+    if (overlap(oq, ok) || overlap(oq, rng(k, T * Dk_local * es)) ||
+        overlap(oq, rng(gamma_k, (int64_t)Dk_local * 4)) || overlap(oq, rng(stats_k, sbytes)) ||
+        overlap(ok, rng(q, T * Dq_local * es)) || overlap(ok, rng(gamma_q, (int64_t)Dq_local * 4)) ||
+        overlap(ok, rng(stats_q, sbytes)))
+        return QKNORM_ERR_INVALID_ARG;
+    const void *x[2] = {q, k};
+    const float *g[2] = {gamma_q, gamma_k};
+    const float *stats[2] = {stats_q, stats_k};
+    void *out[2] = {out_q, out_k};
+    const int32_t D[2] = {Dq_local, Dk_local};
+    return apply_launch(2, x, g, stats, out, D, sgq, T, P_local, ranks, eps, dtype, stream);
 }
 
 int64_t qknorm_fwd_host_workspace(int64_t chunk_tokens, int32_t Dq, int32_t Dk, int32_t dtype) {

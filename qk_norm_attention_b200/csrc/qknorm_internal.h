@@ -38,25 +38,54 @@ TensorShape make_shape(int32_t D, int32_t P, int vec);
 // full: every lane holds exactly vmax vectors in every task (guard-free instance).
 const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads);
 const void *fused_generic_kernel(int dtype);
-const void *stats_kernel(int dtype, int vmax);
+// two: the instance for launches over two tensors.
+const void *stats_kernel(int dtype, int vmax, bool two);
 // multi: the several-rows-per-block instance of apply_k (block != tpr).
-const void *apply_kernel(int dtype, bool multi);
+const void *apply_kernel(int dtype, bool multi, bool two);
 
 // Launchers: enqueue one kernel; return the cudaError_t of the launch.
 cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
                              int block, int64_t grid, cudaStream_t s);
 cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
                                  size_t smem, cudaStream_t s);
-cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64_t T,
-                         const TensorShape &sh, int32_t P, int block, int64_t grid,
+// The split path's kernels take one or two tensors ("sides") per launch:
+// blocks [0, split) work on side 0 and blocks [split, grid) on side 1, each
+// side with its share of the grid. split == grid: one tensor.
+struct StatsSide {
+    const void *x;
+    float *stats;     // [T, P]
+    int32_t D, nv, K; // row width; vectors per shard; lane groups per shard
+};
+struct StatsArgs {
+    StatsSide side[2];
+    int64_t T;
+    int32_t P;
+    int32_t split;
+};
+cudaError_t launch_stats(int dtype, int vmax, const StatsArgs &a, int block, int64_t grid,
                          cudaStream_t s);
 // stats of token t: nb blocks of Pb sums, block b at stats + b * sg + t * Pb;
-// Df the divisor (full width). block must be a multiple of
-// apply_threads_per_row(D, dtype).
+// Df the divisor (full width); tpr threads per row (apply_threads_per_row).
+struct ApplySide {
+    const void *x;
+    const float *g;
+    const float *stats;
+    void *y;
+    int32_t D, tpr;
+    float Df;
+};
+struct ApplyArgs {
+    ApplySide side[2];
+    int64_t T, sg;
+    int32_t Pb, nb;
+    float eps;
+    int32_t split;
+};
 int apply_threads_per_row(int32_t D, int dtype);
-cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
-                         int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg, float Df,
-                         float eps, int block, int64_t grid, cudaStream_t s);
+// multi: the several-rows-per-block instance (needed unless every side's tpr
+// equals block).
+cudaError_t launch_apply(int dtype, bool multi, const ApplyArgs &a, int block, int64_t grid,
+                         cudaStream_t s);
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // tb = tokens per ring stage (1 or 2); mode: 0 any shape, 1 every lane holds

@@ -15,23 +15,40 @@
 //   shard sums of its row in order and forms the factor, then streams its
 //   vectors of the row through (x * gamma) * r. The row's first loads are
 //   issued before the factor so the statistic's latency overlaps them.
+//
+// Both kernels take one or two tensors ("sides") per launch: blocks below
+// split take side 0, the others side 1, each block with its own side's
+// pointers and widths and its share of the grid as its stride. Q and K of
+// one layer (e.g. one rank's slices) then cost one launch per step.
 #include "qknorm_device.cuh"
 #include "qknorm_internal.h"
 
 namespace qkn {
 
-template <class Tag, int VMAX, int R>
-__global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int64_t T, int32_t D,
-                                               int32_t P, int32_t nv, int32_t K) {
+// TWO: the launch may carry two sides (one-side launches compile without
+// the selection, which costs registers).
+template <class Tag, int VMAX, int R, bool TWO>
+__global__ void __launch_bounds__(256) stats_k(const StatsArgs a) {
     constexpr int VEC = Tag::kVec;
     pdl_wait();
     pdl_trigger();
+    const int z = TWO && (int)blockIdx.x >= a.split ? 1 : 0;
+    const int bz = z ? (int)blockIdx.x - a.split : (int)blockIdx.x;   // block within its side
+    const int gz = z ? (int)gridDim.x - a.split : a.split;            // the side's blocks
+    // Each field selected on its own (indexing the parameter array by z
+    // would copy it to the stack).
+    const void *x = z ? a.side[1].x : a.side[0].x;
+    float *stats = z ? a.side[1].stats : a.side[0].stats;
+    const int64_t T = a.T;
+    const int32_t P = a.P;
+    const int32_t nv = z ? a.side[1].nv : a.side[0].nv;
+    const int32_t K = z ? a.side[1].K : a.side[0].K;
     const int lane = threadIdx.x & 31;
-    const int64_t rowvec = D / VEC;
+    const int64_t rowvec = (z ? a.side[1].D : a.side[0].D) / VEC;
     const int64_t ntask = T * (int64_t)P;
-    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t nwarps = (int64_t)gz * (blockDim.x >> 5);
     const int stride = kLanes * K;
-    const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t w0 = (int64_t)bz * (blockDim.x >> 5) + (threadIdx.x >> 5);
     // Task = t * P + p. The (t, p) of a warp's tasks advance by a fixed step
     // (nwarps tasks), so they are carried along instead of divided out.
     const int64_t dt = nwarps / P;
@@ -101,21 +118,25 @@ __global__ void __launch_bounds__(256) stats_k(const void *x, float *stats, int6
 // over the block. MULTI = true: tpr threads per row and blockDim.x / tpr rows
 // per block, so narrow rows (e.g. one rank's slice) still give every thread
 // UNR vectors; the row index then varies within the block, which costs
-// registers (57 against 34), so wide rows keep the uniform form.
+// registers (60 against 34), so wide rows keep the uniform form.
+//
+// apply_rows: the rows of one tensor that block bz of the tensor's gz blocks
+// takes. apply_k runs it for a one-tensor launch, apply2_k for a launch over
+// two tensors.
 template <class Tag, bool MULTI>
-__global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, const float *stats,
-                                               void *y, int64_t T, int32_t D, int32_t Pb, int32_t nb,
-                                               int64_t sg, float Df, float eps, int32_t tpr) {
+__device__ __forceinline__ void apply_rows(const void *x, const float *g, const float *stats, void *y,
+                                           int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg,
+                                           float Df, float eps, int32_t tpr, int64_t bz, int64_t gz) {
     constexpr int VEC = Tag::kVec;
     constexpr int UNR = 4;
-    pdl_wait();
-    pdl_trigger();
     const int64_t rowvec = D / VEC;
+    // tpr threads per row; rows beyond rpb * tpr threads of a block idle.
     const int nthr = MULTI ? tpr : (int)blockDim.x;
     const int rpb = MULTI ? (int)blockDim.x / tpr : 1;
     const int lt = MULTI ? (int)threadIdx.x % tpr : (int)threadIdx.x;
-    const int64_t t0 = MULTI ? (int64_t)blockIdx.x * rpb + threadIdx.x / tpr : (int64_t)blockIdx.x;
-    for (int64_t t = t0; t < T; t += (int64_t)gridDim.x * rpb) {
+    const int64_t t0 = MULTI ? bz * rpb + threadIdx.x / tpr : bz;
+    if (MULTI && (int)threadIdx.x >= rpb * tpr) return;
+    for (int64_t t = t0; t < T; t += gz * rpb) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec;
         uint4 *dst = reinterpret_cast<uint4 *>(y) + t * rowvec;
         float r = 0.f;
@@ -145,58 +166,83 @@ __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, co
     }
 }
 
+// One tensor per launch.
+template <class Tag, bool MULTI>
+__global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, const float *stats,
+                                               void *y, int64_t T, int32_t D, int32_t Pb, int32_t nb,
+                                               int64_t sg, float Df, float eps, int32_t tpr) {
+    pdl_wait();
+    pdl_trigger();
+    apply_rows<Tag, MULTI>(x, g, stats, y, T, D, Pb, nb, sg, Df, eps, tpr, blockIdx.x, gridDim.x);
+}
+
+// Two tensors per launch: blocks below a.split take side 0, the rest side 1.
+template <class Tag, bool MULTI>
+__global__ void __launch_bounds__(256) apply2_k(const ApplyArgs a) {
+    pdl_wait();
+    pdl_trigger();
+    const int z = (int)blockIdx.x >= a.split ? 1 : 0;
+    // Each field selected on its own (indexing the parameter array by z
+    // would copy it to the stack).
+    apply_rows<Tag, MULTI>(z ? a.side[1].x : a.side[0].x, z ? a.side[1].g : a.side[0].g,
+                           z ? a.side[1].stats : a.side[0].stats, z ? a.side[1].y : a.side[0].y, a.T,
+                           z ? a.side[1].D : a.side[0].D, a.Pb, a.nb, a.sg,
+                           z ? a.side[1].Df : a.side[0].Df, a.eps, z ? a.side[1].tpr : a.side[0].tpr,
+                           z ? (int64_t)blockIdx.x - a.split : (int64_t)blockIdx.x,
+                           z ? (int64_t)gridDim.x - a.split : (int64_t)a.split);
+}
+
 // ---------------------------------------------------------------- instance tables
 
 // Tasks per warp turn: as many as keep R x VMAX <= 8 vectors per lane.
 constexpr int stats_r(int vmax) { return vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1); }
 
 template <class Tag, int V>
-const void *stats_fn() {
-    return reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V)>);
+const void *stats_fn(bool two) {
+    return two ? reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), true>)
+               : reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), false>);
 }
 
 template <class Tag>
-const void *stats_table(int vmax) {
+const void *stats_table(int vmax, bool two) {
     switch (vmax) {
-    case 1: return stats_fn<Tag, 1>();
-    case 2: return stats_fn<Tag, 2>();
-    case 3: return stats_fn<Tag, 3>();
-    case 4: return stats_fn<Tag, 4>();
-    case 5: return stats_fn<Tag, 5>();
-    case 6: return stats_fn<Tag, 6>();
-    case 7: return stats_fn<Tag, 7>();
-    case 8: return stats_fn<Tag, 8>();
+    case 1: return stats_fn<Tag, 1>(two);
+    case 2: return stats_fn<Tag, 2>(two);
+    case 3: return stats_fn<Tag, 3>(two);
+    case 4: return stats_fn<Tag, 4>(two);
+    case 5: return stats_fn<Tag, 5>(two);
+    case 6: return stats_fn<Tag, 6>(two);
+    case 7: return stats_fn<Tag, 7>(two);
+    case 8: return stats_fn<Tag, 8>(two);
     default: return nullptr;
     }
 }
 
-const void *stats_kernel(int dtype, int vmax) {
-    if (dtype == 0) return stats_table<F32Tag>(vmax);
-    if (dtype == 1) return stats_table<BF16Tag>(vmax);
-    if (dtype == 2) return stats_table<E4M3Tag>(vmax);
+const void *stats_kernel(int dtype, int vmax, bool two) {
+    if (dtype == 0) return stats_table<F32Tag>(vmax, two);
+    if (dtype == 1) return stats_table<BF16Tag>(vmax, two);
+    if (dtype == 2) return stats_table<E4M3Tag>(vmax, two);
     return nullptr;
 }
 
-template <class Tag>
-const void *apply_fn(bool multi) {
-    return multi ? reinterpret_cast<const void *>(&apply_k<Tag, true>)
-                 : reinterpret_cast<const void *>(&apply_k<Tag, false>);
+template <class Tag, bool MULTI>
+const void *apply_fn(bool two) {
+    return two ? reinterpret_cast<const void *>(&apply2_k<Tag, MULTI>)
+               : reinterpret_cast<const void *>(&apply_k<Tag, MULTI>);
 }
 
-const void *apply_kernel(int dtype, bool multi) {
-    if (dtype == 0) return apply_fn<F32Tag>(multi);
-    if (dtype == 1) return apply_fn<BF16Tag>(multi);
-    if (dtype == 2) return apply_fn<E4M3Tag>(multi);
+const void *apply_kernel(int dtype, bool multi, bool two) {
+    if (dtype == 0) return multi ? apply_fn<F32Tag, true>(two) : apply_fn<F32Tag, false>(two);
+    if (dtype == 1) return multi ? apply_fn<BF16Tag, true>(two) : apply_fn<BF16Tag, false>(two);
+    if (dtype == 2) return multi ? apply_fn<E4M3Tag, true>(two) : apply_fn<E4M3Tag, false>(two);
     return nullptr;
 }
 
-cudaError_t launch_stats(int dtype, int vmax, const void *x, float *stats, int64_t T,
-                         const TensorShape &sh, int32_t P, int block, int64_t grid,
+cudaError_t launch_stats(int dtype, int vmax, const StatsArgs &a, int block, int64_t grid,
                          cudaStream_t s) {
-    const void *fn = stats_kernel(dtype, vmax);
-    if (!fn) return cudaErrorInvalidValue;
-    int32_t D = sh.D, nv = sh.nv, K = sh.K;
-    void *args[] = {const_cast<void **>(&x), &stats, &T, &D, &P, &nv, &K};
+    const void *fn = stats_kernel(dtype, vmax, a.split < grid);
+    if (!fn || a.split < 1 || a.split > grid) return cudaErrorInvalidValue;
+    void *args[] = {const_cast<StatsArgs *>(&a)};
     return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 
@@ -215,14 +261,24 @@ int apply_threads_per_row(int32_t D, int dtype) {
     return (int)(t < 256 ? t : 256);
 }
 
-cudaError_t launch_apply(int dtype, const void *x, const float *g, const float *stats, void *y,
-                         int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg, float Df,
-                         float eps, int block, int64_t grid, cudaStream_t s) {
-    int32_t tpr = apply_threads_per_row(D, dtype);
-    const void *fn = apply_kernel(dtype, block != tpr);
-    if (!fn || block % tpr != 0) return cudaErrorInvalidValue;
-    void *args[] = {const_cast<void **>(&x), const_cast<float **>(&g),
-                    const_cast<float **>(&stats), &y, &T, &D, &Pb, &nb, &sg, &Df, &eps, &tpr};
+cudaError_t launch_apply(int dtype, bool multi, const ApplyArgs &a, int block, int64_t grid,
+                         cudaStream_t s) {
+    const void *fn = apply_kernel(dtype, multi, a.split < grid);
+    if (!fn || a.split < 1 || a.split > grid) return cudaErrorInvalidValue;
+    for (int z = 0; z < (a.split < grid ? 2 : 1); ++z) {
+        const int tpr = a.side[z].tpr;
+        if (tpr < 1 || tpr > block || (!multi && tpr != block)) return cudaErrorInvalidValue;
+    }
+    if (a.split < grid) {
+        void *args[] = {const_cast<ApplyArgs *>(&a)};
+        return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
+    }
+    const ApplySide &d = a.side[0];
+    int64_t T = a.T, sg = a.sg;
+    int32_t D = d.D, Pb = a.Pb, nb = a.nb, tpr = d.tpr;
+    float Df = d.Df, eps = a.eps;
+    void *args[] = {const_cast<void **>(&d.x), const_cast<float **>(&d.g), const_cast<float **>(&d.stats),
+                    const_cast<void **>(&d.y), &T, &D, &Pb, &nb, &sg, &Df, &eps, &tpr};
     return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
 }
 

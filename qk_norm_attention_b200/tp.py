@@ -5,13 +5,14 @@ form. The hidden dimension of Q and K is split across the ranks of a group;
 rank g holds columns [g * D_local, (g + 1) * D_local) of every row, i.e.
 P_local of the P = ranks * P_local shards. Each rank
 
-  Phase A  forms its shard sums of squares (qknorm_partial_sumsq, [T, P_local]),
+  Phase A  forms its shard sums of squares (qknorm_partial_sumsq_qk: Q's and
+           K's [T, P_local] in one launch),
   exchange gathers every rank's sums (one all-gather over the group, Q and K
            together: [ranks, 2, T, P_local]),
   Phase B  adds the P sums of each row in order of the global shard index and
            forms r = rsqrt(S / (ranks * D_local) + eps),
   Phase C  writes (x * gamma) * r for its own slice
-           (B and C: qknorm_apply_tp).
+           (B and C: qknorm_apply_tp_qk, Q and K in one launch).
 
 The result on rank g equals columns g of qknorm_fwd on the whole rows, bit for
 bit: the same shard sums, added in the same order. The exchange is the
@@ -25,7 +26,7 @@ from typing import Optional, Tuple
 import torch
 import torch.distributed as dist
 
-from . import qknorm_apply_tp, qknorm_partial_sumsq
+from . import qknorm_apply_tp_qk, qknorm_partial_sumsq_qk
 
 
 def gathered_stats_shape(ranks: int, T: int, P_local: int) -> Tuple[int, int, int, int]:
@@ -46,15 +47,12 @@ def qknorm_tp_fwd(q_local: torch.Tensor, k_local: torch.Tensor, gamma_q_local: t
     T = q_local.shape[0]
     if k_local.shape[0] != T:
         raise ValueError("q_local and k_local must have the same number of rows")
-    local = torch.empty((2, T, P_local), dtype=torch.float32, device=q_local.device)
-    qknorm_partial_sumsq(q_local, P_local, stats=local[0])
-    qknorm_partial_sumsq(k_local, P_local, stats=local[1])
+    local = qknorm_partial_sumsq_qk(q_local, k_local, P_local)
     if gathered is None:
         gathered = torch.empty(gathered_stats_shape(ranks, T, P_local), dtype=torch.float32,
                                device=q_local.device)
     elif tuple(gathered.shape) != gathered_stats_shape(ranks, T, P_local):
         raise ValueError("gathered must be [ranks, 2, T, P_local]")
     dist.all_gather_into_tensor(gathered.view(-1), local.view(-1), group=group)
-    yq = qknorm_apply_tp(q_local, gamma_q_local, gathered[:, 0], eps, out=out_q)
-    yk = qknorm_apply_tp(k_local, gamma_k_local, gathered[:, 1], eps, out=out_k)
-    return yq, yk
+    return qknorm_apply_tp_qk(q_local, k_local, gamma_q_local, gamma_k_local, gathered, eps,
+                              out_q=out_q, out_k=out_k)

@@ -101,7 +101,7 @@ def test_split_rejects(qk):
     assert L.qknorm_partial_sumsq(A, B, 4, 256, 4, 5, None) == 3
     assert L.qknorm_partial_sumsq(A, B, 4, 256, 64, 1, None) == 3      # 4-wide bf16 shards
     assert L.qknorm_partial_sumsq(A + 2, B, 4, 256, 4, 1, None) == 2
-    assert L.qknorm_partial_sumsq(A, B + 4, 4, 256, 4, 1, None) == 2
+    assert L.qknorm_partial_sumsq(A, B + 2, 4, 256, 4, 1, None) == 2     # stats need 4-byte alignment
     assert L.qknorm_partial_sumsq(A, A + 16, 4, 256, 4, 1, None) == 1  # stats inside x
     assert L.qknorm_partial_sumsq(0, B, 4, 256, 4, 1, None) == 1
     assert L.qknorm_partial_sumsq(0, 0, 0, 256, 4, 1, None) == 0
@@ -153,6 +153,38 @@ def test_apply_tp_rejects(qk):
     assert L.qknorm_apply_tp(A, B, C, 0, Dd, 4, 256, 3, 2, 1e-6, 1, None) == 1    # D_local % P_local
     assert L.qknorm_apply_tp(A, B, C, 0, C + 16, 4, 256, 4, 2, 1e-6, 1, None) == 1  # out on stats
     assert L.qknorm_apply_tp(0, 0, 0, 0, 0, 0, 256, 4, 2, 1e-6, 1, None) == 0     # T = 0
+
+
+@needs_cpu
+def test_two_tensor_calls_reject(qk):
+    """qknorm_partial_sumsq_qk and qknorm_apply_tp_qk check each tensor as the
+    one-tensor calls do, and also reject overlaps across the two tensors."""
+    L = qk.lib
+    # q, k, stats_q, stats_k, T, Dq, Dk, P, dtype, stream  (q 2 KiB at A, k 512 B at A + 4096)
+    sbase = [A, A + 4096, C, C + 4096, 4, 256, 64, 4, 1, None]
+    scall = lambda **kw: L.qknorm_partial_sumsq_qk(*[kw.get(str(i), v) for i, v in enumerate(sbase)])
+    assert scall(**{"4": 0}) == 0                   # T = 0
+    assert scall(**{"3": C + 32}) == 1              # stats_k over stats_q
+    assert scall(**{"3": A}) == 1                   # stats_k over q
+    assert scall(**{"2": A + 4096}) == 1            # stats_q over k
+    assert scall(**{"6": 66}) == 1                  # Dk % P
+    assert scall(**{"6": 60}) == 3                  # shard width not whole 16-byte vectors
+    assert scall(**{"1": A + 4104}) == 2            # k misaligned
+    assert scall(**{"8": 7}) == 3                   # no such dtype
+    # q, k, gq, gk, stats_q, stats_k, stride, out_q, out_k, T, Dq, Dk, P_local, ranks, eps, dtype, stream
+    abase = [A, A + 4096, B, B + 4096, C, C + 16, 32, Dd, Dd + 4096, 4, 256, 64, 4, 2, 1e-6, 1, None]
+    acall = lambda **kw: L.qknorm_apply_tp_qk(*[kw.get(str(i), v) for i, v in enumerate(abase)])
+    assert acall(**{"9": 0}) == 0                   # T = 0
+    assert acall(**{"13": 0}) == 1                  # ranks < 1
+    assert acall(**{"6": -1}) == 1                  # negative stride
+    assert acall(**{"6": 15}) == 1                  # blocks overlap
+    assert acall(**{"8": Dd + 64}) == 1             # out_k over out_q
+    assert acall(**{"7": A + 4096}) == 1            # out_q over k
+    assert acall(**{"8": B}) == 1                   # out_k over gamma_q
+    assert acall(**{"7": C + 16}) == 1              # out_q over stats_k
+    assert acall(**{"8": A}) == 1                   # out_k over q
+    assert acall(**{"14": -1.0}) == 1               # eps < 0
+    assert acall(**{"8": Dd + 4100}) == 2           # out_k misaligned
 
 
 @needs_cpu

@@ -162,6 +162,8 @@ GUARD_CASES = [
     ("generic", 2 * 148 + 41, 5120, 1024, 8, "bf16"),
     ("bulk", 2 * 148 + 41, 5120, 5120, 4, "e4m3"),     # the FP8 half-slot mode
     ("pair", 2 * 148 + 41, 5120, 1024, 8, "e4m3"),
+    ("pair", 2 * 148 + 41, 5120, 4096, 8, "bf16"),     # K shards in pairs, ragged Q lanes
+    (None, 2 * 148 + 41, 4096, 4096, 8, "e4m3"),       # FP8 K pairs, one vector per lane
 ]
 
 

@@ -42,14 +42,24 @@ def _stand_in_apply(x, gamma, stats, eps, out=None):
     return y if out is None else out.copy_(y)
 
 
+def _stand_in_stats_qk(q, k, P, stats=None):
+    out = torch.stack((_stand_in_stats(q, P), _stand_in_stats(k, P)))
+    return out if stats is None else stats.copy_(out)
+
+
+def _stand_in_apply_qk(q, k, gq, gk, stats, eps, out_q=None, out_k=None):
+    return (_stand_in_apply(q, gq, stats[:, 0], eps, out_q),
+            _stand_in_apply(k, gk, stats[:, 1], eps, out_k))
+
+
 def _rank_main(rank, world, port, T, Dq, Dk, P, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
                       RANK=str(rank), LOCAL_RANK=str(rank))
     import torch.distributed as dist
     dist.init_process_group("gloo", rank=rank, world_size=world)
     import qk_norm_attention_b200.tp as tp
-    tp.qknorm_partial_sumsq = _stand_in_stats
-    tp.qknorm_apply_tp = _stand_in_apply
+    tp.qknorm_partial_sumsq_qk = _stand_in_stats_qk
+    tp.qknorm_apply_tp_qk = _stand_in_apply_qk
     rng = np.random.default_rng(5)                    # every rank draws the same full rows
     q = torch.from_numpy(rng.standard_normal((T, Dq)).astype(np.float32))
     k = torch.from_numpy(rng.standard_normal((T, Dk)).astype(np.float32))
