@@ -733,11 +733,14 @@ def run_reference(args, dist):
     """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
     if dist.rank != 0:
         return 0
-    wl = W.WORKLOADS[HEADLINE]
-    T = wl.Ts[0]
+    # The native arm's workload, token count and path (the split path computes
+    # what the fused one does; headwise has its own oracle function).
+    wl = W.WORKLOADS[args.workload]
+    T = args.tokens if args.tokens > 0 else max(wl.Ts)
+    hw = args.path == "headwise"
     cores = host_cores()
     # Calibrate: rows per step so that warmup + steps take about two minutes.
-    p, el = oracle_rows_rate(wl, 64, cores, 0.5)
+    p, el = oracle_rows_rate(wl, 64, cores, 0.5, hw)
     per_row = el / (p * 64)
     budget = 120.0 / max(1, args.steps + args.warmup)
     n = int(min(T, max(16, budget / per_row)))
@@ -747,11 +750,19 @@ def run_reference(args, dist):
     q, k = W.gen_rows(wl, "q", rows), W.gen_rows(wl, "k", rows)
     gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
     eps = float(np.float32(wl.eps))
+
+    def step():
+        if hw:
+            orc.headwise(q, gq[:HEAD_DIM], HEAD_DIM, eps, wl.dtype, nthreads=cores)
+            orc.headwise(k, gk[:HEAD_DIM], HEAD_DIM, eps, wl.dtype, nthreads=cores)
+        else:
+            orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=cores)
+
     for _ in range(args.warmup):
-        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=cores)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.qknorm(q, k, gq, gk, wl.P, eps, wl.dtype, nthreads=cores)
+        step()
     el = time.perf_counter() - t0
     nbytes = W.fused_bytes(n, wl.Dq, wl.Dk, wl.elem_bytes)
     value = args.steps * nbytes / el / 1e9
@@ -760,9 +771,10 @@ def run_reference(args, dist):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1000 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, T, args.gpus),
+        "config": dict(config_of(wl, T, args.gpus), path=args.path),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n} of the {T} tokens (Q and K rows) per step, float64 C "
+                         "sample": f"{n} of the {T} tokens (Q and K rows{', headwise' if hw else ''}) "
+                                   f"per step, float64 C "
                                    f"oracle, OpenMP over tokens on {cores} threads ({cpu_model()})"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
