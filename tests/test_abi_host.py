@@ -448,3 +448,21 @@ def test_headwise_checks(qk):
     assert call(eps=-1.0) == 1 and call(dtype=3) == 3
     assert call(oq=B) == 1                              # output on the other input
     assert call(T=0, q=0, k=0, oq=0, ok=0) == 0
+
+
+def test_two_tensor_wrappers_check_metadata(qk):
+    """The Python wrappers of the two-tensor calls reject mismatched shapes and
+    host tensors before calling into the library."""
+    import torch
+    q, k = torch.zeros(4, 256, dtype=torch.bfloat16), torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        qk.qknorm_partial_sumsq_qk(q, torch.zeros(5, 64, dtype=torch.bfloat16), 4)   # row counts differ
+    with pytest.raises(ValueError):
+        qk.qknorm_partial_sumsq_qk(q, k, 4)                                         # host tensors
+    g = torch.ones(256)
+    with pytest.raises(ValueError):
+        qk.qknorm_apply_tp_qk(q, k, g, g[:64], torch.zeros(2, 4, 4), 1e-6)          # stats not 4-D
+    with pytest.raises(ValueError):
+        qk.qknorm_apply_tp_qk(q, k, g, g[:64], torch.zeros(2, 3, 4, 4), 1e-6)       # not [ranks, 2, ...]
+    with pytest.raises(ValueError):
+        qk.qknorm_apply_tp_qk(q, k, g, g[:64], torch.zeros(2, 2, 4, 4), 1e-6)       # host tensors
