@@ -185,3 +185,36 @@ def test_fp8_saturation(qk, orc):
             inside = np.abs(y_or) < 448
             diff = np.abs(y[inside] - y_or[inside])
             assert (diff <= 2.0 ** -3 * np.abs(y_or[inside]) + 2.0 ** -9).all()
+
+
+@pytest.mark.parametrize("name", ["prefill13b_e4m3", "split_large_e4m3"])
+def test_fp8_bench_workloads_full_size(qk, orc, name):
+    """The FP8 configurations the benchmark times, at full size and in the
+    selector's launch configuration (inputs drawn on the device with the
+    workload's recipe): fused == split on every row, and the oracle on
+    sampled rows (both ends, a regular stride, random rows)."""
+    wl = W.WORKLOADS[name]
+    T = wl.Ts[0]
+    dev = torch.device("cuda")
+    q = W.gen_device_workload(wl, "q", T, dev)
+    k = W.gen_device_workload(wl, "k", T, dev)
+    gq = torch.from_numpy(W.gen_gamma(wl, "q")).to(dev)
+    gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(dev)
+    qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    oq, ok = qk.qknorm_fwd(q, k, gq, gk, wl.P, wl.eps)
+    aq = qk.qknorm_apply(q, gq, qk.qknorm_partial_sumsq(q, wl.P), wl.eps)
+    ak = qk.qknorm_apply(k, gk, qk.qknorm_partial_sumsq(k, wl.P), wl.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(aq), bits(oq)) and torch.equal(bits(ak), bits(ok))
+    rng = np.random.default_rng(98)
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(T - 64, T), np.arange(0, T, 997),
+                                     rng.choice(T, 1500, replace=False)]))
+    rt = torch.from_numpy(rows).to(dev)
+    eps = float(np.float32(wl.eps))
+    for tag, x, g, y in (("q", q, gq, oq), ("k", k, gk, ok)):
+        xs = x.view(torch.uint8).index_select(0, rt).cpu().numpy()     # E4M3 codes
+        y_or, _ = orc.rmsnorm(xs, g.cpu().numpy(), wl.P, eps, "e4m3", nthreads=8)
+        check_outputs(y.view(torch.uint8).index_select(0, rt).cpu().numpy(), y_or, "e4m3",
+                      f"{name} {tag}")
+    del q, k, oq, ok, aq, ak
+    torch.cuda.empty_cache()
