@@ -41,9 +41,10 @@ KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_ge
 
 # dram bytes per launch of the headline kernel from one ncu capture, and the
 # hash of the kernel sources it was taken with (None until captured).
-# From profiles/fused_bulk_prefill13b_full.md: dram__bytes_read.sum 167,837,952
-# + dram__bytes_write.sum 111,811,840 for one launch (cold, serialised capture;
-# ~56 MB of the writes were still in L2 when the kernel ended).
+# Taken from an ncu --set full capture of one launch of the 13B-shaped
+# prefill (cold caches, serialised): dram__bytes_read.sum 167,837,952 +
+# dram__bytes_write.sum 111,811,840 (about 56 MB of the writes were still in
+# L2 when the kernel ended).
 NCU_TRAFFIC = {"src_sha": "aa4e7d5756db0513", "bytes_per_launch": 279488768,
                "plan": {"variant": 3, "block": 256, "grid": 296, "vmax": 5, "stages": 2,
                         "tokens_per_stage": 1, "gamma_regs": 0, "full_lanes": 1}}

@@ -322,9 +322,11 @@ QKNORM_API int qknorm_inv_rms(const void *x, float *inv_rms, int64_t T, int32_t 
  * returns QKNORM_ERR_UNSUPPORTED without launching anything. The call itself
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  * The first call on a device looks up the buffer's device address (with that
- * device current); make that first call before any stream capture. All calls
- * share the buffer: calls that overlap on the GPU race. Nothing in it needs
- * clearing between calls.
+ * device current); make that first call before any stream capture. The first
+ * call after the device's context is destroyed and re-created (e.g. by
+ * cudaDeviceReset) looks the address up again, since the buffer may then sit
+ * elsewhere. All calls share the buffer: calls that overlap on the GPU race.
+ * Nothing in it needs clearing between calls.
  */
 QKNORM_API int qknorm_split_noalloc(const void *x, const float *gamma, void *out, int64_t T,
                                     int32_t D, int32_t P, float eps, int32_t dtype, void *stream);

@@ -512,10 +512,17 @@ def qknorm_split_noalloc(x: torch.Tensor, gamma: torch.Tensor, P: int, eps: floa
     if x.dim() != 2:
         raise ValueError("x must be [T, D]")
     T, D = x.shape
+    code = _dtype_code(x)
+    if gamma.dtype != torch.float32:
+        raise TypeError("gamma must be float32")
+    if gamma.numel() != D:
+        raise ValueError(f"gamma must have D = {D} elements")
     out = torch.empty_like(x) if out is None else out
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must have x's shape and dtype")
     for name, t in (("x", x), ("gamma", gamma), ("out", out)):
         _need_cuda_contig(name, t)
     st = lib.qknorm_split_noalloc(x.data_ptr(), gamma.data_ptr(), out.data_ptr(), T, D, int(P),
-                                  float(eps), _dtype_code(x), _stream_handle(x.device, stream))
+                                  float(eps), code, _stream_handle(x.device, stream))
     _check("qknorm_split_noalloc", st)
     return out

@@ -13,6 +13,7 @@
 // contents. Nothing needs clearing: the statistics pass writes every entry
 // the apply pass reads. Calls that overlap on the GPU (on different streams,
 // say) use the same buffer and race.
+#include <cuda.h>  // CUcontext / CUresult types only; the driver is reached through the runtime
 #include <mutex>
 
 #include "../../include/qknorm.h"
@@ -24,24 +25,68 @@ static __device__ __align__(256) float g_noalloc_stats[kNoallocMaxStats];
 
 namespace {
 
+// The buffer's device address is looked up once per (device, CUDA context):
+// on a device's first call, and again on the first call after the device's
+// context was destroyed and re-created (cudaDeviceReset), when the module is
+// loaded anew and the buffer may sit at another address. Contexts are told
+// apart by the driver's process-unique context ID.
+struct Setup {
+    int dev;
+    unsigned long long ctx_id;
+    float *ptr;
+};
 constexpr int kMaxDevices = 64;
-float *g_stats_ptr[kMaxDevices];
+Setup g_setup[kMaxDevices];
 std::mutex g_setup_mu;
 
-// The device address of g_noalloc_stats on the current device (its host-side
-// name is only a stand-in). Looked up once per device, on that device's first
-// call, with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+bool g_entry_points_resolved = false;
+
+// The ID of the context current on this thread; 0 if there is none yet (the
+// runtime creates the primary context on its first call that needs one) or
+// the driver lacks the query. Called with g_setup_mu held.
+unsigned long long current_ctx_id() {
+    if (!g_entry_points_resolved) {
+        g_entry_points_resolved = true;
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *f1 = nullptr, *f2 = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1) ==
+                cudaSuccess && q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) ==
+                cudaSuccess && q2 == cudaDriverEntryPointSuccess) {
+            g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+            g_ctx_id = reinterpret_cast<CtxGetIdFn>(f2);
+        }
+        cudaGetLastError();  // a failed query must not leak into the caller's error state
+    }
+    if (!g_ctx_current || !g_ctx_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// The device address of g_noalloc_stats in the current device's context (its
+// host-side name is only a stand-in).
 int stats_address(float **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QKNORM_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (g_stats_ptr[dev] == nullptr) {
+    Setup &s = g_setup[dev];
+    const unsigned long long id = current_ctx_id();
+    if (s.ptr == nullptr || id == 0 || id != s.ctx_id) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_stats) != cudaSuccess || p == nullptr)
             return QKNORM_ERR_CUDA;
-        g_stats_ptr[dev] = static_cast<float *>(p);
+        s.dev = dev;
+        s.ptr = static_cast<float *>(p);
+        s.ctx_id = current_ctx_id();  // the lookup made the primary context current if it was not
     }
-    *out = g_stats_ptr[dev];
+    *out = s.ptr;
     return QKNORM_OK;
 }
 

@@ -344,6 +344,39 @@ def pin_headwise(orc):
     assert np.array_equal(y1[:, keep], y2[:, keep])
 
 
+def pin_qknorm(orc):
+    """Layerwise QK-Norm of a layer: one factor over the whole Q row with
+    gamma_q and, separately, one over the whole K row with gamma_k (the
+    review's "Prerequisites", layerwise QK-Norm; Eq. (1) once per tensor).
+    Each output, and each factor, is checked against exact sums and a 50-digit
+    root of its OWN tensor with its OWN weight: the tiny workload (Dq == Dk,
+    gamma_q != gamma_k) and a bf16 GQA-like case with Dk < Dq. A swapped
+    weight, swapped outputs or K normalised with Q's statistic fails here
+    even when the two widths are equal."""
+    wl, q, k, gq, gk = tiny_inputs(4)
+    assert not np.array_equal(gq, gk)
+    cases = [(q, k, gq, gk, wl.P, "f32")]
+    wq = W.custom("pinqk", 3, 48, 16, 2, dtype="bf16", seed=19)
+    qb, kb = W.gen_rows(wq, "q", range(3)), W.gen_rows(wq, "k", range(3))
+    gqb = W.to_storage(np.linspace(0.5, 1.5, 48), "f32")
+    gkb = W.to_storage(np.linspace(-2.0, -0.25, 16), "f32")
+    cases.append((qb, kb, gqb, gkb, 2, "bf16"))
+    # Equal widths, the same rows in Q and K, different weights: only the
+    # weights tell the two outputs apart.
+    cases.append((q, q.copy(), gq, gk, wl.P, "f32"))
+    for xq, xk, g_q, g_k, P, dtype in cases:
+        for eps in (1e-6, 0.3):
+            yq, yk, rq, rk = orc.qknorm(xq, xk, g_q, g_k, P, eps, dtype)
+            assert yq.shape == xq.shape and yk.shape == xk.shape
+            for x, g, y, r, name in ((xq, g_q, yq, rq, "q"), (xk, g_k, yk, rk, "k")):
+                x64 = widen(x, dtype)
+                tol = (x.shape[1] + 8) * U53
+                for t in range(x.shape[0]):
+                    ye, re = exact_y(x64[t], g, eps)
+                    assert rel_err([r[t]], [re]) <= tol, f"qknorm r_{name}[{t}] ({dtype})"
+                    assert rel_err(y[t], ye) <= tol, f"qknorm y_{name}[{t}] ({dtype}, eps={eps})"
+
+
 def e4m3_inputs(T, D, seed, sigma=1.0):
     wl = W.custom("pin8", T, D, D, 1, dtype="e4m3", seed=seed, x_sigma=sigma)
     return W.gen_rows(wl, "q", range(T)), W.gen_gamma(wl, "q")
@@ -395,5 +428,6 @@ ALL_PINS = [
     pin_row_independence,
     pin_xgamma,
     pin_headwise,
+    pin_qknorm,
     pin_e4m3,
 ]

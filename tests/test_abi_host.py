@@ -466,3 +466,24 @@ def test_two_tensor_wrappers_check_metadata(qk):
         qk.qknorm_apply_tp_qk(q, k, g, g[:64], torch.zeros(2, 3, 4, 4), 1e-6)       # not [ranks, 2, ...]
     with pytest.raises(ValueError):
         qk.qknorm_apply_tp_qk(q, k, g, g[:64], torch.zeros(2, 2, 4, 4), 1e-6)       # host tensors
+
+
+def test_noalloc_wrapper_checks_metadata(qk):
+    """The Python wrapper of qknorm_split_noalloc rejects a gamma of the wrong
+    dtype or length and an out of the wrong shape or dtype, and host tensors,
+    before calling into the library."""
+    import torch
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    g = torch.ones(256)
+    with pytest.raises(TypeError):
+        qk.qknorm_split_noalloc(x, g.to(torch.bfloat16), 4, 1e-6)              # bf16 gamma
+    with pytest.raises(ValueError):
+        qk.qknorm_split_noalloc(x, g[:128], 4, 1e-6)                           # short gamma
+    with pytest.raises(ValueError):
+        qk.qknorm_split_noalloc(x, g, 4, 1e-6, out=torch.zeros(2, 256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        qk.qknorm_split_noalloc(x, g, 4, 1e-6, out=torch.zeros(4, 256))        # fp32 out
+    with pytest.raises(TypeError):
+        qk.qknorm_split_noalloc(x.to(torch.float16), g, 4, 1e-6)               # unsupported dtype
+    with pytest.raises(ValueError):
+        qk.qknorm_split_noalloc(x, g, 4, 1e-6)                                 # host tensors

@@ -6,6 +6,7 @@ or stride), compiled to its own library in a temporary directory. The test
 passes when some pin of ``oracle_pins`` rejects the mutant, which shows that
 the pins would catch that mistake in the real oracle.
 """
+import importlib.util
 import os
 
 import pytest
@@ -71,6 +72,51 @@ def _build_mutant(tmpdir, name, edits):
 def test_mutant_is_caught(tmp_path, name):
     lib = _build_mutant(str(tmp_path), name, MUTANTS[name])
     orc = oracle.Oracle(lib)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin rejects the planted mistake {name}"
+
+
+# Mistakes in the Python front end's composition of Q and K (Oracle.qknorm in
+# oracle/__init__.py): each is an edit of that file's text, loaded as its own
+# module over the real compiled oracle.
+PY_MUTANTS = {
+    # Q normalised with K's weight and K with Q's.
+    "qknorm_gamma_swapped": [("self.rmsnorm(q, gamma_q,", "self.rmsnorm(q, gamma_k,"),
+                             ("self.rmsnorm(k, gamma_k,", "self.rmsnorm(k, gamma_q,")],
+    # (yk, yq) returned in place of (yq, yk).
+    "qknorm_outputs_swapped": [("return yq, yk, rq, rk", "return yk, yq, rk, rq")],
+    # K normalised with Q's statistic (the factor of the wrong tensor).
+    "qknorm_k_uses_q_factor": [("return yq, yk, rq, rk",
+                                "return yq, yk * (rq / rk)[:, None], rq, rq")],
+    # eps dropped for K only.
+    "qknorm_k_eps_dropped": [("self.rmsnorm(k, gamma_k, P, eps,", "self.rmsnorm(k, gamma_k, P, 0.0,")],
+}
+
+
+def _load_py_mutant(tmpdir, name, edits):
+    src_path = os.path.join(os.path.dirname(oracle.SOURCE), "__init__.py")
+    with open(src_path) as f:
+        src = f.read()
+    for old, new in edits:
+        assert old in src, f"mutant {name}: pattern {old!r} not in the oracle front end"
+        src = src.replace(old, new)
+    path = os.path.join(tmpdir, f"oracle_{name}.py")
+    with open(path, "w") as f:
+        f.write(src)
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.Oracle(oracle.build())
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_front_end_mutant_is_caught(tmp_path, name):
+    orc = _load_py_mutant(str(tmp_path), name, PY_MUTANTS[name])
     caught = []
     for pin in oracle_pins.ALL_PINS:
         try:

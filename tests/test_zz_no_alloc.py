@@ -52,6 +52,9 @@ def test_noalloc_matches_the_existing_entry_points_twice():
         check_outputs(to_host(got), orc.rmsnorm(x, g, wl.P, float(np.float32(wl.eps)), wl.dtype)[0],
                       wl.dtype, wl.name)
         assert torch.equal(bits(got), bits(ref)) and torch.equal(bits(got), bits(ref2))
+        via_wrapper = qk.qknorm_split_noalloc(xd, gd, wl.P, wl.eps)           # the Python binding
+        torch.cuda.synchronize()
+        assert torch.equal(bits(via_wrapper), bits(got))
 
 
 def test_noalloc_rejects_more_statistics_than_its_buffer():
