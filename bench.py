@@ -36,7 +36,7 @@ METRIC = "QK-Norm GB/s and % of B200 HBM peak (prefill); μs/call at decode T≤
 HEADLINE = "prefill13b"
 FALLBACK_HBM_GBS = 6650.0
 
-KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_generic (one warp)", 2: "fused_generic",
+KERNEL_OF_VARIANT = {0: "fused_cta", 1: "fused_warp", 2: "fused_generic", 6: "fused_gpair",
                      3: "fused_bulk", 4: "fused_rows", 5: "fused_pair"}
 
 # dram bytes per launch of the headline kernel from one ncu capture, and the
@@ -62,7 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS),
                     help="workload of the timed region (default: the 13B-shaped prefill); "
                          "the largest T of the workload is used")
-    ap.add_argument("--variant", default="auto", choices=("auto", "cta", "warp", "generic", "bulk", "rows", "pair"),
+    ap.add_argument("--variant", default="auto",
+                    choices=("auto", "cta", "warp", "generic", "bulk", "rows", "pair", "gpair"),
                     help="force a kernel variant (for profiling; default: the selector's choice)")
     ap.add_argument("--path", default="fused", choices=("fused", "split", "headwise"),
                     help="what a step runs: qknorm_fwd (default), the split path "
@@ -74,7 +75,7 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4, "pair": 5}
+VARIANT_IDS = {"auto": -1, "cta": 0, "warp": 1, "generic": 2, "bulk": 3, "rows": 4, "pair": 5, "gpair": 6}
 
 
 # The source of the headline kernel (the fused_bulk template, from its

@@ -48,7 +48,10 @@
  * an xor butterfly (16, 8, 4, 2, 1); the K group sums are added in order of
  * k, giving S[t,p]; the P shard sums are added in order of p. A vector's sum
  * of squares is e0*e0 followed by fused multiply-adds of e1..e_last; for FP8
- * (16 values) it is that sum over e0..e7 plus that sum over e8..e15.
+ * (16 values) it is h(e0..e7) + h(e8..e15), where h of 8 values is the sum of
+ * two chains formed side by side (as packed f32x2 operations): the even
+ * elements' squares (e0*e0, then fused multiply-adds of e2, e4, e6) plus the
+ * odd elements' (e1*e1, then e3, e5, e7).
  * Then r = rsqrt(S / D + eps) and y = (x * gamma) * r, each step fp32.
  */
 #ifndef QKNORM_H
@@ -347,7 +350,9 @@ typedef enum {
                                    held in registers, persistent grid, next token
                                    prefetched when a CTA has more than one */
     QKNORM_VARIANT_WARP = 1,    /* warp per token: one warp walks all shards of a
-                                   token, then re-reads the row to apply */
+                                   token's Q and K rows, holding them in registers
+                                   (shards of one lane group, at most 32 vectors per
+                                   lane); other shapes loop and re-read the row */
     QKNORM_VARIANT_GENERIC = 2, /* CTA per token, any shape: warps loop over the
                                    shard groups, re-read the row to apply */
     QKNORM_VARIANT_BULK = 3,    /* as CTA, but rows arrive by bulk asynchronous
@@ -358,10 +363,16 @@ typedef enum {
                                    own ring of bulk-copied row stages, walks all
                                    P shards of the row itself and applies from
                                    shared memory; no CTA barrier per row */
-    QKNORM_VARIANT_PAIR = 5     /* as BULK with P warps per token instead of 2P
+    QKNORM_VARIANT_PAIR = 5,    /* as BULK with P warps per token instead of 2P
                                    (GQA-like shapes: P even, K shards of <= 16
                                    vectors): a warp takes two Q shards, or two
                                    K shards on its lane halves */
+    QKNORM_VARIANT_GPAIR = 6    /* as PAIR with gamma staged once per CTA in shared
+                                   memory (no gamma registers): a warp takes two
+                                   shards of one tensor, or (mixed, when Q and K
+                                   shards differ) the same two shards of Q and of
+                                   K; FP8 splits a last slot of <= 16 vectors in
+                                   halves over the lanes */
 } qknorm_variant;
 
 /* A launch plan chosen by the selector (host-side description). */
@@ -375,7 +386,8 @@ typedef struct {
     int32_t groups_k;    /* K for a K shard */
     int32_t stages;      /* ring stages per CTA (bulk) or per warp (rows), else 0 */
     int32_t tokens_per_stage; /* tokens a bulk stage holds (1 or 2), else 0 */
-    int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers */
+    int32_t gamma_regs;  /* 1 if each lane keeps its gamma in registers (bulk, pair; CTA:
+                            loaded together with the row) */
     int32_t full_lanes;  /* 1 if every lane holds exactly vmax vectors per task; 2 (FP8,
                             bulk) if every lane holds vmax - 1 and the last slot's
                             <= 16 vectors are split in halves over the 32 lanes */
@@ -384,6 +396,11 @@ typedef struct {
     int32_t gamma_smem;  /* rows: 1 if gamma is staged in shared memory, 0 if read via L1 */
     int32_t k_pairs;     /* pair: 1 if each K warp takes two K shards like a Q warp, 0 if
                             two K shards of <= 16 vectors share a warp's lane halves */
+    int32_t vmax_k;      /* warp: 16-byte vectors per lane per K shard (vmax is Q's);
+                            0 when the warp variant loops over the row instead;
+                            gpair: whole slots per lane per K shard (vmax: Q's) */
+    int32_t half_slots;  /* gpair: bit 0 Q's, bit 1 K's last slot split in lane halves */
+    int32_t mixed;       /* gpair: 1 if every warp takes Q and K shards */
 } qknorm_plan;
 
 /*
@@ -418,7 +435,8 @@ QKNORM_API int qknorm_launch_plan(int64_t T, int32_t Dq, int32_t Dk, int32_t P, 
  * qknorm_set_tuning -- process-wide tuning of the bulk variant for tests and
  * benchmarks: ring stages per CTA (0 = automatic), tokens per stage (0 =
  * automatic, else 1 or 2), gamma in registers (-1 = automatic, 0 = no,
- * 1 = yes), the bound of every wait in milliseconds (0 = the default of
+ * 1 = yes; also the CTA variant's gamma registers, where an instance has
+ * them), the bound of every wait in milliseconds (0 = the default of
  * 2000 ms). A combination without a kernel instance makes qknorm_fwd return
  * QKNORM_ERR_UNSUPPORTED. Not thread-safe with concurrent calls.
  */

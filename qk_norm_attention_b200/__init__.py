@@ -37,10 +37,11 @@ QKNORM_ERR_MISALIGNED = 2
 QKNORM_ERR_UNSUPPORTED = 3
 QKNORM_ERR_CUDA = 4
 
-VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_ROWS, VARIANT_PAIR = \
-    -1, 0, 1, 2, 3, 4, 5
+VARIANT_AUTO, VARIANT_CTA, VARIANT_WARP, VARIANT_GENERIC, VARIANT_BULK, VARIANT_ROWS, VARIANT_PAIR, \
+    VARIANT_GPAIR = -1, 0, 1, 2, 3, 4, 5, 6
 VARIANT_NAMES = {VARIANT_CTA: "cta", VARIANT_WARP: "warp", VARIANT_GENERIC: "generic",
-                 VARIANT_BULK: "bulk", VARIANT_ROWS: "rows", VARIANT_PAIR: "pair"}
+                 VARIANT_BULK: "bulk", VARIANT_ROWS: "rows", VARIANT_PAIR: "pair",
+                 VARIANT_GPAIR: "gpair"}
 
 _DTYPE = {torch.float32: QKNORM_F32, torch.bfloat16: QKNORM_BF16,
           torch.float8_e4m3fn: QKNORM_E4M3}
@@ -65,7 +66,8 @@ class QKNormPlan(ctypes.Structure):
                 ("tokens_per_stage", ctypes.c_int32), ("gamma_regs", ctypes.c_int32),
                 ("full_lanes", ctypes.c_int32), ("smem_bytes", ctypes.c_int64),
                 ("q_warps", ctypes.c_int32), ("gamma_smem", ctypes.c_int32),
-                ("k_pairs", ctypes.c_int32)]
+                ("k_pairs", ctypes.c_int32), ("vmax_k", ctypes.c_int32),
+                ("half_slots", ctypes.c_int32), ("mixed", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

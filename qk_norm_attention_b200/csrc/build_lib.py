@@ -52,16 +52,35 @@ def nvcc() -> str:
 DECODE_BENCH = os.path.join(PKG, "decode_bench")
 
 
+def _compile_objects(verbose: bool) -> list:
+    """Each .cu to its own object, in parallel (in _build/ under the package)."""
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [f for f in NVCC_FLAGS if f not in ("-shared", "-cudart", "static")]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *flags, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+        jobs.append((cmd, obj))
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with ThreadPoolExecutor(workers) as ex:
+        for r in ex.map(lambda j: subprocess.run(j[0]), jobs):
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
+    return [obj for _, obj in jobs]
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every .cu under csrc/ into libqknorm.so (skipped when up to date),
     and the C++ decode timing program linked against it."""
     if force or verbose or not up_to_date():
         tmp = LIBRARY + ".tmp"
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
-        if verbose:
-            cmd += ["-Xptxas", "-v"]
-        cmd += ["-o", tmp, *sources()]
-        subprocess.run(cmd, check=True)
+        objs = _compile_objects(verbose)
+        subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                        "-cudart", "static", "-o", tmp, *objs], check=True)
         os.replace(tmp, LIBRARY)
     src = os.path.join(CSRC, "decode_bench.cpp")
     if (force or not os.path.exists(DECODE_BENCH) or

@@ -319,6 +319,64 @@ bool pair_fits(const Shapes &sh, int32_t P, int32_t dtype) {
            fused_pair_kernel(dtype, pair_vq(sh), pair_greg(sh, dtype), pair_kw(sh)) != nullptr;
 }
 
+// The CTA kernel keeps a lane's gamma in registers, loaded together with the
+// row, while it is at most 32 floats (one token per CTA: no prefetch).
+bool cta_greg(const Shapes &sh, int32_t dtype, bool full) {
+    if (g_tune_gamma_regs == 0) return false;
+    return fused_cta_kernel(dtype, sh.vmax, false, full, true, nullptr) != nullptr;
+}
+
+// The register-resident warp-per-token kernel: one lane group per shard and
+// an instance for (P, Q vectors per lane, K vectors per lane).
+bool warp_regs_fit(const Shapes &sh, int32_t P, int32_t dtype) {
+    return sh.q.K == 1 && sh.k.K == 1 &&
+           fused_warp_kernel(dtype, P, sh.q.vmax, sh.k.vmax) != nullptr;
+}
+
+// The shard-pair ring with staged gamma: P even, one lane group per shard;
+// Q and K of the same slot geometry take separate warps, others share them
+// (mixed); an instance must exist.
+struct GPairShape {
+    int nwq, nwk;
+    bool hq, hk, mix;
+};
+
+bool gpair_fits(const Shapes &sh, int32_t P, int32_t dtype, GPairShape *g) {
+    if ((P & 1) || P > 32 || sh.q.K != 1 || sh.k.K != 1) return false;
+    gpair_slots(sh.q.nv, dtype, &g->nwq, &g->hq);
+    gpair_slots(sh.k.nv, dtype, &g->nwk, &g->hk);
+    g->mix = sh.q.nv != sh.k.nv;
+    if ((g->mix ? P / 2 : P) * kLanes > 256) return false;
+    return fused_gpair_kernel(dtype, g->nwq, g->hq, g->nwk, g->hk, g->mix) != nullptr;
+}
+
+// Stages of the staged-gamma ring: the most bytes in flight per SM (CTAs x
+// stages x stage bytes) with at least two stages and at most four, within the
+// SM's threads and shared memory; ties go to more CTAs.
+void gpair_stages(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, const GPairShape &g, int block,
+                  qknorm_plan *pl) {
+    int bestS = 2;
+    int64_t best = -1;
+    for (int S = 2; S <= 4; ++S) {
+        const size_t sm = gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, S, (int64_t)Dq * elem_of(dtype),
+                                           (int64_t)Dk * elem_of(dtype), nullptr, nullptr, nullptr, nullptr);
+        if (sm > (size_t)kSmemPerCta) break;
+        int ctas = (int)(kSmemPerSm / (sm + kSmemReservedPerCta));
+        if (ctas > kThreadsPerSm / block) ctas = kThreadsPerSm / block;
+        if (ctas < 1) break;
+        const int64_t inflight = (int64_t)ctas * S;
+        if (inflight > best) {
+            best = inflight;
+            bestS = S;
+        }
+    }
+    if (g_tune_stages > 0) bestS = g_tune_stages;
+    pl->stages = bestS;
+    pl->smem_bytes = (int64_t)gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, bestS,
+                                               (int64_t)Dq * elem_of(dtype), (int64_t)Dk * elem_of(dtype),
+                                               nullptr, nullptr, nullptr, nullptr);
+}
+
 // Static part of the plan: which kernel, block size, template width, stages.
 int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int32_t variant,
                 int num_sms, int regs, qknorm_plan *pl) {
@@ -327,7 +385,7 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
     pl->groups_q = sh.q.K;
     pl->groups_k = sh.k.K;
     int cta_max = 0;
-    fused_cta_kernel(dtype, sh.vmax, false, false, &cta_max);
+    fused_cta_kernel(dtype, sh.vmax, false, false, false, &cta_max);
     pl->full_lanes = lane_mode(sh, dtype);
     const bool cta_ok = sh.ntask * kLanes <= cta_max;
     const int tb = tokens_per_stage_for(sh.vmax);
@@ -364,8 +422,16 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         const bool ragged = !pl->full_lanes && dtype != QKNORM_E4M3;
         const bool kpairs = pair_fits(sh, P, dtype) && pair_kw(sh) && pair_greg(sh, dtype) &&
                             (dtype == QKNORM_E4M3 ? pair_vq(sh) == 1 : ragged);
+        // FP8 with Q and K shards of different widths (GQA-like) takes the
+        // mixed shard-pair ring with gamma staged in shared memory: P/2 warps
+        // per token, each with two Q and two K shards (measured at T = 4096,
+        // 5120/1024, P = 8: 43 % vs 37 % for the shard-pair ring with gamma in
+        // registers).
+        GPairShape gp;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
+        else if (dtype == QKNORM_E4M3 && gpair_fits(sh, P, dtype, &gp) && gp.mix)
+            variant = QKNORM_VARIANT_GPAIR;
         else if (pair_fits(sh, P, dtype) && !pair_kw(sh) && sh.q.nv > kLanes)
             variant = QKNORM_VARIANT_PAIR;
         else if (kpairs)
@@ -382,6 +448,8 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         pl->variant = variant;
         pl->block = (int32_t)(sh.ntask * kLanes);
         pl->vmax = sh.vmax;
+        if (variant == QKNORM_VARIANT_CTA)
+            pl->gamma_regs = cta_greg(sh, dtype, pl->full_lanes == 1) ? 1 : 0;
         if (variant == QKNORM_VARIANT_BULK) {
             pl->gamma_regs = greg ? 1 : 0;
             pl->tokens_per_stage = tb;
@@ -416,6 +484,21 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
             return QKNORM_ERR_UNSUPPORTED;
         return QKNORM_OK;
     }
+    if (variant == QKNORM_VARIANT_GPAIR) {
+        GPairShape g;
+        if (!gpair_fits(sh, P, dtype, &g)) return QKNORM_ERR_UNSUPPORTED;
+        pl->variant = QKNORM_VARIANT_GPAIR;
+        pl->block = (g.mix ? P / 2 : P) * kLanes;
+        pl->vmax = g.nwq;
+        pl->vmax_k = g.nwk;
+        pl->half_slots = (g.hq ? 1 : 0) | (g.hk ? 2 : 0);
+        pl->mixed = g.mix ? 1 : 0;
+        pl->tokens_per_stage = 1;
+        gpair_stages(Dq, Dk, P, dtype, g, pl->block, pl);
+        if (pl->stages < 1 || pl->stages > bulk_max_stages() || pl->smem_bytes > kSmemPerCta)
+            return QKNORM_ERR_UNSUPPORTED;
+        return QKNORM_OK;
+    }
     if (variant == QKNORM_VARIANT_ROWS) {
         const int S = g_rows_stages > 0 ? g_rows_stages : kRowsStagesAuto;
         RowsChoice c = rows_auto(Dq, Dk, dtype, S, g_rows_gsm, regs > 0 ? regs : kRegsHint);
@@ -433,6 +516,13 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         pl->q_warps = c.wq;
         pl->gamma_smem = c.gsm ? 1 : 0;
         pl->smem_bytes = (int64_t)L.smem_bytes;
+        return QKNORM_OK;
+    }
+    if (variant == QKNORM_VARIANT_WARP && warp_regs_fit(sh, P, dtype)) {
+        pl->variant = QKNORM_VARIANT_WARP;
+        pl->block = kLanes;              // one token per CTA: the tokens spread over the SMs
+        pl->vmax = sh.q.vmax;
+        pl->vmax_k = sh.k.vmax;
         return QKNORM_OK;
     }
     if ((size_t)sh.ntask * sizeof(float) > (size_t)kGenericMaxSmem) return QKNORM_ERR_UNSUPPORTED;
@@ -455,6 +545,10 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
 // that give every warp of the smaller pool a row (T Q rows over q_warps
 // warps per CTA, T K rows over the others).
 int64_t plan_units(int64_t T, const qknorm_plan &pl) {
+    if (pl.variant == QKNORM_VARIANT_WARP && pl.vmax > 0) {
+        const int64_t w = pl.block / kLanes;             // tokens per CTA
+        return (T + w - 1) / w;
+    }
     if (pl.variant != QKNORM_VARIANT_ROWS) return T;
     const int64_t wq = pl.q_warps, wk = pl.block / kLanes - pl.q_warps;
     const int64_t w = wq < wk ? wq : wk;
@@ -470,15 +564,21 @@ void plan_grid(int64_t T, int num_sms, int blocks_per_sm, qknorm_plan *pl) {
     pl->grid = T < cap ? T : cap;
     if (pl->grid < 1) pl->grid = 1;
     pl->prefetch = (pl->variant == QKNORM_VARIANT_CTA && T > pl->grid) ? 1 : 0;
+    if (pl->prefetch) pl->gamma_regs = 0;   // the gamma-register instances take one token per CTA
 }
 
 // The kernel a plan launches (for the occupancy query: the register variant
 // with prefetch, whose footprint is the larger).
-const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy) {
+const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, int32_t P, bool for_occupancy) {
     switch (pl.variant) {
     case QKNORM_VARIANT_CTA:
+        if (pl.gamma_regs && !for_occupancy)
+            return fused_cta_kernel(dtype, pl.vmax, false, pl.full_lanes == 1, true, nullptr);
         return fused_cta_kernel(dtype, pl.vmax, for_occupancy || pl.prefetch != 0,
-                                pl.full_lanes == 1, nullptr);
+                                pl.full_lanes == 1, false, nullptr);
+    case QKNORM_VARIANT_WARP:
+        if (pl.vmax > 0) return fused_warp_kernel(dtype, P, pl.vmax, pl.vmax_k);
+        return fused_generic_kernel(dtype);
     case QKNORM_VARIANT_BULK:
         return fused_bulk_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.tokens_per_stage,
                                  pl.full_lanes, nullptr);
@@ -486,6 +586,9 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, bool for_occupancy
         return fused_rows_kernel(dtype);
     case QKNORM_VARIANT_PAIR:
         return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0);
+    case QKNORM_VARIANT_GPAIR:
+        return fused_gpair_kernel(dtype, pl.vmax, (pl.half_slots & 1) != 0, pl.vmax_k,
+                                  (pl.half_slots & 2) != 0, pl.mixed != 0);
     default:
         return fused_generic_kernel(dtype);
     }
@@ -545,17 +648,18 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS ||
         pl->variant == QKNORM_VARIANT_PAIR) {
         int regs = kRegsHint;
-        e = kernel_regs(plan_kernel(*pl, dtype, true), &regs);
+        e = kernel_regs(plan_kernel(*pl, dtype, P, true), &regs);
         if (e != cudaSuccess) return e;
         *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, regs, pl);
         if (*status != QKNORM_OK) return cudaSuccess;
     }
-    const void *fn = plan_kernel(*pl, dtype, true);
+    const void *fn = plan_kernel(*pl, dtype, P, true);
     if (pl->smem_bytes > 48 * 1024 || pl->variant == QKNORM_VARIANT_GENERIC ||
-        pl->variant == QKNORM_VARIANT_WARP) {
+        (pl->variant == QKNORM_VARIANT_WARP && pl->vmax == 0)) {
         e = prepare_kernel(dev, fn, (pl->variant == QKNORM_VARIANT_BULK ||
                                      pl->variant == QKNORM_VARIANT_ROWS ||
-                                     pl->variant == QKNORM_VARIANT_PAIR) ? kSmemPerCta : kGenericMaxSmem);
+                                     pl->variant == QKNORM_VARIANT_PAIR ||
+                                     pl->variant == QKNORM_VARIANT_GPAIR) ? kSmemPerCta : kGenericMaxSmem);
         if (e != cudaSuccess) return e;
     }
     int bres = 1;
@@ -772,7 +876,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 114; }
+int qknorm_version(void) { return 115; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
@@ -788,7 +892,7 @@ const char *qknorm_status_string(int status) {
 const char *qknorm_last_error(void) { return g_last_error; }
 
 int qknorm_force_variant(int32_t variant, int64_t grid) {
-    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_PAIR || grid < 0)
+    if (variant < QKNORM_VARIANT_AUTO || variant > QKNORM_VARIANT_GPAIR || grid < 0)
         return QKNORM_ERR_INVALID_ARG;
     g_forced_variant = variant;
     g_forced_grid = grid;
@@ -889,11 +993,17 @@ int qknorm_fwd_strided(const void *q, const void *k, const float *gamma_q, const
     a.ldy[1] = ldok / vec;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (pl.variant == QKNORM_VARIANT_CTA) {
-        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes == 1, a, pl.block,
-                             pl.grid, s);
+        e = launch_fused_cta(dtype, pl.vmax, pl.prefetch != 0, pl.full_lanes == 1,
+                             pl.gamma_regs != 0, a, pl.block, pl.grid, s);
+    } else if (pl.variant == QKNORM_VARIANT_WARP && pl.vmax > 0) {
+        e = launch_fused_warp(dtype, P, pl.vmax, pl.vmax_k, a, pl.block, pl.grid, s);
     } else if (pl.variant == QKNORM_VARIANT_ROWS) {
         e = launch_fused_rows(dtype, a, pl.q_warps, pl.block / kLanes - pl.q_warps, pl.stages,
                               pl.gamma_smem != 0, pl.grid, g_wait_limit_ns, s);
+    } else if (pl.variant == QKNORM_VARIANT_GPAIR) {
+        e = launch_fused_gpair(dtype, pl.vmax, (pl.half_slots & 1) != 0, pl.vmax_k,
+                               (pl.half_slots & 2) != 0, pl.mixed != 0, a, pl.stages, pl.grid,
+                               g_wait_limit_ns, s);
     } else if (pl.variant == QKNORM_VARIANT_PAIR) {
         e = launch_fused_pair(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0, a, pl.stages,
                               pl.grid, g_wait_limit_ns, s);

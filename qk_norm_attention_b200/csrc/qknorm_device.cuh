@@ -96,25 +96,25 @@ __device__ __forceinline__ float vsumsq(BF16Tag, const uint4 &v) {
 }
 
 // The 8 FP8 values of half a vector (w0, w1; element 0 in the low byte of
-// w0): e0*e0, then e_i*e_i + q fused, i = 1..7 (an E4M3 square is exact in
-// fp32, so each fma rounds only the running sum).
+// w0), as two interleaved chains over its element pairs (e0,e1), (e2,e3),
+// (e4,e5), (e6,e7): the even elements' squares summed in order in one fp32
+// chain and the odd elements' in the other (e0*e0, then e2*e2 + q fused, ...;
+// e1*e1, then e3*e3 + q fused, ...), each step of the two chains one packed
+// f32x2 fused multiply-add; then even sum + odd sum. An E4M3 square is exact
+// in fp32, so each step rounds only the running sums.
 __device__ __forceinline__ float e4m3x8_sumsq(uint32_t w0, uint32_t w1) {
     const float2 a = e4m3x2_to_float2(w0), b = e4m3x2_to_float2(w0 >> 16);
     const float2 c = e4m3x2_to_float2(w1), d = e4m3x2_to_float2(w1 >> 16);
-    float q = __fmul_rn(a.x, a.x);
-    q = __fmaf_rn(a.y, a.y, q);
-    q = __fmaf_rn(b.x, b.x, q);
-    q = __fmaf_rn(b.y, b.y, q);
-    q = __fmaf_rn(c.x, c.x, q);
-    q = __fmaf_rn(c.y, c.y, q);
-    q = __fmaf_rn(d.x, d.x, q);
-    q = __fmaf_rn(d.y, d.y, q);
-    return q;
+    float2 q = __fmul2_rn(a, a);
+    q = __ffma2_rn(b, b, q);
+    q = __ffma2_rn(c, c, q);
+    q = __ffma2_rn(d, d, q);
+    return __fadd_rn(q.x, q.y);
 }
 
 // Same for 16 FP8 values: the sums of the two halves (elements 0-7, 8-15),
-// each in order, then added. Two independent chains; and a half vector is a
-// unit the bulk kernel can hand to another lane.
+// each as above, then added. A half vector is a unit the bulk kernel can hand
+// to another lane.
 __device__ __forceinline__ float vsumsq(E4M3Tag, const uint4 &v) {
     return __fadd_rn(e4m3x8_sumsq(v.x, v.y), e4m3x8_sumsq(v.z, v.w));
 }
@@ -169,26 +169,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// (x * gamma) * r for two values at once: two packed f32x2 multiplies, each
+// lane rounded exactly as wmul's two __fmul_rn (so the bits are wmul's).
+__device__ __forceinline__ float2 wmul2(float2 x, float2 g, float2 rr) {
+    return fmul2_rn(fmul2_rn(x, g), rr);
+}
+
+__device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float *g, float r);
+__device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r);
+
 // y = (x * gamma) * r for one vector; g points at the vector's gamma (fp32).
 __device__ __forceinline__ uint4 vapply(F32Tag, const uint4 &v, const float *g, float r) {
     const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g));
-    uint4 o;
-    o.x = __float_as_uint(wmul(__uint_as_float(v.x), g4.x, r));
-    o.y = __float_as_uint(wmul(__uint_as_float(v.y), g4.y, r));
-    o.z = __float_as_uint(wmul(__uint_as_float(v.z), g4.z, r));
-    o.w = __float_as_uint(wmul(__uint_as_float(v.w), g4.w, r));
-    return o;
+    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+    return vapply_regs(F32Tag{}, v, gg, r);
 }
 
 __device__ __forceinline__ uint4 vapply(BF16Tag, const uint4 &v, const float *g, float r) {
     const float4 ga = __ldg(reinterpret_cast<const float4 *>(g));
     const float4 gb = __ldg(reinterpret_cast<const float4 *>(g) + 1);
-    uint4 o;
-    o.x = pack_bf16x2(wmul(bf_lo(v.x), ga.x, r), wmul(bf_hi(v.x), ga.y, r));
-    o.y = pack_bf16x2(wmul(bf_lo(v.y), ga.z, r), wmul(bf_hi(v.y), ga.w, r));
-    o.z = pack_bf16x2(wmul(bf_lo(v.z), gb.x, r), wmul(bf_hi(v.z), gb.y, r));
-    o.w = pack_bf16x2(wmul(bf_lo(v.w), gb.z, r), wmul(bf_hi(v.w), gb.w, r));
-    return o;
+    const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    return vapply_regs(BF16Tag{}, v, gg, r);
 }
 
 __device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const float *g, float r);
@@ -209,12 +210,10 @@ __device__ __forceinline__ uint4 vapply(E4M3Tag, const uint4 &v, const float *g,
 // Same as vapply with gamma already in registers (g[0..vec-1], indexed with
 // compile-time constants after unrolling).
 __device__ __forceinline__ uint4 vapply_regs(F32Tag, const uint4 &v, const float *g, float r) {
-    uint4 o;
-    o.x = __float_as_uint(wmul(__uint_as_float(v.x), g[0], r));
-    o.y = __float_as_uint(wmul(__uint_as_float(v.y), g[1], r));
-    o.z = __float_as_uint(wmul(__uint_as_float(v.z), g[2], r));
-    o.w = __float_as_uint(wmul(__uint_as_float(v.w), g[3], r));
-    return o;
+    const float2 rr = make_float2(r, r);
+    const float2 a = wmul2(make_float2(__uint_as_float(v.x), __uint_as_float(v.y)), make_float2(g[0], g[1]), rr);
+    const float2 b = wmul2(make_float2(__uint_as_float(v.z), __uint_as_float(v.w)), make_float2(g[2], g[3]), rr);
+    return make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
 }
 
 // FP8, half a vector (8 values, gamma g[0..7]): the two multiplies of each
@@ -229,8 +228,8 @@ __device__ __forceinline__ uint2 vapply_half_regs(E4M3Tag, uint32_t w0, uint32_t
     for (int i = 0; i < 2; ++i) {
         const float2 x01 = e4m3x2_to_float2(w[i]);
         const float2 x23 = e4m3x2_to_float2(w[i] >> 16);
-        const float2 y01 = fmul2_rn(fmul2_rn(x01, make_float2(g[4 * i], g[4 * i + 1])), rr);
-        const float2 y23 = fmul2_rn(fmul2_rn(x23, make_float2(g[4 * i + 2], g[4 * i + 3])), rr);
+        const float2 y01 = wmul2(x01, make_float2(g[4 * i], g[4 * i + 1]), rr);
+        const float2 y23 = wmul2(x23, make_float2(g[4 * i + 2], g[4 * i + 3]), rr);
         o[i] = pack_e4m3x2(y01.x, y01.y) | (pack_e4m3x2(y23.x, y23.y) << 16);
     }
     return make_uint2(o[0], o[1]);
@@ -247,34 +246,38 @@ __device__ __forceinline__ uint4 vapply_regs(E4M3Tag, const uint4 &v, const floa
 }
 
 __device__ __forceinline__ uint4 vapply_regs(BF16Tag, const uint4 &v, const float *g, float r) {
-    uint4 o;
-    o.x = pack_bf16x2(wmul(bf_lo(v.x), g[0], r), wmul(bf_hi(v.x), g[1], r));
-    o.y = pack_bf16x2(wmul(bf_lo(v.y), g[2], r), wmul(bf_hi(v.y), g[3], r));
-    o.z = pack_bf16x2(wmul(bf_lo(v.z), g[4], r), wmul(bf_hi(v.z), g[5], r));
-    o.w = pack_bf16x2(wmul(bf_lo(v.w), g[6], r), wmul(bf_hi(v.w), g[7], r));
-    return o;
+    const float2 rr = make_float2(r, r);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 y = wmul2(make_float2(bf_lo(w[i]), bf_hi(w[i])), make_float2(g[2 * i], g[2 * i + 1]), rr);
+        o[i] = pack_bf16x2(y.x, y.y);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// u = x * gamma for one vector, rounded to the storage type (no factor).
+// u = x * gamma for one vector, rounded to the storage type (no factor);
+// packed f32x2 multiplies, each lane exactly __fmul_rn.
 __device__ __forceinline__ uint4 vxgamma(F32Tag, const uint4 &v, const float *g) {
     const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g));
-    uint4 o;
-    o.x = __float_as_uint(__fmul_rn(__uint_as_float(v.x), g4.x));
-    o.y = __float_as_uint(__fmul_rn(__uint_as_float(v.y), g4.y));
-    o.z = __float_as_uint(__fmul_rn(__uint_as_float(v.z), g4.z));
-    o.w = __float_as_uint(__fmul_rn(__uint_as_float(v.w), g4.w));
-    return o;
+    const float2 a = fmul2_rn(make_float2(__uint_as_float(v.x), __uint_as_float(v.y)), make_float2(g4.x, g4.y));
+    const float2 b = fmul2_rn(make_float2(__uint_as_float(v.z), __uint_as_float(v.w)), make_float2(g4.z, g4.w));
+    return make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
 }
 
 __device__ __forceinline__ uint4 vxgamma(BF16Tag, const uint4 &v, const float *g) {
     const float4 ga = __ldg(reinterpret_cast<const float4 *>(g));
     const float4 gb = __ldg(reinterpret_cast<const float4 *>(g) + 1);
-    uint4 o;
-    o.x = pack_bf16x2(__fmul_rn(bf_lo(v.x), ga.x), __fmul_rn(bf_hi(v.x), ga.y));
-    o.y = pack_bf16x2(__fmul_rn(bf_lo(v.y), ga.z), __fmul_rn(bf_hi(v.y), ga.w));
-    o.z = pack_bf16x2(__fmul_rn(bf_lo(v.z), gb.x), __fmul_rn(bf_hi(v.z), gb.y));
-    o.w = pack_bf16x2(__fmul_rn(bf_lo(v.w), gb.z), __fmul_rn(bf_hi(v.w), gb.w));
-    return o;
+    const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 y = fmul2_rn(make_float2(bf_lo(w[i]), bf_hi(w[i])), make_float2(gg[2 * i], gg[2 * i + 1]));
+        o[i] = pack_bf16x2(y.x, y.y);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint4 vxgamma(E4M3Tag, const uint4 &v, const float *g) {

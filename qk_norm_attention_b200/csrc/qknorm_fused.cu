@@ -48,7 +48,7 @@ __device__ __forceinline__ Task decode_task(const FusedArgs &a, int j) {
     return t;
 }
 
-template <class Tag, int VMAX, bool PREFETCH, bool FULL, int MAXT>
+template <class Tag, int VMAX, bool PREFETCH, bool FULL, int MAXT, bool GREG>
 __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
     constexpr int VEC = Tag::kVec;
     __shared__ float red[2][32];
@@ -82,6 +82,24 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
         for (int i = 0; i < VMAX; ++i)
             if (FULL || i < cnt) cur[i] = ld_stream(src + (int64_t)i * stride);
     }
+    // GREG: the lane's gamma in registers, its loads in flight together with
+    // the row's (otherwise they are issued after the CTA barrier, one more
+    // dependent round trip per token).
+    float gr[GREG ? VMAX : 1][GREG ? VEC : 1];
+    if constexpr (GREG) {
+#pragma unroll
+        for (int i = 0; i < VMAX; ++i)
+            if (FULL || i < cnt) {
+#pragma unroll
+                for (int j = 0; j < VEC; j += 4) {
+                    const float4 g4 = __ldg(reinterpret_cast<const float4 *>(gs + (int64_t)i * stride * VEC + j));
+                    gr[i][j] = g4.x;
+                    gr[i][j + 1] = g4.y;
+                    gr[i][j + 2] = g4.z;
+                    gr[i][j + 3] = g4.w;
+                }
+            }
+    }
     int buf = 0;
     for (; t < T; t += G) {
         const int64_t tn = t + G;
@@ -106,9 +124,13 @@ __global__ void __launch_bounds__(MAXT, 1) fused_cta(const FusedArgs a) {
         uint4 *dst = ys + t * ldy;
 #pragma unroll
         for (int i = 0; i < VMAX; ++i)
-            if (FULL || i < cnt)
-                st_stream(dst + (int64_t)i * stride,
-                          vapply(Tag{}, cur[i], gs + (int64_t)i * stride * VEC, r));
+            if (FULL || i < cnt) {
+                if constexpr (GREG)
+                    st_stream(dst + (int64_t)i * stride, vapply_regs(Tag{}, cur[i], gr[i], r));
+                else
+                    st_stream(dst + (int64_t)i * stride,
+                              vapply(Tag{}, cur[i], gs + (int64_t)i * stride * VEC, r));
+            }
         if (PREFETCH) {
 #pragma unroll
             for (int i = 0; i < VMAX; ++i) cur[i] = nxt[i];
@@ -173,43 +195,53 @@ constexpr int cta_max_threads(int vmax, int vec) { return (vmax <= 2 && vmax * v
 // whose 16 values per vector take twice the registers of bf16 once widened).
 constexpr bool cta_exists(int vmax, int vec) { return vmax >= 1 && vmax <= (vec == 16 ? 4 : kVcap); }
 
-template <class Tag, int VMAX, bool PF, bool FULL>
+// Gamma in registers while a lane's gamma is at most 32 floats, and only for
+// one token per CTA (no prefetch: the decode sizes).
+constexpr bool cta_greg_exists(int vmax, int vec) { return vmax * vec <= 32; }
+
+template <class Tag, int VMAX, bool PF, bool FULL, bool GREG>
 const void *cta_fn() {
-    if constexpr (cta_exists(VMAX, Tag::kVec))
+    if constexpr (cta_exists(VMAX, Tag::kVec) && (!GREG || (!PF && cta_greg_exists(VMAX, Tag::kVec))))
         return reinterpret_cast<const void *>(
-            &fused_cta<Tag, VMAX, PF, FULL, cta_max_threads(VMAX, Tag::kVec)>);
+            &fused_cta<Tag, VMAX, PF, FULL, cta_max_threads(VMAX, Tag::kVec), GREG>);
     else
         return nullptr;
 }
 
-template <class Tag, bool PF, bool FULL>
+template <class Tag, bool PF, bool FULL, bool GREG>
 const void *cta_table(int vmax) {
     switch (vmax) {
-    case 1: return cta_fn<Tag, 1, PF, FULL>();
-    case 2: return cta_fn<Tag, 2, PF, FULL>();
-    case 3: return cta_fn<Tag, 3, PF, FULL>();
-    case 4: return cta_fn<Tag, 4, PF, FULL>();
-    case 5: return cta_fn<Tag, 5, PF, FULL>();
-    case 6: return cta_fn<Tag, 6, PF, FULL>();
-    case 7: return cta_fn<Tag, 7, PF, FULL>();
-    case 8: return cta_fn<Tag, 8, PF, FULL>();
+    case 1: return cta_fn<Tag, 1, PF, FULL, GREG>();
+    case 2: return cta_fn<Tag, 2, PF, FULL, GREG>();
+    case 3: return cta_fn<Tag, 3, PF, FULL, GREG>();
+    case 4: return cta_fn<Tag, 4, PF, FULL, GREG>();
+    case 5: return cta_fn<Tag, 5, PF, FULL, GREG>();
+    case 6: return cta_fn<Tag, 6, PF, FULL, GREG>();
+    case 7: return cta_fn<Tag, 7, PF, FULL, GREG>();
+    case 8: return cta_fn<Tag, 8, PF, FULL, GREG>();
     default: return nullptr;
     }
 }
 
 template <class Tag>
-const void *cta_pick(int vmax, bool prefetch, bool full) {
-    if (prefetch) return full ? cta_table<Tag, true, true>(vmax) : cta_table<Tag, true, false>(vmax);
-    return full ? cta_table<Tag, false, true>(vmax) : cta_table<Tag, false, false>(vmax);
+const void *cta_pick(int vmax, bool prefetch, bool full, bool greg) {
+    if (greg) {
+        if (prefetch) return nullptr;
+        return full ? cta_table<Tag, false, true, true>(vmax) : cta_table<Tag, false, false, true>(vmax);
+    }
+    if (prefetch)
+        return full ? cta_table<Tag, true, true, false>(vmax) : cta_table<Tag, true, false, false>(vmax);
+    return full ? cta_table<Tag, false, true, false>(vmax) : cta_table<Tag, false, false, false>(vmax);
 }
 
-const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads) {
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, bool greg, int *max_threads) {
     const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
     if (!cta_exists(vmax, vec)) return nullptr;
+    if (greg && (prefetch || !cta_greg_exists(vmax, vec))) return nullptr;
     if (max_threads) *max_threads = cta_max_threads(vmax, vec);
-    if (dtype == 0) return cta_pick<F32Tag>(vmax, prefetch, full);
-    if (dtype == 1) return cta_pick<BF16Tag>(vmax, prefetch, full);
-    if (dtype == 2) return cta_pick<E4M3Tag>(vmax, prefetch, full);
+    if (dtype == 0) return cta_pick<F32Tag>(vmax, prefetch, full, greg);
+    if (dtype == 1) return cta_pick<BF16Tag>(vmax, prefetch, full, greg);
+    if (dtype == 2) return cta_pick<E4M3Tag>(vmax, prefetch, full, greg);
     return nullptr;
 }
 
@@ -220,9 +252,9 @@ const void *fused_generic_kernel(int dtype) {
     return nullptr;
 }
 
-cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
-                             int block, int64_t grid, cudaStream_t s) {
-    const void *fn = fused_cta_kernel(dtype, vmax, prefetch, full, nullptr);
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, bool greg,
+                             const FusedArgs &a, int block, int64_t grid, cudaStream_t s) {
+    const void *fn = fused_cta_kernel(dtype, vmax, prefetch, full, greg, nullptr);
     if (!fn) return cudaErrorInvalidValue;
     void *args[] = {const_cast<FusedArgs *>(&a)};
     return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);

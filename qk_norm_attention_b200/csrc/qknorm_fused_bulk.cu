@@ -42,6 +42,14 @@ constexpr uint32_t kRedBytes = 2 * kMaxTB * 32 * sizeof(float);
 constexpr uint32_t kStageBase = kBarBytes + kRedBytes;
 constexpr uint32_t kMaxStages = 16;
 
+}  // namespace qkn
+
+// Gamma staged in shared memory in a lane-permuted layout, and the shard-pair
+// ring built on it (they share this file's device error word).
+#include "qknorm_gpair.cuh"
+
+namespace qkn {
+
 // MODE (how lanes hold vectors): 0 any shape (guards); 1 every lane of every
 // task holds exactly VMAX vectors (no guards); 2 (FP8) every lane holds
 // VMAX - 1 whole vectors and the last slot's r <= 16 vectors are split in

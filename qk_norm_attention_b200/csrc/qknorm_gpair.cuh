@@ -1,0 +1,423 @@
+// qknorm_gpair.cuh -- the shard-pair token ring with gamma staged in shared
+// memory. Included by qknorm_fused_bulk.cu (it shares that file's device
+// error word and bulk-copy ring conventions).
+//
+// SwiftQK technical review, Section 3, Algorithm 1 (Phases A-C per token),
+// as a token ring like fused_bulk, but with each warp taking a PAIR of
+// shards, so that a warp's fixed work per token (the stage wait, the
+// butterflies, the CTA barrier, the factor) is paid once per two shards:
+//
+//   separate (MIX = false): P warps per token; warp w < P/2 takes Q shards
+//     2w and 2w + 1, warp P/2 + w takes K shards 2w and 2w + 1 (Q and K of
+//     the same geometry);
+//   mixed (MIX = true): P/2 warps per token; warp w takes Q shards 2w, 2w + 1
+//     AND K shards 2w, 2w + 1 (GQA-like shapes, whose narrow K shards would
+//     leave a K-only warp mostly idle).
+//
+// Lane l holds, of each of its shards, the vectors l + 32 i (i < NW: the
+// single lane group of the library's reduction order), plus, in the HALF
+// mode (FP8, a last slot of at most 16 vectors), half of vector 32 NW +
+// (l & 15): lane l < 16 the low 8 bytes, lane l + 16 the high 8 bytes. A
+// vector's FP8 sum of squares is the sum of its halves' sums, so lane l
+// adds lane l + 16's half to its own and the chain has the bits it has in
+// every other kernel.
+//
+// The butterflies of a warp's 2 (or 4) shard chains are one transposed
+// butterfly: at the xor-16 step the lane halves trade the chains they do not
+// keep (and, with 4, the xor-8 step again), so each shard's sum is completed
+// by 16 (or 8) lanes; every addition has the same two operands as in the
+// 32-lane butterfly of that shard, so the sums are bit-identical to it.
+//
+// Gamma is staged once per CTA in shared memory, permuted so that the float4
+// a lane needs for (shard, slot, chunk) sits at 32 * index + lane: a warp's
+// gamma reads are conflict-free and no gamma lives in registers.
+#pragma once
+
+namespace qkn {
+
+struct GPairArgs {
+    uint32_t stages;       // S
+    uint32_t qbytes;       // bytes of one Q row
+    uint32_t kbytes;       // bytes of one K row
+    uint32_t stage_stride; // bytes between stages (multiple of 128)
+    uint32_t gq4;          // float4 slots of Q's staged gamma
+    uint32_t gk4;          // float4 slots of K's staged gamma
+    uint32_t stage_base;   // byte offset of the first stage
+    uint64_t timeout_ns;   // bound of every wait
+};
+
+constexpr uint32_t kGPairRedBytes = 2 * 64 * sizeof(float);   // [buf][Q: 0..31, K: 32..63]
+constexpr uint32_t kGPairGammaOff = kBarBytes + kGPairRedBytes;
+
+// Staged-gamma geometry of one tensor: NW whole slots per lane per shard, a
+// half slot (H), C = VEC / 4 float4 chunks per vector.
+template <class Tag, int NW, bool H>
+struct GSlots {
+    static constexpr int C = Tag::kVec / 4;
+    static constexpr int CH = C / 2;
+    __host__ __device__ static int64_t whole(int P) { return (int64_t)P * NW * C * 32; }
+    __host__ __device__ static int64_t total(int P) { return whole(P) + (H ? (int64_t)P * CH * 32 : 0); }
+};
+
+// Source of staged-gamma slot j of one tensor (float offset into gamma), or
+// -1 for a slot whose vector does not exist.
+template <class Tag, int NW, bool H>
+__device__ __forceinline__ int64_t gpair_gamma_src(int j, int whole, int nv) {
+    using G = GSlots<Tag, NW, H>;
+    constexpr int VEC = Tag::kVec;
+    if (j < whole) {
+        const int l = j & 31;
+        int r = j >> 5;
+        const int c = r % G::C;
+        r /= G::C;
+        const int i = r % (NW > 0 ? NW : 1);
+        const int p = r / (NW > 0 ? NW : 1);
+        const int v = l + 32 * i;
+        return v < nv ? ((int64_t)p * nv + v) * VEC + 4 * c : -1;
+    }
+    const int jj = j - whole;
+    const int l = jj & 31;
+    const int r = jj >> 5;
+    const int c = r % G::CH;
+    const int p = r / G::CH;
+    const int v = 32 * NW + (l & 15);
+    return v < nv ? ((int64_t)p * nv + v) * VEC + (VEC / 2) * (l >> 4) + 4 * c : -1;
+}
+
+// Copy one tensor's gamma into its permuted shared-memory layout. Each thread
+// issues kStageLoads independent loads before it stores any, so the copy
+// costs a few L2 round trips, not one per slot.
+template <class Tag, int NW, bool H>
+__device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, int P, int nv, int tid,
+                                                  int nthreads) {
+    using G = GSlots<Tag, NW, H>;
+    constexpr int kStageLoads = 8;
+    const int whole = (int)G::whole(P), total = (int)G::total(P);
+    for (int j0 = tid; j0 < total; j0 += kStageLoads * nthreads) {
+        float4 val[kStageLoads];
+#pragma unroll
+        for (int u = 0; u < kStageLoads; ++u) {
+            const int j = j0 + u * nthreads;
+            const int64_t src = j < total ? gpair_gamma_src<Tag, NW, H>(j, whole, nv) : -1;
+            val[u] = src >= 0 ? __ldg(reinterpret_cast<const float4 *>(g + src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kStageLoads; ++u) {
+            const int j = j0 + u * nthreads;
+            if (j < total) dst[j] = val[u];
+        }
+    }
+}
+
+// The lane's vectors of shards pa, pa + 1 of one tensor (row = the tensor's
+// row in a ring stage, nv vectors per shard) and their two lane chains.
+template <class Tag, int NW, bool H>
+__device__ __forceinline__ void gpair_chains(const unsigned char *row, int nv, int pa, int lane,
+                                             uint4 (&x)[2][NW > 0 ? NW : 1], uint2 (&hx)[2],
+                                             float (&c)[2]) {
+    static_assert(!H || Tag::kVec == 16, "half slots are defined for FP8 vectors only");
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 *sh = reinterpret_cast<const uint4 *>(row) + (pa + h) * nv;
+        float ch = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const int v = lane + 32 * i;
+            x[h][i] = v < nv ? sh[v] : make_uint4(0, 0, 0, 0);
+            ch = __fadd_rn(ch, vsumsq(Tag{}, x[h][i]));   // a missing vector adds +0
+        }
+        if constexpr (H) {
+            const int hv = 32 * NW + (lane & 15);
+            hx[h] = hv < nv ? *reinterpret_cast<const uint2 *>(reinterpret_cast<const unsigned char *>(sh + hv) +
+                                                               8 * (lane >> 4))
+                            : make_uint2(0, 0);
+            const float hs = e4m3x8_sumsq(hx[h].x, hx[h].y);
+            const float hi = __shfl_down_sync(kFull, hs, 16);
+            if (lane < 16) ch = __fadd_rn(ch, __fadd_rn(hs, hi));
+        }
+        c[h] = ch;
+    }
+}
+
+// (x * gamma) * r for the lane's vectors of shards pa, pa + 1 of one tensor,
+// gamma from its staged layout g (P shards), written to the output row dst.
+template <class Tag, int NW, bool H>
+__device__ __forceinline__ void gpair_apply(const uint4 (&x)[2][NW > 0 ? NW : 1], const uint2 (&hx)[2],
+                                            const float4 *g, int P, uint4 *dst, int nv, int pa, int lane,
+                                            float r) {
+    using G = GSlots<Tag, NW, H>;
+    constexpr int VEC = Tag::kVec;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int p = pa + h;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const int v = lane + 32 * i;
+            if (v < nv) {
+                float gg[VEC];
+#pragma unroll
+                for (int c = 0; c < G::C; ++c) {
+                    const float4 t = g[((p * NW + i) * G::C + c) * 32 + lane];
+                    gg[4 * c] = t.x;
+                    gg[4 * c + 1] = t.y;
+                    gg[4 * c + 2] = t.z;
+                    gg[4 * c + 3] = t.w;
+                }
+                st_stream(dst + p * nv + v, vapply_regs(Tag{}, x[h][i], gg, r));
+            }
+        }
+        if constexpr (H) {
+            const int hv = 32 * NW + (lane & 15);
+            if (hv < nv) {
+                float gh[VEC / 2];
+                const float4 *gb = g + G::whole(P);
+#pragma unroll
+                for (int c = 0; c < G::CH; ++c) {
+                    const float4 t = gb[(p * G::CH + c) * 32 + lane];
+                    gh[4 * c] = t.x;
+                    gh[4 * c + 1] = t.y;
+                    gh[4 * c + 2] = t.z;
+                    gh[4 * c + 3] = t.w;
+                }
+                const uint2 y = vapply_half(Tag{}, hx[h], gh, r);
+                __stcs(reinterpret_cast<uint2 *>(reinterpret_cast<unsigned char *>(dst + p * nv + hv) +
+                                                 8 * (lane >> 4)),
+                       y);
+            }
+        }
+    }
+}
+
+// Transposed butterflies (see the top comment). Two chains: lanes 0-15 end
+// with shard 0's sum, lanes 16-31 with shard 1's.
+__device__ __forceinline__ float butterfly_pair(float c0, float c1, int lane) {
+    const bool lo = lane < 16;
+    float v = __fadd_rn(lo ? c0 : c1, __shfl_xor_sync(kFull, lo ? c1 : c0, 16));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 8));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 4));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 2));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 1));
+    return v;
+}
+
+// Four chains (a, b, c, d): lanes 0-7 end with a's sum, 8-15 b's, 16-23 c's,
+// 24-31 d's.
+__device__ __forceinline__ float butterfly_quad(float a, float b, float c, float d, int lane) {
+    const bool lo = lane < 16;
+    const float u0 = __fadd_rn(lo ? a : c, __shfl_xor_sync(kFull, lo ? c : a, 16));
+    const float u1 = __fadd_rn(lo ? b : d, __shfl_xor_sync(kFull, lo ? d : b, 16));
+    const bool l8 = (lane & 8) == 0;
+    float v = __fadd_rn(l8 ? u0 : u1, __shfl_xor_sync(kFull, l8 ? u1 : u0, 8));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 4));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 2));
+    v = __fadd_rn(v, __shfl_xor_sync(kFull, v, 1));
+    return v;
+}
+
+// Separate form: NW whole slots (+ half slot H) per lane per shard for both
+// tensors (their shards have the same vector count).
+// Mixed form: Q with (NWQ, HQ), K with (NWK, HK), both in every warp.
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX>
+__global__ void __launch_bounds__(256, 1) fused_gpair(const FusedArgs a, const GPairArgs b) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    float(*red)[64] = reinterpret_cast<float(*)[64]>(smem + kBarBytes);
+    float4 *gq = reinterpret_cast<float4 *>(smem + kGPairGammaOff);
+    float4 *gk = gq + b.gq4;
+    unsigned char *stages = smem + b.stage_base;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int P = a.P;
+    const int halfP = P >> 1;
+    const int z = MIX ? 0 : (warp < halfP ? 0 : 1);        // separate form: this warp's tensor
+    const int pa = 2 * (MIX ? warp : (z ? warp - halfP : warp));
+    const int nvq = a.nv[0], nvk = a.nv[1];
+    const uint32_t tok_bytes = b.qbytes + b.kbytes;
+
+    const int64_t T = a.T;
+    const int64_t G = gridDim.x;
+    const int S = (int)b.stages;
+    const char *qsrc = static_cast<const char *>(a.x[0]);
+    const char *ksrc = static_cast<const char *>(a.x[1]);
+    const int64_t ldq_b = a.ldx[0] * 16, ldk_b = a.ldx[1] * 16;
+
+    auto issue = [&](int s, int64_t n) {
+        unsigned char *st = stages + (size_t)s * b.stage_stride;
+        const int64_t tt = blockIdx.x + n * G;
+        mbar_arrive_expect_tx(&full[s], tok_bytes);
+        bulk_copy_g2s(st, qsrc + tt * ldq_b, b.qbytes, &full[s]);
+        bulk_copy_g2s(st + b.qbytes, ksrc + tt * ldk_b, b.kbytes, &full[s]);
+    };
+
+    const int64_t npass = (T - blockIdx.x + G - 1) / G;   // >= 1 since blockIdx.x < T
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Shared memory only so far; global reads start after the previous grid.
+    pdl_wait();
+    pdl_trigger();
+    if (tid == 0) {
+        for (int s = 0; s < S && s < npass; ++s) issue(s, s);
+    }
+    // Gamma of both tensors into shared memory (visible after the first barrier).
+    gpair_stage_gamma<Tag, NWQ, HQ>(gq, a.g[0], P, nvq, tid, blockDim.x);
+    gpair_stage_gamma<Tag, NWK, HK>(gk, a.g[1], P, nvk, tid, blockDim.x);
+
+    constexpr int AQ = NWQ > 0 ? NWQ : 1, AK = NWK > 0 ? NWK : 1;
+    int s = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    for (int64_t n = 0; n < npass; ++n) {
+        const int64_t t = blockIdx.x + n * G;
+        const bool ok = mbar_wait_bounded(&full[s], phase, b.timeout_ns);
+        const unsigned char *st = stages + (size_t)s * b.stage_stride;
+        uint4 xq[2][AQ], xk[2][AK];
+        uint2 hq[2], hk[2];
+        float cq[2], ck[2];
+        if constexpr (MIX) {
+            gpair_chains<Tag, NWQ, HQ>(st, nvq, pa, lane, xq, hq, cq);
+            gpair_chains<Tag, NWK, HK>(st + b.qbytes, nvk, pa, lane, xk, hk, ck);
+            const float v = butterfly_quad(cq[0], cq[1], ck[0], ck[1], lane);
+            if ((lane & 7) == 0) red[buf][32 * (lane >> 4) + pa + ((lane >> 3) & 1)] = v;
+        } else {
+            gpair_chains<Tag, NWQ, HQ>(st + (z ? b.qbytes : 0u), z ? nvk : nvq, pa, lane, xq, hq, cq);
+            const float v = butterfly_pair(cq[0], cq[1], lane);
+            if ((lane & 15) == 0) red[buf][32 * z + pa + (lane >> 4)] = v;
+        }
+        if (__syncthreads_or(!ok)) {
+            // A stage never arrived: record it, let copies in flight land, leave.
+            if (tid == 0) {
+                atomicOr(&g_device_errors, kErrWaitTimeout);
+                int ds = s;
+                uint32_t dp = phase;
+                for (int64_t m = n; m < npass && m < n + S; ++m) {
+                    if (!mbar_wait_bounded(&full[ds], dp, b.timeout_ns))
+                        atomicOr(&g_device_errors, kErrDrainTimeout);
+                    if (++ds == S) {
+                        ds = 0;
+                        dp ^= 1u;
+                    }
+                }
+            }
+            return;
+        }
+        // Every lane holds its vectors in registers now: refill this stage.
+        if (tid == 0 && n + S < npass) {
+            fence_proxy_async_smem();
+            issue(s, n + S);
+        }
+        // Phase B: shard sums in order of p, the factor; weight multiply and Phase C.
+        if constexpr (MIX) {
+            const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
+            const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
+            gpair_apply<Tag, NWQ, HQ>(xq, hq, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
+                                      pa, lane, rq);
+            gpair_apply<Tag, NWK, HK>(xk, hk, gk, P, reinterpret_cast<uint4 *>(a.y[1]) + t * a.ldy[1], nvk,
+                                      pa, lane, rk);
+        } else {
+            const float r = factor(combine_fast(&red[buf][32 * z], P, 1), z ? a.Df[1] : a.Df[0], a.eps);
+            gpair_apply<Tag, NWQ, HQ>(xq, hq, z ? gk : gq, P,
+                                      reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]),
+                                      z ? nvk : nvq, pa, lane, r);
+        }
+        buf ^= 1;
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- instances and launch
+
+// (NWQ, HQ, NWK, HK, MIX) of the instances that exist, per dtype:
+//   FP8 separate: (2, half) -- e.g. D = 5120 in 4 shards; (1) -- D = 4096 in 8;
+//                 (2) -- D = 4096 in 4;
+//   FP8 mixed:    Q (1, half), K (0, half) -- e.g. Dq = 5120, Dk = 1024 in 8;
+//   bf16 mixed:   Q (3), K (1) -- the same GQA widths in bf16.
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX>
+const void *gpair_fn() {
+    return reinterpret_cast<const void *>(&fused_gpair<Tag, NWQ, HQ, NWK, HK, MIX>);
+}
+
+const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix) {
+    if (dtype == 2) {
+        if (!mix && nwq == nwk && hq == hk) {
+            if (nwq == 2 && hq) return gpair_fn<E4M3Tag, 2, true, 2, true, false>();
+            if (nwq == 1 && !hq) return gpair_fn<E4M3Tag, 1, false, 1, false, false>();
+            if (nwq == 2 && !hq) return gpair_fn<E4M3Tag, 2, false, 2, false, false>();
+        }
+        if (mix && nwq == 1 && hq && nwk == 0 && hk) return gpair_fn<E4M3Tag, 1, true, 0, true, true>();
+    }
+    if (dtype == 1) {
+        if (mix && nwq == 3 && !hq && nwk == 1 && !hk) return gpair_fn<BF16Tag, 3, false, 1, false, true>();
+    }
+    return nullptr;
+}
+
+// Slots per lane of one tensor: whole slots, and whether the last (at most
+// 16 vectors) is split in halves (FP8 only); a ragged last slot of more than
+// 16 vectors is a guarded whole slot.
+void gpair_slots(int nv, int dtype, int *nw, bool *h) {
+    *nw = nv / 32;
+    const int rem = nv - 32 * *nw;
+    *h = false;
+    if (rem == 0) return;
+    if (dtype == 2 && rem <= 16) {
+        *h = true;
+        return;
+    }
+    *nw += 1;
+}
+
+int64_t gpair_gamma_slots(int dtype, int P, int nw, bool h) {
+    const int C = (dtype == 1 ? 8 : (dtype == 2 ? 16 : 4)) / 4;
+    return (int64_t)P * nw * C * 32 + (h ? (int64_t)P * (C / 2) * 32 : 0);
+}
+
+size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
+                        int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,
+                        uint32_t *gk4, uint32_t *stride) {
+    const int64_t q4 = gpair_gamma_slots(dtype, P, nwq, hq), k4 = gpair_gamma_slots(dtype, P, nwk, hk);
+    const int64_t base = ((int64_t)kGPairGammaOff + 16 * (q4 + k4) + 127) / 128 * 128;
+    const uint32_t st = bulk_stage_stride(qbytes, kbytes, 1);
+    if (stage_base) *stage_base = (uint32_t)base;
+    if (gq4) *gq4 = (uint32_t)q4;
+    if (gk4) *gk4 = (uint32_t)k4;
+    if (stride) *stride = st;
+    return (size_t)base + (size_t)stages * st;
+}
+
+cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix,
+                               const FusedArgs &a, int stages, int64_t grid, uint64_t timeout_ns,
+                               cudaStream_t s) {
+    const void *fn = fused_gpair_kernel(dtype, nwq, hq, nwk, hk, mix);
+    if (!fn || stages < 1 || stages > (int)kMaxStages || (a.P & 1) || a.P > 32 || a.K[0] != 1 ||
+        a.K[1] != 1)
+        return cudaErrorInvalidValue;
+    // The slots must cover every shard exactly as planned.
+    int w;
+    bool h;
+    gpair_slots(a.nv[0], dtype, &w, &h);
+    if (w != nwq || h != hq) return cudaErrorInvalidValue;
+    gpair_slots(a.nv[1], dtype, &w, &h);
+    if (w != nwk || h != hk) return cudaErrorInvalidValue;
+    const int block = 32 * (mix ? a.P / 2 : a.P);
+    if (block > 256) return cudaErrorInvalidValue;
+    const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
+    GPairArgs b;
+    b.stages = (uint32_t)stages;
+    b.qbytes = (uint32_t)(a.D[0] * es);
+    b.kbytes = (uint32_t)(a.D[1] * es);
+    b.timeout_ns = timeout_ns;
+    const size_t smem = gpair_smem_bytes(dtype, a.P, nwq, hq, nwk, hk, stages, b.qbytes, b.kbytes,
+                                         &b.stage_base, &b.gq4, &b.gk4, &b.stage_stride);
+    void *args[] = {const_cast<FusedArgs *>(&a), &b};
+    return launch(fn, dim3((unsigned)grid), dim3(block), smem, s, args);
+}
+
+}  // namespace qkn

@@ -36,7 +36,9 @@ TensorShape make_shape(int32_t D, int32_t P, int vec);
 // Kernel handles for occupancy queries and launches. Each returns nullptr if
 // the combination does not exist.
 // full: every lane holds exactly vmax vectors in every task (guard-free instance).
-const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, int *max_threads);
+// greg: gamma in registers, loaded with the row (no prefetch; vmax * vec <= 32).
+const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, bool greg,
+                             int *max_threads);
 const void *fused_generic_kernel(int dtype);
 // two: the instance for launches over two tensors.
 const void *stats_kernel(int dtype, int vmax, bool two);
@@ -44,8 +46,14 @@ const void *stats_kernel(int dtype, int vmax, bool two);
 const void *apply_kernel(int dtype, bool multi, bool two);
 
 // Launchers: enqueue one kernel; return the cudaError_t of the launch.
-cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, const FusedArgs &a,
-                             int block, int64_t grid, cudaStream_t s);
+cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, bool greg,
+                             const FusedArgs &a, int block, int64_t grid, cudaStream_t s);
+// Warp per token, rows in registers (qknorm_fused_warp.cu): P shards of one
+// group each, vq / vk vectors per lane per Q / K shard; block = 32 x tokens per CTA.
+const void *fused_warp_kernel(int dtype, int P, int vq, int vk);
+int fused_warp_max_threads();
+cudaError_t launch_fused_warp(int dtype, int P, int vq, int vk, const FusedArgs &a, int block,
+                              int64_t grid, cudaStream_t s);
 cudaError_t launch_fused_generic(int dtype, const FusedArgs &a, int block, int64_t grid,
                                  size_t smem, cudaStream_t s);
 // The split path's kernels take one or two tensors ("sides") per launch:
@@ -106,6 +114,18 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, int 
 const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs, bool kw);
 cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const FusedArgs &a,
                               int stages, int64_t grid, uint64_t timeout_ns, cudaStream_t s);
+// The shard-pair ring with gamma staged in shared memory (qknorm_gpair.cuh):
+// each warp takes two shards of one tensor (P warps per token) or, mixed, two
+// shards of Q and the same two of K (P / 2 warps); nw whole slots per lane
+// per shard and, for FP8, h = the last slot (<= 16 vectors) split in halves.
+const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix);
+void gpair_slots(int nv, int dtype, int *nw, bool *h);
+size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
+                        int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,
+                        uint32_t *gk4, uint32_t *stride);
+cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix,
+                               const FusedArgs &a, int stages, int64_t grid, uint64_t timeout_ns,
+                               cudaStream_t s);
 // The warp-per-row bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // wq warps take Q rows and wk warps take K rows in each CTA.
 struct RowsLayout {

@@ -102,6 +102,10 @@ WORKLOADS = {
         "prefill13b_e4m3", Ts=(8192,), Dq=5120, Dk=5120, P=4, eps=1e-6,
         dtype="e4m3", seed=3, x_sigma=1.5,
         note="13B-shaped prefill in FP8 E4M3: T=8192, D=5120, P=4"),
+    "gqa_e4m3": Workload(
+        "gqa_e4m3", Ts=(4096,), Dq=5120, Dk=1024, P=8, eps=1e-6,
+        dtype="e4m3", seed=13, x_sigma=1.5,
+        note="GQA-shaped prefill in FP8 E4M3: T=4096, Dq=5120, Dk=1024, P=8"),
     "split_large": Workload(
         "split_large", Ts=(65536,), Dq=4096, Dk=4096, P=8, eps=1e-5,
         dtype="bf16", seed=5, token_scale_log10=(-2.0, 2.0),

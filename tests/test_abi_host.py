@@ -282,6 +282,28 @@ def test_forced_variants(qk):
         qk.qknorm_force_variant(qk.VARIANT_WARP, 0)
         pl = qk.qknorm_plan_fwd(64, 4096, 4096, 4, qk.QKNORM_BF16, 148, 32)
         assert (pl["variant"], pl["block"], pl["grid"]) == (qk.VARIANT_WARP, 32, 64)
+        # The register-resident warp kernel: (vectors per lane per Q shard, per K shard).
+        assert (pl["vmax"], pl["vmax_k"], pl["smem_bytes"]) == (4, 4, 0)
+        pl = qk.qknorm_plan_fwd(64, 5120, 1024, 8, qk.QKNORM_BF16, 148, 32)
+        assert (pl["vmax"], pl["vmax_k"]) == (3, 1)
+        pl = qk.qknorm_plan_fwd(64, 4096, 4096, 4, qk.QKNORM_E4M3, 148, 32)
+        assert (pl["vmax"], pl["vmax_k"]) == (2, 2)
+        # Beyond 32 vectors per lane (5 + 5 in 4 shards), or shards of two lane
+        # groups: the looped one-warp form.
+        for shape in ((5120, 5120, 4), (4096, 4096, 1)):
+            pl = qk.qknorm_plan_fwd(64, *shape, qk.QKNORM_BF16, 148, 32)
+            assert (pl["variant"], pl["vmax"], pl["block"]) == (qk.VARIANT_WARP, 0, 32)
+        # The CTA kernel keeps gamma in registers while it is at most 32 floats
+        # per lane and a CTA takes one token.
+        qk.qknorm_force_variant(qk.VARIANT_CTA, 0)
+        pl = qk.qknorm_plan_fwd(64, 4096, 4096, 4, qk.QKNORM_BF16, 148, 2)
+        assert (pl["gamma_regs"], pl["prefetch"]) == (1, 0)
+        pl = qk.qknorm_plan_fwd(64, 5120, 5120, 4, qk.QKNORM_BF16, 148, 2)    # 5 x 8 floats
+        assert pl["gamma_regs"] == 0
+        qk.qknorm_force_variant(qk.VARIANT_CTA, 8)
+        pl = qk.qknorm_plan_fwd(64, 4096, 4096, 4, qk.QKNORM_BF16, 148, 2)    # 8 tokens per CTA
+        assert (pl["gamma_regs"], pl["prefetch"]) == (0, 1)
+        qk.qknorm_force_variant(qk.VARIANT_WARP, 0)
         qk.qknorm_force_variant(qk.VARIANT_CTA, 7)
         pl = qk.qknorm_plan_fwd(100, 4096, 4096, 4, qk.QKNORM_BF16, 148, 4)
         assert (pl["grid"], pl["prefetch"]) == (7, 1)
@@ -290,7 +312,7 @@ def test_forced_variants(qk):
             qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         with pytest.raises(qk.QKNormError):
-            qk.qknorm_force_variant(6, 0)
+            qk.qknorm_force_variant(7, 0)
         # The shard-pair ring: P warps, GQA-like shapes only.
         qk.qknorm_force_variant(qk.VARIANT_PAIR, 0)
         pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)
@@ -487,3 +509,32 @@ def test_noalloc_wrapper_checks_metadata(qk):
         qk.qknorm_split_noalloc(x.to(torch.float16), g, 4, 1e-6)               # unsupported dtype
     with pytest.raises(ValueError):
         qk.qknorm_split_noalloc(x, g, 4, 1e-6)                                 # host tensors
+
+
+def test_gpair_plans(qk):
+    """The shard-pair ring with staged gamma: separate warps for Q and K of one
+    geometry, mixed warps (both tensors) otherwise; FP8 splits a last slot of
+    at most 16 vectors in lane halves; the selector takes it for FP8 GQA-like
+    shapes only."""
+    qk.qknorm_force_variant(qk.VARIANT_GPAIR, 0)
+    try:
+        pl = qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)     # 80 vectors per shard
+        assert (pl["variant"], pl["block"], pl["vmax"], pl["vmax_k"], pl["half_slots"], pl["mixed"]) == \
+            (qk.VARIANT_GPAIR, 4 * 32, 2, 2, 3, 0)
+        pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)     # 40 and 8 vectors
+        assert (pl["block"], pl["vmax"], pl["vmax_k"], pl["half_slots"], pl["mixed"]) == (4 * 32, 1, 0, 3, 1)
+        pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)     # 80 and 16: guarded slots
+        assert (pl["block"], pl["vmax"], pl["vmax_k"], pl["half_slots"], pl["mixed"]) == (4 * 32, 3, 1, 0, 1)
+        assert pl["stages"] >= 2 and pl["smem_bytes"] > 24 * 1024            # gamma is staged
+        for bad in ((5120, 5120, 4, qk.QKNORM_BF16),    # no instance
+                    (3072, 3072, 3, qk.QKNORM_E4M3),    # odd P
+                    (4096, 4096, 1, qk.QKNORM_E4M3)):   # one shard
+            with pytest.raises(qk.QKNormError) as ei:
+                qk.qknorm_plan_fwd(4096, *bad, 148)
+            assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
+    assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR
+    assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_BULK
+    assert qk.qknorm_plan_fwd(64, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_CTA

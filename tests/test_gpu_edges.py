@@ -14,7 +14,7 @@ from gpu_util import bits, check_outputs, check_stats, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ("cta", "bulk", "rows", "pair", "warp", "generic")
+VARIANTS = ("cta", "bulk", "rows", "pair", "gpair", "warp", "generic")
 
 
 @pytest.fixture(scope="module")
@@ -39,7 +39,7 @@ def _inputs(wl, T):
 def _fwd(qk, wl, q, k, gq, gk, variant=None, grid=0):
     vid = {"cta": qk.VARIANT_CTA, "warp": qk.VARIANT_WARP, "generic": qk.VARIANT_GENERIC,
            "bulk": qk.VARIANT_BULK, "rows": qk.VARIANT_ROWS, "pair": qk.VARIANT_PAIR,
-           None: qk.VARIANT_AUTO}[variant]
+           "gpair": qk.VARIANT_GPAIR, None: qk.VARIANT_AUTO}[variant]
     qk.qknorm_force_variant(vid, grid)
     try:
         oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk),
@@ -84,7 +84,7 @@ def test_shapes_and_variants(qk, orc, shape):
         except qk.QKNormError as e:
             # Only the register-resident kernels (cta, bulk, pair) and the
             # shared-memory staged ones (bulk, rows, pair) have shape limits.
-            assert v in ("cta", "bulk", "rows", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
+            assert v in ("cta", "bulk", "rows", "pair", "gpair") and e.status == qk.QKNORM_ERR_UNSUPPORTED, str(e)
     base = outs["generic"]
     for v, (oq, ok) in outs.items():
         assert torch.equal(bits(oq), bits(base[0])), f"{v} Q differs from generic"

@@ -57,17 +57,17 @@ SHAPES = [
 
 
 @pytest.mark.parametrize("name,T,Dq,Dk,P", SHAPES)
-@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "pair", "generic"])
+@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "pair", "gpair", "warp", "generic"])
 def test_fp8_fused_and_split(qk, orc, name, T, Dq, Dk, P, variant):
     wl, q, k, gq, gk = _inputs(name, T, Dq, Dk, P, sigma=1.5)
-    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "pair": 5, "generic": 2}[variant]
+    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "pair": 5, "gpair": 6, "warp": 1, "generic": 2}[variant]
     qd, kd, gqd, gkd = to_device(q), to_device(k), to_device(gq), to_device(gk)
     qk.qknorm_force_variant(vid, 0)
     try:
         oq, ok = qk.qknorm_fwd(qd, kd, gqd, gkd, P, 1e-6)
         torch.cuda.synchronize()
     except qk.QKNormError as e:
-        assert variant in ("cta", "bulk", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
+        assert variant in ("cta", "bulk", "pair", "gpair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
         return
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
@@ -112,7 +112,7 @@ def _code_rows(T, D, seed):
     return x
 
 
-@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "generic"])
+@pytest.mark.parametrize("variant", ["auto", "cta", "bulk", "rows", "warp", "generic"])
 def test_fp8_every_code(qk, orc, variant):
     """Every finite E4M3 code in, subnormal-only rows (whose factor is large,
     so their outputs are far from zero) and rows near +-448, with gamma of
@@ -122,7 +122,7 @@ def test_fp8_every_code(qk, orc, variant):
     rng = np.random.default_rng(13)
     gq = rng.uniform(0.5, 1.5, D).astype(np.float32) * rng.choice([-1.0, 1.0], D).astype(np.float32)
     gk = rng.uniform(0.5, 1.5, D).astype(np.float32)
-    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "generic": 2}[variant]
+    vid = {"auto": -1, "cta": 0, "bulk": 3, "rows": 4, "warp": 1, "generic": 2}[variant]
     qk.qknorm_force_variant(vid, 0)
     try:
         oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(gq), to_device(gk), P, 1e-6)
@@ -144,12 +144,12 @@ def test_fp8_variants_bit_identical(qk, D, P):
     g = torch.from_numpy(np.random.default_rng(23).uniform(-1.5, 1.5, D).astype(np.float32)).cuda()
     qd, kd = to_device(q), to_device(k)
     outs = {}
-    for name, vid in (("cta", 0), ("bulk", 3), ("rows", 4), ("pair", 5), ("generic", 2)):
+    for name, vid in (("cta", 0), ("bulk", 3), ("rows", 4), ("pair", 5), ("gpair", 6), ("warp", 1), ("generic", 2)):
         qk.qknorm_force_variant(vid, 0)
         try:
             outs[name] = qk.qknorm_fwd(qd, kd, g, g, P, 1e-6)
         except qk.QKNormError as e:
-            assert name in ("cta", "bulk", "pair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
+            assert name in ("cta", "bulk", "pair", "gpair") and e.status == qk.QKNORM_ERR_UNSUPPORTED
         finally:
             qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     outs["split"] = tuple(qk.qknorm_apply(x, g, qk.qknorm_partial_sumsq(x, P), 1e-6) for x in (qd, kd))
@@ -168,13 +168,13 @@ def test_fp8_saturation(qk, orc):
     rng = np.random.default_rng(33)
     g = rng.uniform(0.5, 1.5, D).astype(np.float32)
     g[::7] *= -300.0                                   # these channels overflow the format
-    for vid in (-1, 0, 2, 3, 4, 5):
+    for vid in (-1, 0, 1, 2, 3, 4, 5, 6):
         qk.qknorm_force_variant(vid, 0)
         try:
             oq, ok = qk.qknorm_fwd(to_device(q), to_device(k), to_device(g), to_device(g), P, 1e-6)
             torch.cuda.synchronize()
         except qk.QKNormError as e:
-            assert vid in (0, 3, 5) and e.status == qk.QKNORM_ERR_UNSUPPORTED
+            assert vid in (0, 3, 5, 6) and e.status == qk.QKNORM_ERR_UNSUPPORTED
             continue
         finally:
             qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
@@ -220,3 +220,53 @@ def test_fp8_bench_workloads_full_size(qk, orc, name):
                           f"{name} {tag} rows {r0}..")
     del q, k, oq, ok, aq, ak
     torch.cuda.empty_cache()
+
+
+GPAIR_SHAPES = [
+    # T, Dq, Dk, P, dtype: separate warps with half slots; mixed with half slots;
+    # separate, one whole slot; mixed bf16 with guarded ragged slots
+    (257, 5120, 5120, 4, "e4m3"),
+    (301, 5120, 1024, 8, "e4m3"),
+    (199, 4096, 4096, 8, "e4m3"),
+    (2 * 148 + 5, 4096, 4096, 4, "e4m3"),
+    (77, 5120, 1024, 8, "bf16"),
+]
+
+
+@pytest.mark.parametrize("T,Dq,Dk,P,dtype", GPAIR_SHAPES)
+def test_gpair_bit_identical_and_oracle(qk, orc, T, Dq, Dk, P, dtype):
+    """The shard-pair ring with staged gamma on every instance: the default
+    plan, forced small grids (each CTA walks many tokens through its ring) and
+    row-strided inputs (Q and K inside one buffer), bit-identical to the
+    generic kernel and within tolerance of the oracle."""
+    wl = W.custom(f"gp{Dq}_{Dk}_{P}", T, Dq, Dk, P, dtype=dtype, seed=Dq + Dk + P + T, x_sigma=1.5)
+    q, k = W.gen_rows(wl, "q", range(T)), W.gen_rows(wl, "k", range(T))
+    gq, gk = W.gen_gamma(wl, "q"), W.gen_gamma(wl, "k")
+    qd, kd, gqd, gkd = to_device(q), to_device(k), to_device(gq), to_device(gk)
+    outs = {}
+    for name, vid, grid in (("generic", 2, 0), ("gpair", 6, 0), ("gpair_g7", 6, 7), ("gpair_g148", 6, 148)):
+        qk.qknorm_force_variant(vid, grid)
+        try:
+            outs[name] = qk.qknorm_fwd(qd, kd, gqd, gkd, P, 1e-6)
+            torch.cuda.synchronize()
+        finally:
+            qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    # Strided: Q and K as column slices of one [T, Dq + Dk + 64] buffer, in place.
+    pad = 64
+    buf = torch.cat([qd, kd, torch.zeros_like(kd[:, :pad])], dim=1).contiguous()
+    qs, ks = buf[:, :Dq], buf[:, Dq:Dq + Dk]
+    qk.qknorm_force_variant(6, 0)
+    try:
+        qk.qknorm_fwd_strided(qs, ks, gqd, gkd, P, 1e-6, out_q=qs, out_k=ks)
+        torch.cuda.synchronize()
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    outs["gpair_strided"] = (qs.contiguous(), ks.contiguous())
+    ref = outs["generic"]
+    for name, (oq, ok) in outs.items():
+        assert torch.equal(bits(oq), bits(ref[0])), f"{name} q"
+        assert torch.equal(bits(ok), bits(ref[1])), f"{name} k"
+    assert torch.equal(bits(buf[:, Dq + Dk:]), bits(torch.zeros_like(kd[:, :pad])))   # padding untouched
+    yq, yk, _, _ = orc.qknorm(q, k, gq, gk, P, EPS, dtype, nthreads=8)
+    check_outputs(to_host(ref[0]), yq, dtype, f"gpair {Dq}/{Dk} q")
+    check_outputs(to_host(ref[1]), yk, dtype, f"gpair {Dq}/{Dk} k")
