@@ -488,7 +488,8 @@ def fp8_prefill(torch, qk, device, peak, steps=200):
     """The 13B-shaped prefill (T = 8192, Dq = Dk = 5120, P = 4) in FP8 E4M3:
     E4M3 in and out, fp32 statistics; half the bytes of the bf16 step. Also
     the large split shape in FP8 (T = 65536, D = 4096, P = 8: one vector per
-    lane, where the shard-pair ring takes Q and K)."""
+    lane, where the shard-pair ring takes Q and K) and the GQA shape in FP8
+    (T = 4096, Dq = 5120, Dk = 1024, P = 8)."""
     wl = W.WORKLOADS["prefill13b_e4m3"]
     gq = torch.from_numpy(W.gen_gamma(wl, "q")).to(device)
     gk = torch.from_numpy(W.gen_gamma(wl, "k")).to(device)
@@ -500,6 +501,12 @@ def fp8_prefill(torch, qk, device, peak, steps=200):
     r = {"workload": "T=65536, Dq=Dk=4096, P=8 in FP8 E4M3"}
     r.update(_fp8_case(torch, qk, device, peak, wl8, g8q, g8k, steps // 4))
     out["split_large_e4m3"] = r
+    wlg = W.WORKLOADS["gqa_e4m3"]
+    ggq = torch.from_numpy(W.gen_gamma(wlg, "q")).to(device)
+    ggk = torch.from_numpy(W.gen_gamma(wlg, "k")).to(device)
+    r = {"workload": "GQA-shaped prefill in FP8 E4M3: T=4096, Dq=5120, Dk=1024, P=8"}
+    r.update(_fp8_case(torch, qk, device, peak, wlg, ggq, ggk, steps))
+    out["gqa_e4m3"] = r
     return out
 
 

@@ -346,35 +346,23 @@ bool gpair_fits(const Shapes &sh, int32_t P, int32_t dtype, GPairShape *g) {
     gpair_slots(sh.q.nv, dtype, &g->nwq, &g->hq);
     gpair_slots(sh.k.nv, dtype, &g->nwk, &g->hk);
     g->mix = sh.q.nv != sh.k.nv;
-    if ((g->mix ? P / 2 : P) * kLanes > 256) return false;
+    if ((g->mix ? P / 2 : P) * kLanes > gpair_max_threads()) return false;
     return fused_gpair_kernel(dtype, g->nwq, g->hq, g->nwk, g->hk, g->mix) != nullptr;
 }
 
-// Stages of the staged-gamma ring: the most bytes in flight per SM (CTAs x
-// stages x stage bytes) with at least two stages and at most four, within the
-// SM's threads and shared memory; ties go to more CTAs.
-void gpair_stages(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, const GPairShape &g, int block,
-                  qknorm_plan *pl) {
-    int bestS = 2;
-    int64_t best = -1;
-    for (int S = 2; S <= 4; ++S) {
-        const size_t sm = gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, S, (int64_t)Dq * elem_of(dtype),
-                                           (int64_t)Dk * elem_of(dtype), nullptr, nullptr, nullptr, nullptr);
-        if (sm > (size_t)kSmemPerCta) break;
-        int ctas = (int)(kSmemPerSm / (sm + kSmemReservedPerCta));
-        if (ctas > kThreadsPerSm / block) ctas = kThreadsPerSm / block;
-        if (ctas < 1) break;
-        const int64_t inflight = (int64_t)ctas * S;
-        if (inflight > best) {
-            best = inflight;
-            bestS = S;
-        }
-    }
-    if (g_tune_stages > 0) bestS = g_tune_stages;
-    pl->stages = bestS;
-    pl->smem_bytes = (int64_t)gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, bestS,
-                                               (int64_t)Dq * elem_of(dtype), (int64_t)Dk * elem_of(dtype),
-                                               nullptr, nullptr, nullptr, nullptr);
+// Stages of the staged-gamma ring: two per CTA, so that as many CTAs as the
+// SM's shared memory, registers and threads allow are resident (measured at
+// the 13B shape in FP8: 3 CTAs x 2 stages 80.8 %, 3 x 3 78.6 %; D = 4096,
+// P = 4: 88.8 % vs 84.0 %; groups of warps sharing one staged gamma in a
+// larger CTA were slower at every setting); three if two do not fit.
+void gpair_stages(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, const GPairShape &g, qknorm_plan *pl) {
+    const int64_t qb = (int64_t)Dq * elem_of(dtype), kb = (int64_t)Dk * elem_of(dtype);
+    int S = g_tune_stages > 0 ? g_tune_stages : 2;
+    pl->block = (g.mix ? P / 2 : P) * kLanes;
+    pl->tokens_per_stage = 1;
+    pl->stages = S;
+    pl->smem_bytes = (int64_t)gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, S, qb, kb, nullptr,
+                                               nullptr, nullptr, nullptr);
 }
 
 // Static part of the plan: which kernel, block size, template width, stages.
@@ -422,15 +410,17 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         const bool ragged = !pl->full_lanes && dtype != QKNORM_E4M3;
         const bool kpairs = pair_fits(sh, P, dtype) && pair_kw(sh) && pair_greg(sh, dtype) &&
                             (dtype == QKNORM_E4M3 ? pair_vq(sh) == 1 : ragged);
-        // FP8 with Q and K shards of different widths (GQA-like) takes the
-        // mixed shard-pair ring with gamma staged in shared memory: P/2 warps
-        // per token, each with two Q and two K shards (measured at T = 4096,
-        // 5120/1024, P = 8: 43 % vs 37 % for the shard-pair ring with gamma in
-        // registers).
+        // FP8 takes the shard-pair ring with gamma staged in shared memory
+        // (two shards per warp, no gamma registers, so 3 CTAs fit an SM) where
+        // a lane holds more than one vector per shard or Q and K shards differ
+        // (mixed warps). Measured: 13B shape 80.8 % vs 73.9 % for the bulk
+        // ring; D = 4096, P = 4, T = 16384: 88.8 % vs 78.1 %; GQA widths, P = 8:
+        // 45.8 % vs 37 %. At one vector per lane (D = 4096, P = 8) the
+        // shard-pair ring with gamma in registers stays (82.5 % vs 76 %).
         GPairShape gp;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
-        else if (dtype == QKNORM_E4M3 && gpair_fits(sh, P, dtype, &gp) && gp.mix)
+        else if (dtype == QKNORM_E4M3 && gpair_fits(sh, P, dtype, &gp) && (gp.mix || gp.hq || gp.nwq >= 2))
             variant = QKNORM_VARIANT_GPAIR;
         else if (pair_fits(sh, P, dtype) && !pair_kw(sh) && sh.q.nv > kLanes)
             variant = QKNORM_VARIANT_PAIR;
@@ -488,14 +478,13 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         GPairShape g;
         if (!gpair_fits(sh, P, dtype, &g)) return QKNORM_ERR_UNSUPPORTED;
         pl->variant = QKNORM_VARIANT_GPAIR;
-        pl->block = (g.mix ? P / 2 : P) * kLanes;
         pl->vmax = g.nwq;
         pl->vmax_k = g.nwk;
         pl->half_slots = (g.hq ? 1 : 0) | (g.hk ? 2 : 0);
         pl->mixed = g.mix ? 1 : 0;
-        pl->tokens_per_stage = 1;
-        gpair_stages(Dq, Dk, P, dtype, g, pl->block, pl);
-        if (pl->stages < 1 || pl->stages > bulk_max_stages() || pl->smem_bytes > kSmemPerCta)
+        gpair_stages(Dq, Dk, P, dtype, g, pl);
+        if (pl->stages < 1 || pl->stages > bulk_max_stages() || pl->smem_bytes > kSmemPerCta ||
+            pl->block > gpair_max_threads())
             return QKNORM_ERR_UNSUPPORTED;
         return QKNORM_OK;
     }
@@ -646,7 +635,7 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, kRegsHint, pl);
     if (*status != QKNORM_OK) return cudaSuccess;
     if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS ||
-        pl->variant == QKNORM_VARIANT_PAIR) {
+        pl->variant == QKNORM_VARIANT_PAIR || pl->variant == QKNORM_VARIANT_GPAIR) {
         int regs = kRegsHint;
         e = kernel_regs(plan_kernel(*pl, dtype, P, true), &regs);
         if (e != cudaSuccess) return e;

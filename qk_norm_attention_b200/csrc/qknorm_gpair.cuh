@@ -59,52 +59,43 @@ struct GSlots {
     __host__ __device__ static int64_t total(int P) { return whole(P) + (H ? (int64_t)P * CH * 32 : 0); }
 };
 
-// Source of staged-gamma slot j of one tensor (float offset into gamma), or
-// -1 for a slot whose vector does not exist.
+// Copy one tensor's gamma into its permuted shared-memory layout. Warp w
+// takes shards w, w + nwarps, ...; lane l copies its own slots of a shard
+// (vector l + 32 i, chunk c; and its half-slot chunks), all of a shard's
+// loads issued before any store, with the slot indices fixed at compile time
+// so that only the shard offset is computed at run time. Slots of vectors
+// the shard does not have are zero.
 template <class Tag, int NW, bool H>
-__device__ __forceinline__ int64_t gpair_gamma_src(int j, int whole, int nv) {
+__device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, int P, int nv, int warp,
+                                                  int nwarps, int lane) {
     using G = GSlots<Tag, NW, H>;
     constexpr int VEC = Tag::kVec;
-    if (j < whole) {
-        const int l = j & 31;
-        int r = j >> 5;
-        const int c = r % G::C;
-        r /= G::C;
-        const int i = r % (NW > 0 ? NW : 1);
-        const int p = r / (NW > 0 ? NW : 1);
-        const int v = l + 32 * i;
-        return v < nv ? ((int64_t)p * nv + v) * VEC + 4 * c : -1;
-    }
-    const int jj = j - whole;
-    const int l = jj & 31;
-    const int r = jj >> 5;
-    const int c = r % G::CH;
-    const int p = r / G::CH;
-    const int v = 32 * NW + (l & 15);
-    return v < nv ? ((int64_t)p * nv + v) * VEC + (VEC / 2) * (l >> 4) + 4 * c : -1;
-}
-
-// Copy one tensor's gamma into its permuted shared-memory layout. Each thread
-// issues kStageLoads independent loads before it stores any, so the copy
-// costs a few L2 round trips, not one per slot.
-template <class Tag, int NW, bool H>
-__device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, int P, int nv, int tid,
-                                                  int nthreads) {
-    using G = GSlots<Tag, NW, H>;
-    constexpr int kStageLoads = 8;
-    const int whole = (int)G::whole(P), total = (int)G::total(P);
-    for (int j0 = tid; j0 < total; j0 += kStageLoads * nthreads) {
-        float4 val[kStageLoads];
+    constexpr int NL = NW * G::C + (H ? G::CH : 0);     // float4 slots per lane per shard
+    const int64_t whole = G::whole(P);
+    const int hv = 32 * NW + (lane & 15);
+    for (int p = warp; p < P; p += nwarps) {
+        const float4 *gp = reinterpret_cast<const float4 *>(g + (int64_t)p * nv * VEC);
+        float4 val[NL > 0 ? NL : 1];
 #pragma unroll
-        for (int u = 0; u < kStageLoads; ++u) {
-            const int j = j0 + u * nthreads;
-            const int64_t src = j < total ? gpair_gamma_src<Tag, NW, H>(j, whole, nv) : -1;
-            val[u] = src >= 0 ? __ldg(reinterpret_cast<const float4 *>(g + src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < NW; ++i)
+#pragma unroll
+            for (int c = 0; c < G::C; ++c) {
+                const int v = lane + 32 * i;
+                val[i * G::C + c] = v < nv ? __ldg(gp + v * G::C + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        if constexpr (H) {
+#pragma unroll
+            for (int c = 0; c < G::CH; ++c)
+                val[NW * G::C + c] = hv < nv ? __ldg(gp + hv * G::C + (lane >> 4) * G::CH + c)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < kStageLoads; ++u) {
-            const int j = j0 + u * nthreads;
-            if (j < total) dst[j] = val[u];
+        for (int i = 0; i < NW; ++i)
+#pragma unroll
+            for (int c = 0; c < G::C; ++c) dst[((p * NW + i) * G::C + c) * 32 + lane] = val[i * G::C + c];
+        if constexpr (H) {
+#pragma unroll
+            for (int c = 0; c < G::CH; ++c) dst[whole + (p * G::CH + c) * 32 + lane] = val[NW * G::C + c];
         }
     }
 }
@@ -217,8 +208,10 @@ __device__ __forceinline__ float butterfly_quad(float a, float b, float c, float
 // Separate form: NW whole slots (+ half slot H) per lane per shard for both
 // tensors (their shards have the same vector count).
 // Mixed form: Q with (NWQ, HQ), K with (NWK, HK), both in every warp.
+constexpr int kGPairMaxThreads = 256;
+
 template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX>
-__global__ void __launch_bounds__(256, 1) fused_gpair(const FusedArgs a, const GPairArgs b) {
+__global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedArgs a, const GPairArgs b) {
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     float(*red)[64] = reinterpret_cast<float(*)[64]>(smem + kBarBytes);
@@ -264,8 +257,8 @@ __global__ void __launch_bounds__(256, 1) fused_gpair(const FusedArgs a, const G
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
     // Gamma of both tensors into shared memory (visible after the first barrier).
-    gpair_stage_gamma<Tag, NWQ, HQ>(gq, a.g[0], P, nvq, tid, blockDim.x);
-    gpair_stage_gamma<Tag, NWK, HK>(gk, a.g[1], P, nvk, tid, blockDim.x);
+    gpair_stage_gamma<Tag, NWQ, HQ>(gq, a.g[0], P, nvq, warp, blockDim.x >> 5, lane);
+    gpair_stage_gamma<Tag, NWK, HK>(gk, a.g[1], P, nvk, warp, blockDim.x >> 5, lane);
 
     constexpr int AQ = NWQ > 0 ? NWQ : 1, AK = NWK > 0 ? NWK : 1;
     int s = 0;
@@ -392,6 +385,8 @@ size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, in
     return (size_t)base + (size_t)stages * st;
 }
 
+int gpair_max_threads() { return kGPairMaxThreads; }
+
 cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix,
                                const FusedArgs &a, int stages, int64_t grid, uint64_t timeout_ns,
                                cudaStream_t s) {
@@ -407,7 +402,7 @@ cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bo
     gpair_slots(a.nv[1], dtype, &w, &h);
     if (w != nwk || h != hk) return cudaErrorInvalidValue;
     const int block = 32 * (mix ? a.P / 2 : a.P);
-    if (block > 256) return cudaErrorInvalidValue;
+    if (block > kGPairMaxThreads) return cudaErrorInvalidValue;
     const int64_t es = dtype == 1 ? 2 : (dtype == 2 ? 1 : 4);
     GPairArgs b;
     b.stages = (uint32_t)stages;

@@ -123,6 +123,7 @@ void gpair_slots(int nv, int dtype, int *nw, bool *h);
 size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
                         int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,
                         uint32_t *gk4, uint32_t *stride);
+int gpair_max_threads();
 cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix,
                                const FusedArgs &a, int stages, int64_t grid, uint64_t timeout_ns,
                                cudaStream_t s);

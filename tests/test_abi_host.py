@@ -198,15 +198,16 @@ def test_valid_call_without_gpu_reports_cuda_error(qk):
 
 def test_auto_k_pairs(qk):
     """The selector puts K shards in pairs (P warps per token) for FP8 at one
-    vector per lane and for ragged bf16 lanes, and keeps the ring with 2P
-    warps for full bf16 lanes and for FP8 at two or more vectors per lane."""
+    vector per lane and for ragged bf16 lanes, keeps the ring with 2P warps
+    for full bf16 lanes, and gives FP8 at two or more vectors per lane the
+    shard pairs with gamma staged in shared memory."""
     qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
     cases = [((65536, 4096, 4096, 8, qk.QKNORM_E4M3), (qk.VARIANT_PAIR, 1)),
              ((16384, 2048, 2048, 4, qk.QKNORM_E4M3), (qk.VARIANT_PAIR, 1)),
              ((8192, 5120, 4096, 8, qk.QKNORM_BF16), (qk.VARIANT_PAIR, 1)),
-             ((16384, 4096, 4096, 4, qk.QKNORM_E4M3), (qk.VARIANT_BULK, 0)),
+             ((16384, 4096, 4096, 4, qk.QKNORM_E4M3), (qk.VARIANT_GPAIR, 0)),
              ((65536, 4096, 4096, 8, qk.QKNORM_BF16), (qk.VARIANT_BULK, 0)),
-             ((8192, 5120, 5120, 4, qk.QKNORM_E4M3), (qk.VARIANT_BULK, 0))]
+             ((8192, 5120, 5120, 4, qk.QKNORM_E4M3), (qk.VARIANT_GPAIR, 0))]
     for shape, (variant, kp) in cases:
         pl = qk.qknorm_plan_fwd(*shape, 148, 2)
         assert (pl["variant"], pl["k_pairs"]) == (variant, kp), shape
@@ -341,7 +342,9 @@ def test_forced_variants(qk):
             qk.qknorm_plan_fwd(10, 4096, 4096, 2, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
         with pytest.raises(qk.QKNormError):
-            qk.qknorm_set_tuning(tokens_per_stage=4)
+            qk.qknorm_set_tuning(tokens_per_stage=3)
+        with pytest.raises(qk.QKNormError):
+            qk.qknorm_set_tuning(tokens_per_stage=-1)
         with pytest.raises(qk.QKNormError) as ei:      # 64 tasks do not fit one CTA
             qk.qknorm_plan_fwd(10, 4096, 4096, 32, qk.QKNORM_BF16, 148)
         assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
@@ -525,7 +528,10 @@ def test_gpair_plans(qk):
         assert (pl["block"], pl["vmax"], pl["vmax_k"], pl["half_slots"], pl["mixed"]) == (4 * 32, 1, 0, 3, 1)
         pl = qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)     # 80 and 16: guarded slots
         assert (pl["block"], pl["vmax"], pl["vmax_k"], pl["half_slots"], pl["mixed"]) == (4 * 32, 3, 1, 0, 1)
-        assert pl["stages"] >= 2 and pl["smem_bytes"] > 24 * 1024            # gamma is staged
+        assert pl["stages"] == 2 and pl["smem_bytes"] > 24 * 1024            # gamma is staged
+        qk.qknorm_set_tuning(stages=3)
+        assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["stages"] == 3
+        qk.qknorm_set_tuning()
         for bad in ((5120, 5120, 4, qk.QKNORM_BF16),    # no instance
                     (3072, 3072, 3, qk.QKNORM_E4M3),    # odd P
                     (4096, 4096, 1, qk.QKNORM_E4M3)):   # one shard
@@ -534,7 +540,11 @@ def test_gpair_plans(qk):
             assert ei.value.status == qk.QKNORM_ERR_UNSUPPORTED
     finally:
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+        qk.qknorm_set_tuning()
     assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
     assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR
-    assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_BULK
+    assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
+    assert qk.qknorm_plan_fwd(8192, 4096, 4096, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
+    assert qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_PAIR
+    assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_BULK
     assert qk.qknorm_plan_fwd(64, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_CTA
