@@ -59,23 +59,18 @@ struct GSlots {
     __host__ __device__ static int64_t total(int P) { return whole(P) + (H ? (int64_t)P * CH * 32 : 0); }
 };
 
-// Copy one tensor's gamma into its permuted shared-memory layout. Warp w
-// takes shards w, w + nwarps, ...; lane l copies its own slots of a shard
-// (vector l + 32 i, chunk c; and its half-slot chunks), all of a shard's
-// loads issued before any store, with the slot indices fixed at compile time
-// so that only the shard offset is computed at run time. Slots of vectors
-// the shard does not have are zero.
+// One tensor's gamma slots of shard p that lane `lane` copies into the
+// permuted shared-memory layout: vector l + 32 i, chunk c of each whole slot,
+// and the lane's half-slot chunks; zero for vectors the shard does not have.
 template <class Tag, int NW, bool H>
-__device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, int P, int nv, int warp,
-                                                  int nwarps, int lane) {
+struct GStage {
     using G = GSlots<Tag, NW, H>;
-    constexpr int VEC = Tag::kVec;
-    constexpr int NL = NW * G::C + (H ? G::CH : 0);     // float4 slots per lane per shard
-    const int64_t whole = G::whole(P);
-    const int hv = 32 * NW + (lane & 15);
-    for (int p = warp; p < P; p += nwarps) {
+    static constexpr int NL = NW * G::C + (H ? G::CH : 0);   // float4 slots per lane per shard
+
+    __device__ __forceinline__ static void load(float4 (&val)[NL > 0 ? NL : 1], const float *g, int p, int nv,
+                                                int lane) {
+        constexpr int VEC = Tag::kVec;
         const float4 *gp = reinterpret_cast<const float4 *>(g + (int64_t)p * nv * VEC);
-        float4 val[NL > 0 ? NL : 1];
 #pragma unroll
         for (int i = 0; i < NW; ++i)
 #pragma unroll
@@ -84,11 +79,17 @@ __device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, i
                 val[i * G::C + c] = v < nv ? __ldg(gp + v * G::C + c) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         if constexpr (H) {
+            const int hv = 32 * NW + (lane & 15);
 #pragma unroll
             for (int c = 0; c < G::CH; ++c)
                 val[NW * G::C + c] = hv < nv ? __ldg(gp + hv * G::C + (lane >> 4) * G::CH + c)
                                              : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+    }
+
+    __device__ __forceinline__ static void store(float4 *dst, const float4 (&val)[NL > 0 ? NL : 1], int P, int p,
+                                                 int lane) {
+        const int64_t whole = G::whole(P);
 #pragma unroll
         for (int i = 0; i < NW; ++i)
 #pragma unroll
@@ -97,6 +98,25 @@ __device__ __forceinline__ void gpair_stage_gamma(float4 *dst, const float *g, i
 #pragma unroll
             for (int c = 0; c < G::CH; ++c) dst[whole + (p * G::CH + c) * 32 + lane] = val[NW * G::C + c];
         }
+    }
+};
+
+// Copy both tensors' gamma into their permuted shared-memory layouts. Warp w
+// takes shards w, w + nwarps, ...; lane l copies its own slots of a shard of
+// Q and of K, all of those loads issued before any store (one L2 round trip
+// per shard, not one per slot), with the slot indices fixed at compile time
+// so that only the shard offset is computed at run time.
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK>
+__device__ __forceinline__ void gpair_stage_gamma(float4 *gq, float4 *gk, const float *gammaq, const float *gammak,
+                                                  int P, int nvq, int nvk, int warp, int nwarps, int lane) {
+    using SQ = GStage<Tag, NWQ, HQ>;
+    using SK = GStage<Tag, NWK, HK>;
+    for (int p = warp; p < P; p += nwarps) {
+        float4 vq[SQ::NL > 0 ? SQ::NL : 1], vk[SK::NL > 0 ? SK::NL : 1];
+        SQ::load(vq, gammaq, p, nvq, lane);
+        SK::load(vk, gammak, p, nvk, lane);
+        SQ::store(gq, vq, P, p, lane);
+        SK::store(gk, vk, P, p, lane);
     }
 }
 
@@ -257,8 +277,7 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
     // Gamma of both tensors into shared memory (visible after the first barrier).
-    gpair_stage_gamma<Tag, NWQ, HQ>(gq, a.g[0], P, nvq, warp, blockDim.x >> 5, lane);
-    gpair_stage_gamma<Tag, NWK, HK>(gk, a.g[1], P, nvk, warp, blockDim.x >> 5, lane);
+    gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp, blockDim.x >> 5, lane);
 
     constexpr int AQ = NWQ > 0 ? NWQ : 1, AK = NWK > 0 ? NWK : 1;
     int s = 0;
