@@ -25,16 +25,10 @@
 
 namespace qkn {
 
-// Registers for 4 resident blocks per SM where a lane's R x VMAX vectors of
-// a turn leave room for it without spilling (at most 7), else the default
-// (measured on one tensor-parallel rank's slices at 2 ranks, 2 x 2560
-// columns: 66.6 -> 74.3 % of the HBM peak for the statistics launch).
-constexpr int stats_min_blocks(int vmax, int r) { return vmax * r <= 7 ? 4 : 1; }
-
 // TWO: the launch may carry two sides (one-side launches compile without
 // the selection, which costs registers).
 template <class Tag, int VMAX, int R, bool TWO>
-__global__ void __launch_bounds__(256, stats_min_blocks(VMAX, R)) stats_k(const StatsArgs a) {
+__device__ __forceinline__ void stats_body(const StatsArgs &a) {
     constexpr int VEC = Tag::kVec;
     pdl_wait();
     pdl_trigger();
@@ -110,6 +104,25 @@ __global__ void __launch_bounds__(256, stats_min_blocks(VMAX, R)) stats_k(const 
             }
         }
     }
+}
+
+template <class Tag, int VMAX, int R, bool TWO>
+__global__ void __launch_bounds__(256) stats_k(const StatsArgs a) {
+    stats_body<Tag, VMAX, R, TWO>(a);
+}
+
+// The same kernel with registers for 4 resident blocks per SM, for the
+// instances whose lane holds at most 7 vectors per turn (no spills; measured
+// on one tensor-parallel rank's slices at 2 ranks, 2 x 2560 columns: 66.6 ->
+// 74.3 % of the HBM peak for the statistics launch). The others keep the
+// bound above: stating a minimum of one block makes the compiler take more
+// registers (80 -> 102 at 2 vectors x 4 tasks, 95 -> 114 us on T = 65536,
+// D = 4096, P = 8).
+constexpr bool stats_four_blocks(int vmax, int r) { return vmax * r <= 7; }
+
+template <class Tag, int VMAX, int R, bool TWO>
+__global__ void __launch_bounds__(256, 4) stats_k4(const StatsArgs a) {
+    stats_body<Tag, VMAX, R, TWO>(a);
 }
 
 // The statistics of token t are nb blocks of Pb shard sums, block b at
@@ -205,8 +218,12 @@ constexpr int stats_r(int vmax) { return vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1); }
 
 template <class Tag, int V>
 const void *stats_fn(bool two) {
-    return two ? reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), true>)
-               : reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), false>);
+    if constexpr (stats_four_blocks(V, stats_r(V)))
+        return two ? reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), true>)
+                   : reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), false>);
+    else
+        return two ? reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), true>)
+                   : reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), false>);
 }
 
 template <class Tag>
