@@ -167,14 +167,10 @@ __device__ __forceinline__ void apply_rows(const void *x, const float *g, const 
                 if (v < rowvec) xv[u] = ld_stream(src + v);
             }
             if (v0 == 0) {
-                // Phase B: S = sum of the shard sums, in order of the shard.
-                float S = 0.f;
-                const float *st = stats + t * Pb;
-                for (int b = 0; b < nb; ++b, st += sg) {
-#pragma unroll 8
-                    for (int p = 0; p < Pb; ++p) S = __fadd_rn(S, __ldg(st + p));
-                }
-                r = factor(S, Df, eps);
+                // Phase B: S = sum of the shard sums in order of the global
+                // shard index, loaded by the warp's lanes at once (tpr is a
+                // multiple of 32, so a warp's lanes share the row).
+                r = factor(stat_sum_warp(stats, t, Pb, nb, sg, threadIdx.x & 31), Df, eps);
             }
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {

@@ -61,6 +61,11 @@ CASES = [
     ("one", 65, 4096, 1024, 4, "bf16", 1),
     ("wide_narrow", 333, 8192, 1024, 2, "bf16", 2),     # one side a CTA per row, one several rows
     ("fp8_narrow", 77, 2048, 1536, 8, "e4m3", 2),
+    ("13b", 8 * 148 + 5, 5120, 5120, 8, "bf16", 8),
+    ("fold64", 97, 4096, 4096, 64, "bf16", 8),         # 64 shard sums per row: two rounds of 32
+    ("fold40", 51, 2560, 640, 40, "f32", 4),           # 40 sums: a round of 32 and one of 8
+    ("v4", 333, 4096, 4096, 8, "bf16", 4),             # 128-vector slices: 4 vectors per lane
+    ("fp8_v4", 150, 4096, 4096, 8, "e4m3", 2),
 ]
 
 
@@ -96,7 +101,7 @@ def test_tp_slices_equal_fused(qk, name, T, Dq, Dk, P, dtype, ranks, two):
     torch.cuda.synchronize()
     assert torch.equal(bits(tq), bits(oq)), "TP Q slices differ from the fused Q"
     assert torch.equal(bits(tk), bits(ok)), "TP K slices differ from the fused K"
-    if name in ("gqa", "tiny"):
+    if name in ("gqa", "tiny", "fold64", "fold40"):
         orc = oracle.get()
         eps = float(np.float32(1e-6))
         yq, _ = orc.rmsnorm(q, gq, P, eps, dtype, nthreads=8)
