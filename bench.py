@@ -401,6 +401,31 @@ def decode_c_abi(wl):
     return out
 
 
+def copy_floor(peak):
+    """A plain streaming copy and a plain streaming read of the byte counts
+    the workloads move in one launch (the yardstick built beside the
+    library, `copy_floor`): device us per launch, back to back with eight
+    rotating buffer sets, and the fraction of the measured peak they reach.
+    Sizes: 21 MB (one tensor-parallel rank's statistics read at 8 ranks),
+    42 MB (its apply), 50.3 MB (FP8 GQA, T = 4096), 100.7 MB (GQA),
+    168 MB (FP8 13B), 336 MB (13B)."""
+    exe = os.path.join(ROOT, "qk_norm_attention_b200", "copy_floor")
+    if not os.path.exists(exe):
+        return {"unavailable": "copy_floor not built"}
+    import subprocess
+    sizes = ["21", "42", "50.3", "100.7", "168", "336"]
+    r = subprocess.run([exe, *sizes], capture_output=True, text=True, timeout=120)
+    if r.returncode != 0:
+        return {"unavailable": r.stderr.strip()[-200:]}
+    out = json.loads(r.stdout)
+    for kind in ("copy", "read"):
+        out[kind] = {mb: {"us": us, "pct_hbm_peak": round(100 * float(mb) * 1e6 / (us * 1e3) / peak, 1)}
+                     for mb, us in out[kind].items()}
+    out["how"] = ("grid-stride kernels, 256 threads x 8 blocks per SM, four 16-byte streaming loads in "
+                  "flight per thread, PDL; copy MB = bytes read + bytes written")
+    return out
+
+
 def throughput(torch, qk, wl, T, device, sets, steps=50):
     """GB/s of the fused path on T tokens with `sets` rotating buffer sets."""
     stream = torch.cuda.current_stream(device)
@@ -923,6 +948,7 @@ def run_native(args, dist):
         extras["headwise"] = headwise(torch, qk, device, peak)
         extras["fp8_prefill13b"] = fp8_prefill(torch, qk, device, peak)
         extras["tp_rank"] = tp_rank_step(torch, qk, device, peak)
+        extras["copy_floor"] = copy_floor(peak)
     dist.barrier()
 
     traffic = None

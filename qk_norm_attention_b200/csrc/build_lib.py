@@ -50,6 +50,7 @@ def nvcc() -> str:
 
 
 DECODE_BENCH = os.path.join(PKG, "decode_bench")
+COPY_FLOOR = os.path.join(PKG, "copy_floor")
 
 
 def _compile_objects(verbose: bool) -> list:
@@ -75,7 +76,8 @@ def _compile_objects(verbose: bool) -> list:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every .cu under csrc/ into libqknorm.so (skipped when up to date),
-    and the C++ decode timing program linked against it."""
+    the C++ decode timing program linked against it, and the copy/read
+    yardstick (copy_floor, standalone)."""
     if force or verbose or not up_to_date():
         tmp = LIBRARY + ".tmp"
         objs = _compile_objects(verbose)
@@ -90,6 +92,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
                         "-I", os.path.join(ROOT, "include"), "-o", tmp, src,
                         "-L", PKG, "-lqknorm", "-Xlinker", "-rpath,$ORIGIN"], check=True)
         os.replace(tmp, DECODE_BENCH)
+    src = os.path.join(CSRC, "copy_floor.cpp")
+    if force or not os.path.exists(COPY_FLOOR) or os.path.getmtime(COPY_FLOOR) < os.path.getmtime(src):
+        tmp = COPY_FLOOR + ".tmp"
+        subprocess.run([nvcc(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-x", "cu", "-o", tmp, src], check=True)
+        os.replace(tmp, COPY_FLOOR)
     return LIBRARY
 
 

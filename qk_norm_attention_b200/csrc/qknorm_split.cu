@@ -25,6 +25,35 @@
 
 namespace qkn {
 
+// The gathered shard sums of row t, n = Pb * nb of them in blocks of Pb at
+// stride sg (block b, shard p at st[b * sg + t * Pb + p]), loaded by the 32
+// lanes of a warp at once: lane l takes global shard index c0 + l (0 past
+// the end). stat_fold then adds the m lanes' values in lane order, which is
+// the order of the global shard index; every lane ends with the same S. One
+// round trip to memory per 32 sums instead of one per sum.
+__device__ __forceinline__ float stat_load(const float *st, int64_t t, int Pb, int n, int64_t sg,
+                                           int c0, int lane) {
+    const int j = c0 + lane;
+    if (j >= n) return 0.f;
+    const int b = j / Pb;
+    return __ldg(st + b * sg + t * Pb + (j - b * Pb));
+}
+
+__device__ __forceinline__ float stat_fold(float S, float v, int m) {
+    for (int u = 0; u < m; ++u) S = __fadd_rn(S, __shfl_sync(kFull, v, u));
+    return S;
+}
+
+// S of row t from its gathered shard sums, by a whole warp.
+__device__ __forceinline__ float stat_sum_warp(const float *st, int64_t t, int Pb, int nb, int64_t sg,
+                                               int lane) {
+    const int n = Pb * nb;
+    float S = 0.f;
+    for (int c0 = 0; c0 < n; c0 += 32)
+        S = stat_fold(S, stat_load(st, t, Pb, n, sg, c0, lane), n - c0 < 32 ? n - c0 : 32);
+    return S;
+}
+
 // TWO: the launch may carry two sides (one-side launches compile without
 // the selection, which costs registers).
 template <class Tag, int VMAX, int R, bool TWO>
