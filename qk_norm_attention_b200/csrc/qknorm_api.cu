@@ -417,10 +417,17 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         // ring; D = 4096, P = 4, T = 16384: 88.8 % vs 78.1 %; GQA widths, P = 8:
         // 45.8 % vs 37 %. At one vector per lane (D = 4096, P = 8) the
         // shard-pair ring with gamma in registers stays (82.5 % vs 76 %).
+        // The instances compiled for an exact shape take it in bf16 as well
+        // (GQA widths, P = 8: 87.1 % vs 83.9 % for the shard-pair ring with
+        // gamma in registers, same box).
         GPairShape gp;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
         else if (dtype == QKNORM_E4M3 && gpair_fits(sh, P, dtype, &gp) && (gp.mix || gp.hq || gp.nwq >= 2))
+            variant = QKNORM_VARIANT_GPAIR;
+        else if (dtype == QKNORM_BF16 && gpair_fits(sh, P, dtype, &gp) &&
+                 fused_gpair_kernel_for(dtype, gp.nwq, gp.hq, gp.nwk, gp.hk, gp.mix, P, sh.q.nv, sh.k.nv) !=
+                     fused_gpair_kernel(dtype, gp.nwq, gp.hq, gp.nwk, gp.hk, gp.mix))
             variant = QKNORM_VARIANT_GPAIR;
         else if (pair_fits(sh, P, dtype) && !pair_kw(sh) && sh.q.nv > kLanes)
             variant = QKNORM_VARIANT_PAIR;
@@ -558,7 +565,8 @@ void plan_grid(int64_t T, int num_sms, int blocks_per_sm, qknorm_plan *pl) {
 
 // The kernel a plan launches (for the occupancy query: the register variant
 // with prefetch, whose footprint is the larger).
-const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, int32_t P, bool for_occupancy) {
+const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, int32_t P, int32_t Dq, int32_t Dk,
+                        bool for_occupancy) {
     switch (pl.variant) {
     case QKNORM_VARIANT_CTA:
         if (pl.gamma_regs && !for_occupancy)
@@ -576,8 +584,9 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, int32_t P, bool fo
     case QKNORM_VARIANT_PAIR:
         return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0);
     case QKNORM_VARIANT_GPAIR:
-        return fused_gpair_kernel(dtype, pl.vmax, (pl.half_slots & 1) != 0, pl.vmax_k,
-                                  (pl.half_slots & 2) != 0, pl.mixed != 0);
+        return fused_gpair_kernel_for(dtype, pl.vmax, (pl.half_slots & 1) != 0, pl.vmax_k,
+                                      (pl.half_slots & 2) != 0, pl.mixed != 0, P, Dq / P / vec_of(dtype),
+                                      Dk / P / vec_of(dtype));
     default:
         return fused_generic_kernel(dtype);
     }
@@ -637,12 +646,12 @@ cudaError_t plan_device(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dt
     if (pl->variant == QKNORM_VARIANT_BULK || pl->variant == QKNORM_VARIANT_ROWS ||
         pl->variant == QKNORM_VARIANT_PAIR || pl->variant == QKNORM_VARIANT_GPAIR) {
         int regs = kRegsHint;
-        e = kernel_regs(plan_kernel(*pl, dtype, P, true), &regs);
+        e = kernel_regs(plan_kernel(*pl, dtype, P, Dq, Dk, true), &regs);
         if (e != cudaSuccess) return e;
         *status = plan_static(T, Dq, Dk, P, dtype, g_forced_variant, sms, regs, pl);
         if (*status != QKNORM_OK) return cudaSuccess;
     }
-    const void *fn = plan_kernel(*pl, dtype, P, true);
+    const void *fn = plan_kernel(*pl, dtype, P, Dq, Dk, true);
     if (pl->smem_bytes > 48 * 1024 || pl->variant == QKNORM_VARIANT_GENERIC ||
         (pl->variant == QKNORM_VARIANT_WARP && pl->vmax == 0)) {
         e = prepare_kernel(dev, fn, (pl->variant == QKNORM_VARIANT_BULK ||
@@ -834,7 +843,7 @@ static int apply_launch(int n, const void *const *x, const float *const *gamma,
     }
     const int block = n == 1 ? tpr[0] * (256 / tpr[0]) : (has96 && !wide ? 192 : 256);
     int bres = 1;
-    e = resident_blocks(dev, apply_kernel(dtype, multi, n == 2), block, 0, &bres);
+    e = resident_blocks(dev, apply_kernel(dtype, multi, n == 2, apply_fold(nb)), block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
     int64_t need[2], bytes[2], grid = 0;
     ApplyArgs a;
@@ -865,7 +874,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 116; }
+int qknorm_version(void) { return 117; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {

@@ -230,7 +230,11 @@ __device__ __forceinline__ float butterfly_quad(float a, float b, float c, float
 // Mixed form: Q with (NWQ, HQ), K with (NWK, HK), both in every warp.
 constexpr int kGPairMaxThreads = 256;
 
-template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX>
+// CP, CNQ, CNK: the shard count and the vectors per Q / K shard fixed at
+// compile time for the shapes that have their own instance (0: read from the
+// arguments). Fixed, every slot index, output offset and guard of a token
+// folds to a constant; the arithmetic and its order are the same.
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX, int CP = 0, int CNQ = 0, int CNK = 0>
 __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedArgs a, const GPairArgs b) {
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -242,11 +246,11 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int P = a.P;
+    const int P = CP ? CP : a.P;
     const int halfP = P >> 1;
     const int z = MIX ? 0 : (warp < halfP ? 0 : 1);        // separate form: this warp's tensor
     const int pa = 2 * (MIX ? warp : (z ? warp - halfP : warp));
-    const int nvq = a.nv[0], nvk = a.nv[1];
+    const int nvq = CNQ ? CNQ : a.nv[0], nvk = CNK ? CNK : a.nv[1];
     const uint32_t tok_bytes = b.qbytes + b.kbytes;
 
     const int64_t T = a.T;
@@ -351,9 +355,9 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
 //                 (2) -- D = 4096 in 4;
 //   FP8 mixed:    Q (1, half), K (0, half) -- e.g. Dq = 5120, Dk = 1024 in 8;
 //   bf16 mixed:   Q (3), K (1) -- the same GQA widths in bf16.
-template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX>
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX, int CP = 0, int CNQ = 0, int CNK = 0>
 const void *gpair_fn() {
-    return reinterpret_cast<const void *>(&fused_gpair<Tag, NWQ, HQ, NWK, HK, MIX>);
+    return reinterpret_cast<const void *>(&fused_gpair<Tag, NWQ, HQ, NWK, HK, MIX, CP, CNQ, CNK>);
 }
 
 const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix) {
@@ -369,6 +373,24 @@ const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bo
         if (mix && nwq == 3 && !hq && nwk == 1 && !hk) return gpair_fn<BF16Tag, 3, false, 1, false, true>();
     }
     return nullptr;
+}
+
+// The instance for this exact shape where one exists (P shards of nvq and
+// nvk vectors, compiled with them as constants), else the general one:
+//   FP8 13B-shaped, D = 5120 in 4 shards (80 vectors each);
+//   FP8 GQA-shaped, Dq = 5120, Dk = 1024 in 8 shards (40 and 8 vectors);
+//   bf16 GQA-shaped, the same widths (80 and 16 vectors).
+const void *fused_gpair_kernel_for(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix, int P, int nvq,
+                                   int nvk) {
+    const void *gen = fused_gpair_kernel(dtype, nwq, hq, nwk, hk, mix);
+    if (!gen) return nullptr;
+    if (dtype == 2 && !mix && nwq == 2 && hq && P == 4 && nvq == 80 && nvk == 80)
+        return gpair_fn<E4M3Tag, 2, true, 2, true, false, 4, 80, 80>();
+    if (dtype == 2 && mix && nwq == 1 && hq && nwk == 0 && hk && P == 8 && nvq == 40 && nvk == 8)
+        return gpair_fn<E4M3Tag, 1, true, 0, true, true, 8, 40, 8>();
+    if (dtype == 1 && mix && nwq == 3 && !hq && nwk == 1 && !hk && P == 8 && nvq == 80 && nvk == 16)
+        return gpair_fn<BF16Tag, 3, false, 1, false, true, 8, 80, 16>();
+    return gen;
 }
 
 // Slots per lane of one tensor: whole slots, and whether the last (at most
@@ -409,7 +431,7 @@ int gpair_max_threads() { return kGPairMaxThreads; }
 cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix,
                                const FusedArgs &a, int stages, int64_t grid, uint64_t timeout_ns,
                                cudaStream_t s) {
-    const void *fn = fused_gpair_kernel(dtype, nwq, hq, nwk, hk, mix);
+    const void *fn = fused_gpair_kernel_for(dtype, nwq, hq, nwk, hk, mix, a.P, a.nv[0], a.nv[1]);
     if (!fn || stages < 1 || stages > (int)kMaxStages || (a.P & 1) || a.P > 32 || a.K[0] != 1 ||
         a.K[1] != 1)
         return cudaErrorInvalidValue;

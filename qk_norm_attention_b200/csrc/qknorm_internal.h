@@ -42,8 +42,11 @@ const void *fused_cta_kernel(int dtype, int vmax, bool prefetch, bool full, bool
 const void *fused_generic_kernel(int dtype);
 // two: the instance for launches over two tensors.
 const void *stats_kernel(int dtype, int vmax, bool two);
-// multi: the several-rows-per-block instance of apply_k (block != tpr).
-const void *apply_kernel(int dtype, bool multi, bool two);
+// multi: the several-rows-per-block instance of apply_k (block != tpr);
+// fold: the row's shard sums loaded by a warp's lanes at once (apply_fold).
+const void *apply_kernel(int dtype, bool multi, bool two, bool fold);
+// Whether an apply over nb blocks of gathered sums takes the lane-parallel form.
+bool apply_fold(int32_t nb);
 
 // Launchers: enqueue one kernel; return the cudaError_t of the launch.
 cudaError_t launch_fused_cta(int dtype, int vmax, bool prefetch, bool full, bool greg,
@@ -119,6 +122,10 @@ cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const
 // shards of Q and the same two of K (P / 2 warps); nw whole slots per lane
 // per shard and, for FP8, h = the last slot (<= 16 vectors) split in halves.
 const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix);
+// The same, or the instance compiled for this exact shape (P shards of nvq
+// and nvk vectors) where one exists: what launch_fused_gpair launches.
+const void *fused_gpair_kernel_for(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix, int P, int nvq,
+                                   int nvk);
 void gpair_slots(int nv, int dtype, int *nw, bool *h);
 size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
                         int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,

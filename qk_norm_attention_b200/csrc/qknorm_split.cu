@@ -29,8 +29,7 @@ namespace qkn {
 // stride sg (block b, shard p at st[b * sg + t * Pb + p]), loaded by the 32
 // lanes of a warp at once: lane l takes global shard index c0 + l (0 past
 // the end). stat_fold then adds the m lanes' values in lane order, which is
-// the order of the global shard index; every lane ends with the same S. One
-// round trip to memory per 32 sums instead of one per sum.
+// the order of the global shard index; every lane ends with the same S.
 __device__ __forceinline__ float stat_load(const float *st, int64_t t, int Pb, int n, int64_t sg,
                                            int c0, int lane) {
     const int j = c0 + lane;
@@ -44,13 +43,29 @@ __device__ __forceinline__ float stat_fold(float S, float v, int m) {
     return S;
 }
 
-// S of row t from its gathered shard sums, by a whole warp.
-__device__ __forceinline__ float stat_sum_warp(const float *st, int64_t t, int Pb, int nb, int64_t sg,
-                                               int lane) {
-    const int n = Pb * nb;
+// S of row t from its gathered shard sums, in order of the global shard
+// index. FOLD = false: block by block, each block's Pb sums loaded by every
+// thread (one round trip per block). FOLD = true: the warp's lanes load 32
+// sums at a time and stat_fold adds them (one round trip per 32 sums, at the
+// cost of registers: 62 against 48 for the narrow two-tensor apply, one
+// resident block per SM fewer). Measured on one tensor-parallel rank's apply
+// at the 13B shape: 8 ranks (8 blocks of 1) 12.8 -> 11.2 us with the fold;
+// 2 and 4 ranks (2 x 4, 4 x 2) 29.5 and 17.7 us with the blocks against
+// 31.1 and 18.7 us with the fold.
+template <bool FOLD>
+__device__ __forceinline__ float stat_sum(const float *st, int64_t t, int Pb, int nb, int64_t sg, int lane) {
     float S = 0.f;
-    for (int c0 = 0; c0 < n; c0 += 32)
-        S = stat_fold(S, stat_load(st, t, Pb, n, sg, c0, lane), n - c0 < 32 ? n - c0 : 32);
+    if constexpr (FOLD) {
+        const int n = Pb * nb;
+        for (int c0 = 0; c0 < n; c0 += 32)
+            S = stat_fold(S, stat_load(st, t, Pb, n, sg, c0, lane), n - c0 < 32 ? n - c0 : 32);
+    } else {
+        st += t * Pb;
+        for (int b = 0; b < nb; ++b, st += sg) {
+#pragma unroll 8
+            for (int p = 0; p < Pb; ++p) S = __fadd_rn(S, __ldg(st + p));
+        }
+    }
     return S;
 }
 
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(256, 4) stats_k4(const StatsArgs a) {
 // apply_rows: the rows of one tensor that block bz of the tensor's gz blocks
 // takes. apply_k runs it for a one-tensor launch, apply2_k for a launch over
 // two tensors.
-template <class Tag, bool MULTI>
+template <class Tag, bool MULTI, bool FOLD>
 __device__ __forceinline__ void apply_rows(const void *x, const float *g, const float *stats, void *y,
                                            int64_t T, int32_t D, int32_t Pb, int32_t nb, int64_t sg,
                                            float Df, float eps, int32_t tpr, int64_t bz, int64_t gz) {
@@ -197,9 +212,9 @@ __device__ __forceinline__ void apply_rows(const void *x, const float *g, const 
             }
             if (v0 == 0) {
                 // Phase B: S = sum of the shard sums in order of the global
-                // shard index, loaded by the warp's lanes at once (tpr is a
-                // multiple of 32, so a warp's lanes share the row).
-                r = factor(stat_sum_warp(stats, t, Pb, nb, sg, threadIdx.x & 31), Df, eps);
+                // shard index (tpr is a multiple of 32, so the lanes of a warp
+                // share the row, as the fold needs).
+                r = factor(stat_sum<FOLD>(stats, t, Pb, nb, sg, threadIdx.x & 31), Df, eps);
             }
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
@@ -211,24 +226,24 @@ __device__ __forceinline__ void apply_rows(const void *x, const float *g, const 
 }
 
 // One tensor per launch.
-template <class Tag, bool MULTI>
+template <class Tag, bool MULTI, bool FOLD>
 __global__ void __launch_bounds__(256) apply_k(const void *x, const float *g, const float *stats,
                                                void *y, int64_t T, int32_t D, int32_t Pb, int32_t nb,
                                                int64_t sg, float Df, float eps, int32_t tpr) {
     pdl_wait();
     pdl_trigger();
-    apply_rows<Tag, MULTI>(x, g, stats, y, T, D, Pb, nb, sg, Df, eps, tpr, blockIdx.x, gridDim.x);
+    apply_rows<Tag, MULTI, FOLD>(x, g, stats, y, T, D, Pb, nb, sg, Df, eps, tpr, blockIdx.x, gridDim.x);
 }
 
 // Two tensors per launch: blocks below a.split take side 0, the rest side 1.
-template <class Tag, bool MULTI>
+template <class Tag, bool MULTI, bool FOLD>
 __global__ void __launch_bounds__(256) apply2_k(const ApplyArgs a) {
     pdl_wait();
     pdl_trigger();
     const int z = (int)blockIdx.x >= a.split ? 1 : 0;
     // Each field selected on its own (indexing the parameter array by z
     // would copy it to the stack).
-    apply_rows<Tag, MULTI>(z ? a.side[1].x : a.side[0].x, z ? a.side[1].g : a.side[0].g,
+    apply_rows<Tag, MULTI, FOLD>(z ? a.side[1].x : a.side[0].x, z ? a.side[1].g : a.side[0].g,
                            z ? a.side[1].stats : a.side[0].stats, z ? a.side[1].y : a.side[0].y, a.T,
                            z ? a.side[1].D : a.side[0].D, a.Pb, a.nb, a.sg,
                            z ? a.side[1].Df : a.side[0].Df, a.eps, z ? a.side[1].tpr : a.side[0].tpr,
@@ -273,18 +288,26 @@ const void *stats_kernel(int dtype, int vmax, bool two) {
     return nullptr;
 }
 
-template <class Tag, bool MULTI>
+template <class Tag, bool MULTI, bool FOLD>
 const void *apply_fn(bool two) {
-    return two ? reinterpret_cast<const void *>(&apply2_k<Tag, MULTI>)
-               : reinterpret_cast<const void *>(&apply_k<Tag, MULTI>);
+    return two ? reinterpret_cast<const void *>(&apply2_k<Tag, MULTI, FOLD>)
+               : reinterpret_cast<const void *>(&apply_k<Tag, MULTI, FOLD>);
 }
 
-const void *apply_kernel(int dtype, bool multi, bool two) {
-    if (dtype == 0) return multi ? apply_fn<F32Tag, true>(two) : apply_fn<F32Tag, false>(two);
-    if (dtype == 1) return multi ? apply_fn<BF16Tag, true>(two) : apply_fn<BF16Tag, false>(two);
-    if (dtype == 2) return multi ? apply_fn<E4M3Tag, true>(two) : apply_fn<E4M3Tag, false>(two);
+template <class Tag>
+const void *apply_table(bool multi, bool two, bool fold) {
+    if (multi) return fold ? apply_fn<Tag, true, true>(two) : apply_fn<Tag, true, false>(two);
+    return fold ? apply_fn<Tag, false, true>(two) : apply_fn<Tag, false, false>(two);
+}
+
+const void *apply_kernel(int dtype, bool multi, bool two, bool fold) {
+    if (dtype == 0) return apply_table<F32Tag>(multi, two, fold);
+    if (dtype == 1) return apply_table<BF16Tag>(multi, two, fold);
+    if (dtype == 2) return apply_table<E4M3Tag>(multi, two, fold);
     return nullptr;
 }
+
+bool apply_fold(int32_t nb) { return nb > 4; }
 
 cudaError_t launch_stats(int dtype, int vmax, const StatsArgs &a, int block, int64_t grid,
                          cudaStream_t s) {
@@ -311,7 +334,7 @@ int apply_threads_per_row(int32_t D, int dtype) {
 
 cudaError_t launch_apply(int dtype, bool multi, const ApplyArgs &a, int block, int64_t grid,
                          cudaStream_t s) {
-    const void *fn = apply_kernel(dtype, multi, a.split < grid);
+    const void *fn = apply_kernel(dtype, multi, a.split < grid, apply_fold(a.nb));
     if (!fn || a.split < 1 || a.split > grid) return cudaErrorInvalidValue;
     for (int z = 0; z < (a.split < grid ? 2 : 1); ++z) {
         const int tpr = a.side[z].tpr;

@@ -228,16 +228,18 @@ def test_plan_for_each_workload(qk):
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
             # One token per CTA: registers only. Several: the token ring (one
             # token per stage, gamma in registers while vmax <= 3), or for the
-            # GQA widths the shard-pair ring (P warps per token).
+            # GQA widths the staged-gamma shard-pair ring compiled for that
+            # shape (P / 2 mixed warps per token: two Q and two K shards each).
             if T <= 2 * 148:
                 want = qk.VARIANT_CTA
             else:
-                want = qk.VARIANT_PAIR if name == "gqa" else qk.VARIANT_BULK
+                want = qk.VARIANT_GPAIR if name == "gqa" else qk.VARIANT_BULK
             assert pl["variant"] == want, (name, T)
             assert pl["groups_q"] == pl["groups_k"] == 1
-            if want == qk.VARIANT_PAIR:
-                assert pl["block"] == wl.P * 32 and pl["vmax"] == 3 and pl["gamma_regs"] == 1
-                assert pl["stages"] == (3 if T >= 40 * 148 else 2) and pl["tokens_per_stage"] == 1
+            if want == qk.VARIANT_GPAIR:
+                assert pl["block"] == wl.P // 2 * 32 and pl["mixed"] == 1 and pl["gamma_regs"] == 0
+                assert (pl["vmax"], pl["vmax_k"], pl["half_slots"]) == (3, 1, 0)
+                assert pl["stages"] == 2 and pl["tokens_per_stage"] == 1
                 continue
             assert pl["block"] == want_block[name], name
             assert pl["vmax"] == want_vmax[name], name
@@ -517,8 +519,8 @@ def test_noalloc_wrapper_checks_metadata(qk):
 def test_gpair_plans(qk):
     """The shard-pair ring with staged gamma: separate warps for Q and K of one
     geometry, mixed warps (both tensors) otherwise; FP8 splits a last slot of
-    at most 16 vectors in lane halves; the selector takes it for FP8 GQA-like
-    shapes only."""
+    at most 16 vectors in lane halves; the selector takes it for FP8, and for
+    bf16 where an instance is compiled for the exact shape (GQA widths, P = 8)."""
     qk.qknorm_force_variant(qk.VARIANT_GPAIR, 0)
     try:
         pl = qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)     # 80 vectors per shard
@@ -542,7 +544,8 @@ def test_gpair_plans(qk):
         qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
         qk.qknorm_set_tuning()
     assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
-    assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR
+    assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_GPAIR
+    assert qk.qknorm_plan_fwd(4096, 5120, 768, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR   # 12 K vectors
     assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
     assert qk.qknorm_plan_fwd(8192, 4096, 4096, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
     assert qk.qknorm_plan_fwd(65536, 4096, 4096, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_PAIR
