@@ -568,24 +568,31 @@ def tp_rank_step(torch, qk, device, peak, steps=100):
         stride = gathered.stride(0)
         gq_, gk_ = gathered[:, 0].data_ptr(), gathered[:, 1].data_ptr()
 
-        def step_two(a, b, oa, ob, st):
+        # The raw C-ABI calls of one step, arguments marshalled once (as in
+        # Fused / Split), so the eager loop times the kernels, not Python.
+        def calls_two(a, b, oa, ob, st, hs):
+            return [(L.qknorm_partial_sumsq_qk, (a.data_ptr(), b.data_ptr(), st[0].data_ptr(), st[1].data_ptr(),
+                                                 T, Dl, Dl, Pl, 1, hs)),
+                    (L.qknorm_apply_tp_qk, (a.data_ptr(), b.data_ptr(), gl.data_ptr(), gl.data_ptr(), gq_, gk_,
+                                            stride, oa.data_ptr(), ob.data_ptr(), T, Dl, Dl, Pl, ranks, 1e-6,
+                                            1, hs))]
+
+        def calls_four(a, b, oa, ob, st, hs):
+            return [(L.qknorm_partial_sumsq, (a.data_ptr(), st[0].data_ptr(), T, Dl, Pl, 1, hs)),
+                    (L.qknorm_partial_sumsq, (b.data_ptr(), st[1].data_ptr(), T, Dl, Pl, 1, hs)),
+                    (L.qknorm_apply_tp, (a.data_ptr(), gl.data_ptr(), gq_, stride, oa.data_ptr(), T, Dl, Pl,
+                                         ranks, 1e-6, 1, hs)),
+                    (L.qknorm_apply_tp, (b.data_ptr(), gl.data_ptr(), gk_, stride, ob.data_ptr(), T, Dl, Pl,
+                                         ranks, 1e-6, 1, hs))]
+
+        def as_step(calls):
             def step():
-                ok(L.qknorm_partial_sumsq_qk(a.data_ptr(), b.data_ptr(), st[0].data_ptr(), st[1].data_ptr(),
-                                             T, Dl, Dl, Pl, 1, h))
-                ok(L.qknorm_apply_tp_qk(a.data_ptr(), b.data_ptr(), gl.data_ptr(), gl.data_ptr(), gq_, gk_,
-                                        stride, oa.data_ptr(), ob.data_ptr(), T, Dl, Dl, Pl, ranks, 1e-6,
-                                        1, h))
+                for fn, args in calls:
+                    ok(fn(*args))
             return step
 
-        def step_four(a, b, oa, ob, st):
-            def step():
-                ok(L.qknorm_partial_sumsq(a.data_ptr(), st[0].data_ptr(), T, Dl, Pl, 1, h))
-                ok(L.qknorm_partial_sumsq(b.data_ptr(), st[1].data_ptr(), T, Dl, Pl, 1, h))
-                ok(L.qknorm_apply_tp(a.data_ptr(), gl.data_ptr(), gq_, stride, oa.data_ptr(), T, Dl, Pl,
-                                     ranks, 1e-6, 1, h))
-                ok(L.qknorm_apply_tp(b.data_ptr(), gl.data_ptr(), gk_, stride, ob.data_ptr(), T, Dl, Pl,
-                                     ranks, 1e-6, 1, h))
-            return step
+        step_two = lambda *st: as_step(calls_two(*st, h))
+        step_four = lambda *st: as_step(calls_four(*st, h))
 
         nbytes = 2 * (3 * T * Dl * 2 + 4 * T * Pl + 4 * ranks * T * Pl + 4 * Dl)
         res = {}
@@ -598,7 +605,31 @@ def tp_rank_step(torch, qk, device, peak, steps=100):
             ms = tot / steps
             res[label] = {"us_per_step": round(ms * 1000, 2), "GB_s": round(nbytes / ms / 1e6, 1),
                           "pct_hbm_peak": round(100 * nbytes / ms / 1e6 / peak, 1)}
+        # The two-launch step of every rank's slices captured in one CUDA graph
+        # (how a serving step runs), replayed; us per step.
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=side):
+                hs = side.cuda_stream
+                for rep in range(4):
+                    for st in sets:
+                        as_step(calls_two(*st, hs))()
+        stream.wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        gms = e0.elapsed_time(e1) / (10 * 4 * ranks)
+        del graph
         out[str(ranks)] = dict(res["two_launches"], four_launches=res["four_launches"],
+                               graph={"us_per_step": round(gms * 1000, 2), "GB_s": round(nbytes / gms / 1e6, 1),
+                                      "pct_hbm_peak": round(100 * nbytes / gms / 1e6 / peak, 1)},
                                algorithmic_bytes=nbytes, exchange_bytes_per_rank=2 * 4 * T * Pl)
         del qs, ks, gathered, sets
     return {"workload": "13B-shaped Q and K (T=8192, D=5120, P=8) split over a tensor-parallel group; "

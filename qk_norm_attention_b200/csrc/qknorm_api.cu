@@ -361,8 +361,9 @@ void gpair_stages(int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, const GPairS
     pl->block = (g.mix ? P / 2 : P) * kLanes;
     pl->tokens_per_stage = 1;
     pl->stages = S;
-    pl->smem_bytes = (int64_t)gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, S, qb, kb, nullptr,
-                                               nullptr, nullptr, nullptr);
+    pl->smem_bytes = (int64_t)gpair_smem_bytes(dtype, P, g.nwq, g.hq, g.nwk, g.hk, Dq / P / vec_of(dtype),
+                                               Dk / P / vec_of(dtype), S, qb, kb, nullptr, nullptr, nullptr,
+                                               nullptr);
 }
 
 // Static part of the plan: which kernel, block size, template width, stages.
@@ -418,14 +419,17 @@ int plan_static(int64_t T, int32_t Dq, int32_t Dk, int32_t P, int32_t dtype, int
         // 45.8 % vs 37 %. At one vector per lane (D = 4096, P = 8) the
         // shard-pair ring with gamma in registers stays (82.5 % vs 76 %).
         // The instances compiled for an exact shape take it in bf16 as well
-        // (GQA widths, P = 8: 87.1 % vs 83.9 % for the shard-pair ring with
-        // gamma in registers, same box).
+        // below 48 tokens per SM (GQA widths, P = 8, one box: T = 4096 93.7 %
+        // vs 83.5 % for the shard-pair ring with gamma in registers; 6144:
+        // 93.8 vs 88.2 %; 8192: 85.4 vs 91.4 %; 16384: 83.2 vs 98.7 %: the
+        // staged-gamma ring's steady rate stays near 85 %, so the register
+        // ring takes the large batches).
         GPairShape gp;
         if (T <= 2 * (int64_t)num_sms)
             variant = cta_ok ? QKNORM_VARIANT_CTA : QKNORM_VARIANT_GENERIC;
         else if (dtype == QKNORM_E4M3 && gpair_fits(sh, P, dtype, &gp) && (gp.mix || gp.hq || gp.nwq >= 2))
             variant = QKNORM_VARIANT_GPAIR;
-        else if (dtype == QKNORM_BF16 && gpair_fits(sh, P, dtype, &gp) &&
+        else if (dtype == QKNORM_BF16 && T < 48 * (int64_t)num_sms && gpair_fits(sh, P, dtype, &gp) &&
                  fused_gpair_kernel_for(dtype, gp.nwq, gp.hq, gp.nwk, gp.hk, gp.mix, P, sh.q.nv, sh.k.nv) !=
                      fused_gpair_kernel(dtype, gp.nwq, gp.hq, gp.nwk, gp.hk, gp.mix))
             variant = QKNORM_VARIANT_GPAIR;

@@ -50,21 +50,52 @@ constexpr uint32_t kGPairRedBytes = 2 * 64 * sizeof(float);   // [buf][Q: 0..31,
 constexpr uint32_t kGPairGammaOff = kBarBytes + kGPairRedBytes;
 
 // Staged-gamma geometry of one tensor: NW whole slots per lane per shard, a
-// half slot (H), C = VEC / 4 float4 chunks per vector.
-template <class Tag, int NW, bool H>
+// half slot (H), C = VEC / 4 float4 chunks per vector. Whole slot i, chunk c
+// of shard p is read by lane l at float4 index
+//   NV = 0 (shard width known at run time): ((p * NW + i) * C + c) * 32 + l,
+//     every slot 32 lanes wide (a ragged last slot padded with zeros);
+//   compact (compiled for NV vectors per shard, no half slot): p * NV * C
+//     + 32 * i * C + c * L_i + l, with L_i = min(32, NV - 32 i) lanes in
+//     slot i, so the shard's block is exactly its NV * C float4 (no padding;
+//     with a half slot the whole slots are full and both forms agree).
+// Either way the lanes of a slot read consecutive float4: conflict-free.
+// The half slot (FP8, the last R <= 16 vectors of a shard, lanes l and l + 16
+// on the two halves of vector 32 NW + (l & 15)) is read at
+//   ((p * CH + c) * 32 + l) padded, or, compiled for NV vectors,
+//   p * CH * 2R + c * 2R + (l >> 4) * R + (l & 15): only its 2R lanes.
+template <class Tag, int NW, bool H, int NV = 0>
 struct GSlots {
     static constexpr int C = Tag::kVec / 4;
     static constexpr int CH = C / 2;
-    __host__ __device__ static int64_t whole(int P) { return (int64_t)P * NW * C * 32; }
-    __host__ __device__ static int64_t total(int P) { return whole(P) + (H ? (int64_t)P * CH * 32 : 0); }
+    static constexpr bool kCompact = NV > 0 && !H;
+    static constexpr bool kCompactH = NV > 0 && H;
+    static constexpr int R = H && NV > 0 ? NV - 32 * NW : 16;   // vectors in the half slot
+    __host__ __device__ static int64_t whole(int P) {
+        return kCompact ? (int64_t)P * NV * C : (int64_t)P * NW * C * 32;
+    }
+    __host__ __device__ static int64_t total(int P) {
+        return whole(P) + (H ? (int64_t)P * CH * 2 * R : 0);
+    }
+    __device__ __forceinline__ static int hidx(int p, int c, int lane) {
+        if constexpr (kCompactH) return p * CH * 2 * R + c * 2 * R + (lane >> 4) * R + (lane & 15);
+        else return (p * CH + c) * 32 + lane;
+    }
+    __device__ __forceinline__ static int idx(int p, int i, int c, int lane) {
+        if constexpr (kCompact) {
+            const int L = NV - 32 * i < 32 ? NV - 32 * i : 32;
+            return p * NV * C + 32 * i * C + c * L + lane;
+        } else {
+            return ((p * NW + i) * C + c) * 32 + lane;
+        }
+    }
 };
 
 // One tensor's gamma slots of shard p that lane `lane` copies into the
 // permuted shared-memory layout: vector l + 32 i, chunk c of each whole slot,
 // and the lane's half-slot chunks; zero for vectors the shard does not have.
-template <class Tag, int NW, bool H>
+template <class Tag, int NW, bool H, int NV = 0>
 struct GStage {
-    using G = GSlots<Tag, NW, H>;
+    using G = GSlots<Tag, NW, H, NV>;
     static constexpr int NL = NW * G::C + (H ? G::CH : 0);   // float4 slots per lane per shard
 
     __device__ __forceinline__ static void load(float4 (&val)[NL > 0 ? NL : 1], const float *g, int p, int nv,
@@ -92,11 +123,15 @@ struct GStage {
         const int64_t whole = G::whole(P);
 #pragma unroll
         for (int i = 0; i < NW; ++i)
+            if (!G::kCompact || lane + 32 * i < NV) {
 #pragma unroll
-            for (int c = 0; c < G::C; ++c) dst[((p * NW + i) * G::C + c) * 32 + lane] = val[i * G::C + c];
+                for (int c = 0; c < G::C; ++c) dst[G::idx(p, i, c, lane)] = val[i * G::C + c];
+            }
         if constexpr (H) {
+            if (!G::kCompactH || (lane & 15) < G::R) {
 #pragma unroll
-            for (int c = 0; c < G::CH; ++c) dst[whole + (p * G::CH + c) * 32 + lane] = val[NW * G::C + c];
+                for (int c = 0; c < G::CH; ++c) dst[whole + G::hidx(p, c, lane)] = val[NW * G::C + c];
+            }
         }
     }
 };
@@ -106,11 +141,11 @@ struct GStage {
 // Q and of K, all of those loads issued before any store (one L2 round trip
 // per shard, not one per slot), with the slot indices fixed at compile time
 // so that only the shard offset is computed at run time.
-template <class Tag, int NWQ, bool HQ, int NWK, bool HK>
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, int CNQ = 0, int CNK = 0>
 __device__ __forceinline__ void gpair_stage_gamma(float4 *gq, float4 *gk, const float *gammaq, const float *gammak,
                                                   int P, int nvq, int nvk, int warp, int nwarps, int lane) {
-    using SQ = GStage<Tag, NWQ, HQ>;
-    using SK = GStage<Tag, NWK, HK>;
+    using SQ = GStage<Tag, NWQ, HQ, CNQ>;
+    using SK = GStage<Tag, NWK, HK, CNK>;
     for (int p = warp; p < P; p += nwarps) {
         float4 vq[SQ::NL > 0 ? SQ::NL : 1], vk[SK::NL > 0 ? SK::NL : 1];
         SQ::load(vq, gammaq, p, nvq, lane);
@@ -152,11 +187,11 @@ __device__ __forceinline__ void gpair_chains(const unsigned char *row, int nv, i
 
 // (x * gamma) * r for the lane's vectors of shards pa, pa + 1 of one tensor,
 // gamma from its staged layout g (P shards), written to the output row dst.
-template <class Tag, int NW, bool H>
+template <class Tag, int NW, bool H, int NV = 0>
 __device__ __forceinline__ void gpair_apply(const uint4 (&x)[2][NW > 0 ? NW : 1], const uint2 (&hx)[2],
                                             const float4 *g, int P, uint4 *dst, int nv, int pa, int lane,
                                             float r) {
-    using G = GSlots<Tag, NW, H>;
+    using G = GSlots<Tag, NW, H, NV>;
     constexpr int VEC = Tag::kVec;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -168,7 +203,7 @@ __device__ __forceinline__ void gpair_apply(const uint4 (&x)[2][NW > 0 ? NW : 1]
                 float gg[VEC];
 #pragma unroll
                 for (int c = 0; c < G::C; ++c) {
-                    const float4 t = g[((p * NW + i) * G::C + c) * 32 + lane];
+                    const float4 t = g[G::idx(p, i, c, lane)];
                     gg[4 * c] = t.x;
                     gg[4 * c + 1] = t.y;
                     gg[4 * c + 2] = t.z;
@@ -184,7 +219,7 @@ __device__ __forceinline__ void gpair_apply(const uint4 (&x)[2][NW > 0 ? NW : 1]
                 const float4 *gb = g + G::whole(P);
 #pragma unroll
                 for (int c = 0; c < G::CH; ++c) {
-                    const float4 t = gb[(p * G::CH + c) * 32 + lane];
+                    const float4 t = gb[G::hidx(p, c, lane)];
                     gh[4 * c] = t.x;
                     gh[4 * c + 1] = t.y;
                     gh[4 * c + 2] = t.z;
@@ -281,7 +316,8 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
     // Gamma of both tensors into shared memory (visible after the first barrier).
-    gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp, blockDim.x >> 5, lane);
+    gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK, CNQ, CNK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp, blockDim.x >> 5,
+                                                      lane);
 
     constexpr int AQ = NWQ > 0 ? NWQ : 1, AK = NWK > 0 ? NWK : 1;
     int s = 0;
@@ -330,13 +366,13 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         if constexpr (MIX) {
             const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
             const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
-            gpair_apply<Tag, NWQ, HQ>(xq, hq, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
-                                      pa, lane, rq);
-            gpair_apply<Tag, NWK, HK>(xk, hk, gk, P, reinterpret_cast<uint4 *>(a.y[1]) + t * a.ldy[1], nvk,
-                                      pa, lane, rk);
+            gpair_apply<Tag, NWQ, HQ, CNQ>(xq, hq, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
+                                           pa, lane, rq);
+            gpair_apply<Tag, NWK, HK, CNK>(xk, hk, gk, P, reinterpret_cast<uint4 *>(a.y[1]) + t * a.ldy[1], nvk,
+                                           pa, lane, rk);
         } else {
             const float r = factor(combine_fast(&red[buf][32 * z], P, 1), z ? a.Df[1] : a.Df[0], a.eps);
-            gpair_apply<Tag, NWQ, HQ>(xq, hq, z ? gk : gq, P,
+            gpair_apply<Tag, NWQ, HQ, CNQ>(xq, hq, z ? gk : gq, P,
                                       reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]),
                                       z ? nvk : nvq, pa, lane, r);
         }
@@ -408,15 +444,24 @@ void gpair_slots(int nv, int dtype, int *nw, bool *h) {
     *nw += 1;
 }
 
-int64_t gpair_gamma_slots(int dtype, int P, int nw, bool h) {
+// Float4 slots of one tensor's staged gamma (GSlots::total): compact (nv
+// vectors per shard exactly) for an instance compiled for the shape without
+// a half slot, else 32 lanes per slot.
+int64_t gpair_gamma_slots(int dtype, int P, int nw, bool h, int nv, bool compiled) {
     const int C = (dtype == 1 ? 8 : (dtype == 2 ? 16 : 4)) / 4;
-    return (int64_t)P * nw * C * 32 + (h ? (int64_t)P * (C / 2) * 32 : 0);
+    const int64_t whole = compiled && !h ? (int64_t)P * nv * C : (int64_t)P * nw * C * 32;
+    const int64_t R = compiled && h ? nv - 32 * nw : 16;   // vectors in the half slot
+    return whole + (h ? (int64_t)P * (C / 2) * 2 * R : 0);
 }
 
-size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
+size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int nvq, int nvk, int stages,
                         int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,
                         uint32_t *gk4, uint32_t *stride) {
-    const int64_t q4 = gpair_gamma_slots(dtype, P, nwq, hq), k4 = gpair_gamma_slots(dtype, P, nwk, hk);
+    const bool mix = nvq != nvk;
+    const bool compiled = fused_gpair_kernel_for(dtype, nwq, hq, nwk, hk, mix, P, nvq, nvk) !=
+                          fused_gpair_kernel(dtype, nwq, hq, nwk, hk, mix);
+    const int64_t q4 = gpair_gamma_slots(dtype, P, nwq, hq, nvq, compiled),
+                  k4 = gpair_gamma_slots(dtype, P, nwk, hk, nvk, compiled);
     const int64_t base = ((int64_t)kGPairGammaOff + 16 * (q4 + k4) + 127) / 128 * 128;
     const uint32_t st = bulk_stage_stride(qbytes, kbytes, 1);
     if (stage_base) *stage_base = (uint32_t)base;
@@ -450,8 +495,8 @@ cudaError_t launch_fused_gpair(int dtype, int nwq, bool hq, int nwk, bool hk, bo
     b.qbytes = (uint32_t)(a.D[0] * es);
     b.kbytes = (uint32_t)(a.D[1] * es);
     b.timeout_ns = timeout_ns;
-    const size_t smem = gpair_smem_bytes(dtype, a.P, nwq, hq, nwk, hk, stages, b.qbytes, b.kbytes,
-                                         &b.stage_base, &b.gq4, &b.gk4, &b.stage_stride);
+    const size_t smem = gpair_smem_bytes(dtype, a.P, nwq, hq, nwk, hk, a.nv[0], a.nv[1], stages, b.qbytes,
+                                         b.kbytes, &b.stage_base, &b.gq4, &b.gk4, &b.stage_stride);
     void *args[] = {const_cast<FusedArgs *>(&a), &b};
     return launch(fn, dim3((unsigned)grid), dim3(block), smem, s, args);
 }

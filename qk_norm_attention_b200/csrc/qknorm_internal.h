@@ -127,7 +127,7 @@ const void *fused_gpair_kernel(int dtype, int nwq, bool hq, int nwk, bool hk, bo
 const void *fused_gpair_kernel_for(int dtype, int nwq, bool hq, int nwk, bool hk, bool mix, int P, int nvq,
                                    int nvk);
 void gpair_slots(int nv, int dtype, int *nw, bool *h);
-size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int stages,
+size_t gpair_smem_bytes(int dtype, int P, int nwq, bool hq, int nwk, bool hk, int nvq, int nvk, int stages,
                         int64_t qbytes, int64_t kbytes, uint32_t *stage_base, uint32_t *gq4,
                         uint32_t *gk4, uint32_t *stride);
 int gpair_max_threads();

@@ -228,8 +228,9 @@ def test_plan_for_each_workload(qk):
             pl = qk.qknorm_plan_fwd(T, wl.Dq, wl.Dk, wl.P, dt[wl.dtype], 148, 4)
             # One token per CTA: registers only. Several: the token ring (one
             # token per stage, gamma in registers while vmax <= 3), or for the
-            # GQA widths the staged-gamma shard-pair ring compiled for that
-            # shape (P / 2 mixed warps per token: two Q and two K shards each).
+            # GQA widths below 48 tokens per SM the staged-gamma shard-pair
+            # ring compiled for that shape (P / 2 mixed warps per token: two Q
+            # and two K shards each).
             if T <= 2 * 148:
                 want = qk.VARIANT_CTA
             else:
@@ -545,6 +546,7 @@ def test_gpair_plans(qk):
         qk.qknorm_set_tuning()
     assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
     assert qk.qknorm_plan_fwd(4096, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_GPAIR
+    assert qk.qknorm_plan_fwd(48 * 148, 5120, 1024, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR
     assert qk.qknorm_plan_fwd(4096, 5120, 768, 8, qk.QKNORM_BF16, 148)["variant"] == qk.VARIANT_PAIR   # 12 K vectors
     assert qk.qknorm_plan_fwd(8192, 5120, 5120, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
     assert qk.qknorm_plan_fwd(8192, 4096, 4096, 4, qk.QKNORM_E4M3, 148)["variant"] == qk.VARIANT_GPAIR
