@@ -775,8 +775,11 @@ static int stats_launch(int n, const void *const *x, float *const *stats, const 
     cudaError_t e = device_sms(&dev, &sms);
     if (e != cudaSuccess) return finish(e);
     const int block = 256;
+    int64_t in_bytes = 0;
+    for (int z = 0; z < n; ++z) in_bytes += T * D[z] * elem_of(dtype);
+    const bool keep = in_bytes <= kStatsKeepBytes;
     int bres = 1;
-    e = resident_blocks(dev, stats_kernel(dtype, vmax, n == 2), block, 0, &bres);
+    e = resident_blocks(dev, stats_kernel(dtype, vmax, n == 2, keep), block, 0, &bres);
     if (e != cudaSuccess) return finish(e);
     // A block takes (block / 32) warps x R tasks per turn.
     const int64_t per_block = (block / kLanes) * (vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1));
@@ -793,7 +796,7 @@ static int stats_launch(int n, const void *const *x, float *const *stats, const 
     a.T = T;
     a.P = P;
     a.split = (int32_t)split_grid(n, need, bytes, (int64_t)sms * bres, &grid);
-    return finish(launch_stats(dtype, vmax, a, block, grid, reinterpret_cast<cudaStream_t>(stream)));
+    return finish(launch_stats(dtype, vmax, keep, a, block, grid, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // Argument checks of the apply step for one tensor, stats laid out as nb

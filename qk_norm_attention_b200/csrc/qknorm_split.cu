@@ -70,8 +70,10 @@ __device__ __forceinline__ float stat_sum(const float *st, int64_t t, int Pb, in
 }
 
 // TWO: the launch may carry two sides (one-side launches compile without
-// the selection, which costs registers).
-template <class Tag, int VMAX, int R, bool TWO>
+// the selection, which costs registers). KEEP: rows read with the default L2
+// policy instead of evict-first, so that an apply launch soon after finds
+// them in L2 (taken for launches that read at most kStatsKeepBytes).
+template <class Tag, int VMAX, int R, bool TWO, bool KEEP>
 __device__ __forceinline__ void stats_body(const StatsArgs &a) {
     constexpr int VEC = Tag::kVec;
     pdl_wait();
@@ -128,7 +130,9 @@ __device__ __forceinline__ void stats_body(const StatsArgs &a) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(x) + t * rowvec + (int64_t)p * nv;
 #pragma unroll
                 for (int i = 0; i < VMAX; ++i)
-                    if (task < ntask && i < cnt) v[j][i] = ld_stream(src + first + (int64_t)i * stride);
+                    if (task < ntask && i < cnt)
+                        v[j][i] = KEEP ? __ldg(src + first + (int64_t)i * stride)
+                                       : ld_stream(src + first + (int64_t)i * stride);
             }
 #pragma unroll
             for (int j = 0; j < R; ++j) {
@@ -150,9 +154,9 @@ __device__ __forceinline__ void stats_body(const StatsArgs &a) {
     }
 }
 
-template <class Tag, int VMAX, int R, bool TWO>
+template <class Tag, int VMAX, int R, bool TWO, bool KEEP>
 __global__ void __launch_bounds__(256) stats_k(const StatsArgs a) {
-    stats_body<Tag, VMAX, R, TWO>(a);
+    stats_body<Tag, VMAX, R, TWO, KEEP>(a);
 }
 
 // The same kernel with registers for 4 resident blocks per SM, for the
@@ -164,9 +168,9 @@ __global__ void __launch_bounds__(256) stats_k(const StatsArgs a) {
 // D = 4096, P = 8).
 constexpr bool stats_four_blocks(int vmax, int r) { return vmax * r <= 7; }
 
-template <class Tag, int VMAX, int R, bool TWO>
+template <class Tag, int VMAX, int R, bool TWO, bool KEEP>
 __global__ void __launch_bounds__(256, 4) stats_k4(const StatsArgs a) {
-    stats_body<Tag, VMAX, R, TWO>(a);
+    stats_body<Tag, VMAX, R, TWO, KEEP>(a);
 }
 
 // The statistics of token t are nb blocks of Pb shard sums, block b at
@@ -256,35 +260,35 @@ __global__ void __launch_bounds__(256) apply2_k(const ApplyArgs a) {
 // Tasks per warp turn: as many as keep R x VMAX <= 8 vectors per lane.
 constexpr int stats_r(int vmax) { return vmax <= 2 ? 4 : (vmax <= 4 ? 2 : 1); }
 
-template <class Tag, int V>
+template <class Tag, int V, bool KEEP>
 const void *stats_fn(bool two) {
     if constexpr (stats_four_blocks(V, stats_r(V)))
-        return two ? reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), true>)
-                   : reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), false>);
+        return two ? reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), true, KEEP>)
+                   : reinterpret_cast<const void *>(&stats_k4<Tag, V, stats_r(V), false, KEEP>);
     else
-        return two ? reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), true>)
-                   : reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), false>);
+        return two ? reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), true, KEEP>)
+                   : reinterpret_cast<const void *>(&stats_k<Tag, V, stats_r(V), false, KEEP>);
 }
 
-template <class Tag>
+template <class Tag, bool KEEP>
 const void *stats_table(int vmax, bool two) {
     switch (vmax) {
-    case 1: return stats_fn<Tag, 1>(two);
-    case 2: return stats_fn<Tag, 2>(two);
-    case 3: return stats_fn<Tag, 3>(two);
-    case 4: return stats_fn<Tag, 4>(two);
-    case 5: return stats_fn<Tag, 5>(two);
-    case 6: return stats_fn<Tag, 6>(two);
-    case 7: return stats_fn<Tag, 7>(two);
-    case 8: return stats_fn<Tag, 8>(two);
+    case 1: return stats_fn<Tag, 1, KEEP>(two);
+    case 2: return stats_fn<Tag, 2, KEEP>(two);
+    case 3: return stats_fn<Tag, 3, KEEP>(two);
+    case 4: return stats_fn<Tag, 4, KEEP>(two);
+    case 5: return stats_fn<Tag, 5, KEEP>(two);
+    case 6: return stats_fn<Tag, 6, KEEP>(two);
+    case 7: return stats_fn<Tag, 7, KEEP>(two);
+    case 8: return stats_fn<Tag, 8, KEEP>(two);
     default: return nullptr;
     }
 }
 
-const void *stats_kernel(int dtype, int vmax, bool two) {
-    if (dtype == 0) return stats_table<F32Tag>(vmax, two);
-    if (dtype == 1) return stats_table<BF16Tag>(vmax, two);
-    if (dtype == 2) return stats_table<E4M3Tag>(vmax, two);
+const void *stats_kernel(int dtype, int vmax, bool two, bool keep) {
+    if (dtype == 0) return keep ? stats_table<F32Tag, true>(vmax, two) : stats_table<F32Tag, false>(vmax, two);
+    if (dtype == 1) return keep ? stats_table<BF16Tag, true>(vmax, two) : stats_table<BF16Tag, false>(vmax, two);
+    if (dtype == 2) return keep ? stats_table<E4M3Tag, true>(vmax, two) : stats_table<E4M3Tag, false>(vmax, two);
     return nullptr;
 }
 
@@ -309,9 +313,9 @@ const void *apply_kernel(int dtype, bool multi, bool two, bool fold) {
 
 bool apply_fold(int32_t nb) { return nb > 4; }
 
-cudaError_t launch_stats(int dtype, int vmax, const StatsArgs &a, int block, int64_t grid,
+cudaError_t launch_stats(int dtype, int vmax, bool keep, const StatsArgs &a, int block, int64_t grid,
                          cudaStream_t s) {
-    const void *fn = stats_kernel(dtype, vmax, a.split < grid);
+    const void *fn = stats_kernel(dtype, vmax, a.split < grid, keep);
     if (!fn || a.split < 1 || a.split > grid) return cudaErrorInvalidValue;
     void *args[] = {const_cast<StatsArgs *>(&a)};
     return launch(fn, dim3((unsigned)grid), dim3(block), 0, s, args);
