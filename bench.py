@@ -928,9 +928,9 @@ def run_native(args, dist):
             oqh.copy_(oqd, non_blocking=True)
             okh.copy_(okd, non_blocking=True)
     else:
-        # The library's host-buffer entry point: chunks of 512 tokens copied in,
-        # normalised and copied out, the two copy directions overlapping.
-        e2e_path = ("qknorm_fwd_host: pinned host rows in, 512-token chunks over 3 device "
+        # The library's host-buffer entry point: chunks of 1024 tokens copied
+        # in, normalised and copied out, the two copy directions overlapping.
+        e2e_path = ("qknorm_fwd_host: pinned host rows in, 1024-token chunks over 3 device "
                     "workspace sets, host->device copy / kernel / device->host copy overlapped")
         ws = torch.empty(qk.qknorm_fwd_host_workspace(wl.Dq, wl.Dk, q.dtype), dtype=torch.uint8,
                          device=device)

@@ -248,7 +248,7 @@ QKNORM_API int qknorm_apply_tp_qk(const void *q, const void *k, const float *gam
  * go to the device, are normalised there and come back (no counterpart in
  * the paper; it is the path a caller with host-resident activations takes).
  *
- * The T tokens are processed in chunks of chunk_tokens (0 = 512). Each chunk
+ * The T tokens are processed in chunks of chunk_tokens (0 = 1024). Each chunk
  * is copied host-to-device into one of three workspace sets, normalised in
  * place by qknorm_fwd on `stream`, and copied back, with the copies on two
  * streams of the library's own, so the host-to-device copy of one chunk, the

@@ -117,7 +117,7 @@ def test_split_rejects(qk):
 
 def test_host_workspace_size(qk):
     L = qk.lib
-    assert L.qknorm_fwd_host_workspace(0, 5120, 5120, 1) == 3 * 512 * 10240 * 2
+    assert L.qknorm_fwd_host_workspace(0, 5120, 5120, 1) == 3 * 1024 * 10240 * 2
     assert L.qknorm_fwd_host_workspace(7, 256, 128, 0) == 3 * 7 * 384 * 4
     assert L.qknorm_fwd_host_workspace(7, 256, 128, 2) == 3 * 7 * 384
     assert L.qknorm_fwd_host_workspace(7, 0, 128, 1) == -1

@@ -25,7 +25,7 @@ def _host(t: torch.Tensor, pinned: bool) -> torch.Tensor:
 
 
 @pytest.mark.parametrize("T,Dq,Dk,P,dtype,chunk,pinned", [
-    (1000, 5120, 1024, 8, "bf16", 0, True),       # default chunks: 512 + 488 tokens
+    (1500, 5120, 1024, 8, "bf16", 0, True),       # default chunks: 1024 + 476 tokens
     (1000, 4096, 4096, 4, "bf16", 7, True),       # many chunks, ragged last
     (333, 256, 256, 2, "f32", 100, False),        # pageable memory
     (640, 4096, 1024, 8, "e4m3", 64, True),
