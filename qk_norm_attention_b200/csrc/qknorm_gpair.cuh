@@ -33,6 +33,8 @@
 // gamma reads are conflict-free and no gamma lives in registers.
 #pragma once
 
+#include <type_traits>
+
 namespace qkn {
 
 struct GPairArgs {
@@ -234,6 +236,94 @@ __device__ __forceinline__ void gpair_apply(const uint4 (&x)[2][NW > 0 ? NW : 1]
     }
 }
 
+// Combined half slot (FP8, mixed, shapes compiled with a Q remainder of
+// RQ <= 8 vectors after NWQ whole slots and K shards of RK <= 8 vectors):
+// the last Q vectors and the K vectors of a shard share one 32-lane slot
+// instead of a half-empty slot each. Lane l takes tensor l >> 4 (Q, K),
+// half (l >> 3) & 1 of vector vv = l & 7 (Q: vector 32 NWQ + vv of the
+// shard, K: vector vv); lanes l and l + 8 hold the two halves of a vector.
+// The vector's sum is its halves' sums added (the FP8 vector sum's
+// definition), formed in lane l; a K vector's sum then moves to lane vv,
+// the lane that owns it in the shard's butterfly. Every addition has the
+// operands it has in the half-slot form, so the bits are the same.
+template <int NWQ, int CNQ, int CNK>
+struct GComb {
+    static constexpr int RQ = CNQ - 32 * NWQ, RK = CNK;
+    __device__ __forceinline__ static bool valid(int lane) {
+        return (lane >> 4) ? (lane & 7) < RK : (lane & 7) < RQ;
+    }
+    // Byte offset of the lane's half inside a row, shard p.
+    __device__ __forceinline__ static int off(int p, int lane) {
+        const int vv = lane & 7, hh = (lane >> 3) & 1;
+        return (lane >> 4) ? (p * CNK + vv) * 16 + 8 * hh : (p * CNQ + 32 * NWQ + vv) * 16 + 8 * hh;
+    }
+};
+
+// Gamma of the combined slots: per shard p, 2 float4 per lane at
+// (p * 2 + c) * 32 + lane (all 32 lanes; zeros where a lane has no vector).
+template <int NWQ, int CNQ, int CNK>
+__device__ __forceinline__ void gpair_stage_comb(float4 *gq, float4 *gcomb, const float *gammaq, const float *gammak,
+                                                 int P, int warp, int nwarps, int lane) {
+    using CB = GComb<NWQ, CNQ, CNK>;
+    using SQ = GStage<E4M3Tag, NWQ, false>;
+    for (int p = warp; p < P; p += nwarps) {
+        float4 vq[SQ::NL > 0 ? SQ::NL : 1];
+        SQ::load(vq, gammaq, p, CNQ, lane);
+        const bool ok = CB::valid(lane);
+        const float *src = ((lane >> 4) ? gammak : gammaq) + CB::off(p, lane);   // floats: 16 per vector = bytes
+        const float4 c0 = ok ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 c1 = ok ? __ldg(reinterpret_cast<const float4 *>(src) + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        SQ::store(gq, vq, P, p, lane);
+        gcomb[(p * 2 + 0) * 32 + lane] = c0;
+        gcomb[(p * 2 + 1) * 32 + lane] = c1;
+    }
+}
+
+// The lane's vectors of Q shards pa, pa + 1 (whole slots) and its combined
+// half of each shard; the Q and K lane chains of both shards.
+template <int NWQ, int CNQ, int CNK>
+__device__ __forceinline__ void gpair_chains_comb(const unsigned char *rowq, const unsigned char *rowk, int pa,
+                                                  int lane, uint4 (&xq)[2][NWQ > 0 ? NWQ : 1], uint2 (&hx)[2],
+                                                  float (&cq)[2], float (&ck)[2]) {
+    using CB = GComb<NWQ, CNQ, CNK>;
+    const bool ok = CB::valid(lane);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int p = pa + h;
+        const uint4 *sh = reinterpret_cast<const uint4 *>(rowq) + p * CNQ;
+        float ch = 0.f;
+#pragma unroll
+        for (int i = 0; i < NWQ; ++i) {
+            xq[h][i] = sh[lane + 32 * i];
+            ch = __fadd_rn(ch, vsumsq(E4M3Tag{}, xq[h][i]));
+        }
+        hx[h] = ok ? *reinterpret_cast<const uint2 *>(((lane >> 4) ? rowk : rowq) + CB::off(p, lane))
+                   : make_uint2(0, 0);
+        const float hf = e4m3x8_sumsq(hx[h].x, hx[h].y);
+        const float vs = __fadd_rn(hf, __shfl_down_sync(kFull, hf, 8));   // half 0 + half 1 in lanes l & 8 == 0
+        if (lane < CB::RQ) ch = __fadd_rn(ch, vs);
+        const float kv = __shfl_sync(kFull, vs, (lane & 7) + 16);
+        cq[h] = ch;
+        ck[h] = lane < CB::RK ? kv : 0.f;
+    }
+}
+
+// (x * gamma) * r for the combined halves of shards pa, pa + 1.
+template <int NWQ, int CNQ, int CNK>
+__device__ __forceinline__ void gpair_apply_comb(const uint2 (&hx)[2], const float4 *gcomb, unsigned char *yq,
+                                                 unsigned char *yk, int pa, int lane, float rq, float rk) {
+    using CB = GComb<NWQ, CNQ, CNK>;
+    if (!CB::valid(lane)) return;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int p = pa + h;
+        const float4 t0 = gcomb[(p * 2 + 0) * 32 + lane], t1 = gcomb[(p * 2 + 1) * 32 + lane];
+        const float gh[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+        const uint2 y = vapply_half(E4M3Tag{}, hx[h], gh, (lane >> 4) ? rk : rq);
+        __stcs(reinterpret_cast<uint2 *>(((lane >> 4) ? yk : yq) + CB::off(p, lane)), y);
+    }
+}
+
 // Transposed butterflies (see the top comment). Two chains: lanes 0-15 end
 // with shard 0's sum, lanes 16-31 with shard 1's.
 __device__ __forceinline__ float butterfly_pair(float c0, float c1, int lane) {
@@ -287,6 +377,11 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
     const int pa = 2 * (MIX ? warp : (z ? warp - halfP : warp));
     const int nvq = CNQ ? CNQ : a.nv[0], nvk = CNK ? CNK : a.nv[1];
     const uint32_t tok_bytes = b.qbytes + b.kbytes;
+    // The combined half slot (see GComb) for the FP8 GQA-shaped instance; its
+    // gamma follows Q's whole slots, in the space of Q's and K's half slots.
+    constexpr bool COMB = std::is_same<Tag, E4M3Tag>::value && MIX && HQ && HK && NWK == 0 && CNQ > 0 &&
+                          CNK > 0 && CNQ - 32 * NWQ <= 8 && CNK <= 8;
+    float4 *gcomb = gq + (int64_t)(CP > 0 ? CP : 1) * NWQ * (Tag::kVec / 4) * 32;
 
     const int64_t T = a.T;
     const int64_t G = gridDim.x;
@@ -316,8 +411,11 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
     // Gamma of both tensors into shared memory (visible after the first barrier).
-    gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK, CNQ, CNK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp, blockDim.x >> 5,
-                                                      lane);
+    if constexpr (COMB)
+        gpair_stage_comb<NWQ, CNQ, CNK>(gq, gcomb, a.g[0], a.g[1], P, warp, blockDim.x >> 5, lane);
+    else
+        gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK, CNQ, CNK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp,
+                                                          blockDim.x >> 5, lane);
 
     constexpr int AQ = NWQ > 0 ? NWQ : 1, AK = NWK > 0 ? NWK : 1;
     int s = 0;
@@ -330,7 +428,11 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         uint4 xq[2][AQ], xk[2][AK];
         uint2 hq[2], hk[2];
         float cq[2], ck[2];
-        if constexpr (MIX) {
+        if constexpr (COMB) {
+            gpair_chains_comb<NWQ, CNQ, CNK>(st, st + b.qbytes, pa, lane, xq, hq, cq, ck);
+            const float v = butterfly_quad(cq[0], cq[1], ck[0], ck[1], lane);
+            if ((lane & 7) == 0) red[buf][32 * (lane >> 4) + pa + ((lane >> 3) & 1)] = v;
+        } else if constexpr (MIX) {
             gpair_chains<Tag, NWQ, HQ>(st, nvq, pa, lane, xq, hq, cq);
             gpair_chains<Tag, NWK, HK>(st + b.qbytes, nvk, pa, lane, xk, hk, ck);
             const float v = butterfly_quad(cq[0], cq[1], ck[0], ck[1], lane);
@@ -363,7 +465,16 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
             issue(s, n + S);
         }
         // Phase B: shard sums in order of p, the factor; weight multiply and Phase C.
-        if constexpr (MIX) {
+        if constexpr (COMB) {
+            const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
+            const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
+            uint2 hdummy[2] = {make_uint2(0, 0), make_uint2(0, 0)};
+            gpair_apply<Tag, NWQ, false>(xq, hdummy, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
+                                         pa, lane, rq);
+            gpair_apply_comb<NWQ, CNQ, CNK>(hq, gcomb, reinterpret_cast<unsigned char *>(a.y[0]) + t * a.ldy[0] * 16,
+                                            reinterpret_cast<unsigned char *>(a.y[1]) + t * a.ldy[1] * 16, pa, lane,
+                                            rq, rk);
+        } else if constexpr (MIX) {
             const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
             const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
             gpair_apply<Tag, NWQ, HQ, CNQ>(xq, hq, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
