@@ -842,6 +842,30 @@ static int apply_launch(int n, const void *const *x, const float *const *gamma,
     int dev = 0, sms = 0;
     cudaError_t e = device_sms(&dev, &sms);
     if (e != cudaSuccess) return finish(e);
+    // Rows of at most 32 x kApplyNarrowMaxV vectors: a warp per row (apply_w).
+    int64_t rowvec = 0;
+    for (int z = 0; z < n; ++z)
+        if (D[z] / vec_of(dtype) > rowvec) rowvec = D[z] / vec_of(dtype);
+    if (rowvec <= 32 * kApplyNarrowMaxV) {
+        const int v = (int)((rowvec + 31) / 32);
+        int bres = 1;
+        e = resident_blocks(dev, apply_narrow_kernel(dtype, v, n == 2, apply_fold(nb)), 256, 0, &bres);
+        if (e != cudaSuccess) return finish(e);
+        ApplyArgs a;
+        for (int z = 0; z < 2; ++z) {
+            const int w = z < n ? z : 0;
+            a.side[z] = ApplySide{x[w], gamma[w], stats[w], out[w], D[w], kLanes, (float)((int64_t)D[w] * nb)};
+        }
+        a.T = T;
+        a.sg = sg;
+        a.Pb = Pb;
+        a.nb = nb;
+        a.eps = eps;
+        a.split = 0;
+        const int64_t need = (T * n + 7) / 8, cap = (int64_t)sms * (bres > 0 ? bres : 1);
+        return finish(launch_apply_narrow(dtype, v, a, n == 2, need < cap ? need : cap,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+    }
     // apply_threads_per_row(D) threads per row. One tensor: as many rows per
     // 256-thread block as fit. Two: a block size both sides' row groups
     // divide (192 for 96-thread rows, else 256; a side's spare threads idle).
@@ -886,7 +910,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 118; }
+int qknorm_version(void) { return 119; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {

@@ -103,6 +103,11 @@ int apply_threads_per_row(int32_t D, int dtype);
 // equals block).
 cudaError_t launch_apply(int dtype, bool multi, const ApplyArgs &a, int block, int64_t grid,
                          cudaStream_t s);
+// Rows of at most 32 * v vectors (v = 1..kApplyNarrowMaxV): one warp per row
+// over the flat row space of one or two tensors (apply_w), 256 threads.
+constexpr int kApplyNarrowMaxV = 5;
+const void *apply_narrow_kernel(int dtype, int v, bool two, bool fold);
+cudaError_t launch_apply_narrow(int dtype, int v, const ApplyArgs &a, bool two, int64_t grid, cudaStream_t s);
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).
 // tb = tokens per ring stage (1 or 2); mode: 0 any shape, 1 every lane holds

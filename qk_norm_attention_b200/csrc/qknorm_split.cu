@@ -255,6 +255,51 @@ __global__ void __launch_bounds__(256) apply2_k(const ApplyArgs a) {
                            z ? (int64_t)gridDim.x - a.split : (int64_t)a.split);
 }
 
+// Narrow rows of at most 32 * V vectors (one rank's slice of a
+// tensor-parallel group, e.g. 640 bf16 columns at 8 ranks): one warp per row
+// over the flat row space of the launch (rows 0 .. T-1 of side 0, then
+// T .. 2T-1 of side 1, so the warps share the two tensors' rows evenly),
+// lane l taking vectors l, l + 32, ...; the row's loads are issued before
+// its shard sums are read. Registers are bounded so that 6-8 blocks are
+// resident per SM: a narrow row gives a thread few vectors, so what an SM
+// keeps in flight comes from its thread count (the several-rows-per-block
+// apply above holds 4 blocks at 58 registers). Measured on one rank's step
+// at the 13B shape, same box: 8 ranks (80 vectors per row) 61.0 -> 64.3 %
+// eager, 63.2 -> 66.0 % in a graph; 4 ranks (160) 68.1 -> 69.2 % eager,
+// 72.7 -> 77.3 % in a graph.
+constexpr int apply_w_blocks(int v) { return v <= 2 ? 8 : (v <= 4 ? 6 : 5); }
+
+template <class Tag, int V, bool TWO, bool FOLD>
+__global__ void __launch_bounds__(256, apply_w_blocks(V)) apply_w(const ApplyArgs a) {
+    constexpr int VEC = Tag::kVec;
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t T = a.T;
+    const int64_t nrows = TWO ? 2 * T : T;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < nrows; w += nw) {
+        const int z = TWO && w >= T ? 1 : 0;
+        const int64_t t = z ? w - T : w;
+        const int rowvec = (z ? a.side[1].D : a.side[0].D) / VEC;
+        const uint4 *src = reinterpret_cast<const uint4 *>(z ? a.side[1].x : a.side[0].x) + t * rowvec;
+        uint4 xv[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+            if (lane + 32 * i < rowvec) xv[i] = ld_stream(src + lane + 32 * i);
+        // Phase B: the shard sums in order of the global shard index.
+        const float r = factor(stat_sum<FOLD>(z ? a.side[1].stats : a.side[0].stats, t, a.Pb, a.nb, a.sg, lane),
+                               z ? a.side[1].Df : a.side[0].Df, a.eps);
+        uint4 *dst = reinterpret_cast<uint4 *>(z ? a.side[1].y : a.side[0].y) + t * rowvec;
+        const float *g = z ? a.side[1].g : a.side[0].g;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int v = lane + 32 * i;
+            if (v < rowvec) st_stream(dst + v, vapply(Tag{}, xv[i], g + (int64_t)v * VEC, r));
+        }
+    }
+}
+
 // ---------------------------------------------------------------- instance tables
 
 // Tasks per warp turn: as many as keep R x VMAX <= 8 vectors per lane.
@@ -312,6 +357,40 @@ const void *apply_kernel(int dtype, bool multi, bool two, bool fold) {
 }
 
 bool apply_fold(int32_t nb) { return nb > 4; }
+
+template <class Tag, bool TWO, bool FOLD>
+const void *apply_w_fn(int v) {
+    switch (v) {
+    case 1: return reinterpret_cast<const void *>(&apply_w<Tag, 1, TWO, FOLD>);
+    case 2: return reinterpret_cast<const void *>(&apply_w<Tag, 2, TWO, FOLD>);
+    case 3: return reinterpret_cast<const void *>(&apply_w<Tag, 3, TWO, FOLD>);
+    case 4: return reinterpret_cast<const void *>(&apply_w<Tag, 4, TWO, FOLD>);
+    case 5: return reinterpret_cast<const void *>(&apply_w<Tag, 5, TWO, FOLD>);
+    default: return nullptr;
+    }
+}
+
+template <class Tag>
+const void *apply_w_table(int v, bool two, bool fold) {
+    if (two) return fold ? apply_w_fn<Tag, true, true>(v) : apply_w_fn<Tag, true, false>(v);
+    return fold ? apply_w_fn<Tag, false, true>(v) : apply_w_fn<Tag, false, false>(v);
+}
+
+const void *apply_narrow_kernel(int dtype, int v, bool two, bool fold) {
+    if (dtype == 0) return apply_w_table<F32Tag>(v, two, fold);
+    if (dtype == 1) return apply_w_table<BF16Tag>(v, two, fold);
+    if (dtype == 2) return apply_w_table<E4M3Tag>(v, two, fold);
+    return nullptr;
+}
+
+cudaError_t launch_apply_narrow(int dtype, int v, const ApplyArgs &a, bool two, int64_t grid, cudaStream_t s) {
+    const void *fn = apply_narrow_kernel(dtype, v, two, apply_fold(a.nb));
+    const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
+    if (!fn || grid < 1 || a.side[0].D / vec > 32 * v || (two && a.side[1].D / vec > 32 * v))
+        return cudaErrorInvalidValue;
+    void *args[] = {const_cast<ApplyArgs *>(&a)};
+    return launch(fn, dim3((unsigned)grid), dim3(256), 0, s, args);
+}
 
 cudaError_t launch_stats(int dtype, int vmax, bool keep, const StatsArgs &a, int block, int64_t grid,
                          cudaStream_t s) {
