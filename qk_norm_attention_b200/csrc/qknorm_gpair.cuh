@@ -324,6 +324,16 @@ __device__ __forceinline__ void gpair_apply_comb(const uint2 (&hx)[2], const flo
     }
 }
 
+// The factor with the width fixed at compile time (W > 0): for a power of
+// two, S * (1 / W) is the same correctly rounded number as S / W (the
+// quotient is S scaled by a power of two), so the multiply replaces the
+// division bit for bit; otherwise, or with W unknown, factor() as everywhere.
+template <int W>
+__device__ __forceinline__ float factor_w(float S, float Df, float eps) {
+    if constexpr (W > 0 && (W & (W - 1)) == 0) return rsqrtf(__fadd_rn(__fmul_rn(S, 1.0f / W), eps));
+    else return factor(S, Df, eps);
+}
+
 // Transposed butterflies (see the top comment). Two chains: lanes 0-15 end
 // with shard 0's sum, lanes 16-31 with shard 1's.
 __device__ __forceinline__ float butterfly_pair(float c0, float c1, int lane) {
@@ -466,8 +476,8 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         }
         // Phase B: shard sums in order of p, the factor; weight multiply and Phase C.
         if constexpr (COMB) {
-            const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
-            const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
+            const float rq = factor_w<CP * CNQ * Tag::kVec>(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
+            const float rk = factor_w<CP * CNK * Tag::kVec>(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
             uint2 hdummy[2] = {make_uint2(0, 0), make_uint2(0, 0)};
             gpair_apply<Tag, NWQ, false>(xq, hdummy, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
                                          pa, lane, rq);
@@ -475,8 +485,8 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
                                             reinterpret_cast<unsigned char *>(a.y[1]) + t * a.ldy[1] * 16, pa, lane,
                                             rq, rk);
         } else if constexpr (MIX) {
-            const float rq = factor(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
-            const float rk = factor(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
+            const float rq = factor_w<CP * CNQ * Tag::kVec>(combine_fast(&red[buf][0], P, 1), a.Df[0], a.eps);
+            const float rk = factor_w<CP * CNK * Tag::kVec>(combine_fast(&red[buf][32], P, 1), a.Df[1], a.eps);
             gpair_apply<Tag, NWQ, HQ, CNQ>(xq, hq, gq, P, reinterpret_cast<uint4 *>(a.y[0]) + t * a.ldy[0], nvq,
                                            pa, lane, rq);
             gpair_apply<Tag, NWK, HK, CNK>(xk, hk, gk, P, reinterpret_cast<uint4 *>(a.y[1]) + t * a.ldy[1], nvk,
