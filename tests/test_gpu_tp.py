@@ -124,3 +124,27 @@ def test_tp_rejects_bad_layouts(qk):
     bad = (x.data_ptr(), g.data_ptr(), st.data_ptr() + 2, 0, y.data_ptr(), 8, 1024, 4, 2, 1e-6, 1, h)
     assert L.qknorm_apply_tp(*bad) == qk.QKNORM_ERR_MISALIGNED             # stats not 4-byte aligned
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "e4m3"])
+@pytest.mark.parametrize("rowvec", [32, 33, 128, 129, 160, 161])
+def test_narrow_apply_boundaries(qk, dtype, rowvec):
+    """The split apply around the widths where the warp-per-row form changes
+    its vectors per lane (32 x 1 .. 5) and where it hands over to the
+    several-rows form (161 vectors): one tensor and two tensors per launch,
+    bit-identical to the fused kernel. One shard (P = 1) so every width is a
+    valid shape."""
+    vec = {"bf16": 8, "f32": 4, "e4m3": 16}[dtype]
+    D, Dk, T, P = rowvec * vec, 32 * vec, 2 * 148 + 3, 1
+    wl = W.custom("narrow", T, D, Dk, P, dtype=dtype, seed=rowvec)
+    q, k = to_device(W.gen_rows(wl, "q", range(T))), to_device(W.gen_rows(wl, "k", range(T)))
+    gq, gk = to_device(W.gen_gamma(wl, "q")), to_device(W.gen_gamma(wl, "k"))
+    oq, ok = qk.qknorm_fwd(q, k, gq, gk, P, 1e-6)
+    sq = qk.qknorm_partial_sumsq(q, P)
+    yq = qk.qknorm_apply(q, gq, sq, 1e-6)
+    st2 = qk.qknorm_partial_sumsq_qk(q, k, P)
+    tq, tk = qk.qknorm_apply_tp_qk(q, k, gq, gk, st2[None], 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(yq), bits(oq)), "one-tensor apply"
+    assert torch.equal(bits(tq), bits(oq)) and torch.equal(bits(tk), bits(ok)), "two-tensor apply"
+    assert qk.qknorm_device_errors() == 0
