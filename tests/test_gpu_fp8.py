@@ -189,7 +189,7 @@ def test_fp8_saturation(qk, orc):
             assert (diff <= 2.0 ** -3 * np.abs(y_or[inside]) + 2.0 ** -9).all()
 
 
-@pytest.mark.parametrize("name", ["prefill13b_e4m3", "split_large_e4m3"])
+@pytest.mark.parametrize("name", ["prefill13b_e4m3", "split_large_e4m3", "gqa_e4m3"])
 def test_fp8_bench_workloads_full_size(qk, orc, name):
     """The FP8 configurations the benchmark times, at full size and in the
     selector's launch configuration (inputs drawn on the device with the
