@@ -586,7 +586,8 @@ const void *plan_kernel(const qknorm_plan &pl, int32_t dtype, int32_t P, int32_t
     case QKNORM_VARIANT_ROWS:
         return fused_rows_kernel(dtype);
     case QKNORM_VARIANT_PAIR:
-        return fused_pair_kernel(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0);
+        return fused_pair_kernel_for(dtype, pl.vmax, pl.gamma_regs != 0, pl.k_pairs != 0, P,
+                                     Dq / P / vec_of(dtype), Dk / P / vec_of(dtype));
     case QKNORM_VARIANT_GPAIR:
         return fused_gpair_kernel_for(dtype, pl.vmax, (pl.half_slots & 1) != 0, pl.vmax_k,
                                       (pl.half_slots & 2) != 0, pl.mixed != 0, P, Dq / P / vec_of(dtype),
@@ -910,7 +911,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 119; }
+int qknorm_version(void) { return 120; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {

@@ -473,7 +473,11 @@ __global__ void __launch_bounds__(512, 1) fused_rows(const FusedArgs a, const Ro
 // butterflies. This halves the warps per token of the ring for equal-width
 // tensors, which pays where a warp's fixed work per token (wait, butterfly,
 // barrier, factor) weighs most: one or two vectors per lane, FP8.
-template <class Tag, int VQ, bool GREG, bool KW>
+// CP, CNQ, CNK: shard count and vectors per Q / K shard fixed at compile
+// time for the shape that has its own instance (0: from the arguments);
+// every slot count, offset and the combine then fold to constants, and a
+// power-of-two width forms the factor by a multiply (same bits).
+template <class Tag, int VQ, bool GREG, bool KW, int CP = 0, int CNQ = 0, int CNK = 0>
 __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const BulkArgs b) {
     constexpr int VEC = Tag::kVec;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -484,11 +488,12 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int half = a.P >> 1;
+    const int P = CP ? CP : a.P;
+    const int half = P >> 1;
     const int z = warp < half ? 0 : 1;
     const int w = z ? warp - half : warp;
     const int pa = 2 * w;                                // first shard of the pair
-    const int nvq = a.nv[0], nvk = a.nv[1];
+    const int nvq = CNQ ? CNQ : a.nv[0], nvk = CNK ? CNK : a.nv[1];
     // Shard pairs (Q warps; K warps too with KW): this lane's vectors of
     // shards pa, pa + 1 of tensor z: lane + 32 i, i < cnt.
     const bool pairs = KW || z == 0;
@@ -623,7 +628,8 @@ __global__ void __launch_bounds__(512, 1) fused_pair(const FusedArgs a, const Bu
             fence_proxy_async_smem();
             issue(s, n + S);
         }
-        const float r = factor(combine_fast(&red[buf][z ? 32 : 0], a.P, 1), Df, eps);
+        const float Sz = combine_fast(&red[buf][z ? 32 : 0], P, 1);
+        const float r = z ? factor_w<CP * CNK * VEC>(Sz, Df, eps) : factor_w<CP * CNQ * VEC>(Sz, Df, eps);
         if (pairs) {
             uint4 *dst = reinterpret_cast<uint4 *>(z ? a.y[1] : a.y[0]) + t * (z ? a.ldy[1] : a.ldy[0]) +
                          (int64_t)pa * nvz + lane;
@@ -847,9 +853,19 @@ const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs, bool kw) {
     return nullptr;
 }
 
+// The instance compiled for this exact shape where one exists (FP8, one
+// vector per lane, K in pairs, 8 shards of 32 vectors: e.g. D = 4096, P = 8),
+// else the general one.
+const void *fused_pair_kernel_for(int dtype, int vq, bool gamma_regs, bool kw, int P, int nvq, int nvk) {
+    const void *gen = fused_pair_kernel(dtype, vq, gamma_regs, kw);
+    if (gen && dtype == 2 && vq == 1 && gamma_regs && kw && P == 8 && nvq == 32 && nvk == 32)
+        return reinterpret_cast<const void *>(&fused_pair<E4M3Tag, 1, true, true, 8, 32, 32>);
+    return gen;
+}
+
 cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const FusedArgs &a,
                               int stages, int64_t grid, uint64_t timeout_ns, cudaStream_t s) {
-    const void *fn = fused_pair_kernel(dtype, vq, gamma_regs, kw);
+    const void *fn = fused_pair_kernel_for(dtype, vq, gamma_regs, kw, a.P, a.nv[0], a.nv[1]);
     if (!fn || stages < 1 || stages > (int)kMaxStages || (a.P & 1) || a.P > 16) return cudaErrorInvalidValue;
     // Each lane's slots must cover its shards: lane halves take at most 16 K vectors.
     if (a.K[0] != 1 || a.K[1] != 1 || a.nv[0] > kLanes * vq || a.nv[1] > (kw ? kLanes * vq : kLanes / 2))

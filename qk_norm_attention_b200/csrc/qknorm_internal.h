@@ -126,6 +126,9 @@ cudaError_t launch_fused_bulk(int dtype, int vmax, bool gamma_regs, int tb, int 
 // shards of <= 16 vectors on lane halves (kw false, GQA-like shapes), or of
 // <= 32 * vq vectors in pairs like Q's (kw true).
 const void *fused_pair_kernel(int dtype, int vq, bool gamma_regs, bool kw);
+// The same, or the instance compiled for this exact shape where one exists:
+// what launch_fused_pair launches.
+const void *fused_pair_kernel_for(int dtype, int vq, bool gamma_regs, bool kw, int P, int nvq, int nvk);
 cudaError_t launch_fused_pair(int dtype, int vq, bool gamma_regs, bool kw, const FusedArgs &a,
                               int stages, int64_t grid, uint64_t timeout_ns, cudaStream_t s);
 // The shard-pair ring with gamma staged in shared memory (qknorm_gpair.cuh):
