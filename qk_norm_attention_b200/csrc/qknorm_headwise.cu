@@ -47,12 +47,15 @@ constexpr int headwise_min_blocks(int vec, int vmax) {
 // One group: units u0 .. u0 + R - 1 of tensor Z (< Uz) of token t. The
 // tensor is a template argument, so its row pointers are formed once per
 // group and its gamma registers are used without a select.
-template <class Tag, int SEG, int VMAX, int R, int Z>
+// CNV: vectors per head fixed at compile time (the instance for heads of 128
+// values), 0 read from the arguments; the slot guards and head offsets then
+// fold to constants (the arithmetic and its order are the same).
+template <class Tag, int SEG, int VMAX, int R, int Z, int CNV>
 __device__ __forceinline__ void headwise_group(const HeadArgs &a, int64_t t, int u0, int Uz, int slot,
                                                int hsub, const float *gz) {
     constexpr int VEC = Tag::kVec;
     constexpr int HPW = 32 / SEG;
-    const int nv = a.nv;
+    const int nv = CNV ? CNV : a.nv;
     const uint4 *xrow = reinterpret_cast<const uint4 *>(a.x[Z]) + t * a.ldx[Z];
     uint4 *yrow = reinterpret_cast<uint4 *>(a.y[Z]) + t * a.ldy[Z];
     uint4 v[R][VMAX];
@@ -94,7 +97,7 @@ __device__ __forceinline__ void headwise_group(const HeadArgs &a, int64_t t, int
     }
 }
 
-template <class Tag, int SEG, int VMAX, int R>
+template <class Tag, int SEG, int VMAX, int R, int CNV = 0>
 __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) headwise_k(const HeadArgs a) {
     constexpr int VEC = Tag::kVec;
     constexpr int HPW = 32 / SEG;  // heads per unit
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) hea
     const int lane = threadIdx.x & 31;
     const int slot = lane & (SEG - 1);
     const int hsub = lane / SEG;
-    const int nv = a.nv;
+    const int nv = CNV ? CNV : a.nv;
     const int64_t NW = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int Uq = (a.H[0] + HPW - 1) / HPW;
     const int Uk = (a.H[1] + HPW - 1) / HPW;
@@ -133,9 +136,9 @@ __global__ void __launch_bounds__(256, headwise_min_blocks(Tag::kVec, VMAX)) hea
     int gsub = (int)(w0 - t * G);
     while (t < a.T) {
         if (gsub < Gq)
-            headwise_group<Tag, SEG, VMAX, R, 0>(a, t, gsub * R, Uq, slot, hsub, gr[0]);
+            headwise_group<Tag, SEG, VMAX, R, 0, CNV>(a, t, gsub * R, Uq, slot, hsub, gr[0]);
         else
-            headwise_group<Tag, SEG, VMAX, R, 1>(a, t, (gsub - Gq) * R, Uk, slot, hsub, gr[1]);
+            headwise_group<Tag, SEG, VMAX, R, 1, CNV>(a, t, (gsub - Gq) * R, Uk, slot, hsub, gr[1]);
         t += dt;
         gsub += dg;
         if (gsub >= G) {
@@ -192,8 +195,13 @@ int64_t headwise_groups(int64_t T, int32_t Hq, int32_t Hk, int32_t nv) {
     return T * ((uq + r - 1) / r + (uk + r - 1) / r);
 }
 
+// Heads of 128 values (the common head_dim) have an instance with the vectors
+// per head compiled in: 32 fp32, 16 bf16, 8 FP8 vectors.
 const void *headwise_kernel(int dtype, int nv) {
     if (nv < 1 || nv > 256) return nullptr;
+    if (dtype == 0 && nv == 32) return reinterpret_cast<const void *>(&headwise_k<F32Tag, 32, 1, 4, 32>);
+    if (dtype == 1 && nv == 16) return reinterpret_cast<const void *>(&headwise_k<BF16Tag, 16, 1, 4, 16>);
+    if (dtype == 2 && nv == 8) return reinterpret_cast<const void *>(&headwise_k<E4M3Tag, 8, 1, 4, 8>);
     if (dtype == 0) return headwise_table<F32Tag>(nv);
     if (dtype == 1) return headwise_table<BF16Tag>(nv);
     if (dtype == 2) return headwise_table<E4M3Tag>(nv);
