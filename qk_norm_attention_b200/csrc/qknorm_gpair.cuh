@@ -261,11 +261,35 @@ struct GComb {
 
 // Gamma of the combined slots: per shard p, 2 float4 per lane at
 // (p * 2 + c) * 32 + lane (all 32 lanes; zeros where a lane has no vector).
+// When the warps take two shards each (P = 2 x warps), both shards' loads
+// are issued before either's stores: one L2 round trip instead of two
+// (measured at T = 4096: 12.53 -> 12.15 us per launch).
 template <int NWQ, int CNQ, int CNK>
 __device__ __forceinline__ void gpair_stage_comb(float4 *gq, float4 *gcomb, const float *gammaq, const float *gammak,
                                                  int P, int warp, int nwarps, int lane) {
     using CB = GComb<NWQ, CNQ, CNK>;
     using SQ = GStage<E4M3Tag, NWQ, false>;
+    if (2 * nwarps == P) {
+        const bool ok = CB::valid(lane);
+        float4 vq[2][SQ::NL > 0 ? SQ::NL : 1];
+        float4 c0[2], c1[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int p = warp + h * nwarps;
+            SQ::load(vq[h], gammaq, p, CNQ, lane);
+            const float *src = ((lane >> 4) ? gammak : gammaq) + CB::off(p, lane);   // 16 floats per vector
+            c0[h] = ok ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            c1[h] = ok ? __ldg(reinterpret_cast<const float4 *>(src) + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int p = warp + h * nwarps;
+            SQ::store(gq, vq[h], P, p, lane);
+            gcomb[(p * 2 + 0) * 32 + lane] = c0[h];
+            gcomb[(p * 2 + 1) * 32 + lane] = c1[h];
+        }
+        return;
+    }
     for (int p = warp; p < P; p += nwarps) {
         float4 vq[SQ::NL > 0 ? SQ::NL : 1];
         SQ::load(vq, gammaq, p, CNQ, lane);
