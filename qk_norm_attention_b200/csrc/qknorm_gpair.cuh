@@ -90,6 +90,13 @@ struct GSlots {
             return ((p * NW + i) * C + c) * 32 + lane;
         }
     }
+    // Where chunk c of vector v of shard p sits: a whole slot's lane v & 31,
+    // or a half slot's (half c / CH on lanes r and r + 16).
+    __device__ __forceinline__ static int at(int P, int p, int v, int c) {
+        if (!H || v < 32 * NW) return idx(p, v >> 5, c, v & 31);
+        const int r = v - 32 * NW, hh = c / CH;
+        return (int)whole(P) + hidx(p, c - hh * CH, r + 16 * hh);
+    }
 };
 
 // One tensor's gamma slots of shard p that lane `lane` copies into the
@@ -154,6 +161,64 @@ __device__ __forceinline__ void gpair_stage_gamma(float4 *gq, float4 *gk, const 
         SK::load(vk, gammak, p, nvk, lane);
         SQ::store(gq, vq, P, p, lane);
         SK::store(gk, vk, P, p, lane);
+    }
+}
+
+// Staging for the instances compiled for their shape (CP shards of CNQ and
+// CNK vectors): a warp reads each of its shards' gamma in memory order, 32
+// consecutive float4 per load (4 cache lines, where the lane-slot order above
+// touches 16 with its 64-byte lane stride and so costs the L1 four times the
+// cycles), all of its loads before any store, and each store puts a float4
+// where the slot layout wants it. Warp w takes shards w, w + nwarps, ... (two
+// in the mixed form, one in the separate). With COMB, Q's vectors after its
+// whole slots and all of K's go to the combined half slots (see GComb).
+template <class Tag, int NWQ, bool HQ, int NWK, bool HK, bool MIX, int CP, int CNQ, int CNK, bool COMB>
+__device__ __forceinline__ void gpair_stage_rows(float4 *gq, float4 *gk, float4 *gcomb, const float *gammaq,
+                                                 const float *gammak, int warp, int nwarps, int lane) {
+    constexpr int C = Tag::kVec / 4;
+    constexpr int NQ4 = CNQ * C, NK4 = CNK * C;              // float4 of one shard
+    constexpr int LQ = (NQ4 + 31) / 32, LK = (NK4 + 31) / 32;  // per lane
+    constexpr int HPW = MIX ? 2 : 1;                         // shards per warp
+    using GQ = GSlots<Tag, NWQ, COMB ? false : HQ, COMB ? 0 : CNQ>;
+    using GK = GSlots<Tag, NWK, HK, CNK>;
+    float4 vq[HPW][LQ], vk[HPW][LK];
+#pragma unroll
+    for (int h = 0; h < HPW; ++h) {
+        const int p = warp + h * nwarps;
+        if (p < CP) {
+            const float4 *sq = reinterpret_cast<const float4 *>(gammaq) + p * NQ4;
+            const float4 *sk = reinterpret_cast<const float4 *>(gammak) + p * NK4;
+#pragma unroll
+            for (int m = 0; m < LQ; ++m)
+                if (lane + 32 * m < NQ4) vq[h][m] = __ldg(sq + lane + 32 * m);
+#pragma unroll
+            for (int m = 0; m < LK; ++m)
+                if (lane + 32 * m < NK4) vk[h][m] = __ldg(sk + lane + 32 * m);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < HPW; ++h) {
+        const int p = warp + h * nwarps;
+        if (p < CP) {
+#pragma unroll
+            for (int m = 0; m < LQ; ++m) {
+                const int g = lane + 32 * m, v = g / C, c = g % C;
+                if (g >= NQ4) continue;
+                if (COMB && v >= 32 * NWQ)   // combined slot: lane (v - 32 NWQ) + 8 x half, chunk c & 1
+                    gcomb[(p * 2 + (c & 1)) * 32 + (v - 32 * NWQ) + 8 * (c >> 1)] = vq[h][m];
+                else
+                    gq[GQ::at(CP, p, v, c)] = vq[h][m];
+            }
+#pragma unroll
+            for (int m = 0; m < LK; ++m) {
+                const int g = lane + 32 * m, v = g / C, c = g % C;
+                if (g >= NK4) continue;
+                if (COMB)
+                    gcomb[(p * 2 + (c & 1)) * 32 + 16 + v + 8 * (c >> 1)] = vk[h][m];
+                else
+                    gk[GK::at(CP, p, v, c)] = vk[h][m];
+            }
+        }
     }
 }
 
@@ -445,7 +510,10 @@ __global__ void __launch_bounds__(kGPairMaxThreads, 1) fused_gpair(const FusedAr
         for (int s = 0; s < S && s < npass; ++s) issue(s, s);
     }
     // Gamma of both tensors into shared memory (visible after the first barrier).
-    if constexpr (COMB)
+    if constexpr (CP > 0 && CNQ > 0 && CNK > 0)
+        gpair_stage_rows<Tag, NWQ, HQ, NWK, HK, MIX, CP, CNQ, CNK, COMB>(gq, gk, gcomb, a.g[0], a.g[1], warp,
+                                                                       blockDim.x >> 5, lane);
+    else if constexpr (COMB)
         gpair_stage_comb<NWQ, CNQ, CNK>(gq, gcomb, a.g[0], a.g[1], P, warp, blockDim.x >> 5, lane);
     else
         gpair_stage_gamma<Tag, NWQ, HQ, NWK, HK, CNQ, CNK>(gq, gk, a.g[0], a.g[1], P, nvq, nvk, warp,
