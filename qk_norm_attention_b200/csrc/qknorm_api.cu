@@ -911,7 +911,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 122; }
+int qknorm_version(void) { return 123; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {
