@@ -270,3 +270,39 @@ def test_gpair_bit_identical_and_oracle(qk, orc, T, Dq, Dk, P, dtype):
     yq, yk, _, _ = orc.qknorm(q, k, gq, gk, P, EPS, dtype, nthreads=8)
     check_outputs(to_host(ref[0]), yq, dtype, f"gpair {Dq}/{Dk} q")
     check_outputs(to_host(ref[1]), yk, dtype, f"gpair {Dq}/{Dk} k")
+
+
+@pytest.mark.parametrize("T,Dq,Dk,P,dtype", [(3001, 5120, 1024, 8, "e4m3"), (2 * 1184 + 3, 5120, 5120, 4, "e4m3"),
+                                             (1500, 5120, 1024, 8, "bf16")])
+def test_gpair_many_launches_two_streams(qk, T, Dq, Dk, P, dtype):
+    """The staged-gamma ring launched many times back to back (programmatic
+    dependent launch between them), on two streams at once and with different
+    grids (each CTA walking from 2 to over 400 tokens through its ring): every
+    launch gives exactly the generic kernel's bits on every row."""
+    wl = W.custom(f"dyn{Dq}_{Dk}_{P}", T, Dq, Dk, P, dtype=dtype, seed=T + Dq, x_sigma=1.2)
+    q, k = W.gen_rows(wl, "q", range(T)), W.gen_rows(wl, "k", range(T))
+    qd, kd = to_device(q), to_device(k)
+    gqd, gkd = to_device(W.gen_gamma(wl, "q")), to_device(W.gen_gamma(wl, "k"))
+    qk.qknorm_force_variant(2, 0)
+    try:
+        ref = qk.qknorm_fwd(qd, kd, gqd, gkd, P, 1e-6)
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    try:
+        for i in range(24):
+            qk.qknorm_force_variant(6, (0, 0, 7, 300)[i % 4])
+            s = streams[i % 2]
+            with torch.cuda.stream(s):
+                oq, ok = torch.empty_like(qd), torch.empty_like(kd)
+                qk.qknorm_fwd(qd, kd, gqd, gkd, P, 1e-6, out_q=oq, out_k=ok, stream=s.cuda_stream)
+            outs.append((oq, ok))
+    finally:
+        qk.qknorm_force_variant(qk.VARIANT_AUTO, 0)
+    torch.cuda.synchronize()
+    assert qk.qknorm_device_errors() == 0
+    for i, (oq, ok) in enumerate(outs):
+        assert torch.equal(bits(oq), bits(ref[0])), f"launch {i} q"
+        assert torch.equal(bits(ok), bits(ref[1])), f"launch {i} k"
