@@ -850,7 +850,10 @@ static int apply_launch(int n, const void *const *x, const float *const *gamma,
     if (rowvec <= 32 * kApplyNarrowMaxV) {
         const int v = (int)((rowvec + 31) / 32);
         int bres = 1;
-        e = resident_blocks(dev, apply_narrow_kernel(dtype, v, n == 2, apply_fold(nb)), 256, 0, &bres);
+        const int vec = vec_of(dtype);
+        e = resident_blocks(dev,
+                            apply_narrow_kernel_for(dtype, v, n == 2, D[0] / vec, D[n == 2 ? 1 : 0] / vec, Pb, nb),
+                            256, 0, &bres);
         if (e != cudaSuccess) return finish(e);
         ApplyArgs a;
         for (int z = 0; z < 2; ++z) {
@@ -911,7 +914,7 @@ static int apply_blocks(const void *x, const float *gamma, const float *stats, i
 
 extern "C" {
 
-int qknorm_version(void) { return 123; }
+int qknorm_version(void) { return 125; }
 
 const char *qknorm_status_string(int status) {
     switch (status) {

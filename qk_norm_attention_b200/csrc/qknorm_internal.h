@@ -107,6 +107,10 @@ cudaError_t launch_apply(int dtype, bool multi, const ApplyArgs &a, int block, i
 // over the flat row space of one or two tensors (apply_w), 256 threads.
 constexpr int kApplyNarrowMaxV = 5;
 const void *apply_narrow_kernel(int dtype, int v, bool two, bool fold);
+// The same, or the instance compiled for this shape (rows of rv0 and rv1
+// vectors, nb blocks of Pb sums) where one exists: what launch_apply_narrow
+// launches.
+const void *apply_narrow_kernel_for(int dtype, int v, bool two, int rv0, int rv1, int Pb, int nb);
 cudaError_t launch_apply_narrow(int dtype, int v, const ApplyArgs &a, bool two, int64_t grid, cudaStream_t s);
 
 // The bulk-copy fed fused kernel (qknorm_fused_bulk.cu).

@@ -267,9 +267,13 @@ __global__ void __launch_bounds__(256) apply2_k(const ApplyArgs a) {
 // at the 13B shape, same box: 8 ranks (80 vectors per row) 61.0 -> 64.3 %
 // eager, 63.2 -> 66.0 % in a graph; 4 ranks (160) 68.1 -> 69.2 % eager,
 // 72.7 -> 77.3 % in a graph.
+// CRV, CPB, CNB: the row's vectors, the sums per block and the blocks fixed
+// at compile time for the shapes that have their own instance (0: read from
+// the arguments); fixed, the guards, the block index of each sum and the
+// fold's length are constants, the arithmetic and its order the same.
 constexpr int apply_w_blocks(int v) { return v <= 2 ? 8 : (v <= 4 ? 6 : 5); }
 
-template <class Tag, int V, bool TWO, bool FOLD>
+template <class Tag, int V, bool TWO, bool FOLD, int CRV = 0, int CPB = 0, int CNB = 0>
 __global__ void __launch_bounds__(256, apply_w_blocks(V)) apply_w(const ApplyArgs a) {
     constexpr int VEC = Tag::kVec;
     pdl_wait();
@@ -281,14 +285,15 @@ __global__ void __launch_bounds__(256, apply_w_blocks(V)) apply_w(const ApplyArg
     for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < nrows; w += nw) {
         const int z = TWO && w >= T ? 1 : 0;
         const int64_t t = z ? w - T : w;
-        const int rowvec = (z ? a.side[1].D : a.side[0].D) / VEC;
+        const int rowvec = CRV ? CRV : (z ? a.side[1].D : a.side[0].D) / VEC;
         const uint4 *src = reinterpret_cast<const uint4 *>(z ? a.side[1].x : a.side[0].x) + t * rowvec;
         uint4 xv[V];
 #pragma unroll
         for (int i = 0; i < V; ++i)
             if (lane + 32 * i < rowvec) xv[i] = ld_stream(src + lane + 32 * i);
         // Phase B: the shard sums in order of the global shard index.
-        const float r = factor(stat_sum<FOLD>(z ? a.side[1].stats : a.side[0].stats, t, a.Pb, a.nb, a.sg, lane),
+        const float r = factor(stat_sum<FOLD>(z ? a.side[1].stats : a.side[0].stats, t, CPB ? CPB : a.Pb,
+                                              CNB ? CNB : a.nb, a.sg, lane),
                                z ? a.side[1].Df : a.side[0].Df, a.eps);
         uint4 *dst = reinterpret_cast<uint4 *>(z ? a.side[1].y : a.side[0].y) + t * rowvec;
         const float *g = z ? a.side[1].g : a.side[0].g;
@@ -383,9 +388,27 @@ const void *apply_narrow_kernel(int dtype, int v, bool two, bool fold) {
     return nullptr;
 }
 
+// The instance for these shapes where one exists (two sides, bf16), else
+// the general one. A tensor-parallel rank of the 13B shape (Dq = Dk = 5120,
+// P = 8): at 8 ranks, 8 blocks of 1 sum (the row's width, 80 vectors, stays
+// a run-time value: fixing it as well made ptxas spill under the register
+// bound of 6 blocks per SM, 61.7 %), measured 64.1 -> 65.8 % eager and
+// 66.0 -> 67.8 % in a graph for the rank's step; at 4 ranks, rows of 160
+// vectors and 4 blocks of 2 sums, 69.0 -> 72.1 % and 77.3 -> 79.1 % (same box).
+const void *apply_narrow_kernel_for(int dtype, int v, bool two, int rv0, int rv1, int Pb, int nb) {
+    const bool fold = apply_fold(nb);
+    if (dtype == 1 && two) {
+        if (v == 3 && fold && Pb == 1 && nb == 8)
+            return reinterpret_cast<const void *>(&apply_w<BF16Tag, 3, true, true, 0, 1, 8>);
+        if (v == 5 && !fold && rv0 == 160 && rv1 == 160 && Pb == 2 && nb == 4)
+            return reinterpret_cast<const void *>(&apply_w<BF16Tag, 5, true, false, 160, 2, 4>);
+    }
+    return apply_narrow_kernel(dtype, v, two, fold);
+}
+
 cudaError_t launch_apply_narrow(int dtype, int v, const ApplyArgs &a, bool two, int64_t grid, cudaStream_t s) {
-    const void *fn = apply_narrow_kernel(dtype, v, two, apply_fold(a.nb));
     const int vec = dtype == 1 ? 8 : (dtype == 2 ? 16 : 4);
+    const void *fn = apply_narrow_kernel_for(dtype, v, two, a.side[0].D / vec, a.side[1].D / vec, a.Pb, a.nb);
     if (!fn || grid < 1 || a.side[0].D / vec > 32 * v || (two && a.side[1].D / vec > 32 * v))
         return cudaErrorInvalidValue;
     void *args[] = {const_cast<ApplyArgs *>(&a)};

@@ -66,6 +66,7 @@ CASES = [
     ("fold40", 51, 2560, 640, 40, "f32", 4),           # 40 sums: a round of 32 and one of 8
     ("v4", 333, 4096, 4096, 8, "bf16", 4),             # 128-vector slices: 4 vectors per lane
     ("fp8_v4", 150, 4096, 4096, 8, "e4m3", 2),
+    ("13b_p8_r4", 2 * 148 + 3, 5120, 5120, 8, "bf16", 4),   # 160-vector slices, 4 blocks of 2 sums
 ]
 
 
